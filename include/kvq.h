@@ -1,0 +1,257 @@
+/*
+ * kvq.h -- C ABI of the B200 (sm_100a) per-token KV-cache epilogue library.
+ *
+ * One call per operation.  Each call validates its arguments on the host and,
+ * if they are valid, enqueues exactly one kernel on the given CUDA stream and
+ * returns.  Nothing is allocated, nothing is synchronised, no workspace is
+ * needed; the caller owns every buffer.  Caches (and cache_scale) are updated
+ * IN PLACE: only the rows addressed by a valid slot are written, and within a
+ * row only the bytes the operation defines; every other byte keeps its value.
+ * Execution is deterministic: each row has exactly one writer and no atomics
+ * touch the outputs.
+ *
+ * Tensors are passed as kvq_tensor descriptors: a DEVICE pointer to element
+ * [0, ..., 0], a dtype, and shape/stride in ELEMENTS (not bytes).  The
+ * library never dereferences a descriptor's data on the host.
+ *
+ * Errors.  A host-detected problem (null pointer, wrong rank, shape, dtype,
+ * attribute, layout or capacity) returns a nonzero kvq_status and launches
+ * nothing.  After a launch the call returns KVQ_ERR_CUDA if the launch itself
+ * failed (cudaGetLastError), else KVQ_OK.  Data faults the device can see --
+ * a slot index outside [0, num_slots) that is not -1 -- skip the affected row
+ * and set a bit in a per-device fault word that kvq_get_error() returns and
+ * clears.  Duplicate slots are not detected (the pages declare the result
+ * undefined); rows then have two writers and either may win.
+ *
+ * Sources (page title and section):
+ *   aclnnKvCompressEpilog        -- 接口功能, 计算公式, 约束说明
+ *   aclnnKvRmsNormRopeCache      -- 接口功能, 计算公式, 约束说明
+ *   indexer_quant_cache          -- 接口功能, 语义说明, 约束说明 (torch_npu op)
+ *   aclnnDequantRopeQuantKvcache 算子深度解析 -- 计算步骤公式, 两段式接口与函数原型,
+ *                                   约束说明, Shape 推导逻辑, Kernel 实现要点
+ * The pages' two-stage GetWorkspaceSize + execute pattern becomes one call:
+ * the workspace is always 0 bytes and validation happens before the launch.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Symbols of the ABI are exported; everything else in the library is hidden. */
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+/* A CUDA stream (the same object as cudaStream_t / CUstream).  NULL is the
+ * legacy default stream. */
+struct CUstream_st;
+typedef struct CUstream_st* kvq_stream;
+
+typedef enum {
+    KVQ_BF16 = 0,
+    KVQ_F16 = 1,
+    KVQ_F32 = 2,
+    KVQ_I32 = 3,
+    KVQ_I64 = 4,
+    KVQ_I8 = 5,
+    KVQ_U8 = 6,
+    KVQ_F8E4M3 = 7,   /* FLOAT8 E4M3FN: no infinities, max 448 */
+    KVQ_F8E5M2 = 8,   /* FLOAT8 E5M2: max finite 57344 */
+    KVQ_E8M0 = 9      /* unsigned 8-bit power-of-two scale 2^(b-127) */
+} kvq_dtype;
+
+#define KVQ_MAX_DIMS 8
+
+typedef struct {
+    void* data;                       /* device pointer to element [0,...,0] */
+    int32_t dtype;                    /* kvq_dtype */
+    int32_t ndim;                     /* 0 .. KVQ_MAX_DIMS */
+    int64_t shape[KVQ_MAX_DIMS];
+    int64_t stride[KVQ_MAX_DIMS];     /* in elements */
+} kvq_tensor;
+
+typedef enum {
+    KVQ_OK = 0,
+    KVQ_ERR_NULL = 1,         /* a required tensor or its data pointer is NULL */
+    KVQ_ERR_NDIM = 2,         /* wrong number of dimensions */
+    KVQ_ERR_SHAPE = 3,        /* inconsistent sizes */
+    KVQ_ERR_DTYPE = 4,        /* dtype not allowed here */
+    KVQ_ERR_ATTR = 5,         /* bad attribute value (mode, group size, ...) */
+    KVQ_ERR_LAYOUT = 6,       /* non-contiguous where contiguity is required */
+    KVQ_ERR_CAPACITY = 7,     /* cache row (headDim) too small for the packed row */
+    KVQ_ERR_CUDA = 8,         /* the CUDA runtime reported an error */
+    KVQ_ERR_UNSUPPORTED = 9   /* a valid combination this library does not implement */
+} kvq_status;
+
+/* Fault bits of the device fault word. */
+#define KVQ_FAULT_SLOT_RANGE 0x1u   /* a slot/index outside [0, num_slots) and not -1 */
+
+/* ------------------------------------------------------------------------ */
+/* kv_compress_epilog                                                        */
+/* Source: aclnnKvCompressEpilog, 接口功能 / 计算公式 / 约束说明.               */
+/*                                                                           */
+/* x            bf16 [..., d]; the last dimension contiguous, the leading     */
+/*              dimensions flattenable to T rows with one row stride.         */
+/*              64 < d <= 8192, d % 64 == 0.  Columns [0, d-64) are the nope  */
+/*              segment, [d-64, d) the rope segment.                          */
+/* slot_mapping int32 or int64, T elements (x's leading dims flattened),     */
+/*              contiguous.  -1 skips the token; other values in             */
+/*              [0, blockNum*blockSize) and distinct.                         */
+/* cache        uint8 [blockNum, blockSize, 1, headDim], headDim >= kvCacheCol */
+/*              (kvq_kv_cache_col).  Rows contiguous inside a block; only    */
+/*              the blockNum dimension may be strided.                        */
+/* quant_mode   0: groups of 64 -> FP8 E4M3, bf16 scale = amax/448;          */
+/*              1: groups of 64 -> FP8 E4M3, E8M0 scale = amax/448 rounded up */
+/*                 to a power of two;                                         */
+/*              2: nope groups of quant_group_size -> FP4 E2M1, bf16 scale =  */
+/*                 amax/6; rope -> FP8 E4M3 of x * x_scale (this library's   */
+/*                 stand-in for the pages' hifloat8).                         */
+/* quant_group_size  16, 32 or 64 in mode 2 ((d-64) % G == 0); ignored else. */
+/* x_scale      mode 2 rope multiplier; ignored else.                         */
+/* Codes are round-to-nearest-even with saturation of x divided by the       */
+/* STORED scale; a stored bf16 scale of 0 gives all-zero codes.              */
+/* Packed row (kvCacheCol bytes, written from byte 0 of the slot row):       */
+/*   modes 0/1: [d-64 code bytes][64 bf16 rope values][(d-64)/64 scales]     */
+/*   mode 2:    [(d-64)/2 bytes of FP4 pairs, even element in the low nibble] */
+/*              [64 E4M3 rope codes][(d-64)/G bf16 scales]                   */
+/*   then 0x00 up to kvCacheCol (32-byte alignment in modes 0 and 2).        */
+/* ------------------------------------------------------------------------ */
+KVQ_API kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_mapping, kvq_tensor* cache,
+                                  int32_t quant_mode, int32_t quant_group_size, float x_scale,
+                                  kvq_stream stream);
+
+/* Bytes of one packed row (kvCacheCol) for kv_compress_epilog, or -1 for an
+ * invalid (d, quant_mode, quant_group_size).  Closed form of
+ * aclnnKvCompressEpilog 约束说明 (headDim constraint); d=256, mode 1 -> 323. */
+KVQ_API int64_t kvq_kv_cache_col(int64_t d, int32_t quant_mode, int32_t quant_group_size);
+
+/* ------------------------------------------------------------------------ */
+/* indexer_quant_cache                                                       */
+/* Source: indexer_quant_cache, 接口功能 / 语义说明 / 约束说明.                 */
+/*                                                                           */
+/* x            bf16 or f16 [..., d], last dimension contiguous, leading dims */
+/*              flattenable to T rows.                                        */
+/* cache        [blockNum, blockSize, 1, headDim]: FLOAT8 E4M3 or E5M2 for    */
+/*              mxfp8/fp8 (headDim >= d), uint8 for mxfp4 (headDim >=         */
+/*              ceil(d/2) bytes, two E2M1 codes per byte, even element low).  */
+/* cache_scale  [blockNum, blockSize, 1, scaleHeadDim] with the same blockNum */
+/*              and blockSize: E8M0 (or uint8) for mxfp8/mxfp4, scaleHeadDim  */
+/*              >= ceil(d/32); FLOAT32 for fp8, scaleHeadDim >= 1.            */
+/* slot_mapping int32/int64, T elements, -1 skips.                            */
+/* quant_mode   0 mxfp8 (groups of 32, E8M0 scale rounded up, codes          */
+/*                FP8(x / 2^(b-127)), format from cache dtype);               */
+/*              1 fp8 (one group per row, fp32 scale = amax / FP8_MAX);      */
+/*              2 hifloat8 -> KVQ_ERR_UNSUPPORTED (no NVIDIA type);          */
+/*              3 mxfp4 (groups of 32, E8M0 scale, E2M1 codes).               */
+/* ------------------------------------------------------------------------ */
+KVQ_API kvq_status kvq_indexer_quant_cache(const kvq_tensor* x, kvq_tensor* cache, kvq_tensor* cache_scale,
+                                   const kvq_tensor* slot_mapping, int32_t quant_mode, kvq_stream stream);
+
+/* scaleCol of indexer_quant_cache: ceil(d/32) for mxfp8/mxfp4, 1 for fp8 and
+ * hifloat8, -1 otherwise.  The page's example: d=128, mode 0 -> 4. */
+KVQ_API int64_t kvq_indexer_scale_col(int64_t d, int32_t quant_mode);
+
+/* ------------------------------------------------------------------------ */
+/* kv_rmsnorm_rope_cache                                                     */
+/* Source: aclnnKvRmsNormRopeCache, 接口功能 / 计算公式 / 约束说明.             */
+/*                                                                           */
+/* kv        bf16 or f16 [B, 1, S, D] contiguous (N = 1).  D = Dv + Dk with   */
+/*           Dv = ckv_cache's last dim, Dk = k_cache's last dim, Dk even.     */
+/* gamma     [Dv], same dtype as kv.                                          */
+/* cos, sin  [B, 1, S, Dk], same dtype as kv, contiguous.                     */
+/* index     int32/int64.  cache_mode 0 Norm: [B, S], values in [-1, Scache), */
+/*           caches [Bc, 1, Scache, Dc] with Bc >= B; 1 PA and 2 PA_BNSD:     */
+/*           [B*S], values in [-1, blockNum*blockSize), caches               */
+/*           [blockNum, blockSize, 1, Dc] or [blockNum, 1, blockSize, Dc];   */
+/*           3 PA_BLK_BNSD: [B*ceil(S/blockSize)], entry v places token s of  */
+/*           batch b in block v/blockSize at offset s % blockSize.  -1 skips. */
+/* k_cache   receives RoPE(kv[..., Dv:]) (interleaved pairs, de-interleaved   */
+/* ckv_cache output order); ckv_cache receives RMSNorm(kv[..., :Dv]) * gamma. */
+/*           dtypes: bf16/f16 (stored rounded to nearest even), or FLOAT8     */
+/*           E4M3/E5M2 or int8 (static quantisation fp(y / scale), int8 also  */
+/*           + offset, round half even, saturating); a quantised cache needs  */
+/*           its scale tensor (f32, 1 or Dc elements); offsets only for int8. */
+/*           blockSize % 32 == 0 for 1-byte caches, % 16 for 2-byte caches.   */
+/* RMSNorm: rms = sqrt(mean(x*x) + epsilon), y = (x / rms) * gamma.  The sum */
+/* of squares uses a fixed order: element i belongs to 8-element chunk i/8,   */
+/* chunk c to lane c % 32; lanes add their elements in index order; the 32    */
+/* partial sums combine by the butterfly p[l] += p[l ^ k], k = 16..1.         */
+/* ------------------------------------------------------------------------ */
+KVQ_API kvq_status kvq_kv_rmsnorm_rope_cache(const kvq_tensor* kv, const kvq_tensor* gamma, const kvq_tensor* cos,
+                                     const kvq_tensor* sin, const kvq_tensor* index, kvq_tensor* k_cache,
+                                     kvq_tensor* ckv_cache, const kvq_tensor* k_scale,
+                                     const kvq_tensor* ckv_scale, const kvq_tensor* k_offset,
+                                     const kvq_tensor* ckv_offset, float epsilon, int32_t cache_mode,
+                                     kvq_stream stream);
+
+/* ------------------------------------------------------------------------ */
+/* dequant_rope_quant_kvcache                                                */
+/* Source: aclnnDequantRopeQuantKvcache 算子深度解析, 计算步骤公式, 两种 KV     */
+/* Cache 更新模式, 两段式接口与函数原型 (argument order), 约束说明, Shape 推导.   */
+/*                                                                           */
+/* x          int32, bf16 or f16, [B, S, H] or [B, H] (S = 1), contiguous.    */
+/* cos, sin   bf16 or f16 [B, S, 1, D] (or [B, 1, D] / [B, 1, 1, D] for 2-D  */
+/*            x), contiguous; for a 16-bit x the same dtype as x.            */
+/* k_cache,   int8 [c0, c1, Nkv, D], (Nkv, D) contiguous, only dim 0 strided. */
+/* v_cache    D % 32 == 0.                                                    */
+/* indices    int32/int64.  page (cache_mode 1): [B*S], row                   */
+/*            cache.view(-1, Nkv, D)[indices[t]], values in [0, c0*c1);       */
+/*            contiguous (0): [B], token s of batch b -> cache[b][indices[b]+s]. */
+/*            -1 skips (page mode: the token; contiguous: the batch).         */
+/* scale_k, scale_v     f32, Nkv*D elements; offset_k/v optional, f32.        */
+/* weight_scale         f32 [H], required for int32 x;                        */
+/* activation_scale     f32 [B*S], optional; bias [H] optional, f32/f16/bf16/ */
+/*                      int32.  For a 16-bit x these three are ignored.       */
+/* size_splits          {Nq*D, Nkv*D, Nkv*D}, n_splits == 3, sum == H.        */
+/* quant_mode 0 ("static"), layout 0 ("BSND") are the only values.            */
+/* kv_output  nonzero: k_out / v_out [B, S, Nkv, D] (cos dtype) are written.  */
+/* q_out      [B, S, Nq, D] (or [B, Nq, D]) in the cos dtype.                 */
+/* Per token: v = ((float)x * weight_scale[h]) * activation_scale[t] + bias[h]; */
+/* split; half-rotation RoPE on q and k heads: o_j = u_j c_j - u_{j+D/2} s_j,  */
+/* o_{j+D/2} = u_{j+D/2} c_{j+D/2} + u_j s_{j+D/2}; int8 quantisation of k     */
+/* (after RoPE, binary32) and v: clamp(rint(w / scale + offset), -128, 127).  */
+/* ------------------------------------------------------------------------ */
+KVQ_API kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor* cos, const kvq_tensor* sin,
+                                          kvq_tensor* k_cache, kvq_tensor* v_cache, const kvq_tensor* indices,
+                                          const kvq_tensor* scale_k, const kvq_tensor* scale_v,
+                                          const kvq_tensor* offset_k, const kvq_tensor* offset_v,
+                                          const kvq_tensor* weight_scale, const kvq_tensor* activation_scale,
+                                          const kvq_tensor* bias, const int64_t* size_splits, int32_t n_splits,
+                                          int32_t quant_mode, int32_t layout, int32_t kv_output,
+                                          int32_t cache_mode, kvq_tensor* q_out, kvq_tensor* k_out,
+                                          kvq_tensor* v_out, kvq_stream stream);
+
+/* ------------------------------------------------------------------------ */
+/* Utilities                                                                 */
+/* ------------------------------------------------------------------------ */
+
+/* Enqueue a read of this device's fault word, wait for `stream`, store the
+ * bits in *fault_bits and clear the word.  Returns KVQ_ERR_CUDA if the stream
+ * reported an error (the bits are then 0). */
+KVQ_API kvq_status kvq_get_error(kvq_stream stream, uint32_t* fault_bits);
+
+/* Element-wise conversion of n binary32 values on the device with the same
+ * device codecs the kernels use (no counterpart on the pages; it lets the
+ * codecs be checked exhaustively).  fmt: 0 E4M3 (satfinite, 1 byte each),
+ * 1 E5M2 (satfinite), 2 E2M1 (satfinite, one code per byte in the low
+ * nibble), 3 bf16 (2 bytes, RNE), 4 E8M0 rounded up (1 byte), 5 int8 static
+ * (1 byte, rint then clamp).  in, out: device pointers. */
+KVQ_API kvq_status kvq_convert(int32_t fmt, const float* in, int64_t n, void* out, kvq_stream stream);
+
+/* Static description of a status code. */
+KVQ_API const char* kvq_status_string(kvq_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+KVQ_API int32_t kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

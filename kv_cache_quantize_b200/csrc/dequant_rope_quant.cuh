@@ -1,0 +1,216 @@
+// dequant_rope_quant.cuh -- dequant_rope_quant_kvcache kernel
+// (aclnnDequantRopeQuantKvcache 算子深度解析: 计算步骤公式 steps 1-5, 两种 KV
+// Cache 更新模式, Kernel 实现要点: dequant Cast -> Mul -> Muls -> Add, RoPE with
+// the sine negated first, quant Div -> Add offset -> round to int8).
+//
+// A CTA walks tokens (grid-stride); its DQ_WARPS warps split the token's
+// Nq + 2*Nkv heads (warp w takes heads w, w + DQ_WARPS, ...).  Within a head of
+// D values each lane holds E = D/32 consecutive values, so the first half of
+// the head sits in lanes 0-15 and the second half in lanes 16-31 at the same
+// register positions: the half-rotation partner of every value is one
+// __shfl_xor(16) away.  Up to DQ_PASS of a warp's heads are loaded before
+// any of them is processed.
+#pragma once
+
+#include "kvq_device.cuh"
+
+namespace kvq {
+
+struct DrqArgs {
+    const void* x;          // [B*S, H]
+    int32_t x_kind;         // 0 int32, 1 bf16, 2 f16
+    int64_t B, S, H;
+    const uint16_t* cos;    // [B*S, D]
+    const uint16_t* sin;
+    int32_t cos_f16;        // cos/sin and the 16-bit outputs are f16 (else bf16)
+    PagedRows kc, vc;       // rows of Nkv*D int8
+    const void* indices;
+    int32_t indices_i64;
+    int32_t cache_mode;     // 0 contiguous, 1 page
+    const float* scale_k;
+    const float* scale_v;
+    const float* offset_k;  // nullable
+    const float* offset_v;
+    const float* weight_scale;      // [H], int32 x only
+    const float* activation_scale;  // [B*S] nullable
+    const void* bias;               // [H] nullable
+    int32_t bias_kind;              // 0 f32, 1 f16, 2 bf16, 3 int32
+    int32_t Nq, Nkv, D;
+    uint16_t* q_out;        // [B*S, Nq*D]
+    uint16_t* k_out;        // [B*S, Nkv*D] or null
+    uint16_t* v_out;
+};
+
+constexpr int DQ_WARPS = 8;
+constexpr int DQ_MAX_HEADS_PER_WARP = 8;
+constexpr int DQ_PASS = 4;
+
+template <int E>
+__device__ __forceinline__ void dq_load(const DrqArgs& a, int64_t e0, float (&u)[E], const int32_t* xi) {
+    if (a.x_kind == 0) {
+        int32_t v[E];
+        if (E % 4 == 0) {
+#pragma unroll
+            for (int k = 0; k < E; k += 4) {
+                const int4 w = __ldcs(reinterpret_cast<const int4*>(xi + e0 + k));
+                v[k] = w.x; v[k + 1] = w.y; v[k + 2] = w.z; v[k + 3] = w.w;
+            }
+        } else if (E % 2 == 0) {
+#pragma unroll
+            for (int k = 0; k < E; k += 2) {
+                const int2 w = __ldcs(reinterpret_cast<const int2*>(xi + e0 + k));
+                v[k] = w.x; v[k + 1] = w.y;
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < E; ++k) v[k] = __ldcs(xi + e0 + k);
+        }
+#pragma unroll
+        for (int k = 0; k < E; ++k) u[k] = __int2float_rn(v[k]);
+    } else {
+        const uint16_t* xh = reinterpret_cast<const uint16_t*>(a.x);
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+            const uint32_t hb = __ldcs(xh + e0 + k);
+            u[k] = a.x_kind == 2 ? __half2float(__ushort_as_half((unsigned short)hb)) : __uint_as_float(hb << 16);
+        }
+    }
+}
+
+__device__ __forceinline__ float dq_bias(const DrqArgs& a, int64_t i) {
+    switch (a.bias_kind) {
+        case 0: return reinterpret_cast<const float*>(a.bias)[i];
+        case 1: return __half2float(__ushort_as_half(reinterpret_cast<const unsigned short*>(a.bias)[i]));
+        case 2: return __uint_as_float((uint32_t) reinterpret_cast<const uint16_t*>(a.bias)[i] << 16);
+        default: return __int2float_rn(reinterpret_cast<const int32_t*>(a.bias)[i]);
+    }
+}
+
+__device__ __forceinline__ uint32_t dq_round16(const DrqArgs& a, float v) {
+    return a.cos_f16 ? to_f16_bits(v) : to_bf16_bits(v);
+}
+
+template <int E>
+__device__ __forceinline__ void dq_store16(uint16_t* p, const DrqArgs& a, const float (&o)[E]) {
+#pragma unroll
+    for (int k = 0; k < E; ++k) p[k] = (uint16_t)dq_round16(a, o[k]);
+}
+
+// One head of one token: dequant, RoPE (q and k heads), outputs, int8 quant
+// and the cache write.  Called with the whole warp (the RoPE shuffle).
+template <int E>
+__device__ __forceinline__ void dq_head(const DrqArgs& a, int64_t t, int hd, float (&u)[E], const float (&cs)[E],
+                                        const float (&sn)[E], float act, int64_t slot, int pos, bool second_half) {
+    const int D = a.D;
+    const int ch0 = hd * D + pos;    // channel index within H
+    // 1 dequant: ((float)x * weight_scale) * activation_scale + bias
+    if (a.x_kind == 0) {
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+            float v = __fmul_rn(u[k], a.weight_scale[ch0 + k]);
+            if (a.activation_scale) v = __fmul_rn(v, act);
+            if (a.bias) v = __fadd_rn(v, dq_bias(a, ch0 + k));
+            u[k] = v;
+        }
+    }
+    float o[E];
+    if (hd < a.Nq + a.Nkv) {
+        // 3 RoPE, half rotation: the partner value is 16 lanes away
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+            const float p = __shfl_xor_sync(FULL_MASK, u[k], 16);
+            const float sgn_s = second_half ? sn[k] : -sn[k];
+            o[k] = __fadd_rn(__fmul_rn(u[k], cs[k]), __fmul_rn(p, sgn_s));
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < E; ++k) o[k] = u[k];
+    }
+    if (hd < a.Nq) {
+        dq_store16<E>(a.q_out + t * (int64_t)(a.Nq * D) + ch0, a, o);
+        return;
+    }
+    const bool is_k = hd < a.Nq + a.Nkv;
+    const int c0 = (is_k ? hd - a.Nq : hd - a.Nq - a.Nkv) * D + pos;   // channel in [0, Nkv*D)
+    if (a.k_out) dq_store16<E>((is_k ? a.k_out : a.v_out) + t * (int64_t)(a.Nkv * D) + c0, a, o);
+    if (slot < 0) return;
+    // 4 quant: int8(rint(w / scale + offset)), saturating
+    const float* sc = is_k ? a.scale_k : a.scale_v;
+    const float* of = is_k ? a.offset_k : a.offset_v;
+    uint32_t packed[(E + 3) / 4];
+#pragma unroll
+    for (int k = 0; k < (E + 3) / 4; ++k) packed[k] = 0u;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        float q = __fdiv_rn(o[k], sc[c0 + k]);
+        if (of) q = __fadd_rn(q, of[c0 + k]);
+        packed[k / 4] |= ((uint32_t)int8_rne_sat(q) & 0xffu) << (8 * (k % 4));
+    }
+    // 5 cache write
+    uint8_t* row = slot_row(is_k ? a.kc : a.vc, slot) + c0;
+    if (E % 4 == 0) {
+#pragma unroll
+        for (int k = 0; k < E / 4; ++k) st_b32(row + 4 * k, packed[k]);
+    } else {
+#pragma unroll
+        for (int k = 0; k < E; ++k) row[k] = (uint8_t)(packed[k / 4] >> (8 * (k % 4)));
+    }
+}
+
+template <int E>
+__global__ void __launch_bounds__(DQ_WARPS * 32) dequant_rope_quant_kernel(const DrqArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int NH = a.Nq + 2 * a.Nkv;
+    const int64_t ntok = a.B * a.S;
+    const int D = a.D;
+    const int pos = lane * E;                // first position of this lane inside a head
+    const bool second_half = lane >= 16;
+    const int32_t* xi = reinterpret_cast<const int32_t*>(a.x);
+
+    for (int64_t t = blockIdx.x; t < ntok; t += gridDim.x) {
+        // destination row of this token (or -1 skip / -2 fault)
+        int64_t slot;
+        if (a.cache_mode == 1) {
+            slot = load_slot(a.indices, a.indices_i64, t);
+            if (slot != -1 && !slot_ok(slot, a.kc.num_slots)) slot = -2;
+        } else {
+            const int64_t b = t / a.S, s = t - b * a.S;
+            const int64_t start = load_slot(a.indices, a.indices_i64, b);
+            const int64_t c1 = a.kc.block_size;
+            if (start == -1) slot = -1;
+            else if (start < 0 || start + s >= c1 || b * c1 >= a.kc.num_slots) slot = -2;
+            else slot = b * c1 + start + s;
+        }
+        if (slot == -2 && threadIdx.x == 0) raise_fault(FAULT_SLOT_RANGE);
+
+        float cs[E], sn[E];
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+            const uint32_t cb = a.cos[t * D + pos + k], sb = a.sin[t * D + pos + k];
+            cs[k] = a.cos_f16 ? __half2float(__ushort_as_half((unsigned short)cb)) : __uint_as_float(cb << 16);
+            sn[k] = a.cos_f16 ? __half2float(__ushort_as_half((unsigned short)sb)) : __uint_as_float(sb << 16);
+        }
+        const float act = (a.x_kind == 0 && a.activation_scale) ? a.activation_scale[t] : 1.0f;
+
+        // the warp's heads are hd = warp + i * DQ_WARPS; DQ_PASS of them are
+        // loaded before any is processed
+        const int nh = (NH - warp + DQ_WARPS - 1) / DQ_WARPS;
+        for (int i0 = 0; i0 < nh; i0 += DQ_PASS) {
+            float u[DQ_PASS][E];
+#pragma unroll
+            for (int i = 0; i < DQ_PASS; ++i) {
+                const int hd = warp + (i0 + i) * DQ_WARPS;
+                if (i0 + i < nh) dq_load<E>(a, t * a.H + (int64_t)hd * D + pos, u[i], xi);
+            }
+#pragma unroll
+            for (int i = 0; i < DQ_PASS; ++i) {
+                if (i0 + i >= nh) break;
+                const int hd = warp + (i0 + i) * DQ_WARPS;
+                dq_head<E>(a, t, hd, u[i], cs, sn, act, slot, pos, second_half);
+            }
+        }
+    }
+}
+
+}  // namespace kvq

@@ -1,0 +1,168 @@
+// indexer_quant.cuh -- indexer_quant_cache kernel (indexer_quant_cache,
+// 接口功能: mxfp8 / mxfp4 groups of 32 with an E8M0 scale, fp8 one group per
+// row with a binary32 scale; 约束说明 for the cache / cache_scale rows).
+//
+// A row is handled by a TEAM of TEAM lanes (4, 8, 16 or 32), one 16-byte chunk
+// of 8 values per lane, so a 32-value group is 4 adjacent lanes and its
+// maximum is two butterfly shuffles.  Rows longer than 8*TEAM values (TEAM 32
+// only) are walked in blocks of 8*TEAM values.  A warp owns a tile of 32 rows
+// whose slots it loads once; 32/TEAM rows are in flight per step and
+// IX_UNROLL steps are loaded before they are processed.
+#pragma once
+
+#include "kvq_device.cuh"
+
+namespace kvq {
+
+struct IndexerArgs {
+    const uint16_t* x;
+    int64_t x_row_stride;
+    int64_t T;
+    int32_t d;
+    int32_t nchunks;      // ceil(d / 8)
+    int32_t x_f16;
+    int32_t x_vec;        // every full chunk is 16-byte aligned
+    const void* slots;
+    int32_t slots_i64;
+    PagedRows cache;      // codes
+    PagedRows scale;      // cache_scale rows
+    int32_t e5m2;         // FP8 codes in E5M2 (else E4M3)
+};
+
+constexpr int IX_THREADS = 256;
+constexpr int IX_UNROLL = 2;
+
+// Load the values [8c, 8c + 8) of a row, zero beyond d.
+__device__ __forceinline__ uint4 ix_load_chunk(const IndexerArgs& a, const uint16_t* xrow, int c) {
+    const int nvalid = a.d - 8 * c;
+    if (nvalid >= 8 && a.x_vec) return ld_stream16(xrow + 8 * c);
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        if (i < nvalid) w[i >> 1] |= (uint32_t)__ldcs(xrow + 8 * c + i) << (16 * (i & 1));
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ void ix_widen(const IndexerArgs& a, const uint4& v, float (&f)[8]) {
+    if (a.x_f16) widen8<true>(v, f); else widen8<false>(v, f);
+}
+
+__device__ __forceinline__ uint2 ix_fp8x8(const IndexerArgs& a, const float (&q)[8]) {
+    return a.e5m2 ? fp8x8<true>(q) : fp8x8<false>(q);
+}
+
+// mx modes: quantise chunk c of a row whose group maximum (bits) is m.
+template <int MODE>
+__device__ __forceinline__ void ix_mx_chunk(const IndexerArgs& a, const uint4& v, uint32_t m, uint8_t* crow,
+                                            uint8_t* srow, int c, int tl) {
+    const int nvalid = a.d - 8 * c;
+    if (nvalid <= 0) return;
+    const float amax = a.x_f16 ? __half2float(__ushort_as_half((unsigned short)m)) : __uint_as_float(m << 16);
+    const float fmax = MODE == 3 ? 6.0f : (a.e5m2 ? 57344.0f : 448.0f);
+    const uint32_t b = e8m0_ceil(__fdiv_rn(amax, fmax));
+    const float mul = e8m0_reciprocal(b);
+    float f[8], q[8];
+    ix_widen(a, v, f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(f[i], mul);
+    if (MODE == 0) {
+        const uint2 codes = ix_fp8x8(a, q);
+        if (nvalid >= 8) st_b64(crow + 8 * c, codes);
+        else st_partial(crow + 8 * c, make_uint4(codes.x, codes.y, 0u, 0u), nvalid);
+    } else {
+        const uint32_t codes = e2m1x8(q);
+        if (nvalid >= 8) st_b32(crow + 4 * c, codes);
+        else st_partial(crow + 4 * c, make_uint4(codes, 0u, 0u, 0u), (nvalid + 1) / 2);
+    }
+    if ((tl & 3) == 0) st_b8(srow + (c >> 2), b);
+}
+
+template <int MODE, int TEAM>
+__global__ void __launch_bounds__(IX_THREADS) indexer_quant_kernel(const IndexerArgs a) {
+    constexpr int RPS = 32 / TEAM;   // rows per warp step
+    const int lane = threadIdx.x & 31;
+    const int tm = lane / TEAM;
+    const int tl = lane % TEAM;
+    const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t ntiles = (a.T + 31) / 32;
+    const int nblocks = (a.nchunks + TEAM - 1) / TEAM;
+
+    for (int64_t tile = gwarp; tile < ntiles; tile += nwarps) {
+        const int64_t row0 = tile * 32;
+        const int rows = (int)(a.T - row0 < 32 ? a.T - row0 : 32);
+        int64_t my_slot = -1;
+        if (lane < rows) {
+            my_slot = load_slot(a.slots, a.slots_i64, row0 + lane);
+            if (my_slot != -1 && !slot_ok(my_slot, a.cache.num_slots)) {
+                raise_fault(FAULT_SLOT_RANGE);
+                my_slot = -1;
+            }
+        }
+        for (int r0 = 0; r0 < rows; r0 += RPS * IX_UNROLL) {
+            int64_t sl[IX_UNROLL];
+            bool live[IX_UNROLL];
+            const uint16_t* xrow[IX_UNROLL];
+#pragma unroll
+            for (int u = 0; u < IX_UNROLL; ++u) {
+                const int r = r0 + u * RPS + tm;
+                const bool act = r < rows;
+                sl[u] = __shfl_sync(FULL_MASK, my_slot, act ? r : 0);
+                live[u] = act && sl[u] >= 0;
+                xrow[u] = a.x + (row0 + (act ? r : 0)) * a.x_row_stride;
+            }
+            if (MODE == 1) {
+                // fp8: one group per row -> row maximum, then quantise
+#pragma unroll
+                for (int u = 0; u < IX_UNROLL; ++u) {
+                    uint32_t m = 0u;
+                    for (int cb = 0; cb < nblocks; ++cb) {
+                        const int c = cb * TEAM + tl;
+                        if (live[u] && c < a.nchunks) m = max(m, absmax_bits8(ix_load_chunk(a, xrow[u], c)));
+                    }
+#pragma unroll
+                    for (int k = TEAM / 2; k >= 1; k >>= 1) m = max(m, __shfl_xor_sync(FULL_MASK, m, k));
+                    if (!live[u]) continue;
+                    const float amax = a.x_f16 ? __half2float(__ushort_as_half((unsigned short)m))
+                                               : __uint_as_float(m << 16);
+                    const float scale = __fdiv_rn(amax, a.e5m2 ? 57344.0f : 448.0f);
+                    uint8_t* crow = slot_row(a.cache, sl[u]);
+                    for (int cb = 0; cb < nblocks; ++cb) {
+                        const int c = cb * TEAM + tl;
+                        if (c >= a.nchunks) continue;
+                        float f[8], q[8];
+                        ix_widen(a, ix_load_chunk(a, xrow[u], c), f);
+                        uint2 codes = make_uint2(0u, 0u);
+                        if (scale != 0.0f) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], scale);
+                            codes = ix_fp8x8(a, q);
+                        }
+                        const int nvalid = a.d - 8 * c;
+                        if (nvalid >= 8) st_b64(crow + 8 * c, codes);
+                        else st_partial(crow + 8 * c, make_uint4(codes.x, codes.y, 0u, 0u), nvalid);
+                    }
+                    if (tl == 0) st_b32(slot_row(a.scale, sl[u]), __float_as_uint(scale));
+                }
+            } else {
+                for (int cb = 0; cb < nblocks; ++cb) {
+                    const int c = cb * TEAM + tl;
+                    uint4 v[IX_UNROLL];
+#pragma unroll
+                    for (int u = 0; u < IX_UNROLL; ++u)
+                        v[u] = (live[u] && c < a.nchunks) ? ix_load_chunk(a, xrow[u], c) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int u = 0; u < IX_UNROLL; ++u) {
+                        uint32_t m = absmax_bits8(v[u]);
+                        m = max(m, __shfl_xor_sync(FULL_MASK, m, 1));
+                        m = max(m, __shfl_xor_sync(FULL_MASK, m, 2));
+                        if (live[u] && c < a.nchunks)
+                            ix_mx_chunk<MODE>(a, v[u], m, slot_row(a.cache, sl[u]), slot_row(a.scale, sl[u]), c, tl);
+                    }
+                }
+            }
+        }
+    }
+}
+
+}  // namespace kvq

@@ -1,0 +1,646 @@
+// kvq.cu -- host side of the C ABI declared in include/kvq.h: argument
+// validation, kernel selection and launch.  Single translation unit: the
+// kernels live in the .cuh files included below.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "kvq.h"
+#include "compress_epilog.cuh"
+#include "dequant_rope_quant.cuh"
+#include "indexer_quant.cuh"
+#include "rmsnorm_rope.cuh"
+
+namespace {
+
+using namespace kvq;
+
+// ---------------------------------------------------------------------------
+// descriptor helpers
+// ---------------------------------------------------------------------------
+int64_t elem_bytes(int32_t dt) {
+    switch (dt) {
+        case KVQ_BF16: case KVQ_F16: return 2;
+        case KVQ_F32: case KVQ_I32: return 4;
+        case KVQ_I64: return 8;
+        case KVQ_I8: case KVQ_U8: case KVQ_F8E4M3: case KVQ_F8E5M2: case KVQ_E8M0: return 1;
+        default: return 0;
+    }
+}
+
+bool valid_desc(const kvq_tensor* t) {
+    if (!t || t->ndim < 0 || t->ndim > KVQ_MAX_DIMS || elem_bytes(t->dtype) == 0) return false;
+    for (int i = 0; i < t->ndim; ++i)
+        if (t->shape[i] < 0) return false;
+    return true;
+}
+
+int64_t numel(const kvq_tensor* t) {
+    int64_t n = 1;
+    for (int i = 0; i < t->ndim; ++i) n *= t->shape[i];
+    return n;
+}
+
+// Row-major contiguous (dimensions of size 1 may carry any stride).
+bool contiguous(const kvq_tensor* t) {
+    int64_t expect = 1;
+    for (int i = t->ndim - 1; i >= 0; --i) {
+        if (t->shape[i] == 1) continue;
+        if (t->stride[i] != expect) return false;
+        expect *= t->shape[i];
+    }
+    return true;
+}
+
+// Last dimension contiguous and the leading dimensions flattenable into rows
+// with one row stride (in elements).
+bool flatten_rows(const kvq_tensor* t, int64_t* rows, int64_t* row_stride) {
+    if (t->ndim < 1) return false;
+    const int64_t d = t->shape[t->ndim - 1];
+    if (d > 1 && t->stride[t->ndim - 1] != 1) return false;
+    int64_t r = 1, rs = -1, expect = -1;
+    for (int i = t->ndim - 2; i >= 0; --i) {
+        r *= t->shape[i];
+        if (t->shape[i] == 1) continue;
+        if (rs < 0) {
+            rs = t->stride[i];
+        } else if (t->stride[i] != expect) {
+            return false;
+        }
+        expect = t->stride[i] * t->shape[i];
+    }
+    if (rs < 0) rs = d;
+    if (r > 1 && rs < d) return false;
+    *rows = r;
+    *row_stride = rs;
+    return true;
+}
+
+// A cache [blockNum, a, b, headDim] with one of a/b equal to 1 (the other is
+// blockSize) -- or, when inner > 1, [blockNum, blockSize, inner, headDim].
+// Rows of inner*headDim elements are contiguous inside a block; only the
+// block dimension may be strided.
+kvq_status paged_from(const kvq_tensor* c, int64_t inner, PagedRows* out, int64_t* head_dim) {
+    if (c->ndim != 4) return KVQ_ERR_NDIM;
+    const int64_t eb = elem_bytes(c->dtype);
+    const int64_t hd = c->shape[3];
+    int64_t bs;
+    int bs_dim;
+    if (inner > 1) {
+        if (c->shape[2] != inner) return KVQ_ERR_SHAPE;
+        bs = c->shape[1];
+        bs_dim = 1;
+        if (hd > 1 && c->stride[3] != 1) return KVQ_ERR_LAYOUT;
+        if (inner > 1 && c->stride[2] != hd) return KVQ_ERR_LAYOUT;
+        if (bs > 1 && c->stride[1] != inner * hd) return KVQ_ERR_LAYOUT;
+    } else {
+        if (c->shape[2] == 1) { bs = c->shape[1]; bs_dim = 1; }
+        else if (c->shape[1] == 1) { bs = c->shape[2]; bs_dim = 2; }
+        else return KVQ_ERR_SHAPE;
+        if (hd > 1 && c->stride[3] != 1) return KVQ_ERR_LAYOUT;
+        if (bs > 1 && c->stride[bs_dim] != hd) return KVQ_ERR_LAYOUT;
+    }
+    const int64_t nb = c->shape[0];
+    const int64_t row = inner * hd;
+    if (nb > 1 && c->stride[0] < bs * row) return KVQ_ERR_LAYOUT;
+    out->base = static_cast<uint8_t*>(c->data);
+    out->num_slots = nb * bs;
+    out->block_size = bs;
+    out->row_bytes = row * eb;
+    out->block_stride = (nb > 1 ? c->stride[0] : bs * row) * eb;
+    *head_dim = hd;
+    return KVQ_OK;
+}
+
+bool is_index_dtype(int32_t dt) { return dt == KVQ_I32 || dt == KVQ_I64; }
+
+// ---------------------------------------------------------------------------
+// launch sizing: a grid of (SMs x resident blocks) persistent blocks at most
+// ---------------------------------------------------------------------------
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+template <typename K>
+int64_t persistent_grid(K kernel, int threads, int64_t needed_blocks) {
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, 0) != cudaSuccess || occ < 1) occ = 1;
+    const int64_t cap = (int64_t)sm_count() * occ;
+    int64_t g = needed_blocks < cap ? needed_blocks : cap;
+    return g < 1 ? 1 : g;
+}
+
+kvq_status launched() {
+    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// conversion kernel (kvq_convert)
+// ---------------------------------------------------------------------------
+__global__ void convert_kernel(int32_t fmt, const float* in, int64_t n, uint8_t* out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const float v = in[i];
+        switch (fmt) {
+            case 0: out[i] = (uint8_t)e4m3x2(v, 0.0f); break;
+            case 1: out[i] = (uint8_t)e5m2x2(v, 0.0f); break;
+            case 2: {
+                const float q[8] = {v, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                out[i] = (uint8_t)(e2m1x8(q) & 0xfu);
+                break;
+            }
+            case 3: reinterpret_cast<uint16_t*>(out)[i] = (uint16_t)to_bf16_bits(v); break;
+            case 4: out[i] = (uint8_t)e8m0_ceil(v); break;
+            default: out[i] = (uint8_t)int8_rne_sat(v); break;
+        }
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t kvq_version(void) { return 100; }
+
+const char* kvq_status_string(kvq_status s) {
+    switch (s) {
+        case KVQ_OK: return "ok";
+        case KVQ_ERR_NULL: return "a required tensor or data pointer is NULL";
+        case KVQ_ERR_NDIM: return "wrong number of dimensions";
+        case KVQ_ERR_SHAPE: return "inconsistent tensor sizes";
+        case KVQ_ERR_DTYPE: return "dtype not allowed";
+        case KVQ_ERR_ATTR: return "bad attribute value";
+        case KVQ_ERR_LAYOUT: return "non-contiguous where contiguity is required";
+        case KVQ_ERR_CAPACITY: return "cache row too small for the packed row";
+        case KVQ_ERR_CUDA: return "CUDA runtime error";
+        case KVQ_ERR_UNSUPPORTED: return "valid but not implemented by this library";
+        default: return "unknown status";
+    }
+}
+
+int64_t kvq_kv_cache_col(int64_t d, int32_t quant_mode, int32_t quant_group_size) {
+    if (d <= 64 || d % 64 != 0 || d > 8192) return -1;
+    const int64_t n = d - 64;
+    int64_t concat;
+    if (quant_mode == 0 || quant_mode == 1) {
+        concat = n + 128 + ((n + 63) / 64) * (quant_mode == 0 ? 2 : 1);
+    } else if (quant_mode == 2) {
+        if (quant_group_size != 16 && quant_group_size != 32 && quant_group_size != 64) return -1;
+        if (n % quant_group_size != 0) return -1;
+        concat = 64 + n / 2 + (n / quant_group_size) * 2;
+    } else {
+        return -1;
+    }
+    return quant_mode == 1 ? concat : (concat + 31) / 32 * 32;
+}
+
+int64_t kvq_indexer_scale_col(int64_t d, int32_t quant_mode) {
+    if (d < 1) return -1;
+    if (quant_mode == 0 || quant_mode == 3) return (d + 31) / 32;
+    if (quant_mode == 1 || quant_mode == 2) return 1;
+    return -1;
+}
+
+// ---------------------------------------------------------------------------
+kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_mapping, kvq_tensor* cache,
+                                  int32_t quant_mode, int32_t quant_group_size, float x_scale,
+                                  kvq_stream stream) {
+    if (!x || !slot_mapping || !cache) return KVQ_ERR_NULL;
+    if (!valid_desc(x) || !valid_desc(slot_mapping) || !valid_desc(cache)) return KVQ_ERR_DTYPE;
+    if (x->dtype != KVQ_BF16) return KVQ_ERR_DTYPE;
+    if (x->ndim < 1) return KVQ_ERR_NDIM;
+    int64_t T, rs;
+    if (!flatten_rows(x, &T, &rs)) return KVQ_ERR_LAYOUT;
+    const int64_t d = x->shape[x->ndim - 1];
+    if (d <= 64 || d % 64 != 0 || d > 8192) return KVQ_ERR_SHAPE;
+    if (quant_mode < 0 || quant_mode > 2) return KVQ_ERR_ATTR;
+    const int32_t G = quant_mode == 2 ? quant_group_size : 64;
+    if (quant_mode == 2 && ((G != 16 && G != 32 && G != 64) || (d - 64) % G != 0)) return KVQ_ERR_ATTR;
+    if (!is_index_dtype(slot_mapping->dtype)) return KVQ_ERR_DTYPE;
+    if (numel(slot_mapping) != T) return KVQ_ERR_SHAPE;
+    if (!contiguous(slot_mapping)) return KVQ_ERR_LAYOUT;
+    if (cache->dtype != KVQ_U8 && cache->dtype != KVQ_I8) return KVQ_ERR_DTYPE;
+    if (cache->ndim != 4) return KVQ_ERR_NDIM;
+    if (cache->shape[2] != 1) return KVQ_ERR_SHAPE;
+    PagedRows rows;
+    int64_t head_dim;
+    kvq_status st = paged_from(cache, 1, &rows, &head_dim);
+    if (st != KVQ_OK) return st;
+    const int64_t col = kvq_kv_cache_col(d, quant_mode, G);
+    if (head_dim < col) return KVQ_ERR_CAPACITY;
+    if (T == 0) return KVQ_OK;
+    if (!x->data || !slot_mapping->data || (!cache->data && rows.num_slots > 0)) return KVQ_ERR_NULL;
+
+    CompressArgs a;
+    a.x = static_cast<const uint16_t*>(x->data);
+    a.x_row_stride = rs;
+    a.T = T;
+    a.slots = slot_mapping->data;
+    a.slots_i64 = slot_mapping->dtype == KVQ_I64;
+    a.cache = rows;
+    a.nseg = (int32_t)(d / 64);
+    a.n = (int32_t)(d - 64);
+    a.col = (int32_t)col;
+    a.concat = quant_mode == 2 ? (int32_t)(64 + (d - 64) / 2 + ((d - 64) / G) * 2)
+                               : (int32_t)((d - 64) + 128 + ((d - 64) / 64) * (quant_mode == 0 ? 2 : 1));
+    a.x_scale = x_scale;
+    a.x_vec = (reinterpret_cast<uintptr_t>(x->data) % 16 == 0) && ((rs * 2) % 16 == 0);
+
+    const int64_t tiles = (T + CE_TILE - 1) / CE_TILE;
+    const int64_t need = (tiles + (CE_THREADS / 32) - 1) / (CE_THREADS / 32);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+#define KVQ_LAUNCH_CE(M, GG)                                                                   \
+    do {                                                                                       \
+        auto k = compress_epilog_kernel<M, GG>;                                                \
+        k<<<(unsigned)persistent_grid(k, CE_THREADS, need), CE_THREADS, 0, s>>>(a);             \
+    } while (0)
+    if (quant_mode == 0) KVQ_LAUNCH_CE(0, 64);
+    else if (quant_mode == 1) KVQ_LAUNCH_CE(1, 64);
+    else if (G == 16) KVQ_LAUNCH_CE(2, 16);
+    else if (G == 32) KVQ_LAUNCH_CE(2, 32);
+    else KVQ_LAUNCH_CE(2, 64);
+#undef KVQ_LAUNCH_CE
+    return launched();
+}
+
+// ---------------------------------------------------------------------------
+kvq_status kvq_indexer_quant_cache(const kvq_tensor* x, kvq_tensor* cache, kvq_tensor* cache_scale,
+                                   const kvq_tensor* slot_mapping, int32_t quant_mode, kvq_stream stream) {
+    if (!x || !cache || !cache_scale || !slot_mapping) return KVQ_ERR_NULL;
+    if (!valid_desc(x) || !valid_desc(cache) || !valid_desc(cache_scale) || !valid_desc(slot_mapping))
+        return KVQ_ERR_DTYPE;
+    if (x->dtype != KVQ_BF16 && x->dtype != KVQ_F16) return KVQ_ERR_DTYPE;
+    if (x->ndim < 1) return KVQ_ERR_NDIM;
+    int64_t T, rs;
+    if (!flatten_rows(x, &T, &rs)) return KVQ_ERR_LAYOUT;
+    const int64_t d = x->shape[x->ndim - 1];
+    if (d < 1) return KVQ_ERR_SHAPE;
+    if (quant_mode == 2) return KVQ_ERR_UNSUPPORTED;
+    if (quant_mode != 0 && quant_mode != 1 && quant_mode != 3) return KVQ_ERR_ATTR;
+    if (quant_mode == 3) {
+        if (cache->dtype != KVQ_U8 && cache->dtype != KVQ_I8) return KVQ_ERR_DTYPE;
+    } else if (cache->dtype != KVQ_F8E4M3 && cache->dtype != KVQ_F8E5M2) {
+        return KVQ_ERR_DTYPE;
+    }
+    if (quant_mode == 1) {
+        if (cache_scale->dtype != KVQ_F32) return KVQ_ERR_DTYPE;
+    } else if (cache_scale->dtype != KVQ_E8M0 && cache_scale->dtype != KVQ_U8) {
+        return KVQ_ERR_DTYPE;
+    }
+    if (!is_index_dtype(slot_mapping->dtype)) return KVQ_ERR_DTYPE;
+    if (numel(slot_mapping) != T) return KVQ_ERR_SHAPE;
+    if (!contiguous(slot_mapping)) return KVQ_ERR_LAYOUT;
+    if (cache->ndim != 4 || cache_scale->ndim != 4) return KVQ_ERR_NDIM;
+    if (cache->shape[2] != 1 || cache_scale->shape[2] != 1) return KVQ_ERR_SHAPE;
+    PagedRows crow, srow;
+    int64_t chd, shd;
+    kvq_status st = paged_from(cache, 1, &crow, &chd);
+    if (st != KVQ_OK) return st;
+    st = paged_from(cache_scale, 1, &srow, &shd);
+    if (st != KVQ_OK) return st;
+    if (cache->shape[0] != cache_scale->shape[0] || cache->shape[1] != cache_scale->shape[1]) return KVQ_ERR_SHAPE;
+    const int64_t need_codes = quant_mode == 3 ? (d + 1) / 2 : d;
+    if (chd < need_codes || shd < kvq_indexer_scale_col(d, quant_mode)) return KVQ_ERR_CAPACITY;
+    if (T == 0) return KVQ_OK;
+    if (!x->data || !slot_mapping->data || !cache->data || !cache_scale->data) return KVQ_ERR_NULL;
+
+    IndexerArgs a;
+    a.x = static_cast<const uint16_t*>(x->data);
+    a.x_row_stride = rs;
+    a.T = T;
+    a.d = (int32_t)d;
+    a.nchunks = (int32_t)((d + 7) / 8);
+    a.x_f16 = x->dtype == KVQ_F16;
+    a.x_vec = (reinterpret_cast<uintptr_t>(x->data) % 16 == 0) && ((rs * 2) % 16 == 0);
+    a.slots = slot_mapping->data;
+    a.slots_i64 = slot_mapping->dtype == KVQ_I64;
+    a.cache = crow;
+    a.scale = srow;
+    a.e5m2 = cache->dtype == KVQ_F8E5M2;
+
+    int team = 32;
+    if (a.nchunks <= 4) team = 4;
+    else if (a.nchunks <= 8) team = 8;
+    else if (a.nchunks <= 16) team = 16;
+    const int64_t tiles = (T + 31) / 32;
+    const int64_t need = (tiles + (IX_THREADS / 32) - 1) / (IX_THREADS / 32);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+#define KVQ_LAUNCH_IX(M, TM)                                                                   \
+    do {                                                                                       \
+        auto k = indexer_quant_kernel<M, TM>;                                                  \
+        k<<<(unsigned)persistent_grid(k, IX_THREADS, need), IX_THREADS, 0, s>>>(a);             \
+    } while (0)
+#define KVQ_LAUNCH_IX_TEAM(M)                                                                  \
+    do {                                                                                       \
+        if (team == 4) KVQ_LAUNCH_IX(M, 4);                                                    \
+        else if (team == 8) KVQ_LAUNCH_IX(M, 8);                                               \
+        else if (team == 16) KVQ_LAUNCH_IX(M, 16);                                             \
+        else KVQ_LAUNCH_IX(M, 32);                                                             \
+    } while (0)
+    if (quant_mode == 0) KVQ_LAUNCH_IX_TEAM(0);
+    else if (quant_mode == 1) KVQ_LAUNCH_IX_TEAM(1);
+    else KVQ_LAUNCH_IX_TEAM(3);
+#undef KVQ_LAUNCH_IX_TEAM
+#undef KVQ_LAUNCH_IX
+    return launched();
+}
+
+// ---------------------------------------------------------------------------
+namespace {
+
+int32_t cache_dt(int32_t dt) {
+    switch (dt) {
+        case KVQ_BF16: return CDT_BF16;
+        case KVQ_F16: return CDT_F16;
+        case KVQ_F8E4M3: return CDT_E4M3;
+        case KVQ_F8E5M2: return CDT_E5M2;
+        case KVQ_I8: return CDT_I8;
+        default: return -1;
+    }
+}
+
+// scale / offset of a quantised cache: f32, 1 or Dc elements, contiguous
+kvq_status cache_param(const kvq_tensor* p, int64_t dc, const float** out, int32_t* n) {
+    *out = nullptr;
+    *n = 0;
+    if (!p) return KVQ_OK;
+    if (!valid_desc(p) || p->dtype != KVQ_F32) return KVQ_ERR_DTYPE;
+    const int64_t k = numel(p);
+    if (k != 1 && k != dc) return KVQ_ERR_SHAPE;
+    if (!contiguous(p)) return KVQ_ERR_LAYOUT;
+    *out = static_cast<const float*>(p->data);
+    *n = (int32_t)k;
+    return KVQ_OK;
+}
+
+kvq_status setup_cache_out(const kvq_tensor* c, const kvq_tensor* scale, const kvq_tensor* offset,
+                           CacheOut* out, int64_t* head_dim) {
+    if (!valid_desc(c)) return KVQ_ERR_DTYPE;
+    out->dt = cache_dt(c->dtype);
+    if (out->dt < 0) return KVQ_ERR_DTYPE;
+    kvq_status st = paged_from(c, 1, &out->rows, head_dim);
+    if (st != KVQ_OK) return st;
+    const bool quant = out->dt == CDT_E4M3 || out->dt == CDT_E5M2 || out->dt == CDT_I8;
+    if (quant && !scale) return KVQ_ERR_NULL;
+    if (offset && out->dt != CDT_I8) return KVQ_ERR_ATTR;
+    st = cache_param(quant ? scale : nullptr, *head_dim, &out->scale, &out->scale_n);
+    if (st != KVQ_OK) return st;
+    return cache_param(offset, *head_dim, &out->offset, &out->offset_n);
+}
+
+}  // namespace
+
+kvq_status kvq_kv_rmsnorm_rope_cache(const kvq_tensor* kv, const kvq_tensor* gamma, const kvq_tensor* cos,
+                                     const kvq_tensor* sin, const kvq_tensor* index, kvq_tensor* k_cache,
+                                     kvq_tensor* ckv_cache, const kvq_tensor* k_scale,
+                                     const kvq_tensor* ckv_scale, const kvq_tensor* k_offset,
+                                     const kvq_tensor* ckv_offset, float epsilon, int32_t cache_mode,
+                                     kvq_stream stream) {
+    if (!kv || !gamma || !cos || !sin || !index || !k_cache || !ckv_cache) return KVQ_ERR_NULL;
+    if (!valid_desc(kv) || !valid_desc(gamma) || !valid_desc(cos) || !valid_desc(sin) || !valid_desc(index))
+        return KVQ_ERR_DTYPE;
+    if (cache_mode == 4 || cache_mode == 5) return KVQ_ERR_UNSUPPORTED;   // PA_NZ, PA_BLK_NZ
+    if (cache_mode < 0 || cache_mode > 3) return KVQ_ERR_ATTR;
+    if (kv->dtype != KVQ_BF16 && kv->dtype != KVQ_F16) return KVQ_ERR_DTYPE;
+    if (gamma->dtype != kv->dtype || cos->dtype != kv->dtype || sin->dtype != kv->dtype) return KVQ_ERR_DTYPE;
+    if (kv->ndim != 4) return KVQ_ERR_NDIM;
+    if (kv->shape[1] != 1) return KVQ_ERR_SHAPE;
+    if (!contiguous(kv) || !contiguous(gamma) || !contiguous(cos) || !contiguous(sin) || !contiguous(index))
+        return KVQ_ERR_LAYOUT;
+    const int64_t B = kv->shape[0], S = kv->shape[2], D = kv->shape[3];
+    CacheOut kc, cc;
+    int64_t Dk, Dv;
+    kvq_status st = setup_cache_out(k_cache, k_scale, k_offset, &kc, &Dk);
+    if (st != KVQ_OK) return st;
+    st = setup_cache_out(ckv_cache, ckv_scale, ckv_offset, &cc, &Dv);
+    if (st != KVQ_OK) return st;
+    if (Dk + Dv != D || Dk % 2 != 0 || Dk < 2 || Dv < 1) return KVQ_ERR_SHAPE;
+    const bool kq = kc.dt >= CDT_E4M3, cq = cc.dt >= CDT_E4M3;
+    if (kq && cq && kc.dt != cc.dt) return KVQ_ERR_DTYPE;     // scenario 3 needs one dtype
+    if (k_cache->shape[0] != ckv_cache->shape[0] || kc.rows.block_size != cc.rows.block_size) return KVQ_ERR_SHAPE;
+    const int64_t bs = kc.rows.block_size;
+    if (cache_mode != 0) {
+        // PA block size rule: % 32 for 1-byte caches, % 16 for 2-byte ones
+        const bool one_byte = kq || cq, two_byte = !kq || !cq;
+        if ((one_byte && bs % 32 != 0) || (two_byte && bs % 16 != 0)) return KVQ_ERR_SHAPE;
+    }
+    if (numel(gamma) != Dv || numel(cos) != B * S * Dk || numel(sin) != B * S * Dk) return KVQ_ERR_SHAPE;
+    if (!is_index_dtype(index->dtype)) return KVQ_ERR_DTYPE;
+    const int64_t nidx = cache_mode == 3 ? B * ((S + bs - 1) / (bs > 0 ? bs : 1)) : B * S;
+    if (numel(index) != nidx) return KVQ_ERR_SHAPE;
+    if (B * S == 0) return KVQ_OK;
+    if (!kv->data || !gamma->data || !cos->data || !sin->data || !index->data || !k_cache->data ||
+        !ckv_cache->data || (kc.scale_n && !kc.scale) || (cc.scale_n && !cc.scale) ||
+        (kc.offset_n && !kc.offset) || (cc.offset_n && !cc.offset))
+        return KVQ_ERR_NULL;
+
+    RmsRopeArgs a;
+    a.kv = static_cast<const uint16_t*>(kv->data);
+    a.kv_f16 = kv->dtype == KVQ_F16;
+    a.B = B;
+    a.S = S;
+    a.D = (int32_t)D;
+    a.Dv = (int32_t)Dv;
+    a.Dk = (int32_t)Dk;
+    a.gamma = static_cast<const uint16_t*>(gamma->data);
+    a.cos = static_cast<const uint16_t*>(cos->data);
+    a.sin = static_cast<const uint16_t*>(sin->data);
+    a.index = index->data;
+    a.index_i64 = index->dtype == KVQ_I64;
+    a.cache_mode = cache_mode;
+    a.k = kc;
+    a.ckv = cc;
+    a.eps = epsilon;
+    const int64_t warps_per_block = RR_THREADS / 32;
+    const int64_t need = (B * S + warps_per_block - 1) / warps_per_block;
+    rmsnorm_rope_kernel<<<(unsigned)persistent_grid(rmsnorm_rope_kernel, RR_THREADS, need), RR_THREADS, 0,
+                          reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    return launched();
+}
+
+// ---------------------------------------------------------------------------
+kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor* cos, const kvq_tensor* sin,
+                                          kvq_tensor* k_cache, kvq_tensor* v_cache, const kvq_tensor* indices,
+                                          const kvq_tensor* scale_k, const kvq_tensor* scale_v,
+                                          const kvq_tensor* offset_k, const kvq_tensor* offset_v,
+                                          const kvq_tensor* weight_scale, const kvq_tensor* activation_scale,
+                                          const kvq_tensor* bias, const int64_t* size_splits, int32_t n_splits,
+                                          int32_t quant_mode, int32_t layout, int32_t kv_output,
+                                          int32_t cache_mode, kvq_tensor* q_out, kvq_tensor* k_out,
+                                          kvq_tensor* v_out, kvq_stream stream) {
+    if (!x || !cos || !sin || !k_cache || !v_cache || !indices || !scale_k || !scale_v || !q_out || !size_splits)
+        return KVQ_ERR_NULL;
+    if (!valid_desc(x) || !valid_desc(cos) || !valid_desc(sin) || !valid_desc(k_cache) || !valid_desc(v_cache) ||
+        !valid_desc(indices) || !valid_desc(scale_k) || !valid_desc(scale_v) || !valid_desc(q_out))
+        return KVQ_ERR_DTYPE;
+    if (quant_mode != 0 || layout != 0 || (cache_mode != 0 && cache_mode != 1) || n_splits != 3)
+        return KVQ_ERR_ATTR;
+    if (x->dtype != KVQ_I32 && x->dtype != KVQ_BF16 && x->dtype != KVQ_F16) return KVQ_ERR_DTYPE;
+    if (cos->dtype != KVQ_BF16 && cos->dtype != KVQ_F16) return KVQ_ERR_DTYPE;
+    if (sin->dtype != cos->dtype || q_out->dtype != cos->dtype) return KVQ_ERR_DTYPE;
+    if (x->dtype != KVQ_I32 && x->dtype != cos->dtype) return KVQ_ERR_DTYPE;
+    if (x->ndim != 2 && x->ndim != 3) return KVQ_ERR_NDIM;
+    if (k_cache->ndim != 4 || v_cache->ndim != 4) return KVQ_ERR_NDIM;
+    if (k_cache->dtype != KVQ_I8 || v_cache->dtype != KVQ_I8) return KVQ_ERR_DTYPE;
+    const int64_t B = x->shape[0];
+    const int64_t S = x->ndim == 3 ? x->shape[1] : 1;
+    const int64_t H = x->shape[x->ndim - 1];
+    if (size_splits[1] != size_splits[2]) return KVQ_ERR_ATTR;
+    const int64_t D = k_cache->shape[3];
+    if (D <= 0 || D % 16 != 0) return KVQ_ERR_SHAPE;
+    if (size_splits[0] <= 0 || size_splits[1] <= 0 || size_splits[0] % D || size_splits[1] % D) return KVQ_ERR_SHAPE;
+    if (size_splits[0] + size_splits[1] + size_splits[2] != H) return KVQ_ERR_SHAPE;
+    if (H > 4096 || H % 64 != 0) return KVQ_ERR_SHAPE;
+    const int64_t Nq = size_splits[0] / D, Nkv = size_splits[1] / D;
+    if (k_cache->shape[2] != Nkv) return KVQ_ERR_SHAPE;
+    for (int i = 0; i < 4; ++i)
+        if (k_cache->shape[i] != v_cache->shape[i]) return KVQ_ERR_SHAPE;
+    PagedRows kr, vr;
+    int64_t hd;
+    kvq_status st = paged_from(k_cache, Nkv, &kr, &hd);
+    if (st != KVQ_OK) return st;
+    st = paged_from(v_cache, Nkv, &vr, &hd);
+    if (st != KVQ_OK) return st;
+    if (D % 32 != 0 || D > 256 || Nq + 2 * Nkv > DQ_WARPS * DQ_MAX_HEADS_PER_WARP) return KVQ_ERR_UNSUPPORTED;
+    if (!contiguous(x) || !contiguous(cos) || !contiguous(sin) || !contiguous(indices) || !contiguous(q_out))
+        return KVQ_ERR_LAYOUT;
+    if (numel(cos) != B * S * D || numel(sin) != B * S * D) return KVQ_ERR_SHAPE;
+    if (numel(q_out) != B * S * Nq * D) return KVQ_ERR_SHAPE;
+    if (!is_index_dtype(indices->dtype)) return KVQ_ERR_DTYPE;
+    if (numel(indices) != (cache_mode == 1 ? B * S : B)) return KVQ_ERR_SHAPE;
+    if (cache_mode == 0 && (k_cache->shape[0] < B || k_cache->shape[1] < S)) return KVQ_ERR_SHAPE;
+    const float *sk = nullptr, *sv = nullptr, *ok = nullptr, *ov = nullptr, *ws = nullptr, *as = nullptr;
+    auto f32param = [](const kvq_tensor* p, int64_t n, bool required, const float** out) -> kvq_status {
+        if (!p) return required ? KVQ_ERR_NULL : KVQ_OK;
+        if (!valid_desc(p) || p->dtype != KVQ_F32) return KVQ_ERR_DTYPE;
+        if (numel(p) != n) return KVQ_ERR_SHAPE;
+        if (!contiguous(p)) return KVQ_ERR_LAYOUT;
+        *out = static_cast<const float*>(p->data);
+        return KVQ_OK;
+    };
+    const bool dq = x->dtype == KVQ_I32;
+    if ((st = f32param(scale_k, Nkv * D, true, &sk)) != KVQ_OK) return st;
+    if ((st = f32param(scale_v, Nkv * D, true, &sv)) != KVQ_OK) return st;
+    if ((st = f32param(offset_k, Nkv * D, false, &ok)) != KVQ_OK) return st;
+    if ((st = f32param(offset_v, Nkv * D, false, &ov)) != KVQ_OK) return st;
+    if (dq) {
+        if ((st = f32param(weight_scale, H, true, &ws)) != KVQ_OK) return st;
+        if ((st = f32param(activation_scale, B * S, false, &as)) != KVQ_OK) return st;
+    }
+    int32_t bias_kind = 0;
+    const void* bias_ptr = nullptr;
+    if (dq && bias) {
+        if (!valid_desc(bias)) return KVQ_ERR_DTYPE;
+        switch (bias->dtype) {
+            case KVQ_F32: bias_kind = 0; break;
+            case KVQ_F16: bias_kind = 1; break;
+            case KVQ_BF16: bias_kind = 2; break;
+            case KVQ_I32: bias_kind = 3; break;
+            default: return KVQ_ERR_DTYPE;
+        }
+        if (numel(bias) != H) return KVQ_ERR_SHAPE;
+        if (!contiguous(bias)) return KVQ_ERR_LAYOUT;
+        bias_ptr = bias->data;
+    }
+    uint16_t *kop = nullptr, *vop = nullptr;
+    if (kv_output) {
+        if (!k_out || !v_out) return KVQ_ERR_NULL;
+        if (!valid_desc(k_out) || !valid_desc(v_out)) return KVQ_ERR_DTYPE;
+        if (k_out->dtype != cos->dtype || v_out->dtype != cos->dtype) return KVQ_ERR_DTYPE;
+        if (numel(k_out) != B * S * Nkv * D || numel(v_out) != B * S * Nkv * D) return KVQ_ERR_SHAPE;
+        if (!contiguous(k_out) || !contiguous(v_out)) return KVQ_ERR_LAYOUT;
+        kop = static_cast<uint16_t*>(k_out->data);
+        vop = static_cast<uint16_t*>(v_out->data);
+    }
+    if (B * S == 0) return KVQ_OK;
+    if (!x->data || !cos->data || !sin->data || !indices->data || !q_out->data || !k_cache->data || !v_cache->data ||
+        (kv_output && (!kop || !vop)) || !sk || !sv || (offset_k && !ok) || (offset_v && !ov) || (dq && !ws) ||
+        (dq && activation_scale && !as) || (dq && bias && !bias_ptr))
+        return KVQ_ERR_NULL;
+
+    DrqArgs a;
+    a.x = x->data;
+    a.x_kind = dq ? 0 : (x->dtype == KVQ_BF16 ? 1 : 2);
+    a.B = B;
+    a.S = S;
+    a.H = H;
+    a.cos = static_cast<const uint16_t*>(cos->data);
+    a.sin = static_cast<const uint16_t*>(sin->data);
+    a.cos_f16 = cos->dtype == KVQ_F16;
+    a.kc = kr;
+    a.vc = vr;
+    a.indices = indices->data;
+    a.indices_i64 = indices->dtype == KVQ_I64;
+    a.cache_mode = cache_mode;
+    a.scale_k = sk;
+    a.scale_v = sv;
+    a.offset_k = ok;
+    a.offset_v = ov;
+    a.weight_scale = ws;
+    a.activation_scale = as;
+    a.bias = bias_ptr;
+    a.bias_kind = bias_kind;
+    a.Nq = (int32_t)Nq;
+    a.Nkv = (int32_t)Nkv;
+    a.D = (int32_t)D;
+    a.q_out = static_cast<uint16_t*>(q_out->data);
+    a.k_out = kop;
+    a.v_out = vop;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t need = B * S;
+#define KVQ_LAUNCH_DQ(E)                                                                       \
+    do {                                                                                       \
+        auto k = dequant_rope_quant_kernel<E>;                                                 \
+        k<<<(unsigned)persistent_grid(k, DQ_WARPS * 32, need), DQ_WARPS * 32, 0, s>>>(a);       \
+    } while (0)
+    switch (D / 32) {
+        case 1: KVQ_LAUNCH_DQ(1); break;
+        case 2: KVQ_LAUNCH_DQ(2); break;
+        case 3: KVQ_LAUNCH_DQ(3); break;
+        case 4: KVQ_LAUNCH_DQ(4); break;
+        case 5: KVQ_LAUNCH_DQ(5); break;
+        case 6: KVQ_LAUNCH_DQ(6); break;
+        case 7: KVQ_LAUNCH_DQ(7); break;
+        default: KVQ_LAUNCH_DQ(8); break;
+    }
+#undef KVQ_LAUNCH_DQ
+    return launched();
+}
+
+// ---------------------------------------------------------------------------
+kvq_status kvq_get_error(kvq_stream stream, uint32_t* fault_bits) {
+    if (!fault_bits) return KVQ_ERR_NULL;
+    *fault_bits = 0u;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned int h = 0u;
+    const unsigned int zero = 0u;
+    if (cudaMemcpyFromSymbolAsync(&h, g_fault_word, sizeof(h), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    if (cudaMemcpyToSymbolAsync(g_fault_word, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return KVQ_ERR_CUDA;
+    *fault_bits = h;
+    return KVQ_OK;
+}
+
+kvq_status kvq_convert(int32_t fmt, const float* in, int64_t n, void* out, kvq_stream stream) {
+    if (fmt < 0 || fmt > 5) return KVQ_ERR_ATTR;
+    if (n < 0) return KVQ_ERR_SHAPE;
+    if (n == 0) return KVQ_OK;
+    if (!in || !out) return KVQ_ERR_NULL;
+    const int64_t need = (n + 255) / 256;
+    convert_kernel<<<(unsigned)persistent_grid(convert_kernel, 256, need), 256, 0,
+                     reinterpret_cast<cudaStream_t>(stream)>>>(fmt, in, n, static_cast<uint8_t*>(out));
+    return launched();
+}
+
+}  // extern "C"

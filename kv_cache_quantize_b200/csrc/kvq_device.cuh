@@ -1,0 +1,227 @@
+// kvq_device.cuh -- device helpers shared by the epilogue kernels (sm_100a).
+//
+// Number formats use the hardware conversions: cvt.rn.satfinite.{e4m3x2,
+// e5m2x2,e2m1x2}.f32 (round to nearest even, saturate to the largest finite
+// value), cvt.rn.bf16.f32 / cvt.rn.f16.f32, cvt.rni.s32.f32.  binary32
+// arithmetic uses the explicitly rounded intrinsics (__fdiv_rn, __fmul_rn,
+// __fadd_rn, __fsqrt_rn) and the library is compiled with -fmad=false, so
+// no multiply-add is contracted and every expression is evaluated in the
+// order written.  Subnormals are kept (no -ftz).
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace kvq {
+
+constexpr unsigned FULL_MASK = 0xffffffffu;
+
+// ---------------------------------------------------------------------------
+// Device fault word: data faults (a bad slot) set bits here; the host reads
+// and clears it with kvq_get_error.  One word per device (module global).
+// ---------------------------------------------------------------------------
+__device__ unsigned int g_fault_word;
+constexpr unsigned FAULT_SLOT_RANGE = 0x1u;
+
+__device__ __forceinline__ void raise_fault(unsigned bits) { atomicOr(&g_fault_word, bits); }
+
+// ---------------------------------------------------------------------------
+// 16-bit float widening (exact) and narrowing (round to nearest even)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float f16_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
+__device__ __forceinline__ float f16_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
+
+template <bool F16>
+__device__ __forceinline__ void widen8(const uint4& v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = F16 ? f16_lo(w[i]) : bf16_lo(w[i]);
+        f[2 * i + 1] = F16 ? f16_hi(w[i]) : bf16_hi(w[i]);
+    }
+}
+
+__device__ __forceinline__ uint32_t to_bf16_bits(float f) {
+    unsigned short r;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(f));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t to_f16_bits(float f) {
+    unsigned short r;
+    asm("cvt.rn.f16.f32 %0, %1;" : "=h"(r) : "f"(f));
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// FP8 / FP4 codes.  The x2 conversions put their FIRST source operand in the
+// HIGH half of the result, so (hi, lo) are passed in that order and the
+// element with the lower index lands in the lower byte / nibble.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    unsigned short r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t e5m2x2(float lo, float hi) {
+    unsigned short r;
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+template <bool E5M2>
+__device__ __forceinline__ uint32_t fp8x2(float lo, float hi) {
+    return E5M2 ? e5m2x2(lo, hi) : e4m3x2(lo, hi);
+}
+
+// Eight E2M1 codes packed into 32 bits, element 0 in bits [3:0].
+__device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
+    uint32_t r;
+    asm("{\n\t"
+        ".reg .b8 q0, q1, q2, q3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t"
+        "}"
+        : "=r"(r)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return r;
+}
+
+// Eight FP8 codes packed into two 32-bit words, element 0 in byte 0.
+template <bool E5M2>
+__device__ __forceinline__ uint2 fp8x8(const float (&v)[8]) {
+    uint2 r;
+    r.x = fp8x2<E5M2>(v[0], v[1]) | (fp8x2<E5M2>(v[2], v[3]) << 16);
+    r.y = fp8x2<E5M2>(v[4], v[5]) | (fp8x2<E5M2>(v[6], v[7]) << 16);
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// E8M0 scale rounded up: the smallest b in [0, 254] with 2^(b-127) >= q, for a
+// finite q >= 0, read off the binary32 fields of q.  A normal q = 2^(E-127) *
+// 1.M needs b = E when M == 0 and E + 1 otherwise; a subnormal q < 2^-126
+// needs b = 0 when q <= 2^-127 (fraction <= 2^22) and b = 1 otherwise.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e8m0_ceil(float q) {
+    const uint32_t u = __float_as_uint(q) & 0x7fffffffu;
+    const uint32_t E = u >> 23, M = u & 0x7fffffu;
+    uint32_t b = (E == 0) ? (M > 0x400000u ? 1u : 0u) : E + (M != 0 ? 1u : 0u);
+    return b > 254u ? 254u : b;
+}
+
+// 2^(127-b) as binary32 (exact; 2^-127 is the subnormal 0x00400000).
+__device__ __forceinline__ float e8m0_reciprocal(uint32_t b) {
+    const int k = 127 - (int)b;
+    return k >= -126 ? __uint_as_float((uint32_t)(k + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// Static int8: round half to even, saturate to [-128, 127]; NaN -> 0.
+__device__ __forceinline__ int32_t int8_rne_sat(float v) {
+    int r;
+    asm("cvt.rni.s32.f32 %0, %1;" : "=r"(r) : "f"(v));
+    return r < -128 ? -128 : (r > 127 ? 127 : r);
+}
+
+// Largest |x| of eight 16-bit floats as the bits of one of them (for finite
+// inputs the magnitude order equals the integer order of the bit patterns).
+__device__ __forceinline__ uint32_t absmax_bits8(const uint4& v) {
+    const uint32_t m = 0x7fff7fffu;
+    uint32_t a = __vmaxu2(v.x & m, v.y & m);
+    uint32_t b = __vmaxu2(v.z & m, v.w & m);
+    a = __vmaxu2(a, b);
+    return max(a & 0xffffu, a >> 16);
+}
+
+// ---------------------------------------------------------------------------
+// Loads and stores.  Every store checks the alignment of its own address, so
+// packed rows of any byte length (e.g. 323) are written correctly; aligned
+// rows take the vector path.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+    return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+
+__device__ __forceinline__ void st_b8(uint8_t* p, uint32_t v) { *p = (uint8_t)v; }
+
+__device__ __forceinline__ void st_b16(uint8_t* p, uint32_t v) {
+    if ((reinterpret_cast<uintptr_t>(p) & 1) == 0) {
+        *reinterpret_cast<uint16_t*>(p) = (uint16_t)v;
+    } else {
+        p[0] = (uint8_t)v;
+        p[1] = (uint8_t)(v >> 8);
+    }
+}
+
+__device__ __forceinline__ void st_b32(uint8_t* p, uint32_t v) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    if ((a & 3) == 0) {
+        *reinterpret_cast<uint32_t*>(p) = v;
+    } else if ((a & 1) == 0) {
+        reinterpret_cast<uint16_t*>(p)[0] = (uint16_t)v;
+        reinterpret_cast<uint16_t*>(p)[1] = (uint16_t)(v >> 16);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) p[k] = (uint8_t)(v >> (8 * k));
+    }
+}
+
+__device__ __forceinline__ void st_b64(uint8_t* p, uint2 v) {
+    if ((reinterpret_cast<uintptr_t>(p) & 7) == 0) {
+        *reinterpret_cast<uint2*>(p) = v;
+    } else {
+        st_b32(p, v.x);
+        st_b32(p + 4, v.y);
+    }
+}
+
+__device__ __forceinline__ void st_b128(uint8_t* p, uint4 v) {
+    if ((reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+        *reinterpret_cast<uint4*>(p) = v;
+    } else {
+        st_b64(p, make_uint2(v.x, v.y));
+        st_b64(p + 8, make_uint2(v.z, v.w));
+    }
+}
+
+// Store the first nbytes (0..16) of v at p, byte by byte.
+__device__ __forceinline__ void st_partial(uint8_t* p, uint4 v, int nbytes) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+        if (k < nbytes) p[k] = (uint8_t)(w[k >> 2] >> (8 * (k & 3)));
+}
+
+// ---------------------------------------------------------------------------
+// Paged cache rows: slot s -> block s / block_size, row s % block_size.
+// ---------------------------------------------------------------------------
+struct PagedRows {
+    uint8_t* base;
+    int64_t num_slots;
+    int64_t block_size;
+    int64_t row_bytes;
+    int64_t block_stride;  // bytes
+};
+
+__device__ __forceinline__ uint8_t* slot_row(const PagedRows& c, int64_t s) {
+    if (c.num_slots <= 0x7fffffff) {
+        const uint32_t us = (uint32_t)s, bs = (uint32_t)c.block_size;
+        const uint32_t blk = us / bs;
+        return c.base + (int64_t)blk * c.block_stride + (int64_t)(us - blk * bs) * c.row_bytes;
+    }
+    const int64_t blk = s / c.block_size;
+    return c.base + blk * c.block_stride + (s - blk * c.block_size) * c.row_bytes;
+}
+
+// -1 -> skip silently; other values outside [0, num_slots) -> skip and flag.
+__device__ __forceinline__ bool slot_ok(int64_t s, int64_t num_slots) {
+    return s >= 0 && s < num_slots;
+}
+
+}  // namespace kvq

@@ -1,0 +1,155 @@
+// rmsnorm_rope.cuh -- kv_rmsnorm_rope_cache kernel (aclnnKvRmsNormRopeCache,
+// 计算公式 (1) interleaveRope and (2) rmsNorm; 约束说明 for index modes and
+// cache dtype scenarios).
+//
+// One warp per token.  The sum of squares follows the library's fixed order:
+// value i of the RMSNorm segment belongs to 8-value chunk i/8, chunk c to lane
+// c % 32; each lane adds x*x of its values in index order (x*x is exact for
+// 16-bit inputs), then the lanes combine by the butterfly p += p[lane ^ k],
+// k = 16, 8, 4, 2, 1.  The row is read a second time (from L1) to write the
+// normalised values.  The rope segment is handled one interleaved pair per
+// lane.  gamma, cos and sin are small and stay in L1/L2 across tokens.
+#pragma once
+
+#include "kvq_device.cuh"
+
+namespace kvq {
+
+enum CacheDt : int32_t { CDT_BF16 = 0, CDT_F16 = 1, CDT_E4M3 = 2, CDT_E5M2 = 3, CDT_I8 = 4 };
+
+struct CacheOut {
+    PagedRows rows;
+    int32_t dt;             // CacheDt
+    const float* scale;     // null, 1 value, or one per channel
+    int32_t scale_n;
+    const float* offset;    // int8 only: null, 1 value, or one per channel
+    int32_t offset_n;
+};
+
+struct RmsRopeArgs {
+    const uint16_t* kv;     // [B, 1, S, D] contiguous
+    int32_t kv_f16;
+    int64_t B, S;
+    int32_t D, Dv, Dk;
+    const uint16_t* gamma;  // [Dv]
+    const uint16_t* cos;    // [B*S, Dk]
+    const uint16_t* sin;
+    const void* index;
+    int32_t index_i64;
+    int32_t cache_mode;     // 0 Norm, 1 PA, 2 PA_BNSD, 3 PA_BLK_BNSD
+    CacheOut k;             // Dk values per row
+    CacheOut ckv;           // Dv values per row
+    float eps;
+};
+
+constexpr int RR_THREADS = 128;
+
+__device__ __forceinline__ float half_at(const uint16_t* p, int64_t i, int f16) {
+    const uint32_t h = p[i];
+    return f16 ? __half2float(__ushort_as_half((unsigned short)h)) : __uint_as_float(h << 16);
+}
+
+// Store y as element j of a cache row (unquantised: rounded to the dtype;
+// quantised: fp(y / scale) or int8(rint(y / scale + offset))).
+__device__ __forceinline__ void store_elem(const CacheOut& c, uint8_t* row, int j, float y) {
+    switch (c.dt) {
+        case CDT_BF16: st_b16(row + 2 * j, to_bf16_bits(y)); break;
+        case CDT_F16: st_b16(row + 2 * j, to_f16_bits(y)); break;
+        case CDT_E4M3:
+        case CDT_E5M2: {
+            const float s = c.scale[c.scale_n == 1 ? 0 : j];
+            const float q = __fdiv_rn(y, s);
+            row[j] = (uint8_t)(c.dt == CDT_E4M3 ? e4m3x2(q, 0.0f) : e5m2x2(q, 0.0f));
+            break;
+        }
+        case CDT_I8: {
+            const float s = c.scale[c.scale_n == 1 ? 0 : j];
+            float q = __fdiv_rn(y, s);
+            if (c.offset) q = __fadd_rn(q, c.offset[c.offset_n == 1 ? 0 : j]);
+            row[j] = (uint8_t)int8_rne_sat(q);
+            break;
+        }
+        default: break;
+    }
+}
+
+__device__ __forceinline__ int64_t rr_slot(const RmsRopeArgs& a, int64_t b, int64_t s) {
+    const int64_t t = b * a.S + s;
+    const int64_t bs = a.k.rows.block_size;
+    if (a.cache_mode == 0) {                       // Norm: [B, S] positions, one block per batch
+        const int64_t v = load_slot(a.index, a.index_i64, t);
+        if (v == -1) return -1;
+        if (v < 0 || v >= bs || b * bs >= a.k.rows.num_slots) return -2;
+        return b * bs + v;
+    }
+    if (a.cache_mode == 3) {                       // PA_BLK_BNSD: one entry per block of tokens
+        const int64_t nb = (a.S + bs - 1) / bs;
+        const int64_t v = load_slot(a.index, a.index_i64, b * nb + s / bs);
+        if (v == -1) return -1;
+        if (v < 0 || v >= a.k.rows.num_slots) return -2;
+        return (v / bs) * bs + s % bs;
+    }
+    const int64_t v = load_slot(a.index, a.index_i64, t);   // PA, PA_BNSD
+    if (v == -1) return -1;
+    if (v < 0 || v >= a.k.rows.num_slots) return -2;
+    return v;
+}
+
+__global__ void __launch_bounds__(RR_THREADS) rmsnorm_rope_kernel(const RmsRopeArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t ntok = a.B * a.S;
+    const int nch = (a.Dv + 7) / 8;
+    const int h = a.Dk / 2;
+
+    for (int64_t t = gwarp; t < ntok; t += nwarps) {
+        const int64_t b = t / a.S, s = t - (t / a.S) * a.S;
+        const int64_t slot = rr_slot(a, b, s);     // warp-uniform
+        if (slot == -2) {
+            if (lane == 0) raise_fault(FAULT_SLOT_RANGE);
+            continue;
+        }
+        if (slot < 0) continue;
+        const uint16_t* x = a.kv + t * a.D;
+
+        // RMSNorm: sum of squares in the fixed lane order
+        float acc = 0.0f;
+        for (int c = lane; c < nch; c += 32) {
+            for (int i = 8 * c; i < 8 * c + 8 && i < a.Dv; ++i) {
+                const float v = half_at(x, i, a.kv_f16);
+                acc = __fadd_rn(acc, __fmul_rn(v, v));
+            }
+        }
+#pragma unroll
+        for (int k = 16; k >= 1; k >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(FULL_MASK, acc, k));
+        const float mean = __fdiv_rn(acc, (float)a.Dv);
+        const float rms = __fsqrt_rn(__fadd_rn(mean, a.eps));
+
+        uint8_t* crow = slot_row(a.ckv.rows, slot);
+        for (int c = lane; c < nch; c += 32) {
+            for (int i = 8 * c; i < 8 * c + 8 && i < a.Dv; ++i) {
+                const float v = half_at(x, i, a.kv_f16);
+                const float y = __fmul_rn(__fdiv_rn(v, rms), half_at(a.gamma, i, a.kv_f16));
+                store_elem(a.ckv, crow, i, y);
+            }
+        }
+
+        // interleaved RoPE: y_j = z_2j c_j - z_2j+1 s_j, y_h+j = z_2j+1 c_h+j + z_2j s_h+j
+        uint8_t* krow = slot_row(a.k.rows, slot);
+        const uint16_t* z = x + a.Dv;
+        const uint16_t* cs = a.cos + t * a.Dk;
+        const uint16_t* sn = a.sin + t * a.Dk;
+        for (int j = lane; j < h; j += 32) {
+            const float z0 = half_at(z, 2 * j, a.kv_f16), z1 = half_at(z, 2 * j + 1, a.kv_f16);
+            const float c0 = half_at(cs, j, a.kv_f16), c1 = half_at(cs, h + j, a.kv_f16);
+            const float s0 = half_at(sn, j, a.kv_f16), s1 = half_at(sn, h + j, a.kv_f16);
+            const float y0 = __fadd_rn(__fmul_rn(z0, c0), __fmul_rn(-z1, s0));
+            const float y1 = __fadd_rn(__fmul_rn(z1, c1), __fmul_rn(z0, s1));
+            store_elem(a.k, krow, j, y0);
+            store_elem(a.k, krow, h + j, y1);
+        }
+    }
+}
+
+}  // namespace kvq

@@ -312,3 +312,103 @@ CONFIGS = {
     "cfg5a_compress_mode0": cfg5a_compress_mode0,
     "cfg5b_compress_mode2": cfg5b_compress_mode2,
 }
+
+
+# ---------------------------------------------------------------------------
+# device copies of a case and the library call that updates them
+# ---------------------------------------------------------------------------
+DEV = "cuda"
+
+TORCH_DT = {"bf16": torch.bfloat16, "f16": torch.float16, "e4m3": torch.float8_e4m3fn,
+            "e5m2": torch.float8_e5m2, "i8": torch.int8, "u8": torch.uint8, "e8m0": torch.float8_e8m0fnu,
+            "f32": torch.float32}
+
+
+def half_tensor(bits: np.ndarray, dt: str, device=DEV) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.view(TORCH_DT[dt]).to(device)
+
+
+def dev_cache(cb: CacheBuf, dt: torch.dtype):
+    st = torch.from_numpy(cb.storage.copy()).to(DEV)
+    eb = cb.elem_bytes
+    n = (st.numel() - cb.offset) // eb * eb
+    typed = st[cb.offset:cb.offset + n].view(dt)
+    view = typed.as_strided((cb.num_blocks, cb.block_size, cb.inner, cb.head_dim),
+                            (cb.block_stride // eb, cb.inner * cb.head_dim, cb.head_dim, 1))
+    return st, view
+
+
+def f32(a) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(DEV)
+
+
+def idx(a) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def build_call(case: Case):
+    """Device tensors for a case and a closure that runs the library call once.
+
+    Returns (call, storages, outputs): call(stream=None) enqueues the operation;
+    storages maps each cache name to the device copy of its whole byte buffer;
+    outputs collects the dense outputs (q_out, k_out, v_out) after a call.
+    """
+    import kv_cache_quantize_b200 as kvq
+    a, at = case.arrays, case.attrs
+    st, views, outs = {}, {}, {}
+    if case.op == "kv_compress_epilog":
+        st["cache"], views["cache"] = dev_cache(case.caches["cache"], torch.uint8)
+        x, s = half_tensor(a["x"], "bf16"), idx(a["slot_mapping"])
+
+        def call(stream=None):
+            kvq.kv_compress_epilog(x, s, views["cache"], at["quant_mode"], at["quant_group_size"], at["x_scale"],
+                                   stream=stream)
+    elif case.op == "indexer_quant_cache":
+        cdt = TORCH_DT[at["cache_dtype"]]
+        sdt = torch.float32 if at["quant_mode"] == 1 else torch.float8_e8m0fnu
+        st["cache"], views["cache"] = dev_cache(case.caches["cache"], cdt)
+        st["cache_scale"], views["cache_scale"] = dev_cache(case.caches["cache_scale"], sdt)
+        x, s = half_tensor(a["x"], at["x_dtype"]), idx(a["slot_mapping"])
+
+        def call(stream=None):
+            kvq.indexer_quant_cache(x, views["cache"], views["cache_scale"], s, at["quant_mode"], stream=stream)
+    elif case.op == "kv_rmsnorm_rope_cache":
+        kdt = at["kv_dtype"]
+        st["k_cache"], views["k_cache"] = dev_cache(case.caches["k_cache"], TORCH_DT[at["k_dtype"]])
+        st["ckv_cache"], views["ckv_cache"] = dev_cache(case.caches["ckv_cache"], TORCH_DT[at["ckv_dtype"]])
+        kv = half_tensor(a["kv"], kdt)
+        gamma, cos, sin = half_tensor(a["gamma"], kdt), half_tensor(a["cos"], kdt), half_tensor(a["sin"], kdt)
+        index = idx(a["index"])
+        opt = {k: (f32(a[k]) if k in a else None) for k in ("k_scale", "ckv_scale", "k_offset", "ckv_offset")}
+
+        def call(stream=None):
+            kvq.kv_rmsnorm_rope_cache(kv, gamma, cos, sin, index, views["k_cache"], views["ckv_cache"],
+                                      opt["k_scale"], opt["ckv_scale"], opt["k_offset"], opt["ckv_offset"],
+                                      at["epsilon"], at["cache_mode"], stream=stream)
+    elif case.op == "dequant_rope_quant_kvcache":
+        st["k_cache"], views["k_cache"] = dev_cache(case.caches["k_cache"], torch.int8)
+        st["v_cache"], views["v_cache"] = dev_cache(case.caches["v_cache"], torch.int8)
+        if at["x_dtype"] == "i32":
+            x = torch.from_numpy(np.ascontiguousarray(a["x"])).to(DEV)
+        else:
+            x = half_tensor(a["x"], at["x_dtype"])
+        cos, sin = half_tensor(a["cos"], at["cos_dtype"]), half_tensor(a["sin"], at["cos_dtype"])
+        bias = None
+        if "bias" in a:
+            bdt = at["bias_dtype"]
+            bias = f32(a["bias"]) if bdt == "f32" else (idx(a["bias"]) if bdt == "i32" else half_tensor(a["bias"], bdt))
+        opt = {k: (f32(a[k]) if k in a else None)
+               for k in ("offset_k", "offset_v", "weight_scale", "activation_scale")}
+        sk, sv, ind = f32(a["scale_k"]), f32(a["scale_v"]), idx(a["indices"])
+
+        def call(stream=None):
+            q, k, v = kvq.dequant_rope_quant_kvcache(
+                x, cos, sin, views["k_cache"], views["v_cache"], ind, sk, sv, opt["offset_k"], opt["offset_v"],
+                opt["weight_scale"], opt["activation_scale"], bias, at["size_splits"], "static", "BSND",
+                at["kv_output"], at["cache_mode"], outs.get("q_out"), outs.get("k_out"), outs.get("v_out"),
+                stream=stream)
+            outs["q_out"], outs["k_out"], outs["v_out"] = q, k, v
+    else:
+        raise ValueError(case.op)
+    return call, st, outs

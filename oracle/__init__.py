@@ -157,36 +157,67 @@ def _slots(a) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(a).ravel(), dtype=np.int64)
 
 
+def _row_chunks(T: int, threads: int):
+    n = max(1, min(threads, T))
+    bounds = np.linspace(0, T, n + 1).astype(np.int64)
+    return [(int(bounds[i]), int(bounds[i + 1])) for i in range(n) if bounds[i + 1] > bounds[i]]
+
+
+def _parallel_rows(T: int, threads: int, fn) -> int:
+    """Run fn(row_lo, row_hi) -> fault bits over row chunks.  Every row writes only
+    its own slot row, so chunks are independent; ctypes releases the GIL."""
+    chunks = _row_chunks(T, threads)
+    if len(chunks) <= 1:
+        return fn(0, T)
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(len(chunks)) as ex:
+        bits = list(ex.map(lambda c: fn(*c), chunks))
+    out = 0
+    for b in bits:
+        out |= b
+    return out
+
+
 def kv_compress_epilog(x_bits: np.ndarray, slot_mapping, cache: Paged, quant_mode: int,
-                       quant_group_size: int = 64, x_scale: float = 1.0) -> int:
+                       quant_group_size: int = 64, x_scale: float = 1.0, threads: int = 1) -> int:
     """x_bits: uint16 bf16 bit patterns [..., d].  Updates cache.storage; returns fault bits."""
     x = np.ascontiguousarray(x_bits, dtype=np.uint16)
     d = x.shape[-1]
     T = x.size // d
+    x = x.reshape(T, d)
     s = _slots(slot_mapping)
     assert s.size == T
-    faults = np.zeros(1, dtype=np.uint32)
     pc = cache.c()
-    rc = lib().kvqo_kv_compress_epilog(_ptr(x), T, d, d, _ptr(s), ctypes.byref(pc), quant_mode,
-                                       quant_group_size, ctypes.c_float(x_scale), _ptr(faults))
-    _check(rc, "kv_compress_epilog")
-    return int(faults[0])
+
+    def run(lo, hi):
+        faults = np.zeros(1, dtype=np.uint32)
+        rc = lib().kvqo_kv_compress_epilog(x[lo:].ctypes.data, hi - lo, d, d, s[lo:].ctypes.data,
+                                           ctypes.byref(pc), quant_mode, quant_group_size,
+                                           ctypes.c_float(x_scale), _ptr(faults))
+        _check(rc, "kv_compress_epilog")
+        return int(faults[0])
+    return _parallel_rows(T, threads, run)
 
 
 def indexer_quant_cache(x_bits: np.ndarray, x_dtype: str, slot_mapping, cache: Paged, cache_fp8: str,
-                        cache_scale: Paged, quant_mode: int) -> int:
+                        cache_scale: Paged, quant_mode: int, threads: int = 1) -> int:
     x = np.ascontiguousarray(x_bits, dtype=np.uint16)
     d = x.shape[-1]
     T = x.size // d
+    x = x.reshape(T, d)
     s = _slots(slot_mapping)
     assert s.size == T
-    faults = np.zeros(1, dtype=np.uint32)
     pc, ps = cache.c(), cache_scale.c()
-    rc = lib().kvqo_indexer_quant_cache(_ptr(x), IN_DTYPES[x_dtype], T, d, d, _ptr(s), ctypes.byref(pc),
-                                        1 if cache_fp8 == "e5m2" else 0, ctypes.byref(ps), quant_mode,
-                                        _ptr(faults))
-    _check(rc, "indexer_quant_cache")
-    return int(faults[0])
+
+    def run(lo, hi):
+        faults = np.zeros(1, dtype=np.uint32)
+        rc = lib().kvqo_indexer_quant_cache(x[lo:].ctypes.data, IN_DTYPES[x_dtype], hi - lo, d, d,
+                                            s[lo:].ctypes.data, ctypes.byref(pc),
+                                            1 if cache_fp8 == "e5m2" else 0, ctypes.byref(ps), quant_mode,
+                                            _ptr(faults))
+        _check(rc, "indexer_quant_cache")
+        return int(faults[0])
+    return _parallel_rows(T, threads, run)
 
 
 @dataclass

@@ -13,19 +13,20 @@ def paged(c: CacheBuf, storage: np.ndarray) -> oracle.Paged:
     return oracle.Paged(storage, c.offset, c.num_blocks, c.block_size, c.row_bytes, c.block_stride)
 
 
-def run_oracle(case: Case):
+def run_oracle(case: Case, threads: int = 1):
     """Returns (dict of updated cache storages, outputs dict, fault bits)."""
     st = {k: v.storage.copy() for k, v in case.caches.items()}
     a, at = case.arrays, case.attrs
     outs = {}
     if case.op == "kv_compress_epilog":
         f = oracle.kv_compress_epilog(a["x"], a["slot_mapping"], paged(case.caches["cache"], st["cache"]),
-                                      at["quant_mode"], at["quant_group_size"], at["x_scale"])
+                                      at["quant_mode"], at["quant_group_size"], at["x_scale"], threads)
     elif case.op == "indexer_quant_cache":
         f = oracle.indexer_quant_cache(a["x"], at["x_dtype"], a["slot_mapping"],
                                        paged(case.caches["cache"], st["cache"]),
                                        "e5m2" if at["cache_dtype"] == "e5m2" else "e4m3",
-                                       paged(case.caches["cache_scale"], st["cache_scale"]), at["quant_mode"])
+                                       paged(case.caches["cache_scale"], st["cache_scale"]), at["quant_mode"],
+                                       threads)
     elif case.op == "kv_rmsnorm_rope_cache":
         kc, cc = case.caches["k_cache"], case.caches["ckv_cache"]
         ko = oracle.CacheOut(paged(kc, st["k_cache"]), at["k_dtype"], a.get("k_scale"), a.get("k_offset"))

@@ -1,0 +1,254 @@
+"""CUDA library vs the CPU oracle, byte for byte, through the C ABI.
+
+Every comparison covers the cache's whole byte storage (guard bands, block
+padding, headDim tails, skipped and unmapped rows included).  Small cases span
+several warp tiles and a ragged tail; the five named workloads run at full size.
+"""
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_quantize_b200 as kvq
+import oracle
+from _gpu_harness import run_gpu
+from _oracle_harness import run_oracle
+from kv_cache_quantize_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+THREADS = 16
+
+
+def _same(case, check_outputs=True):
+    st_o, out_o, f_o = run_oracle(case, threads=THREADS)
+    st_g, out_g, f_g = run_gpu(case)
+    assert f_g == f_o, f"fault bits gpu={f_g} oracle={f_o}"
+    for k in st_o:
+        a, b = st_g[k], st_o[k]
+        bad = np.nonzero(a != b)[0]
+        assert bad.size == 0, f"{case.name}/{k}: {bad.size} bytes differ, first at {bad[0]} gpu={a[bad[0]]:#x} oracle={b[bad[0]]:#x}"
+    if check_outputs:
+        for k, v in out_o.items():
+            if v is None:
+                continue
+            g = out_g[k].reshape(v.shape)
+            bad = np.nonzero(g != v)[0] if g.ndim == 1 else np.argwhere(g != v)
+            assert len(bad) == 0, f"{case.name}/{k}: {len(bad)} values differ"
+    return st_g, out_g
+
+
+# ---------------------------------------------------------------------------
+# kv_compress_epilog
+# ---------------------------------------------------------------------------
+def _ce(T, d, mode, G=64, kind="normal", pad=0, extra=13, skip=0.1, seed=0, slot_dtype=np.int32, xs=0.1,
+        block_size=16):
+    col = oracle.kv_cache_col(d, mode, G)
+    nblk = max(1, (2 * T + block_size - 1) // block_size)
+    return W.gen_compress(f"ce_m{mode}_g{G}_d{d}_T{T}_{kind}", T=T, d=d, quant_mode=mode, num_blocks=nblk,
+                          block_size=block_size, head_dim=col + extra, group_size=G, x_scale=xs, skip_frac=skip,
+                          outlier_frac=0.05, seed=seed, x_kind=kind, block_pad_bytes=pad, slot_dtype=slot_dtype)
+
+
+@pytest.mark.parametrize("kind", ["normal", "wide"])
+@pytest.mark.parametrize("mode,G", [(0, 64), (1, 64), (2, 16), (2, 32), (2, 64)])
+@pytest.mark.parametrize("d", [128, 576, 1024])
+def test_compress_small(mode, G, d, kind):
+    _same(_ce(203, d, mode, G, kind))
+
+
+@pytest.mark.parametrize("mode,G", [(0, 64), (1, 64), (2, 32)])
+@pytest.mark.parametrize("extra,pad", [(0, 0), (1, 0), (3, 40), (16, 1000), (7, 5)])
+def test_compress_row_alignments(mode, G, extra, pad):
+    """headDim tails and block strides that make rows start at every alignment."""
+    _same(_ce(77, 320, mode, G, extra=extra, pad=pad, seed=5))
+
+
+@pytest.mark.parametrize("T", [0, 1, 7, 8, 9, 31, 33])
+def test_compress_ragged_counts(T):
+    _same(_ce(T, 576, 0, seed=7))
+
+
+def test_compress_max_width_and_int64_slots():
+    _same(_ce(40, 8192, 0, seed=9, slot_dtype=np.int64))
+    _same(_ce(40, 8192, 2, 16, seed=9, slot_dtype=np.int64))
+    _same(_ce(40, 8192, 1, seed=9))
+
+
+def test_compress_strided_and_misaligned_x():
+    case = _ce(50, 256, 0, seed=11)
+    st_o, _, _ = run_oracle(case)
+    x = case.arrays["x"]
+    dev = "cuda"
+    # rows 320 elements apart (non-contiguous leading dim), and a view starting 1 element in
+    for stride_extra, shift in ((64, 0), (0, 1), (3, 1)):
+        row = x.shape[1] + stride_extra
+        buf = np.zeros(x.shape[0] * row + shift + 8, dtype=np.uint16)
+        for t in range(x.shape[0]):
+            buf[shift + t * row: shift + t * row + x.shape[1]] = x[t]
+        tb = torch.from_numpy(buf.view(np.int16)).view(torch.bfloat16).to(dev)
+        xv = tb[shift:shift + x.shape[0] * row].view(x.shape[0], row)[:, :x.shape[1]]
+        cb = case.caches["cache"]
+        st = torch.from_numpy(cb.storage.copy()).to(dev)
+        view = st[cb.offset:].as_strided((cb.num_blocks, cb.block_size, 1, cb.head_dim),
+                                         (cb.block_stride, cb.head_dim, cb.head_dim, 1))
+        kvq.kv_compress_epilog(xv, torch.from_numpy(case.arrays["slot_mapping"]).to(dev), view, 0)
+        torch.cuda.synchronize()
+        assert np.array_equal(st.cpu().numpy(), st_o["cache"]), (stride_extra, shift)
+
+
+def test_compress_bad_slots_raise_fault_and_skip():
+    case = _ce(64, 576, 0, seed=13)
+    s = case.arrays["slot_mapping"]
+    s[3] = case.caches["cache"].num_slots
+    s[10] = -5
+    s[11:20] = -1
+    _same(case)
+
+
+def test_compress_all_skipped():
+    case = _ce(64, 576, 2, 32, seed=15)
+    case.arrays["slot_mapping"][:] = -1
+    st_g, _ = _same(case)
+    assert np.array_equal(st_g["cache"], case.caches["cache"].storage)
+
+
+@pytest.mark.parametrize("name", ["cfg1_compress_mode1", "cfg5a_compress_mode0", "cfg5b_compress_mode2"])
+def test_compress_named_workloads_full_size(name):
+    _same(W.CONFIGS[name]())
+
+
+def test_compress_is_deterministic():
+    case = W.cfg5b_compress_mode2()
+    a, _, _ = run_gpu(case)
+    b, _, _ = run_gpu(case)
+    assert np.array_equal(a["cache"], b["cache"])
+
+
+# ---------------------------------------------------------------------------
+# indexer_quant_cache
+# ---------------------------------------------------------------------------
+def _ix(T, d, mode, cdt="e4m3", xdt="bf16", kind="student_t", pad=0, seed=0, extra=5):
+    scol = oracle.indexer_scale_col(d, mode)
+    code_bytes = (d + 1) // 2 if mode == 3 else d
+    return W.gen_indexer(f"ix_m{mode}_{cdt}_{xdt}_d{d}_T{T}", T=T, d=d, quant_mode=mode,
+                         num_blocks=max(1, (2 * T + 7) // 8), block_size=8, cache_head_dim=code_bytes + extra,
+                         scale_head_dim=scol + 3, cache_dtype=cdt, x_dtype=xdt, skip_frac=0.1, seed=seed,
+                         block_pad_bytes=pad, x_kind=kind)
+
+
+@pytest.mark.parametrize("xdt", ["bf16", "f16"])
+@pytest.mark.parametrize("mode,cdt", [(0, "e4m3"), (0, "e5m2"), (1, "e4m3"), (1, "e5m2"), (3, "u8")])
+@pytest.mark.parametrize("d", [32, 99, 128, 200, 256, 520])
+def test_indexer_small(mode, cdt, d, xdt):
+    _same(_ix(150, d, mode, cdt, xdt, seed=d))
+
+
+@pytest.mark.parametrize("mode,cdt", [(0, "e4m3"), (1, "e5m2"), (3, "u8")])
+def test_indexer_wide_values_and_padding(mode, cdt):
+    _same(_ix(97, 128, mode, cdt, kind="wide", pad=24, extra=0, seed=3))
+
+
+@pytest.mark.parametrize("name", ["cfg3a_indexer_mxfp8", "cfg3b_indexer_mxfp4"])
+def test_indexer_named_workloads_full_size(name):
+    _same(W.CONFIGS[name]())
+
+
+def test_indexer_bad_slot_fault():
+    case = _ix(64, 128, 0)
+    case.arrays["slot_mapping"][5] = case.caches["cache"].num_slots + 3
+    _same(case)
+
+
+# ---------------------------------------------------------------------------
+# kv_rmsnorm_rope_cache
+# ---------------------------------------------------------------------------
+def _rr(cache_mode="PA_BNSD", B=40, S=1, k_dtype="bf16", ckv_dtype="e4m3", kv_dtype="bf16", D=576, Dv=512,
+        seed=0, **kw):
+    opt = {}
+    if ckv_dtype in ("e4m3", "e5m2", "i8"):
+        opt["ckv_scale"] = [1 / 64]
+    if k_dtype in ("e4m3", "e5m2", "i8"):
+        opt["k_scale"] = [1 / 16]
+    if ckv_dtype == "i8":
+        opt["ckv_offset"] = [2.0]
+    opt.update(kw)
+    return W.gen_rmsnorm_rope(f"rr_{cache_mode}_{k_dtype}_{ckv_dtype}_{kv_dtype}_D{D}", B=B, S=S, D=D, Dv=Dv,
+                              num_blocks=max(B + 1, (2 * B * S) // 32 + 2), block_size=32, k_dtype=k_dtype,
+                              ckv_dtype=ckv_dtype, cache_mode=cache_mode, skip_frac=0.1, seed=seed,
+                              kv_dtype=kv_dtype, block_pad_bytes=64, **opt)
+
+
+@pytest.mark.parametrize("cache_mode,S", [("PA_BNSD", 1), ("PA", 3), ("Norm", 5), ("PA_BLK_BNSD", 70)])
+def test_rmsnorm_rope_cache_modes(cache_mode, S):
+    _same(_rr(cache_mode, B=6 if S > 1 else 40, S=S))
+
+
+@pytest.mark.parametrize("k_dtype,ckv_dtype", [("bf16", "bf16"), ("bf16", "e4m3"), ("f16", "e5m2"),
+                                               ("bf16", "i8"), ("e4m3", "bf16"), ("i8", "f16"),
+                                               ("e4m3", "e4m3"), ("i8", "i8")])
+def test_rmsnorm_rope_dtype_scenarios(k_dtype, ckv_dtype):
+    _same(_rr(k_dtype=k_dtype, ckv_dtype=ckv_dtype))
+
+
+@pytest.mark.parametrize("D,Dv", [(192, 128), (96, 32), (1034, 1000)])
+def test_rmsnorm_rope_other_widths_and_f16(D, Dv):
+    _same(_rr(D=D, Dv=Dv, kv_dtype="f16", k_dtype="f16", ckv_dtype="f16"))
+    _same(_rr(D=D, Dv=Dv))
+
+
+def test_rmsnorm_rope_named_workload_full_size():
+    _same(W.cfg2_rmsnorm_rope())
+
+
+# ---------------------------------------------------------------------------
+# dequant_rope_quant_kvcache
+# ---------------------------------------------------------------------------
+def _dq(**kw):
+    base = dict(B=3, S=40, Nq=4, Nkv=2, D=128, c0=8, c1=64, x_range=1 << 12, seed=1, block_pad_bytes=40)
+    base.update(kw)
+    name = "dq_" + "_".join(f"{k}{v}" for k, v in sorted(kw.items()))
+    return W.gen_dequant_rope_quant(name, **base)
+
+
+@pytest.mark.parametrize("cache_mode", ["page", "contiguous"])
+@pytest.mark.parametrize("kv_output", [False, True])
+def test_drq_modes(cache_mode, kv_output):
+    _same(_dq(cache_mode=cache_mode, kv_output=kv_output, skip_frac=0.1 if cache_mode == "page" else 0.0))
+
+
+@pytest.mark.parametrize("D", [32, 64, 96, 256])
+def test_drq_head_dims(D):
+    _same(_dq(D=D, Nq=4, Nkv=1, kv_output=True))   # H = 6*D, a multiple of 64
+
+
+@pytest.mark.parametrize("bias_dtype", ["f32", "bf16", "f16", "i32", None])
+def test_drq_bias_and_optional_inputs(bias_dtype):
+    _same(_dq(bias_dtype=bias_dtype, with_offsets=bias_dtype is not None,
+              with_activation_scale=bias_dtype != "f16"))
+
+
+@pytest.mark.parametrize("x_dtype", ["bf16", "f16"])
+def test_drq_float_input(x_dtype):
+    _same(_dq(x_dtype=x_dtype, cos_dtype=x_dtype, kv_output=True))
+
+
+def test_drq_two_dim_x():
+    _same(_dq(S=1, x_2d=True, kv_output=True, cache_mode="contiguous"))
+
+
+def test_drq_many_heads():
+    _same(_dq(Nq=40, Nkv=8, D=32, S=8))
+
+
+def test_drq_bad_index_fault():
+    case = _dq(cache_mode="page")
+    case.arrays["indices"][7] = case.caches["k_cache"].num_slots
+    _same(case)
+
+
+def test_drq_named_workload_full_size():
+    _same(W.cfg4_dequant_rope_quant())
+
+
+def test_drq_named_workload_narrow_range():
+    """Same shapes with |x| <= 2^12, where few int8 codes saturate."""
+    _same(W.cfg4_dequant_rope_quant(x_range=1 << 12))
