@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Benchmark of the per-token KV-cache epilogue on B200.
+
+A STEP is one pass of the headline workload: kv_compress_epilog over
+T = 262144 bf16 token rows of d = 576 (DeepSeek-V3 MLA width), first with
+quantMode 0 (group-64 FP8 E4M3 + bf16 scale, 672-byte rows) and then with
+quantMode 2 (group-32 FP4 E2M1 + bf16 scale, E4M3 static rope, 352-byte rows),
+scattered into paged caches of 4096 blocks x 128 slots (2 % of slots -1, 1 % of
+rows x50 outliers).  The two passes read separate copies of x, so every step
+reads 604 MB of input -- more than the 126 MB L2 -- and needs no L2 flush.
+
+value = token rows quantised per second over all ranks (2 x 262144 per step and
+GPU); the roofline object reports the dominant kernel's algorithmic HBM bytes
+per launch over its CUDA-event duration.  The other four workloads are timed
+once each (L2 flushed before every launch) and reported under "per_config".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 the script runs under torchrun, one process per GPU; tokens are
+independent, so every rank runs its own copy of the workload (weak scaling, no
+collective on the data path) and the step time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV-epilog tokens/s and achieved HBM GB/s vs ~8 TB/s B200 peak (1 GPU)"
+UNIT = "tokens/s"
+WORKLOAD = ("kv_compress_epilog large sweep: T=262144 tokens, d=576 bf16 N(0,1) with 1% rows x50; "
+            "quantMode=0 (group-64 FP8 E4M3, bf16 scale, 672-B rows) then quantMode=2 (group-32 FP4 E2M1, "
+            "bf16 scale, rope FP8 E4M3 static x_scale=0.1, 352-B rows); cache blockSize=128, 4096 blocks; "
+            "2% slot_mapping -1")
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes: what the method must move (each valid row's input bytes
+# plus its packed-row bytes out, 4 slot bytes per token, per-token cos/sin and
+# activation scale, per-call parameters once); never skipped rows' x, untouched
+# cache or headDim tails
+# ---------------------------------------------------------------------------
+def algorithmic_bytes(case) -> int:
+    a, at = case.arrays, case.attrs
+    if case.op == "kv_compress_epilog":
+        import kv_cache_quantize_b200 as kvq
+        T, d = a["x"].shape
+        valid = int((a["slot_mapping"] != -1).sum())
+        col = kvq.kv_cache_col(d, at["quant_mode"], at["quant_group_size"])
+        return valid * (2 * d + col) + T * a["slot_mapping"].itemsize
+    if case.op == "indexer_quant_cache":
+        import kv_cache_quantize_b200 as kvq
+        T, d = a["x"].shape
+        valid = int((a["slot_mapping"] != -1).sum())
+        mode = at["quant_mode"]
+        codes = (d + 1) // 2 if mode == 3 else d
+        scales = 4 if mode == 1 else kvq.indexer_scale_col(d, mode)
+        return valid * (2 * d + codes + scales) + T * a["slot_mapping"].itemsize
+    if case.op == "kv_rmsnorm_rope_cache":
+        B, _, S, D = a["kv"].shape
+        Dv = at["Dv"]
+        Dk = D - Dv
+        idx = a["index"]
+        valid = int((idx != -1).sum())
+        eb = {"bf16": 2, "f16": 2, "e4m3": 1, "e5m2": 1, "i8": 1}
+        per_row = 2 * D + 2 * 2 * Dk + Dv * eb[at["ckv_dtype"]] + Dk * eb[at["k_dtype"]]
+        params = 2 * Dv + sum(a[k].nbytes for k in ("k_scale", "ckv_scale", "k_offset", "ckv_offset") if k in a)
+        return valid * per_row + idx.size * idx.itemsize + params
+    if case.op == "dequant_rope_quant_kvcache":
+        B, S = a["x"].shape[0], (a["x"].shape[1] if a["x"].ndim == 3 else 1)
+        T = B * S
+        H = a["x"].shape[-1]
+        D, Nq, Nkv = at["D"], at["Nq"], at["Nkv"]
+        per_tok = H * a["x"].itemsize + 2 * 2 * D + Nq * D * 2 + 2 * Nkv * D
+        if at["kv_output"]:
+            per_tok += 2 * Nkv * D * 2
+        per_tok += a["indices"].itemsize if at["cache_mode"] == "page" else 0
+        per_tok += 4 if "activation_scale" in a else 0
+        params = sum(a[k].nbytes for k in ("weight_scale", "bias", "scale_k", "scale_v", "offset_k", "offset_v")
+                     if k in a)
+        return T * per_tok + params
+    raise ValueError(case.op)
+
+
+def token_rows(case) -> int:
+    a = case.arrays
+    if case.op in ("kv_compress_epilog", "indexer_quant_cache"):
+        return int(a["x"].shape[0])
+    if case.op == "kv_rmsnorm_rope_cache":
+        return int(a["kv"].shape[0] * a["kv"].shape[2])
+    return int(a["x"].shape[0] * (a["x"].shape[1] if a["x"].ndim == 3 else 1))
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kv_cache_quantize_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str):
+    """dram bytes per launch from a committed ncu summary, if taken on the current sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = kernel_source_hash()
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 3 and parts[0] == kernel and parts[1] == src:
+            return float(parts[2])
+    return None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML: the same counters nvidia-smi reads)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, b in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (the oracle as it stands, all host cores via row chunks)
+# ---------------------------------------------------------------------------
+def oracle_rows_per_s(cases, budget_s: float, threads: int):
+    """Time the oracle on the workload's passes, 16384-row chunk by chunk (alternating
+    passes), until budget_s is spent or every row is done; returns (rows/s, rows, s)."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import oracle
+    from _oracle_harness import paged
+    chunk, rows, spent = 16384, 0, 0.0
+    T = min(c.arrays["x"].shape[0] for c in cases)
+    for lo in range(0, T, chunk):
+        hi = min(T, lo + chunk)
+        for case in cases:
+            a, at = case.arrays, case.attrs
+            st = case.caches["cache"].storage.copy()
+            t0 = time.perf_counter()
+            oracle.kv_compress_epilog(a["x"][lo:hi], a["slot_mapping"][lo:hi], paged(case.caches["cache"], st),
+                                      at["quant_mode"], at["quant_group_size"], at["x_scale"], threads=threads)
+            spent += time.perf_counter() - t0
+            rows += hi - lo
+        if spent >= budget_s:
+            break
+    return rows / spent, rows, spent
+
+
+def run_reference(args):
+    """The base contract's reference arm: the CPU oracle, timed on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from kv_cache_quantize_b200 import workloads as W
+    threads = os.cpu_count() or 1
+    cases = [W.cfg5a_compress_mode0(), W.cfg5b_compress_mode2()]
+    # size each step so that warmup + steps end within about two minutes
+    rate, _, _ = oracle_rows_per_s(cases, 2.0, threads)
+    per_step_s = min(10.0, 120.0 / max(1, args.steps + args.warmup))
+    rows_per_pass = max(256, min(262144, int(rate * per_step_s / 2)))
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import oracle
+    from _oracle_harness import paged
+
+    def step():
+        for case in cases:
+            a, at = case.arrays, case.attrs
+            st = case.caches["cache"].storage.copy()
+            oracle.kv_compress_epilog(a["x"][:rows_per_pass], a["slot_mapping"][:rows_per_pass],
+                                      paged(case.caches["cache"], st), at["quant_mode"], at["quant_group_size"],
+                                      at["x_scale"], threads=threads)
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        step()
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = 2 * rows_per_pass * args.steps / total
+    sample = (f"first {rows_per_pass} of the 262144 token rows of each quantMode pass per step "
+              f"(oracle in C, rows split over {threads} host threads)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "parallelism": "cpu oracle, rank 0 only"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-per-config", action="store_true", help="skip the per-workload breakdown")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import kv_cache_quantize_b200 as kvq
+    from kv_cache_quantize_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    kvq.lib()
+
+    # ---------------- headline workload ----------------
+    case_a = W.cfg5a_compress_mode0(seed=rank)
+    case_b = W.cfg5b_compress_mode2(seed=rank)
+    call_a, st_a, _ = W.build_call(case_a)
+    call_b, st_b, _ = W.build_call(case_b)
+    stream = torch.cuda.current_stream(dev)
+    bytes_a, bytes_b = algorithmic_bytes(case_a), algorithmic_bytes(case_b)
+    tokens_per_step = token_rows(case_a) + token_rows(case_b)
+
+    for _ in range(args.warmup):
+        call_a(stream)
+        call_b(stream)
+    torch.cuda.synchronize(dev)
+    if kvq.get_error(stream) != 0:
+        raise RuntimeError("device fault bits set during warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for e0, e1, e2 in ev:
+            e0.record(stream)
+            call_a(stream)
+            e1.record(stream)
+            call_b(stream)
+            e2.record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    elapsed = start.elapsed_time(stop) / 1e3
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+        dist.barrier()
+    ms_a = [e0.elapsed_time(e1) for e0, e1, _ in ev]
+    ms_b = [e1.elapsed_time(e2) for _, e1, e2 in ev]
+    faults = kvq.get_error(stream)
+
+    value = world * tokens_per_step * args.steps / elapsed
+    peak, peak_kind = hbm_peak()
+    avg_a, avg_b = statistics.mean(ms_a) / 1e3, statistics.mean(ms_b) / 1e3
+    kernels = {
+        "compress_epilog_kernel<0,64> (quantMode 0)": {
+            "alg_bytes_per_launch": bytes_a, "avg_us": 1e6 * avg_a, "median_us": 1e6 * statistics.median(ms_a) / 1e3,
+            "alg_GBps": bytes_a / avg_a / 1e9, "frac_of_peak": bytes_a / avg_a / 1e9 / peak,
+            "share_of_step": avg_a / (avg_a + avg_b)},
+        "compress_epilog_kernel<2,32> (quantMode 2)": {
+            "alg_bytes_per_launch": bytes_b, "avg_us": 1e6 * avg_b, "median_us": 1e6 * statistics.median(ms_b) / 1e3,
+            "alg_GBps": bytes_b / avg_b / 1e9, "frac_of_peak": bytes_b / avg_b / 1e9 / peak,
+            "share_of_step": avg_b / (avg_a + avg_b)},
+    }
+    dom_name, dom_bytes, dom_avg = ("compress_epilog_kernel<0,64>", bytes_a, avg_a) if avg_a >= avg_b else \
+        ("compress_epilog_kernel<2,32>", bytes_b, avg_b)
+    achieved = dom_bytes / dom_avg / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": profiled_traffic(dom_name), "kernel": dom_name,
+                "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)", "alg_bytes_per_launch": dom_bytes}
+
+    # ---------------- end to end through the public API with host buffers ----------------
+    e2e_steps = min(args.steps, 10)
+    xa_host = torch.from_numpy(case_a.arrays["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    xb_host = torch.from_numpy(case_b.arrays["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    sa_host = torch.from_numpy(case_a.arrays["slot_mapping"]).pin_memory()
+    sb_host = torch.from_numpy(case_b.arrays["slot_mapping"]).pin_memory()
+    xa_dev, xb_dev = torch.empty_like(xa_host, device=dev), torch.empty_like(xb_host, device=dev)
+    sa_dev, sb_dev = torch.empty_like(sa_host, device=dev), torch.empty_like(sb_host, device=dev)
+    from kv_cache_quantize_b200.workloads import dev_cache
+    _, cache_a = dev_cache(case_a.caches["cache"], torch.uint8)
+    _, cache_b = dev_cache(case_b.caches["cache"], torch.uint8)
+    at_a, at_b = case_a.attrs, case_b.attrs
+
+    def e2e_step():
+        xa_dev.copy_(xa_host, non_blocking=True)
+        sa_dev.copy_(sa_host, non_blocking=True)
+        kvq.kv_compress_epilog(xa_dev, sa_dev, cache_a, at_a["quant_mode"], at_a["quant_group_size"],
+                               at_a["x_scale"], stream=stream)
+        xb_dev.copy_(xb_host, non_blocking=True)
+        sb_dev.copy_(sb_host, non_blocking=True)
+        kvq.kv_compress_epilog(xb_dev, sb_dev, cache_b, at_b["quant_mode"], at_b["quant_group_size"],
+                               at_b["x_scale"], stream=stream)
+        return kvq.get_error(stream)      # device -> host read of the step's result (fault word)
+    for _ in range(3):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_s = time.perf_counter() - t0
+    if world > 1:
+        t = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    h2d = xa_host.nbytes + xb_host.nbytes + sa_host.nbytes + sb_host.nbytes
+    e2e = {"value": world * tokens_per_step * e2e_steps / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": 4, "steps": e2e_steps,
+           "note": "pinned host x + slot_mapping copied in, both passes through the C ABI, fault word read back"}
+    del xa_host, xb_host, xa_dev, xb_dev, cache_a, cache_b
+
+    # ---------------- per-workload breakdown (rank 0) ----------------
+    per_config = None
+    if rank == 0 and not args.no_per_config:
+        per_config = {}
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for name, make in W.CONFIGS.items():
+            case = {"cfg5a_compress_mode0": case_a, "cfg5b_compress_mode2": case_b}.get(name) or make()
+            call, _, _ = W.build_call(case)
+            reps = 50
+            times = []
+            for i in range(reps + 3):
+                flush.fill_(i & 0xFF)                 # evict the previous launch's data from L2
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                call(stream)
+                e1.record(stream)
+                if i >= 3:
+                    times.append((e0, e1))
+            torch.cuda.synchronize(dev)
+            us = sorted(1e3 * a.elapsed_time(b) for a, b in times)
+            med = statistics.median(us) / 1e6
+            nb = algorithmic_bytes(case)
+            per_config[name] = {"tokens": token_rows(case), "alg_bytes": nb, "median_us": med * 1e6,
+                                "tokens_per_s": token_rows(case) / med, "alg_GBps": nb / med / 1e9,
+                                "frac_of_peak": nb / med / 1e9 / peak}
+            del call, case
+            torch.cuda.empty_cache()
+        del flush
+
+    # ---------------- CPU oracle baseline (rank 0, N = 1) ----------------
+    cpu = None
+    if rank == 0 and world == 1:
+        threads = os.cpu_count() or 1
+        rate, rows, spent = oracle_rows_per_s([case_a, case_b], args.cpu_budget, threads)
+        cpu = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{rows} token rows of the two quantMode passes in 16384-row chunks, {spent:.1f} s "
+                         f"(oracle in C, rows split over {threads} host threads)"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "tokens_per_step_per_gpu": tokens_per_step,
+                           "alg_bytes_per_step_per_gpu": bytes_a + bytes_b,
+                           "alg_GBps_per_gpu": (bytes_a + bytes_b) * args.steps / elapsed / 1e9,
+                           "l2": "inputs larger than L2 (two 302 MB x buffers per step), no flush",
+                           "parallelism": f"replicas x{world} (independent token batches, no collective)"},
+                "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": 2 * args.steps, "clocks": clocks.summary(), "fault_bits": faults,
+                "per_config": per_config}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -19,6 +19,7 @@ namespace kvq {
 struct DrqArgs {
     const void* x;          // [B*S, H]
     int32_t x_kind;         // 0 int32, 1 bf16, 2 f16
+    int32_t x_vec;          // x is 16-byte aligned (vector loads of int32 values)
     int64_t B, S, H;
     const uint16_t* cos;    // [B*S, D]
     const uint16_t* sin;
@@ -49,13 +50,13 @@ template <int E>
 __device__ __forceinline__ void dq_load(const DrqArgs& a, int64_t e0, float (&u)[E], const int32_t* xi) {
     if (a.x_kind == 0) {
         int32_t v[E];
-        if (E % 4 == 0) {
+        if (E % 4 == 0 && a.x_vec) {
 #pragma unroll
             for (int k = 0; k < E; k += 4) {
                 const int4 w = __ldcs(reinterpret_cast<const int4*>(xi + e0 + k));
                 v[k] = w.x; v[k + 1] = w.y; v[k + 2] = w.z; v[k + 3] = w.w;
             }
-        } else if (E % 2 == 0) {
+        } else if (E % 2 == 0 && a.x_vec) {
 #pragma unroll
             for (int k = 0; k < E; k += 2) {
                 const int2 w = __ldcs(reinterpret_cast<const int2*>(xi + e0 + k));

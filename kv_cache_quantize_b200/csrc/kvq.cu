@@ -43,8 +43,15 @@ int64_t numel(const kvq_tensor* t) {
     return n;
 }
 
+int64_t numel_leading(const kvq_tensor* t) {
+    int64_t n = 1;
+    for (int i = 0; i + 1 < t->ndim; ++i) n *= t->shape[i];
+    return n;
+}
+
 // Row-major contiguous (dimensions of size 1 may carry any stride).
 bool contiguous(const kvq_tensor* t) {
+    if (numel(t) == 0) return true;   // no elements: any strides describe it
     int64_t expect = 1;
     for (int i = t->ndim - 1; i >= 0; --i) {
         if (t->shape[i] == 1) continue;
@@ -59,6 +66,11 @@ bool contiguous(const kvq_tensor* t) {
 bool flatten_rows(const kvq_tensor* t, int64_t* rows, int64_t* row_stride) {
     if (t->ndim < 1) return false;
     const int64_t d = t->shape[t->ndim - 1];
+    if (numel(t) == 0) {             // no elements: any strides describe it
+        *rows = d == 0 ? 0 : numel_leading(t);
+        *row_stride = d;
+        return true;
+    }
     if (d > 1 && t->stride[t->ndim - 1] != 1) return false;
     int64_t r = 1, rs = -1, expect = -1;
     for (int i = t->ndim - 2; i >= 0; --i) {
@@ -570,6 +582,7 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
     DrqArgs a;
     a.x = x->data;
     a.x_kind = dq ? 0 : (x->dtype == KVQ_BF16 ? 1 : 2);
+    a.x_vec = reinterpret_cast<uintptr_t>(x->data) % 16 == 0;
     a.B = B;
     a.S = S;
     a.H = H;

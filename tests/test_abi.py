@@ -208,3 +208,11 @@ def test_dequant_rope_quant_validation(L):
     kc48 = D([512, 128, 4, 48], "i8")
     assert f(kc=kc48, vc=kc48, c=D([16, 1024, 1, 48], "bf16"), x=D([16, 1024, 1152], "i32"),
              splits=(768, 192, 192), q=D([16, 1024, 16, 48], "bf16")) == EUNSUP   # D % 32 != 0
+
+
+def test_empty_inputs_are_accepted_whatever_their_strides(L):
+    x, s, c = D([0, 576], "bf16", [0, 0]), D([0], "i32", [0]), D([8, 16, 1, 672], "u8")
+    assert ce(L, x, s, c) == OK
+    xi, si = D([0, 128], "f16", [0, 0]), D([0], "i64", [0])
+    assert L.kvq_indexer_quant_cache(R(xi), R(D([16, 8, 1, 128], "e4m3")), R(D([16, 8, 1, 4], "e8m0")), R(si), 0,
+                                     None) == OK

@@ -21,7 +21,8 @@ def _inputs(seed: int, nonneg: bool = False) -> np.ndarray:
         v = (bf[:, None] * scales[None, :]).astype(np.float32).ravel()
     rng = np.random.default_rng(seed)
     rnd = rng.integers(0, 1 << 32, size=4_000_000, dtype=np.uint64).astype(np.uint32).view(np.float32)
-    near = (rnd % np.float32(1000.0)).astype(np.float32)
+    with np.errstate(invalid="ignore"):
+        near = (rnd % np.float32(1000.0)).astype(np.float32)
     v = np.concatenate([v, rnd, near, np.array([0.0, -0.0, 1e-45, -1e-45, 448.0, 464.0, 480.0, -500.0,
                                                 6.0, 5.0, 7.0, 0.25, 0.75, 57344.0, 61440.0], np.float32)])
     v = v[np.isfinite(v)]
