@@ -91,6 +91,7 @@ typedef enum {
 
 /* Fault bits of the device fault word. */
 #define KVQ_FAULT_SLOT_RANGE 0x1u   /* a slot/index outside [0, num_slots) and not -1 */
+#define KVQ_FAULT_TIMEOUT 0x2u      /* a pipeline wait gave up (an internal error; the output is incomplete) */
 
 /* ------------------------------------------------------------------------ */
 /* kv_compress_epilog                                                        */
@@ -243,6 +244,18 @@ KVQ_API kvq_status kvq_get_error(kvq_stream stream, uint32_t* fault_bits);
  * nibble), 3 bf16 (2 bytes, RNE), 4 E8M0 rounded up (1 byte), 5 int8 static
  * (1 byte, rint then clamp).  in, out: device pointers. */
 KVQ_API kvq_status kvq_convert(int32_t fmt, const float* in, int64_t n, void* out, kvq_stream stream);
+
+/* Device self-test of the arithmetic shortcuts the kernels rely on (no
+ * counterpart on the pages).  which = 0 / 1: the number of (numerator, scale)
+ * pairs -- every finite bf16 numerator a and every bf16 scale s in
+ * [2^-100, 2^101) with |a| <= 512 s -- where the one-step (0) or two-step (1)
+ * division-by-scale differs from IEEE division in any bit; 2 / 3: the number
+ * of such pairs whose E4M3 (2) or E2M1 (3) code of the one-step quotient
+ * differs from the code of the IEEE quotient; 4: the number of positive
+ * finite bf16 values a for which the constant-divisor form of a / 448,
+ * a / 57344 or a / 6 differs from IEEE division.  Blocks until done; *result
+ * receives the count (0 means the shortcut is exact on the domain). */
+KVQ_API kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream);
 
 /* Static description of a status code. */
 KVQ_API const char* kvq_status_string(kvq_status status);

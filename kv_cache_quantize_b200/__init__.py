@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "KvqError", "lib", "library_path", "kv_compress_epilog", "indexer_quant_cache", "kv_rmsnorm_rope_cache",
-    "dequant_rope_quant_kvcache", "get_error", "kv_cache_col", "indexer_scale_col", "convert",
+    "dequant_rope_quant_kvcache", "get_error", "kv_cache_col", "indexer_scale_col", "convert", "selftest",
     "FAULT_SLOT_RANGE", "STATUS",
 ]
 
@@ -74,6 +74,7 @@ def lib() -> ctypes.CDLL:
                                                      ctypes.POINTER(i64), i32, i32, i32, i32, i32, _P, _P, _P, vp]
         L.kvq_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.kvq_convert.argtypes = [i32, vp, i64, vp, vp]
+        L.kvq_selftest.argtypes = [i32, ctypes.POINTER(ctypes.c_uint64), vp]
         L.kvq_kv_cache_col.argtypes = [i64, i32, i32]
         L.kvq_kv_cache_col.restype = i64
         L.kvq_indexer_scale_col.argtypes = [i64, i32]
@@ -82,7 +83,7 @@ def lib() -> ctypes.CDLL:
         L.kvq_status_string.restype = ctypes.c_char_p
         L.kvq_version.restype = i32
         for name in ("kvq_kv_compress_epilog", "kvq_indexer_quant_cache", "kvq_kv_rmsnorm_rope_cache",
-                     "kvq_dequant_rope_quant_kvcache", "kvq_get_error", "kvq_convert"):
+                     "kvq_dequant_rope_quant_kvcache", "kvq_get_error", "kvq_convert", "kvq_selftest"):
             getattr(L, name).restype = i32
         _LIB = L
     return _LIB
@@ -219,6 +220,15 @@ def kv_cache_col(d: int, quant_mode: int, quant_group_size: int = 64) -> int:
 def indexer_scale_col(d: int, quant_mode) -> int:
     mode = INDEXER_MODES[quant_mode] if isinstance(quant_mode, str) else int(quant_mode)
     return int(lib().kvq_indexer_scale_col(d, mode))
+
+
+def selftest(which: int, stream=None, device=None) -> int:
+    """Run a device self-test of the kernels' arithmetic shortcuts; returns the mismatch count."""
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    out = ctypes.c_uint64(0)
+    _check("selftest", lib().kvq_selftest(int(which), ctypes.byref(out), _stream(stream)))
+    return int(out.value)
 
 
 def convert(fmt: str, values: torch.Tensor, stream=None) -> torch.Tensor:

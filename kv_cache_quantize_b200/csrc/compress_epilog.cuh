@@ -15,6 +15,7 @@
 #pragma once
 
 #include "kvq_device.cuh"
+#include "tma_pipe.cuh"
 
 namespace kvq {
 
@@ -31,7 +32,18 @@ struct CompressArgs {
     int32_t col;            // kvCacheCol
     float x_scale;          // mode 2 rope multiplier
     int32_t x_vec;          // every row chunk is 16-byte aligned
+    // pipelined kernel only
+    int32_t R;              // rows per shared-memory stage (<= 32)
+    int32_t stages;         // ring depth
+    float inv_nseg;         // 1 / nseg in binary32
 };
+
+// Division of a code's numerator by the group scale: the one- or two-step
+// Markstein form (kvq_device.cuh); kvq_selftest confirms the choice is exact
+// against IEEE division on its whole domain.
+#ifndef KVQ_SCALE_DIV
+#define KVQ_SCALE_DIV div_scale2
+#endif
 
 constexpr int CE_TILE = 8;
 constexpr int CE_UNROLL = 3;
@@ -50,17 +62,31 @@ __device__ __forceinline__ int64_t load_slot(const void* slots, int is64, int64_
 
 // One segment.  All lanes call this (the shuffles need the whole warp); lanes
 // whose segment is inactive or skipped carry live == false.
+// x_i / sf for the eight values of a lane: Markstein-corrected multiply by the
+// reciprocal when the scale is in the self-tested range, IEEE division else.
+__device__ __forceinline__ void div_by_scale8(const float (&f)[8], float sf, float (&q)[8]) {
+    if (scale_in_fast_range(sf)) {
+        const float r = __frcp_rn(sf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = KVQ_SCALE_DIV(f[i], sf, r);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], sf);
+    }
+}
+
+// One segment of 64 values, one 16-byte chunk per lane of an 8-lane team.
+// All lanes call this (the shuffles need the whole warp); row == nullptr for
+// lanes whose segment is inactive or whose token is skipped.
 template <int MODE, int G>
-__device__ __forceinline__ void ce_segment(const CompressArgs& a, const uint4& v, bool live, int64_t slot,
-                                           int j, int sub) {
+__device__ __forceinline__ void ce_segment(const CompressArgs& a, const uint4& v, uint8_t* row, int j, int sub) {
     constexpr int GL = (MODE == 2 ? G : 64) / 8;   // lanes per quantisation group
     uint32_t m = absmax_bits8(v);
     if (GL >= 2) m = max(m, __shfl_xor_sync(FULL_MASK, m, 1));
     if (GL >= 4) m = max(m, __shfl_xor_sync(FULL_MASK, m, 2));
     if (GL >= 8) m = max(m, __shfl_xor_sync(FULL_MASK, m, 4));
-    if (!live) return;
+    if (row == nullptr) return;
 
-    uint8_t* row = slot_row(a.cache, slot);
     const bool rope = (j == a.nseg - 1);
     float f[8];
     widen8<false>(v, f);
@@ -74,8 +100,7 @@ __device__ __forceinline__ void ce_segment(const CompressArgs& a, const uint4& v
             uint2 codes = make_uint2(0u, 0u);
             if (sf != 0.0f) {
                 float q[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], sf);
+                div_by_scale8(f, sf, q);
                 codes = fp8x8<false>(q);
             }
             st_b64(row + j * 64 + sub * 8, codes);
@@ -105,8 +130,7 @@ __device__ __forceinline__ void ce_segment(const CompressArgs& a, const uint4& v
             uint32_t codes = 0u;
             if (sf != 0.0f) {
                 float q[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], sf);
+                div_by_scale8(f, sf, q);
                 codes = e2m1x8(q);
             }
             st_b32(row + j * 32 + sub * 4, codes);
@@ -163,8 +187,106 @@ __global__ void __launch_bounds__(CE_THREADS) compress_epilog_kernel(const Compr
                 }
             }
 #pragma unroll
-            for (int u = 0; u < CE_UNROLL; ++u) ce_segment<MODE, G>(a, v[u], live[u], sl[u], jj[u], sub);
+            for (int u = 0; u < CE_UNROLL; ++u)
+                ce_segment<MODE, G>(a, v[u], live[u] ? slot_row(a.cache, sl[u]) : nullptr, jj[u], sub);
         }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Pipelined kernel (16-byte aligned rows).  CTA = CT_CONSUMER_WARPS consumer
+// warps + 1 producer warp.  The producer walks the CTA's tiles of R rows:
+// lanes load the R slots, turn valid ones into destination row pointers (kept
+// in shared memory for the consumers) and issue one bulk copy per valid row
+// into the stage; skipped rows are never read.  Consumers take the tile's
+// segments four per warp (one per team), reading x from shared memory.
+// ---------------------------------------------------------------------------
+constexpr int CT_CONSUMER_WARPS = 8;
+constexpr int CT_THREADS = (CT_CONSUMER_WARPS + 1) * 32;
+
+__host__ __device__ inline uint32_t ct_header_bytes(int stages, int R) {
+    return ((uint32_t)(16 * stages + 8 * stages * R) + 127u) & ~127u;
+}
+
+template <int MODE, int G>
+__global__ void __launch_bounds__(CT_THREADS) compress_tma_kernel(const CompressArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int S = a.stages, R = a.R;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + S;
+    uint8_t** rowptr = reinterpret_cast<uint8_t**>(empty + S);
+    uint8_t* xs = smem + ct_header_bytes(S, R);
+    const uint32_t row_bytes = (uint32_t)a.nseg * 128u;
+    const uint32_t stage_bytes = (uint32_t)R * row_bytes;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t ntiles = (a.T + R - 1) / R;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < S; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], CT_CONSUMER_WARPS);
+        }
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    if (warp == CT_CONSUMER_WARPS) {
+        // ---------------- producer ----------------
+        int it = 0;
+        for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+            const int st = it % S;
+            const uint32_t round = (uint32_t)(it / S);
+            if (!__all_sync(FULL_MASK, mbar_wait(&empty[st], (round & 1u) ^ 1u))) break;
+            const int64_t row0 = tile * R;
+            const int rows = (int)(a.T - row0 < R ? a.T - row0 : R);
+            uint8_t* p = nullptr;
+            if (lane < rows) {
+                const int64_t slot = load_slot(a.slots, a.slots_i64, row0 + lane);
+                if (slot != -1) {
+                    if (slot_ok(slot, a.cache.num_slots)) p = slot_row(a.cache, slot);
+                    else raise_fault(FAULT_SLOT_RANGE);
+                }
+            }
+            if (lane < R) rowptr[st * R + lane] = p;
+            const unsigned valid = __ballot_sync(FULL_MASK, p != nullptr);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)__popc(valid) * row_bytes);
+            __syncwarp();
+            if (p != nullptr)
+                bulk_copy_g2s(xs + (size_t)st * stage_bytes + (size_t)lane * row_bytes,
+                              a.x + (row0 + lane) * a.x_row_stride, row_bytes, &full[st]);
+        }
+        // no copy may still be in flight when the CTA exits
+        if (lane == 0)
+            for (int k = it > S ? it - S : 0; k < it; ++k) mbar_wait(&full[k % S], (uint32_t)(k / S) & 1u);
+        return;
+    }
+
+    // ---------------- consumers ----------------
+    const int team = lane >> 3, sub = lane & 7;
+    int it = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        const int st = it % S;
+        const uint32_t round = (uint32_t)(it / S);
+        if (!__all_sync(FULL_MASK, mbar_wait(&full[st], round & 1u))) break;   // every lane acquires the stage
+        const int64_t row0 = tile * R;
+        const int rows = (int)(a.T - row0 < R ? a.T - row0 : R);
+        const int nsegs = rows * a.nseg;
+        const uint8_t* xst = xs + (size_t)st * stage_bytes;
+        for (int base = warp * 4; base < nsegs; base += CT_CONSUMER_WARPS * 4) {
+            const int seg = base + team;
+            const bool act = seg < nsegs;
+            // seg / nseg: (seg + 1/2) / nseg is never an integer and its binary32
+            // product with 1/nseg is within 2^-11 of it for seg < 2^12, nseg <= 128
+            const int r = act ? (int)(((float)seg + 0.5f) * a.inv_nseg) : 0;
+            const int j = seg - r * a.nseg;
+            uint8_t* row = act ? rowptr[st * R + r] : nullptr;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (row != nullptr) v = *reinterpret_cast<const uint4*>(xst + (size_t)r * row_bytes + j * 128 + sub * 16);
+            ce_segment<MODE, G>(a, v, row, j, sub);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
     }
 }
 

@@ -177,9 +177,75 @@ __global__ void convert_kernel(int32_t fmt, const float* in, int64_t n, uint8_t*
     }
 }
 
+// ---------------------------------------------------------------------------
+// self-test of the division shortcut (kvq_selftest)
+// ---------------------------------------------------------------------------
+__device__ unsigned long long g_selftest_count;
+
+// grid.x: numerator bit patterns (65536); threads walk the scale patterns with
+// biased exponent 27..227 (2^-100 <= s < 2^101), all 128 fractions each.
+__global__ void selftest_div_kernel(int32_t which) {
+    const uint32_t abits = blockIdx.x;
+    if ((abits & 0x7f80u) == 0x7f80u) return;               // inf / NaN numerators
+    const float a = __uint_as_float(abits << 16);
+    unsigned long long bad = 0;
+    for (uint32_t k = threadIdx.x; k < 201u * 128u; k += blockDim.x) {
+        const uint32_t sbits = ((27u + k / 128u) << 7) | (k % 128u);
+        const float s = __uint_as_float(sbits << 16);
+        if (fabsf(a) > 512.0f * s) continue;
+        const float r = __frcp_rn(s);
+        const float ref = __fdiv_rn(a, s);
+        const float q1 = div_scale1(a, s, r);
+        bool diff;
+        switch (which) {
+            case 0: diff = __float_as_uint(q1) != __float_as_uint(ref); break;
+            case 1: diff = __float_as_uint(div_scale2(a, s, r)) != __float_as_uint(ref); break;
+            case 2: diff = e4m3x2(q1, 0.0f) != e4m3x2(ref, 0.0f); break;
+            default: {
+                const float v1[8] = {q1, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                const float v2[8] = {ref, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                diff = (e2m1x8(v1) & 0xfu) != (e2m1x8(v2) & 0xfu);
+            }
+        }
+        bad += diff ? 1ull : 0ull;
+    }
+    if (bad) atomicAdd(&g_selftest_count, bad);
+}
+
+// every positive finite bf16 amax over the three format maxima
+__global__ void selftest_fmax_kernel() {
+    const uint32_t bits = blockIdx.x * blockDim.x + threadIdx.x;   // 0 .. 32767
+    if (bits >= 0x7f80u) return;
+    const float a = __uint_as_float(bits << 16);
+    unsigned long long bad = 0;
+    const float cs[3] = {448.0f, 57344.0f, 6.0f};
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+        bad += __float_as_uint(div_by_fmax(a, cs[i])) != __float_as_uint(__fdiv_rn(a, cs[i])) ? 1ull : 0ull;
+    if (bad) atomicAdd(&g_selftest_count, bad);
+}
+
 }  // namespace
 
 extern "C" {
+
+kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream) {
+    if (!result) return KVQ_ERR_NULL;
+    if (which < 0 || which > 4) return KVQ_ERR_ATTR;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const unsigned long long zero = 0ull;
+    unsigned long long h = 0ull;
+    if (cudaMemcpyToSymbolAsync(g_selftest_count, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    if (which == 4) selftest_fmax_kernel<<<128, 256, 0, s>>>();
+    else selftest_div_kernel<<<65536, 256, 0, s>>>(which);
+    if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+    if (cudaMemcpyFromSymbolAsync(&h, g_selftest_count, sizeof(h), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return KVQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return KVQ_ERR_CUDA;
+    *result = h;
+    return KVQ_OK;
+}
 
 int32_t kvq_version(void) { return 100; }
 
@@ -267,9 +333,36 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
     a.x_scale = x_scale;
     a.x_vec = (reinterpret_cast<uintptr_t>(x->data) % 16 == 0) && ((rs * 2) % 16 == 0);
 
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (a.x_vec) {
+        // pipelined kernel: rows arrive in shared memory by bulk copy
+        const int64_t row_bytes = 2 * d;
+        a.R = row_bytes <= 2048 ? 32 : (int32_t)(32768 / row_bytes > 1 ? 32768 / row_bytes : 1);
+        a.stages = 3;
+        a.inv_nseg = 1.0f / (float)a.nseg;
+        const size_t smem = ct_header_bytes(a.stages, a.R) + (size_t)a.stages * a.R * row_bytes;
+        const int64_t tiles = (T + a.R - 1) / a.R;
+#define KVQ_LAUNCH_CT(M, GG)                                                                   \
+    do {                                                                                       \
+        auto k = compress_tma_kernel<M, GG>;                                                   \
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
+            return KVQ_ERR_CUDA;                                                               \
+        int occ = 0;                                                                           \
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, CT_THREADS, smem) != cudaSuccess || occ < 1) \
+            occ = 1;                                                                           \
+        const int64_t cap = (int64_t)sm_count() * occ;                                         \
+        k<<<(unsigned)(tiles < cap ? tiles : cap), CT_THREADS, smem, s>>>(a);                 \
+    } while (0)
+        if (quant_mode == 0) KVQ_LAUNCH_CT(0, 64);
+        else if (quant_mode == 1) KVQ_LAUNCH_CT(1, 64);
+        else if (G == 16) KVQ_LAUNCH_CT(2, 16);
+        else if (G == 32) KVQ_LAUNCH_CT(2, 32);
+        else KVQ_LAUNCH_CT(2, 64);
+#undef KVQ_LAUNCH_CT
+        return launched();
+    }
     const int64_t tiles = (T + CE_TILE - 1) / CE_TILE;
     const int64_t need = (tiles + (CE_THREADS / 32) - 1) / (CE_THREADS / 32);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 #define KVQ_LAUNCH_CE(M, GG)                                                                   \
     do {                                                                                       \
         auto k = compress_epilog_kernel<M, GG>;                                                \

@@ -122,6 +122,51 @@ __device__ __forceinline__ float e8m0_reciprocal(uint32_t b) {
     return k >= -126 ? __uint_as_float((uint32_t)(k + 127) << 23) : __uint_as_float(0x00400000u);
 }
 
+// ---------------------------------------------------------------------------
+// Division by a per-group scale.  With r = RN(1/s) (one IEEE reciprocal per
+// group), Markstein's correction -- P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1),
+// 1990 -- refines q0 = RN(a r): the residual a - s q0 is exact under a fused
+// multiply-add, and q = RN(q0 + residual * r).  The two-step variant repeats
+// the correction once.  The quotient of a positive scale carries the sign of
+// a, which also fixes the sign of a zero result.  Used only for scales with
+// 2^-100 <= s < 2^101 and |a / s| <= 512; kvq_selftest compares both variants
+// with IEEE division for every bf16 numerator and bf16 scale of that domain,
+// and the constant-divisor form for every bf16 amax over 448, 57344 and 6.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool scale_in_fast_range(float s) {
+    const uint32_t e = (__float_as_uint(s) >> 23) & 0xffu;
+    return e >= 27u && e <= 227u;
+}
+
+__device__ __forceinline__ float with_sign_of(float q, float a) {
+    return __uint_as_float(__float_as_uint(q) | (__float_as_uint(a) & 0x80000000u));
+}
+
+__device__ __forceinline__ float div_scale1(float a, float s, float r) {
+    const float q0 = __fmul_rn(a, r);
+    const float rem = __fmaf_rn(-q0, s, a);
+    return with_sign_of(__fmaf_rn(rem, r, q0), a);
+}
+
+__device__ __forceinline__ float div_scale2(float a, float s, float r) {
+    const float q0 = __fmul_rn(a, r);
+    const float rem0 = __fmaf_rn(-q0, s, a);
+    const float q1 = __fmaf_rn(rem0, r, q0);
+    const float rem1 = __fmaf_rn(-q1, s, a);
+    return with_sign_of(__fmaf_rn(rem1, r, q1), a);
+}
+
+// amax / c for the format maxima c = 448, 57344, 6 (amax >= 0, a bf16 value):
+// the one-step form with the constant RN(1/c).
+__device__ __forceinline__ float div_by_fmax(float amax, float c) {
+    // RN(1/448) = 0x3b124925, RN(1/6) = 0x3e2aaaab, RN(1/57344) = 0x37924925
+    const float r = __uint_as_float(c == 448.0f ? 0x3b124925u : (c == 6.0f ? 0x3e2aaaabu : 0x37924925u));
+    const float q0 = __fmul_rn(amax, r);
+    const float rem = __fmaf_rn(-q0, c, amax);
+    return __fmaf_rn(rem, r, q0);
+}
+
 // Static int8: round half to even, saturate to [-128, 127]; NaN -> 0.
 __device__ __forceinline__ int32_t int8_rne_sat(float v) {
     int r;
