@@ -38,12 +38,10 @@ struct CompressArgs {
     float inv_nseg;         // 1 / nseg in binary32
 };
 
-// Division of a code's numerator by the group scale: the one- or two-step
-// Markstein form (kvq_device.cuh); kvq_selftest confirms the choice is exact
-// against IEEE division on its whole domain.
-#ifndef KVQ_SCALE_DIV
-#define KVQ_SCALE_DIV div_scale2
-#endif
+// Division of a code's numerator by the group scale: the one-step Markstein
+// form (kvq_device.cuh), whose E4M3 / E2M1 codes kvq_selftest shows equal to
+// those of IEEE division on its whole domain.
+#define KVQ_SCALE_DIV div_scale1
 
 constexpr int CE_TILE = 8;
 constexpr int CE_UNROLL = 3;
@@ -95,7 +93,7 @@ __device__ __forceinline__ void ce_segment(const CompressArgs& a, const uint4& v
     if (MODE == 0) {
         if (!rope) {
             // scale_g = amax / FP8_MAX, stored as bf16; codes use the stored scale
-            const uint32_t sb = to_bf16_bits(__fdiv_rn(amax, 448.0f));
+            const uint32_t sb = to_bf16_bits(div_by_fmax(amax, 448.0f));
             const float sf = __uint_as_float(sb << 16);
             uint2 codes = make_uint2(0u, 0u);
             if (sf != 0.0f) {
@@ -112,7 +110,7 @@ __device__ __forceinline__ void ce_segment(const CompressArgs& a, const uint4& v
     } else if (MODE == 1) {
         if (!rope) {
             // E8M0 scale: amax / FP8_MAX rounded up to a power of two
-            const uint32_t b = e8m0_ceil(__fdiv_rn(amax, 448.0f));
+            const uint32_t b = e8m0_ceil(div_by_fmax(amax, 448.0f));
             const float mul = e8m0_reciprocal(b);
             float q[8];
 #pragma unroll
@@ -125,7 +123,7 @@ __device__ __forceinline__ void ce_segment(const CompressArgs& a, const uint4& v
     } else {
         if (!rope) {
             // FP4 E2M1 per group of G, bf16 scale = amax / 6
-            const uint32_t sb = to_bf16_bits(__fdiv_rn(amax, 6.0f));
+            const uint32_t sb = to_bf16_bits(div_by_fmax(amax, 6.0f));
             const float sf = __uint_as_float(sb << 16);
             uint32_t codes = 0u;
             if (sf != 0.0f) {

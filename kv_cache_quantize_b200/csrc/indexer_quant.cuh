@@ -59,7 +59,7 @@ __device__ __forceinline__ void ix_mx_chunk(const IndexerArgs& a, const uint4& v
     if (nvalid <= 0) return;
     const float amax = a.x_f16 ? __half2float(__ushort_as_half((unsigned short)m)) : __uint_as_float(m << 16);
     const float fmax = MODE == 3 ? 6.0f : (a.e5m2 ? 57344.0f : 448.0f);
-    const uint32_t b = e8m0_ceil(__fdiv_rn(amax, fmax));
+    const uint32_t b = e8m0_ceil(div_by_fmax(amax, fmax));
     const float mul = e8m0_reciprocal(b);
     float f[8], q[8];
     ix_widen(a, v, f);
@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(IX_THREADS) indexer_quant_kernel(const Indexer
                     if (!live[u]) continue;
                     const float amax = a.x_f16 ? __half2float(__ushort_as_half((unsigned short)m))
                                                : __uint_as_float(m << 16);
-                    const float scale = __fdiv_rn(amax, a.e5m2 ? 57344.0f : 448.0f);
+                    const float scale = div_by_fmax(amax, a.e5m2 ? 57344.0f : 448.0f);
                     uint8_t* crow = slot_row(a.cache, sl[u]);
                     for (int cb = 0; cb < nblocks; ++cb) {
                         const int c = cb * TEAM + tl;

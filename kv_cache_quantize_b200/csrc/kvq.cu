@@ -199,6 +199,7 @@ __global__ void selftest_div_kernel(int32_t which) {
         bool diff;
         switch (which) {
             case 0: diff = __float_as_uint(q1) != __float_as_uint(ref); break;
+            case 5: diff = fabsf(ref) >= 1.17549435e-38f && __float_as_uint(q1) != __float_as_uint(ref); break;
             case 1: diff = __float_as_uint(div_scale2(a, s, r)) != __float_as_uint(ref); break;
             case 2: diff = e4m3x2(q1, 0.0f) != e4m3x2(ref, 0.0f); break;
             default: {
@@ -212,11 +213,14 @@ __global__ void selftest_div_kernel(int32_t which) {
     if (bad) atomicAdd(&g_selftest_count, bad);
 }
 
-// every positive finite bf16 amax over the three format maxima
+// every positive finite bf16 amax (bits < 0x7f80) and every positive finite
+// f16 amax (bits < 0x7c00) over the three format maxima
 __global__ void selftest_fmax_kernel() {
-    const uint32_t bits = blockIdx.x * blockDim.x + threadIdx.x;   // 0 .. 32767
-    if (bits >= 0x7f80u) return;
-    const float a = __uint_as_float(bits << 16);
+    const uint32_t i = blockIdx.x * blockDim.x + threadIdx.x;       // 0 .. 65535
+    const uint32_t bits = i & 0x7fffu;
+    const bool f16 = i >= 0x8000u;
+    if (bits >= (f16 ? 0x7c00u : 0x7f80u)) return;
+    const float a = f16 ? __half2float(__ushort_as_half((unsigned short)bits)) : __uint_as_float(bits << 16);
     unsigned long long bad = 0;
     const float cs[3] = {448.0f, 57344.0f, 6.0f};
 #pragma unroll
@@ -231,13 +235,13 @@ extern "C" {
 
 kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream) {
     if (!result) return KVQ_ERR_NULL;
-    if (which < 0 || which > 4) return KVQ_ERR_ATTR;
+    if (which < 0 || which > 5) return KVQ_ERR_ATTR;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const unsigned long long zero = 0ull;
     unsigned long long h = 0ull;
     if (cudaMemcpyToSymbolAsync(g_selftest_count, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
         return KVQ_ERR_CUDA;
-    if (which == 4) selftest_fmax_kernel<<<128, 256, 0, s>>>();
+    if (which == 4) selftest_fmax_kernel<<<256, 256, 0, s>>>();
     else selftest_div_kernel<<<65536, 256, 0, s>>>(which);
     if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
     if (cudaMemcpyFromSymbolAsync(&h, g_selftest_count, sizeof(h), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
