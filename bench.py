@@ -255,6 +255,32 @@ def run_reference(args):
     return 0
 
 
+def run_profile_workload(args):
+    """Run one named workload a few times (for ncu captures of a single kernel)."""
+    import torch
+    import kv_cache_quantize_b200 as kvq
+    from kv_cache_quantize_b200 import workloads as W
+    case = W.CONFIGS[args.profile_workload]()
+    call, _, _ = W.build_call(case)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    times = []
+    for i in range(args.profile_reps):
+        flush.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call(stream)
+        e1.record(stream)
+        times.append((e0, e1))
+    torch.cuda.synchronize()
+    if kvq.get_error(stream) != 0:
+        raise RuntimeError("device fault bits set")
+    us = [1e3 * a.elapsed_time(b) for a, b in times]
+    print(f"{args.profile_workload}: {len(us)} launches, median {statistics.median(us):.1f} us, "
+          f"{algorithmic_bytes(case) / statistics.median(us) / 1e3:.0f} GB/s algorithmic")
+    return 0
+
+
 # ---------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
@@ -264,11 +290,17 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-per-config", action="store_true", help="skip the per-workload breakdown")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing for cpu_baseline")
+    ap.add_argument("--profile-workload", default=None,
+                    help="profiling mode: run only this named workload --profile-reps times (L2 flushed "
+                         "before each launch) and print its median launch time; no JSON line")
+    ap.add_argument("--profile-reps", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_workload:
+        return run_profile_workload(args)
 
     import numpy as np
     import torch

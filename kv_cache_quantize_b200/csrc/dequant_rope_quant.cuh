@@ -13,6 +13,7 @@
 #pragma once
 
 #include "kvq_device.cuh"
+#include "tma_pipe.cuh"
 
 namespace kvq {
 
@@ -40,6 +41,9 @@ struct DrqArgs {
     uint16_t* q_out;        // [B*S, Nq*D]
     uint16_t* k_out;        // [B*S, Nkv*D] or null
     uint16_t* v_out;
+    // pipelined kernel only
+    int32_t tps;            // tokens per shared-memory stage
+    int32_t stages;
 };
 
 constexpr int DQ_WARPS = 8;
@@ -158,6 +162,25 @@ __device__ __forceinline__ void dq_head(const DrqArgs& a, int64_t t, int hd, flo
     }
 }
 
+// Destination row of token t: >= 0 a cache slot, -1 skip, -2 bad index.
+__device__ __forceinline__ int64_t dq_slot(const DrqArgs& a, int64_t t) {
+    if (a.cache_mode == 1) {
+        const int64_t slot = load_slot(a.indices, a.indices_i64, t);
+        if (slot != -1 && !slot_ok(slot, a.kc.num_slots)) return -2;
+        return slot;
+    }
+    const int64_t b = t / a.S, s = t - b * a.S;
+    const int64_t start = load_slot(a.indices, a.indices_i64, b);
+    const int64_t c1 = a.kc.block_size;
+    if (start == -1) return -1;
+    if (start < 0 || start + s >= c1 || b * c1 >= a.kc.num_slots) return -2;
+    return b * c1 + start + s;
+}
+
+__device__ __forceinline__ float half_bits_to_f32(uint32_t h, bool f16) {
+    return f16 ? __half2float(__ushort_as_half((unsigned short)h)) : __uint_as_float(h << 16);
+}
+
 template <int E>
 __global__ void __launch_bounds__(DQ_WARPS * 32) dequant_rope_quant_kernel(const DrqArgs a) {
     const int lane = threadIdx.x & 31;
@@ -171,18 +194,7 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) dequant_rope_quant_kernel(const
 
     for (int64_t t = blockIdx.x; t < ntok; t += gridDim.x) {
         // destination row of this token (or -1 skip / -2 fault)
-        int64_t slot;
-        if (a.cache_mode == 1) {
-            slot = load_slot(a.indices, a.indices_i64, t);
-            if (slot != -1 && !slot_ok(slot, a.kc.num_slots)) slot = -2;
-        } else {
-            const int64_t b = t / a.S, s = t - b * a.S;
-            const int64_t start = load_slot(a.indices, a.indices_i64, b);
-            const int64_t c1 = a.kc.block_size;
-            if (start == -1) slot = -1;
-            else if (start < 0 || start + s >= c1 || b * c1 >= a.kc.num_slots) slot = -2;
-            else slot = b * c1 + start + s;
-        }
+        const int64_t slot = dq_slot(a, t);
         if (slot == -2 && threadIdx.x == 0) raise_fault(FAULT_SLOT_RANGE);
 
         float cs[E], sn[E];
@@ -211,6 +223,138 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) dequant_rope_quant_kernel(const
                 dq_head<E>(a, t, hd, u[i], cs, sn, act, slot, pos, second_half);
             }
         }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Pipelined kernel (16-byte aligned x, cos and sin).  CTA = DQ_WARPS consumer
+// warps + 1 producer warp.  A stage holds TPS consecutive tokens: their x rows,
+// cos rows and sin rows arrive by three bulk copies (each a contiguous span),
+// and the producer stores their destination slots next to them.  Consumers
+// keep the head mapping of the direct kernel and read x, cos and sin from
+// shared memory.
+// ---------------------------------------------------------------------------
+constexpr int DT_THREADS = (DQ_WARPS + 1) * 32;
+
+__host__ __device__ inline uint32_t dt_header_bytes(int stages, int tps) {
+    return ((uint32_t)(16 * stages + 8 * stages * tps) + 127u) & ~127u;
+}
+
+__host__ __device__ inline uint32_t dt_stage_bytes(int tps, int64_t H, int x_bytes, int D) {
+    return (uint32_t)(((tps * H * x_bytes + 127) & ~127) + 2 * ((tps * D * 2 + 127) & ~127));
+}
+
+template <int E>
+__global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(const DrqArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int S = a.stages, TPS = a.tps, D = a.D;
+    const int xb = a.x_kind == 0 ? 4 : 2;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + S;
+    int64_t* slots = reinterpret_cast<int64_t*>(empty + S);
+    uint8_t* stages = smem + dt_header_bytes(S, TPS);
+    const uint32_t x_span = (uint32_t)((TPS * a.H * xb + 127) & ~127);
+    const uint32_t cs_span = (uint32_t)((TPS * D * 2 + 127) & ~127);
+    const uint32_t stage_bytes = x_span + 2 * cs_span;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t ntok = a.B * a.S;
+    const int64_t ntiles = (ntok + TPS - 1) / TPS;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < S; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], DQ_WARPS);
+        }
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    if (warp == DQ_WARPS) {
+        // ---------------- producer ----------------
+        int it = 0;
+        for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+            const int st = it % S;
+            const uint32_t round = (uint32_t)(it / S);
+            if (!__all_sync(FULL_MASK, mbar_wait(&empty[st], (round & 1u) ^ 1u))) break;
+            const int64_t t0 = tile * TPS;
+            const int toks = (int)(ntok - t0 < TPS ? ntok - t0 : TPS);
+            for (int k = lane; k < toks; k += 32) {
+                int64_t slot = dq_slot(a, t0 + k);
+                if (slot == -2) {
+                    raise_fault(FAULT_SLOT_RANGE);
+                    slot = -1;
+                }
+                slots[st * TPS + k] = slot;
+            }
+            __syncwarp();
+            if (lane == 0) {
+                uint8_t* base = stages + (size_t)st * stage_bytes;
+                const uint32_t xbytes = (uint32_t)(toks * a.H * xb), cbytes = (uint32_t)(toks * D * 2);
+                mbar_arrive_expect_tx(&full[st], xbytes + 2 * cbytes);
+                bulk_copy_g2s(base, reinterpret_cast<const uint8_t*>(a.x) + (size_t)t0 * a.H * xb, xbytes, &full[st]);
+                bulk_copy_g2s(base + x_span, a.cos + (size_t)t0 * D, cbytes, &full[st]);
+                bulk_copy_g2s(base + x_span + cs_span, a.sin + (size_t)t0 * D, cbytes, &full[st]);
+            }
+            __syncwarp();
+        }
+        if (lane == 0)
+            for (int k = it > S ? it - S : 0; k < it; ++k) mbar_wait(&full[k % S], (uint32_t)(k / S) & 1u);
+        return;
+    }
+
+    // ---------------- consumers ----------------
+    const int NH = a.Nq + 2 * a.Nkv;
+    const int pos = lane * E;
+    const bool second_half = lane >= 16;
+    const bool f16 = a.cos_f16 != 0;
+    const int nh = (NH - warp + DQ_WARPS - 1) / DQ_WARPS;
+    int it = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        const int st = it % S;
+        const uint32_t round = (uint32_t)(it / S);
+        if (!__all_sync(FULL_MASK, mbar_wait(&full[st], round & 1u))) break;
+        const int64_t t0 = tile * TPS;
+        const int toks = (int)(ntok - t0 < TPS ? ntok - t0 : TPS);
+        const uint8_t* base = stages + (size_t)st * stage_bytes;
+        for (int k = 0; k < toks; ++k) {
+            const int64_t t = t0 + k;
+            const int64_t slot = slots[st * TPS + k];
+            const uint16_t* cw = reinterpret_cast<const uint16_t*>(base + x_span) + k * D + pos;
+            const uint16_t* sw = reinterpret_cast<const uint16_t*>(base + x_span + cs_span) + k * D + pos;
+            float cs[E], sn[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                cs[e] = half_bits_to_f32(cw[e], f16);
+                sn[e] = half_bits_to_f32(sw[e], f16);
+            }
+            const float act = (a.x_kind == 0 && a.activation_scale) ? a.activation_scale[t] : 1.0f;
+            for (int i = 0; i < nh; ++i) {
+                const int hd = warp + i * DQ_WARPS;
+                float u[E];
+                const int64_t e0 = (int64_t)k * a.H + (int64_t)hd * D + pos;
+                if (a.x_kind == 0) {
+                    const int32_t* xi = reinterpret_cast<const int32_t*>(base) + e0;
+                    if (E % 4 == 0) {
+#pragma unroll
+                        for (int e = 0; e < E; e += 4) {
+                            const int4 w = *reinterpret_cast<const int4*>(xi + e);
+                            u[e] = __int2float_rn(w.x); u[e + 1] = __int2float_rn(w.y);
+                            u[e + 2] = __int2float_rn(w.z); u[e + 3] = __int2float_rn(w.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < E; ++e) u[e] = __int2float_rn(xi[e]);
+                    }
+                } else {
+                    const uint16_t* xh = reinterpret_cast<const uint16_t*>(base) + e0;
+#pragma unroll
+                    for (int e = 0; e < E; ++e) u[e] = half_bits_to_f32(xh[e], a.x_kind == 2);
+                }
+                dq_head<E>(a, t, hd, u, cs, sn, act, slot, pos, second_half);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
     }
 }
 

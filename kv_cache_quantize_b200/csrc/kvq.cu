@@ -440,11 +440,12 @@ kvq_status kvq_indexer_quant_cache(const kvq_tensor* x, kvq_tensor* cache, kvq_t
     if (a.nchunks <= 4) team = 4;
     else if (a.nchunks <= 8) team = 8;
     else if (a.nchunks <= 16) team = 16;
-    const int64_t tiles = (T + 31) / 32;
-    const int64_t need = (tiles + (IX_THREADS / 32) - 1) / (IX_THREADS / 32);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 #define KVQ_LAUNCH_IX(M, TM)                                                                   \
     do {                                                                                       \
+        constexpr int rps = 32 / TM, u = (32 / rps) < 8 ? (32 / rps) : 8;                      \
+        const int64_t tiles = (T + rps * u - 1) / (rps * u);                                   \
+        const int64_t need = (tiles + (IX_THREADS / 32) - 1) / (IX_THREADS / 32);              \
         auto k = indexer_quant_kernel<M, TM>;                                                  \
         k<<<(unsigned)persistent_grid(k, IX_THREADS, need), IX_THREADS, 0, s>>>(a);             \
     } while (0)
@@ -680,6 +681,8 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
     a.x = x->data;
     a.x_kind = dq ? 0 : (x->dtype == KVQ_BF16 ? 1 : 2);
     a.x_vec = reinterpret_cast<uintptr_t>(x->data) % 16 == 0;
+    a.tps = 0;
+    a.stages = 0;
     a.B = B;
     a.S = S;
     a.H = H;
@@ -707,6 +710,40 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
     a.v_out = vop;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int64_t need = B * S;
+    const int xb = dq ? 4 : 2;
+    const bool aligned = reinterpret_cast<uintptr_t>(x->data) % 16 == 0 &&
+                         reinterpret_cast<uintptr_t>(cos->data) % 16 == 0 &&
+                         reinterpret_cast<uintptr_t>(sin->data) % 16 == 0 && (D * 2) % 16 == 0;
+    if (aligned) {
+        // pipelined kernel: token rows, cos and sin arrive in shared memory by bulk copy
+        a.tps = (int32_t)(H * xb <= 8192 ? 2 : 1);
+        a.stages = 4;
+        const size_t smem = dt_header_bytes(a.stages, a.tps) + (size_t)a.stages * dt_stage_bytes(a.tps, H, xb, (int)D);
+        const int64_t tiles = (need + a.tps - 1) / a.tps;
+#define KVQ_LAUNCH_DT(E)                                                                       \
+    do {                                                                                       \
+        auto k = dequant_rope_quant_tma_kernel<E>;                                             \
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
+            return KVQ_ERR_CUDA;                                                               \
+        int occ = 0;                                                                           \
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, DT_THREADS, smem) != cudaSuccess || occ < 1) \
+            occ = 1;                                                                           \
+        const int64_t cap = (int64_t)sm_count() * occ;                                         \
+        k<<<(unsigned)(tiles < cap ? tiles : cap), DT_THREADS, smem, s>>>(a);                 \
+    } while (0)
+        switch (D / 32) {
+            case 1: KVQ_LAUNCH_DT(1); break;
+            case 2: KVQ_LAUNCH_DT(2); break;
+            case 3: KVQ_LAUNCH_DT(3); break;
+            case 4: KVQ_LAUNCH_DT(4); break;
+            case 5: KVQ_LAUNCH_DT(5); break;
+            case 6: KVQ_LAUNCH_DT(6); break;
+            case 7: KVQ_LAUNCH_DT(7); break;
+            default: KVQ_LAUNCH_DT(8); break;
+        }
+#undef KVQ_LAUNCH_DT
+        return launched();
+    }
 #define KVQ_LAUNCH_DQ(E)                                                                       \
     do {                                                                                       \
         auto k = dequant_rope_quant_kernel<E>;                                                 \
