@@ -33,9 +33,9 @@ struct CompressArgs {
     float x_scale;          // mode 2 rope multiplier
     int32_t x_vec;          // every row chunk is 16-byte aligned
     // pipelined kernel only
-    int32_t R;              // rows per shared-memory stage (<= 32)
     int32_t stages;         // ring depth
-    float inv_nseg;         // 1 / nseg in binary32
+    int32_t ncw;            // consumer warps
+    int32_t rows_aligned;   // every cache row starts on a 16-byte boundary
 };
 
 // Division of a code's numerator by the group scale: the one-step Markstein
@@ -192,51 +192,211 @@ __global__ void __launch_bounds__(CE_THREADS) compress_epilog_kernel(const Compr
 }
 
 // ---------------------------------------------------------------------------
-// Pipelined kernel (16-byte aligned rows).  CTA = CT_CONSUMER_WARPS consumer
-// warps + 1 producer warp.  The producer walks the CTA's tiles of R rows:
-// lanes load the R slots, turn valid ones into destination row pointers (kept
-// in shared memory for the consumers) and issue one bulk copy per valid row
-// into the stage; skipped rows are never read.  Consumers take the tile's
-// segments four per warp (one per team), reading x from shared memory.
+// Pipelined kernel (16-byte aligned rows).  A stage holds a tile of 32 rows,
+// brought into shared memory by the producer warp with one bulk copy per
+// valid row (skipped rows are never read); their destination row pointers sit
+// next to the stage.  Consumer warp w owns the 64-value segment columns
+// j = w, w + NCW, ... of the tile and lane r owns row r, so every lane
+// quantises whole 64-value groups on its own (no shuffles) and the nope /
+// rope branch is uniform across a warp.  Shared-memory rows are padded by 16
+// bytes, which spreads the 32 lanes' 16-byte reads over all banks.
 // ---------------------------------------------------------------------------
-constexpr int CT_CONSUMER_WARPS = 8;
-constexpr int CT_THREADS = (CT_CONSUMER_WARPS + 1) * 32;
+constexpr int CT_ROWS = 32;
+constexpr int CT_MAX_CONSUMER_WARPS = 16;
+constexpr int CT_MAX_THREADS = (CT_MAX_CONSUMER_WARPS + 1) * 32;
 
-__host__ __device__ inline uint32_t ct_header_bytes(int stages, int R) {
-    return ((uint32_t)(16 * stages + 8 * stages * R) + 127u) & ~127u;
+__host__ __device__ inline uint32_t ct_header_bytes(int stages) {
+    return ((uint32_t)(16 * stages + 8 * stages * CT_ROWS) + 127u) & ~127u;
+}
+
+__host__ __device__ inline uint32_t ct_pitch(int nseg) { return (uint32_t)nseg * 128u + 16u; }
+
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+
+// |x| maximum of the 64 bf16 values of one segment (as bits)
+__device__ __forceinline__ uint32_t seg_absmax_bits(const uint8_t* seg, int nchunks) {
+    uint32_t m2 = 0u;
+    for (int k = 0; k < nchunks; ++k) {
+        const uint4 v = lds128(seg + 16 * k);
+        const uint32_t msk = 0x7fff7fffu;
+        m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(v.x & msk, v.y & msk), __vmaxu2(v.z & msk, v.w & msk)));
+    }
+    return max(m2 & 0xffffu, m2 >> 16);
 }
 
 template <int MODE, int G>
-__global__ void __launch_bounds__(CT_THREADS) compress_tma_kernel(const CompressArgs a) {
+__device__ __forceinline__ void ct_nope_segment(const CompressArgs& a, const uint8_t* seg, uint8_t* row, int j,
+                                                bool aligned) {
+    if (MODE == 0 || MODE == 1) {
+        const float amax = __uint_as_float(seg_absmax_bits(seg, 8) << 16);
+        float sf, r = 0.0f;
+        bool fast = true;
+        uint32_t scale_bits;
+        if (MODE == 0) {
+            scale_bits = to_bf16_bits(div_by_fmax(amax, 448.0f));
+            sf = __uint_as_float(scale_bits << 16);
+            fast = scale_in_fast_range(sf);
+            if (fast) r = __frcp_rn(sf);
+        } else {
+            scale_bits = e8m0_ceil(div_by_fmax(amax, 448.0f));
+            sf = e8m0_reciprocal(scale_bits);      // multiplier 2^(127-b)
+        }
+#pragma unroll 2
+        for (int k = 0; k < 8; k += 2) {
+            uint32_t w[4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float f[8], q[8];
+                widen8<false>(lds128(seg + 16 * (k + h)), f);
+                if (MODE == 1) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(f[i], sf);
+                } else if (sf == 0.0f) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) q[i] = 0.0f;
+                } else if (fast) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) q[i] = KVQ_SCALE_DIV(f[i], sf, r);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], sf);
+                }
+                const uint2 c = fp8x8<false>(q);
+                w[2 * h] = c.x;
+                w[2 * h + 1] = c.y;
+            }
+            uint8_t* dst = row + j * 64 + k * 8;
+            if (aligned) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+            else st_b128(dst, make_uint4(w[0], w[1], w[2], w[3]));
+        }
+        if (MODE == 0) st_b16(row + a.n + 128 + 2 * j, scale_bits);
+        else st_b8(row + a.n + 128 + j, scale_bits);
+    } else {
+        constexpr int GC = G / 8;                   // chunks per group
+        uint32_t sbits[64 / G];
+#pragma unroll
+        for (int g = 0; g < 64 / G; ++g) {
+            const uint8_t* gseg = seg + g * G * 2;
+            const float amax = __uint_as_float(seg_absmax_bits(gseg, GC) << 16);
+            sbits[g] = to_bf16_bits(div_by_fmax(amax, 6.0f));
+            const float sf = __uint_as_float(sbits[g] << 16);
+            const bool fast = scale_in_fast_range(sf);
+            const float r = fast ? __frcp_rn(sf) : 0.0f;
+            uint32_t w[GC];
+#pragma unroll
+            for (int k = 0; k < GC; ++k) {
+                float f[8], q[8];
+                widen8<false>(lds128(gseg + 16 * k), f);
+                if (sf == 0.0f) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) q[i] = 0.0f;
+                } else if (fast) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) q[i] = KVQ_SCALE_DIV(f[i], sf, r);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], sf);
+                }
+                w[k] = e2m1x8(q);
+            }
+            uint8_t* dst = row + j * 32 + g * (G / 2);
+            if (GC == 8) {
+                if (aligned) {
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4*>(dst + 16) = make_uint4(w[4 % GC], w[5 % GC], w[6 % GC], w[7 % GC]);
+                } else {
+                    st_b128(dst, make_uint4(w[0], w[1], w[2], w[3]));
+                    st_b128(dst + 16, make_uint4(w[4 % GC], w[5 % GC], w[6 % GC], w[7 % GC]));
+                }
+            } else if (GC == 4) {
+                if (aligned) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1 % GC], w[2 % GC], w[3 % GC]);
+                else st_b128(dst, make_uint4(w[0], w[1 % GC], w[2 % GC], w[3 % GC]));
+            } else {
+                st_b64(dst, make_uint2(w[0], w[1 % GC]));
+            }
+        }
+        // the 64/G bf16 scales of this segment are consecutive
+        uint8_t* sdst = row + a.n / 2 + 64 + 2 * (j * (64 / G));
+        if (G == 64) st_b16(sdst, sbits[0]);
+        else if (G == 32) st_b32(sdst, sbits[0] | (sbits[1 % (64 / G)] << 16));
+        else st_b64(sdst, make_uint2(sbits[0] | (sbits[1 % (64 / G)] << 16), sbits[2 % (64 / G)] | (sbits[3 % (64 / G)] << 16)));
+    }
+}
+
+template <int MODE>
+__device__ __forceinline__ void ct_rope_segment(const CompressArgs& a, const uint8_t* seg, uint8_t* row,
+                                                bool aligned) {
+    if (MODE == 2) {
+        // static rope: FP8 E4M3 of x * xScale, 64 bytes
+#pragma unroll 2
+        for (int k = 0; k < 8; k += 2) {
+            uint32_t w[4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float f[8], q[8];
+                widen8<false>(lds128(seg + 16 * (k + h)), f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(f[i], a.x_scale);
+                const uint2 c = fp8x8<false>(q);
+                w[2 * h] = c.x;
+                w[2 * h + 1] = c.y;
+            }
+            uint8_t* dst = row + a.n / 2 + k * 8;
+            if (aligned) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+            else st_b128(dst, make_uint4(w[0], w[1], w[2], w[3]));
+        }
+    } else {
+        // rope kept as bf16: copy 128 bytes
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            uint8_t* dst = row + a.n + 16 * k;
+            if (aligned) *reinterpret_cast<uint4*>(dst) = lds128(seg + 16 * k);
+            else st_b128(dst, lds128(seg + 16 * k));
+        }
+    }
+    // zero padding [concatCol, kvCacheCol): bytes up to a 16-byte boundary of
+    // the (aligned) row, then 16-byte stores, then the tail
+    int p = a.concat;
+    if (aligned) {
+        for (; p < a.col && (p & 15) != 0; ++p) row[p] = 0;
+        for (; p + 16 <= a.col; p += 16) *reinterpret_cast<uint4*>(row + p) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    for (; p < a.col; ++p) row[p] = 0;
+}
+
+template <int MODE, int G>
+__global__ void __launch_bounds__(CT_MAX_THREADS) compress_tma_kernel(const CompressArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
-    const int S = a.stages, R = a.R;
+    const int S = a.stages;
+    const int NCW = a.ncw;                         // consumer warps
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + S;
     uint8_t** rowptr = reinterpret_cast<uint8_t**>(empty + S);
-    uint8_t* xs = smem + ct_header_bytes(S, R);
+    uint8_t* xs = smem + ct_header_bytes(S);
     const uint32_t row_bytes = (uint32_t)a.nseg * 128u;
-    const uint32_t stage_bytes = (uint32_t)R * row_bytes;
+    const uint32_t pitch = ct_pitch(a.nseg);
+    const uint32_t stage_bytes = CT_ROWS * pitch;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t ntiles = (a.T + R - 1) / R;
+    const int64_t ntiles = (a.T + CT_ROWS - 1) / CT_ROWS;
 
     if (threadIdx.x == 0) {
         for (int st = 0; st < S; ++st) {
             mbar_init(&full[st], 1);
-            mbar_init(&empty[st], CT_CONSUMER_WARPS);
+            mbar_init(&empty[st], NCW);
         }
         mbar_init_fence();
     }
     __syncthreads();
 
-    if (warp == CT_CONSUMER_WARPS) {
+    if (warp == NCW) {
         // ---------------- producer ----------------
         int it = 0;
         for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
             const int st = it % S;
             const uint32_t round = (uint32_t)(it / S);
             if (!__all_sync(FULL_MASK, mbar_wait(&empty[st], (round & 1u) ^ 1u))) break;
-            const int64_t row0 = tile * R;
-            const int rows = (int)(a.T - row0 < R ? a.T - row0 : R);
+            const int64_t row0 = tile * CT_ROWS;
+            const int rows = (int)(a.T - row0 < CT_ROWS ? a.T - row0 : CT_ROWS);
             uint8_t* p = nullptr;
             if (lane < rows) {
                 const int64_t slot = load_slot(a.slots, a.slots_i64, row0 + lane);
@@ -245,13 +405,13 @@ __global__ void __launch_bounds__(CT_THREADS) compress_tma_kernel(const Compress
                     else raise_fault(FAULT_SLOT_RANGE);
                 }
             }
-            if (lane < R) rowptr[st * R + lane] = p;
+            rowptr[st * CT_ROWS + lane] = p;
             const unsigned valid = __ballot_sync(FULL_MASK, p != nullptr);
             __syncwarp();
             if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)__popc(valid) * row_bytes);
             __syncwarp();
             if (p != nullptr)
-                bulk_copy_g2s(xs + (size_t)st * stage_bytes + (size_t)lane * row_bytes,
+                bulk_copy_g2s(xs + (size_t)st * stage_bytes + (size_t)lane * pitch,
                               a.x + (row0 + lane) * a.x_row_stride, row_bytes, &full[st]);
         }
         // no copy may still be in flight when the CTA exits
@@ -260,28 +420,20 @@ __global__ void __launch_bounds__(CT_THREADS) compress_tma_kernel(const Compress
         return;
     }
 
-    // ---------------- consumers ----------------
-    const int team = lane >> 3, sub = lane & 7;
+    // ---------------- consumers: warp -> segment columns, lane -> row ----------------
+    const bool aligned = a.rows_aligned != 0;
     int it = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
         const int st = it % S;
         const uint32_t round = (uint32_t)(it / S);
         if (!__all_sync(FULL_MASK, mbar_wait(&full[st], round & 1u))) break;   // every lane acquires the stage
-        const int64_t row0 = tile * R;
-        const int rows = (int)(a.T - row0 < R ? a.T - row0 : R);
-        const int nsegs = rows * a.nseg;
-        const uint8_t* xst = xs + (size_t)st * stage_bytes;
-        for (int base = warp * 4; base < nsegs; base += CT_CONSUMER_WARPS * 4) {
-            const int seg = base + team;
-            const bool act = seg < nsegs;
-            // seg / nseg: (seg + 1/2) / nseg is never an integer and its binary32
-            // product with 1/nseg is within 2^-11 of it for seg < 2^12, nseg <= 128
-            const int r = act ? (int)(((float)seg + 0.5f) * a.inv_nseg) : 0;
-            const int j = seg - r * a.nseg;
-            uint8_t* row = act ? rowptr[st * R + r] : nullptr;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (row != nullptr) v = *reinterpret_cast<const uint4*>(xst + (size_t)r * row_bytes + j * 128 + sub * 16);
-            ce_segment<MODE, G>(a, v, row, j, sub);
+        uint8_t* row = rowptr[st * CT_ROWS + lane];
+        const uint8_t* xrow = xs + (size_t)st * stage_bytes + (size_t)lane * pitch;
+        if (row != nullptr) {
+            for (int j = warp; j < a.nseg; j += NCW) {
+                if (j < a.nseg - 1) ct_nope_segment<MODE, G>(a, xrow + j * 128, row, j, aligned);
+                else ct_rope_segment<MODE>(a, xrow + j * 128, row, aligned);
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[st]);

@@ -338,24 +338,32 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
     a.x_vec = (reinterpret_cast<uintptr_t>(x->data) % 16 == 0) && ((rs * 2) % 16 == 0);
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (a.x_vec) {
+    // pipelined kernel when x rows are 16-byte aligned and a ring of at least
+    // two 32-row stages fits in shared memory (d <= 1728); else the direct one
+    const size_t smem_limit = 227 * 1024;
+    auto ct_smem = [&](int stages) {
+        return ct_header_bytes(stages) + (size_t)stages * CT_ROWS * ct_pitch((int)(d / 64));
+    };
+    const int ct_stages = ct_smem(3) <= smem_limit ? 3 : (ct_smem(2) <= smem_limit ? 2 : 0);
+    if (a.x_vec && ct_stages > 0) {
         // pipelined kernel: rows arrive in shared memory by bulk copy
-        const int64_t row_bytes = 2 * d;
-        a.R = row_bytes <= 2048 ? 32 : (int32_t)(32768 / row_bytes > 1 ? 32768 / row_bytes : 1);
-        a.stages = 3;
-        a.inv_nseg = 1.0f / (float)a.nseg;
-        const size_t smem = ct_header_bytes(a.stages, a.R) + (size_t)a.stages * a.R * row_bytes;
-        const int64_t tiles = (T + a.R - 1) / a.R;
+        a.ncw = a.nseg < CT_MAX_CONSUMER_WARPS ? a.nseg : CT_MAX_CONSUMER_WARPS;
+        a.stages = ct_stages;
+        a.rows_aligned = (reinterpret_cast<uintptr_t>(cache->data) % 16 == 0) && rows.row_bytes % 16 == 0 &&
+                         rows.block_stride % 16 == 0;
+        const size_t smem = ct_smem(ct_stages);
+        const int64_t tiles = (T + CT_ROWS - 1) / CT_ROWS;
+        const int threads = (a.ncw + 1) * 32;
 #define KVQ_LAUNCH_CT(M, GG)                                                                   \
     do {                                                                                       \
         auto k = compress_tma_kernel<M, GG>;                                                   \
         if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
             return KVQ_ERR_CUDA;                                                               \
         int occ = 0;                                                                           \
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, CT_THREADS, smem) != cudaSuccess || occ < 1) \
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, threads, smem) != cudaSuccess || occ < 1) \
             occ = 1;                                                                           \
         const int64_t cap = (int64_t)sm_count() * occ;                                         \
-        k<<<(unsigned)(tiles < cap ? tiles : cap), CT_THREADS, smem, s>>>(a);                 \
+        k<<<(unsigned)(tiles < cap ? tiles : cap), threads, smem, s>>>(a);                    \
     } while (0)
         if (quant_mode == 0) KVQ_LAUNCH_CT(0, 64);
         else if (quant_mode == 1) KVQ_LAUNCH_CT(1, 64);
