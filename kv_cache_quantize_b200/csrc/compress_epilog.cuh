@@ -36,6 +36,9 @@ struct CompressArgs {
     int32_t stages;         // ring depth
     int32_t ncw;            // consumer warps
     int32_t rows_aligned;   // every cache row starts on a 16-byte boundary
+    int32_t bulk_out;       // packed rows leave by bulk copy (aligned rows, kvCacheCol % 16 == 0, one segment
+                            // per warp, and in modes 0/1 kvCacheCol <= 2(d-64) so the input rope lies past
+                            // the packed row in shared memory)
 };
 
 // Division of a code's numerator by the group scale: the one-step Markstein
@@ -224,65 +227,70 @@ __device__ __forceinline__ uint32_t seg_absmax_bits(const uint8_t* seg, int nchu
     return max(m2 & 0xffffu, m2 >> 16);
 }
 
+// Outputs of one 64-value segment held in registers: the code bytes packed
+// little-endian in 32-bit words, and the segment's scale bits (mode 0: one
+// bf16, mode 1: one E8M0 byte, mode 2: 64/G bf16 packed).  The bf16 rope of
+// modes 0/1 is copied, not computed, and never lands here.
+struct SegOut {
+    uint32_t w[16];
+    uint32_t sc[2];
+};
+
+// Number of output words of a computed segment.
 template <int MODE, int G>
-__device__ __forceinline__ void ct_nope_segment(const CompressArgs& a, const uint8_t* seg, uint8_t* row, int j,
-                                                bool aligned) {
+__device__ __forceinline__ int seg_words(bool rope) {
+    if (rope) return 16;
+    return MODE == 2 ? 8 : 16;
+}
+
+template <int MODE, int G>
+__device__ __forceinline__ void ct_compute_nope(const uint8_t* seg, SegOut& o) {
     if (MODE == 0 || MODE == 1) {
         const float amax = __uint_as_float(seg_absmax_bits(seg, 8) << 16);
         float sf, r = 0.0f;
         bool fast = true;
-        uint32_t scale_bits;
         if (MODE == 0) {
-            scale_bits = to_bf16_bits(div_by_fmax(amax, 448.0f));
-            sf = __uint_as_float(scale_bits << 16);
+            o.sc[0] = to_bf16_bits(div_by_fmax(amax, 448.0f));
+            sf = __uint_as_float(o.sc[0] << 16);
             fast = scale_in_fast_range(sf);
             if (fast) r = __frcp_rn(sf);
         } else {
-            scale_bits = e8m0_ceil(div_by_fmax(amax, 448.0f));
-            sf = e8m0_reciprocal(scale_bits);      // multiplier 2^(127-b)
+            o.sc[0] = e8m0_ceil(div_by_fmax(amax, 448.0f));
+            sf = e8m0_reciprocal(o.sc[0]);      // multiplier 2^(127-b)
         }
-#pragma unroll 2
-        for (int k = 0; k < 8; k += 2) {
-            uint32_t w[4];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float f[8], q[8];
-                widen8<false>(lds128(seg + 16 * (k + h)), f);
-                if (MODE == 1) {
+        for (int k = 0; k < 8; ++k) {
+            float f[8], q[8];
+            widen8<false>(lds128(seg + 16 * k), f);
+            if (MODE == 1) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(f[i], sf);
-                } else if (sf == 0.0f) {
+                for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(f[i], sf);
+            } else if (sf == 0.0f) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) q[i] = 0.0f;
-                } else if (fast) {
+                for (int i = 0; i < 8; ++i) q[i] = 0.0f;
+            } else if (fast) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) q[i] = KVQ_SCALE_DIV(f[i], sf, r);
-                } else {
+                for (int i = 0; i < 8; ++i) q[i] = KVQ_SCALE_DIV(f[i], sf, r);
+            } else {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], sf);
-                }
-                const uint2 c = fp8x8<false>(q);
-                w[2 * h] = c.x;
-                w[2 * h + 1] = c.y;
+                for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], sf);
             }
-            uint8_t* dst = row + j * 64 + k * 8;
-            if (aligned) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-            else st_b128(dst, make_uint4(w[0], w[1], w[2], w[3]));
+            const uint2 c = fp8x8<false>(q);
+            o.w[2 * k] = c.x;
+            o.w[2 * k + 1] = c.y;
         }
-        if (MODE == 0) st_b16(row + a.n + 128 + 2 * j, scale_bits);
-        else st_b8(row + a.n + 128 + j, scale_bits);
     } else {
         constexpr int GC = G / 8;                   // chunks per group
-        uint32_t sbits[64 / G];
+        constexpr int NG = 64 / G;                  // groups per segment
+        uint32_t sb[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int g = 0; g < 64 / G; ++g) {
+        for (int g = 0; g < NG; ++g) {
             const uint8_t* gseg = seg + g * G * 2;
             const float amax = __uint_as_float(seg_absmax_bits(gseg, GC) << 16);
-            sbits[g] = to_bf16_bits(div_by_fmax(amax, 6.0f));
-            const float sf = __uint_as_float(sbits[g] << 16);
+            sb[g] = to_bf16_bits(div_by_fmax(amax, 6.0f));
+            const float sf = __uint_as_float(sb[g] << 16);
             const bool fast = scale_in_fast_range(sf);
             const float r = fast ? __frcp_rn(sf) : 0.0f;
-            uint32_t w[GC];
 #pragma unroll
             for (int k = 0; k < GC; ++k) {
                 float f[8], q[8];
@@ -297,71 +305,93 @@ __device__ __forceinline__ void ct_nope_segment(const CompressArgs& a, const uin
 #pragma unroll
                     for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], sf);
                 }
-                w[k] = e2m1x8(q);
-            }
-            uint8_t* dst = row + j * 32 + g * (G / 2);
-            if (GC == 8) {
-                if (aligned) {
-                    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-                    *reinterpret_cast<uint4*>(dst + 16) = make_uint4(w[4 % GC], w[5 % GC], w[6 % GC], w[7 % GC]);
-                } else {
-                    st_b128(dst, make_uint4(w[0], w[1], w[2], w[3]));
-                    st_b128(dst + 16, make_uint4(w[4 % GC], w[5 % GC], w[6 % GC], w[7 % GC]));
-                }
-            } else if (GC == 4) {
-                if (aligned) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1 % GC], w[2 % GC], w[3 % GC]);
-                else st_b128(dst, make_uint4(w[0], w[1 % GC], w[2 % GC], w[3 % GC]));
-            } else {
-                st_b64(dst, make_uint2(w[0], w[1 % GC]));
+                o.w[g * GC + k] = e2m1x8(q);
             }
         }
-        // the 64/G bf16 scales of this segment are consecutive
-        uint8_t* sdst = row + a.n / 2 + 64 + 2 * (j * (64 / G));
-        if (G == 64) st_b16(sdst, sbits[0]);
-        else if (G == 32) st_b32(sdst, sbits[0] | (sbits[1 % (64 / G)] << 16));
-        else st_b64(sdst, make_uint2(sbits[0] | (sbits[1 % (64 / G)] << 16), sbits[2 % (64 / G)] | (sbits[3 % (64 / G)] << 16)));
+        o.sc[0] = sb[0] | (sb[1] << 16);
+        o.sc[1] = sb[2] | (sb[3] << 16);
     }
 }
 
-template <int MODE>
-__device__ __forceinline__ void ct_rope_segment(const CompressArgs& a, const uint8_t* seg, uint8_t* row,
-                                                bool aligned) {
-    if (MODE == 2) {
-        // static rope: FP8 E4M3 of x * xScale, 64 bytes
-#pragma unroll 2
-        for (int k = 0; k < 8; k += 2) {
-            uint32_t w[4];
+// Mode 2 rope: static FP8 E4M3 of x * xScale, 64 bytes.
+__device__ __forceinline__ void ct_compute_rope2(const CompressArgs& a, const uint8_t* seg, SegOut& o) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float f[8], q[8];
-                widen8<false>(lds128(seg + 16 * (k + h)), f);
+    for (int k = 0; k < 8; ++k) {
+        float f[8], q[8];
+        widen8<false>(lds128(seg + 16 * k), f);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(f[i], a.x_scale);
-                const uint2 c = fp8x8<false>(q);
-                w[2 * h] = c.x;
-                w[2 * h + 1] = c.y;
-            }
-            uint8_t* dst = row + a.n / 2 + k * 8;
-            if (aligned) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-            else st_b128(dst, make_uint4(w[0], w[1], w[2], w[3]));
+        for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(f[i], a.x_scale);
+        const uint2 c = fp8x8<false>(q);
+        o.w[2 * k] = c.x;
+        o.w[2 * k + 1] = c.y;
+    }
+}
+
+// Modes 0/1: the rope segment is kept as bf16 -- copy its 128 bytes.
+template <bool SMEM>
+__device__ __forceinline__ void ct_copy_rope(const uint8_t* src, uint8_t* dst, bool aligned) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        if (SMEM || aligned) *reinterpret_cast<uint4*>(dst + 16 * k) = lds128(src + 16 * k);
+        else st_b128(dst + 16 * k, lds128(src + 16 * k));
+    }
+}
+
+// Byte offsets inside the packed row.
+template <int MODE, int G>
+__device__ __forceinline__ int seg_code_offset(const CompressArgs& a, int j, bool rope) {
+    if (rope) return MODE == 2 ? a.n / 2 : a.n;
+    return MODE == 2 ? j * 32 : j * 64;
+}
+
+template <int MODE, int G>
+__device__ __forceinline__ int seg_scale_offset(const CompressArgs& a, int j) {
+    return MODE == 0 ? a.n + 128 + 2 * j : (MODE == 1 ? a.n + 128 + j : a.n / 2 + 64 + 2 * j * (64 / G));
+}
+
+// Write a segment's outputs to a packed row; SMEM: the row is this CTA's
+// shared memory (16-byte aligned), else global memory (aligned: the row
+// starts on a 16-byte boundary).
+// rope_src: the input rope segment (modes 0/1 copy it to the row).
+template <int MODE, int G, bool SMEM>
+__device__ __forceinline__ void ct_write(const CompressArgs& a, uint8_t* row, int j, bool rope, const SegOut& o,
+                                         const uint8_t* rope_src, bool aligned) {
+    uint8_t* dst = row + seg_code_offset<MODE, G>(a, j, rope);
+    if (rope && MODE != 2) {
+        ct_copy_rope<SMEM>(rope_src, dst, aligned);
+    } else {
+        const int nw = seg_words<MODE, G>(rope);
+#pragma unroll
+        for (int k = 0; k < 16; k += 4) {
+            if (k >= nw) break;
+            const uint4 v = make_uint4(o.w[k], o.w[k + 1], o.w[k + 2], o.w[k + 3]);
+            if (SMEM || aligned) *reinterpret_cast<uint4*>(dst + 4 * k) = v;
+            else st_b128(dst + 4 * k, v);
+        }
+    }
+    if (!rope) {
+        uint8_t* sdst = row + seg_scale_offset<MODE, G>(a, j);
+        if (MODE == 0 || (MODE == 2 && G == 64)) {
+            if (SMEM) *reinterpret_cast<uint16_t*>(sdst) = (uint16_t)o.sc[0];
+            else st_b16(sdst, o.sc[0]);
+        } else if (MODE == 1) {
+            *sdst = (uint8_t)o.sc[0];
+        } else if (G == 32) {
+            if (SMEM) *reinterpret_cast<uint32_t*>(sdst) = o.sc[0];
+            else st_b32(sdst, o.sc[0]);
+        } else {
+            if (SMEM) *reinterpret_cast<uint2*>(sdst) = make_uint2(o.sc[0], o.sc[1]);
+            else st_b64(sdst, make_uint2(o.sc[0], o.sc[1]));
         }
     } else {
-        // rope kept as bf16: copy 128 bytes
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            uint8_t* dst = row + a.n + 16 * k;
-            if (aligned) *reinterpret_cast<uint4*>(dst) = lds128(seg + 16 * k);
-            else st_b128(dst, lds128(seg + 16 * k));
+        // zero padding [concatCol, kvCacheCol)
+        int p = a.concat;
+        if (SMEM || aligned) {
+            for (; p < a.col && (p & 15) != 0; ++p) row[p] = 0;
+            for (; p + 16 <= a.col; p += 16) *reinterpret_cast<uint4*>(row + p) = make_uint4(0u, 0u, 0u, 0u);
         }
+        for (; p < a.col; ++p) row[p] = 0;
     }
-    // zero padding [concatCol, kvCacheCol): bytes up to a 16-byte boundary of
-    // the (aligned) row, then 16-byte stores, then the tail
-    int p = a.concat;
-    if (aligned) {
-        for (; p < a.col && (p & 15) != 0; ++p) row[p] = 0;
-        for (; p + 16 <= a.col; p += 16) *reinterpret_cast<uint4*>(row + p) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    for (; p < a.col; ++p) row[p] = 0;
 }
 
 template <int MODE, int G>
@@ -422,21 +452,73 @@ __global__ void __launch_bounds__(CT_MAX_THREADS) compress_tma_kernel(const Comp
 
     // ---------------- consumers: warp -> segment columns, lane -> row ----------------
     const bool aligned = a.rows_aligned != 0;
+    const bool bulk_out = a.bulk_out != 0;       // one segment per warp, rows stored by bulk copy
     int it = 0;
+    int pending = -1;                             // warp 0: stage whose bulk stores may still read smem
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
         const int st = it % S;
         const uint32_t round = (uint32_t)(it / S);
-        if (!__all_sync(FULL_MASK, mbar_wait(&full[st], round & 1u))) break;   // every lane acquires the stage
+        // every lane acquires the stage; with bulk stores the consumer warps
+        // also agree (they meet at named barriers below) before going on
+        bool ok = __all_sync(FULL_MASK, mbar_wait(&full[st], round & 1u));
+        if (bulk_out) ok = named_barrier_and(NCW * 32, ok);
+        if (!ok) break;
         uint8_t* row = rowptr[st * CT_ROWS + lane];
-        const uint8_t* xrow = xs + (size_t)st * stage_bytes + (size_t)lane * pitch;
-        if (row != nullptr) {
-            for (int j = warp; j < a.nseg; j += NCW) {
-                if (j < a.nseg - 1) ct_nope_segment<MODE, G>(a, xrow + j * 128, row, j, aligned);
-                else ct_rope_segment<MODE>(a, xrow + j * 128, row, aligned);
+        uint8_t* xrow = xs + (size_t)st * stage_bytes + (size_t)lane * pitch;
+        if (bulk_out) {
+            // phase A: read this warp's segment of the lane's row and compute in registers
+            const int j = warp;
+            const bool rope = (j == a.nseg - 1);
+            SegOut o;
+            if (row != nullptr) {
+                if (!rope) ct_compute_nope<MODE, G>(xrow + j * 128, o);
+                else if (MODE == 2) ct_compute_rope2(a, xrow + j * 128, o);
             }
+            if (warp == 0 && pending >= 0) {
+                // the previous stage's rows have been read by the bulk engine: release
+                // it (bulk groups belong to the lane that committed them)
+                bulk_wait_read_all();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[pending]);
+                pending = -1;
+            }
+            named_barrier_sync(NCW * 32);           // every read of the stage is done
+            // phase B: assemble the packed row in place, over the stage's input row
+            if (row != nullptr) {
+                // modes 0/1 copy the rope within the row: its input lies past kvCacheCol
+                ct_write<MODE, G, true>(a, xrow, j, rope, o, xrow + j * 128, true);
+                fence_proxy_async_smem();
+            }
+            named_barrier_sync(NCW * 32);           // every packed row is complete
+            // phase C: one bulk store per valid row
+            if (warp == 0) {
+                if (row != nullptr) bulk_copy_s2g(row, xrow, (uint32_t)a.col);
+                bulk_commit();
+                __syncwarp();
+                pending = st;                        // released after the stores have read it
+            } else {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
+            }
+        } else {
+            if (row != nullptr) {
+                for (int j = warp; j < a.nseg; j += NCW) {
+                    const bool rope = (j == a.nseg - 1);
+                    SegOut o;
+                    if (!rope) ct_compute_nope<MODE, G>(xrow + j * 128, o);
+                    else if (MODE == 2) ct_compute_rope2(a, xrow + j * 128, o);
+                    ct_write<MODE, G, false>(a, row, j, rope, o, xrow + j * 128, aligned);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
         }
+    }
+    if (warp == 0 && bulk_out) {
+        // every bulk store of this CTA is complete before it exits
+        bulk_wait_all();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
+        if (pending >= 0 && lane == 0) mbar_arrive(&empty[pending]);
     }
 }
 

@@ -351,6 +351,8 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
         a.stages = ct_stages;
         a.rows_aligned = (reinterpret_cast<uintptr_t>(cache->data) % 16 == 0) && rows.row_bytes % 16 == 0 &&
                          rows.block_stride % 16 == 0;
+        a.bulk_out = a.rows_aligned && col % 16 == 0 && a.nseg <= CT_MAX_CONSUMER_WARPS &&
+                     (quant_mode == 2 || col <= 2 * (d - 64));
         const size_t smem = ct_smem(ct_stages);
         const int64_t tiles = (T + CT_ROWS - 1) / CT_ROWS;
         const int threads = (a.ncw + 1) * 32;
