@@ -209,7 +209,7 @@ constexpr int CT_MAX_CONSUMER_WARPS = 16;
 constexpr int CT_MAX_THREADS = (CT_MAX_CONSUMER_WARPS + 1) * 32;
 
 __host__ __device__ inline uint32_t ct_header_bytes(int stages) {
-    return ((uint32_t)(16 * stages + 8 * stages * CT_ROWS) + 127u) & ~127u;
+    return ((uint32_t)(16 * stages + 8 + 8 * stages * CT_ROWS) + 127u) & ~127u;
 }
 
 __host__ __device__ inline uint32_t ct_pitch(int nseg) { return (uint32_t)nseg * 128u + 16u; }
@@ -394,18 +394,26 @@ __device__ __forceinline__ void ct_write(const CompressArgs& a, uint8_t* row, in
     }
 }
 
+// Shared memory: barriers (full[S], empty[S], out_free), row pointers
+// [S][32], S input stages of 32 rows (pitch nseg*128 + 16), and -- with bulk
+// stores -- one output buffer of 32 packed rows (pitch odd*16 bytes).
+__host__ __device__ inline uint32_t ct_out_pitch(int col) { return (uint32_t)(((col + 15) / 16) | 1) * 16u; }
+
 template <int MODE, int G>
-__global__ void __launch_bounds__(CT_MAX_THREADS) compress_tma_kernel(const CompressArgs a) {
+__global__ void __launch_bounds__(CT_MAX_THREADS, 1) compress_tma_kernel(const CompressArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int S = a.stages;
     const int NCW = a.ncw;                         // consumer warps
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + S;
-    uint8_t** rowptr = reinterpret_cast<uint8_t**>(empty + S);
+    uint64_t* out_free = empty + S;
+    uint8_t** rowptr = reinterpret_cast<uint8_t**>(smem + 16 * S + 8);
     uint8_t* xs = smem + ct_header_bytes(S);
     const uint32_t row_bytes = (uint32_t)a.nseg * 128u;
     const uint32_t pitch = ct_pitch(a.nseg);
     const uint32_t stage_bytes = CT_ROWS * pitch;
+    uint8_t* obuf = xs + (size_t)S * stage_bytes;
+    const uint32_t opitch = ct_out_pitch(a.col);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t ntiles = (a.T + CT_ROWS - 1) / CT_ROWS;
 
@@ -414,6 +422,7 @@ __global__ void __launch_bounds__(CT_MAX_THREADS) compress_tma_kernel(const Comp
             mbar_init(&full[st], 1);
             mbar_init(&empty[st], NCW);
         }
+        mbar_init(out_free, 1);
         mbar_init_fence();
     }
     __syncthreads();
@@ -450,75 +459,78 @@ __global__ void __launch_bounds__(CT_MAX_THREADS) compress_tma_kernel(const Comp
         return;
     }
 
-    // ---------------- consumers: warp -> segment columns, lane -> row ----------------
+    // ---------------- consumers: warp -> segment column, lane -> row ----------------
     const bool aligned = a.rows_aligned != 0;
-    const bool bulk_out = a.bulk_out != 0;       // one segment per warp, rows stored by bulk copy
     int it = 0;
-    int pending = -1;                             // warp 0: stage whose bulk stores may still read smem
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-        const int st = it % S;
-        const uint32_t round = (uint32_t)(it / S);
-        // every lane acquires the stage; with bulk stores the consumer warps
-        // also agree (they meet at named barriers below) before going on
-        bool ok = __all_sync(FULL_MASK, mbar_wait(&full[st], round & 1u));
-        if (bulk_out) ok = named_barrier_and(NCW * 32, ok);
-        if (!ok) break;
-        uint8_t* row = rowptr[st * CT_ROWS + lane];
-        uint8_t* xrow = xs + (size_t)st * stage_bytes + (size_t)lane * pitch;
-        if (bulk_out) {
-            // phase A: read this warp's segment of the lane's row and compute in registers
-            const int j = warp;
-            const bool rope = (j == a.nseg - 1);
+    if (a.bulk_out) {
+        // warp 0 takes the rope segment (the least work) and owns the output
+        // buffer: it releases it for tile `it` (out_free phase it) once the bulk
+        // engine has read tile it-1's rows, waits for every warp's rows of tile
+        // it (named barrier) and issues one bulk store per row.  Warp w >= 1
+        // takes nope segment w - 1.  Nobody waits for another warp's reads:
+        // each warp releases an input stage as soon as it has read it.
+        // Every consumer warp runs every tile and makes every barrier arrival,
+        // so warp 0's bar.sync always completes; after a timed-out wait a warp
+        // is "dead": it skips all further waits and writes.
+        const int j = warp == 0 ? a.nseg - 1 : warp - 1;
+        const bool rope = (warp == 0);
+        bool dead = false;
+        for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+            const int st = it % S;
+            const uint32_t round = (uint32_t)(it / S);
+            if (!dead) dead = !__all_sync(FULL_MASK, mbar_wait(&full[st], round & 1u));
+            uint8_t* row = dead ? nullptr : rowptr[st * CT_ROWS + lane];
+            const uint8_t* xrow = xs + (size_t)st * stage_bytes + (size_t)lane * pitch;
+            uint8_t* orow = obuf + (size_t)lane * opitch;
             SegOut o;
             if (row != nullptr) {
                 if (!rope) ct_compute_nope<MODE, G>(xrow + j * 128, o);
                 else if (MODE == 2) ct_compute_rope2(a, xrow + j * 128, o);
             }
-            if (warp == 0 && pending >= 0) {
-                // the previous stage's rows have been read by the bulk engine: release
-                // it (bulk groups belong to the lane that committed them)
-                bulk_wait_read_all();
+            if (rope) {
+                if (it > 0) bulk_wait_read_all();    // tile it-1's rows have left the buffer
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[pending]);
-                pending = -1;
-            }
-            named_barrier_sync(NCW * 32);           // every read of the stage is done
-            // phase B: assemble the packed row in place, over the stage's input row
-            if (row != nullptr) {
-                // modes 0/1 copy the rope within the row: its input lies past kvCacheCol
-                ct_write<MODE, G, true>(a, xrow, j, rope, o, xrow + j * 128, true);
-                fence_proxy_async_smem();
-            }
-            named_barrier_sync(NCW * 32);           // every packed row is complete
-            // phase C: one bulk store per valid row
-            if (warp == 0) {
-                if (row != nullptr) bulk_copy_s2g(row, xrow, (uint32_t)a.col);
-                bulk_commit();
-                __syncwarp();
-                pending = st;                        // released after the stores have read it
+                if (lane == 0) mbar_arrive(out_free);
             } else {
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[st]);
+                if (lane == 0 && !dead) mbar_arrive(&empty[st]);   // inputs read
+                if (!dead) dead = !__all_sync(FULL_MASK, mbar_wait(out_free, (uint32_t)it & 1u));
+                if (dead) row = nullptr;
             }
-        } else {
             if (row != nullptr) {
-                for (int j = warp; j < a.nseg; j += NCW) {
-                    const bool rope = (j == a.nseg - 1);
-                    SegOut o;
-                    if (!rope) ct_compute_nope<MODE, G>(xrow + j * 128, o);
-                    else if (MODE == 2) ct_compute_rope2(a, xrow + j * 128, o);
-                    ct_write<MODE, G, false>(a, row, j, rope, o, xrow + j * 128, aligned);
-                }
+                ct_write<MODE, G, true>(a, orow, j, rope, o, xrow + j * 128, true);
+                fence_proxy_async_smem();
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
+            if (rope) {
+                __syncwarp();
+                if (lane == 0 && !dead) mbar_arrive(&empty[st]);   // the bf16 rope was copied
+                named_barrier_sync(NCW * 32);                     // every packed row is complete
+                if (row != nullptr) bulk_copy_s2g(row, orow, (uint32_t)a.col);
+                bulk_commit();
+            } else {
+                named_barrier_arrive(NCW * 32);
+            }
         }
+        if (warp == 0) bulk_wait_all();            // every bulk store is complete before the CTA exits
+        return;
     }
-    if (warp == 0 && bulk_out) {
-        // every bulk store of this CTA is complete before it exits
-        bulk_wait_all();
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        const int st = it % S;
+        const uint32_t round = (uint32_t)(it / S);
+        if (!__all_sync(FULL_MASK, mbar_wait(&full[st], round & 1u))) break;   // every lane acquires the stage
+        uint8_t* row = rowptr[st * CT_ROWS + lane];
+        const uint8_t* xrow = xs + (size_t)st * stage_bytes + (size_t)lane * pitch;
+        if (row != nullptr) {
+            for (int j = warp; j < a.nseg; j += NCW) {
+                const bool rope = (j == a.nseg - 1);
+                SegOut o;
+                if (!rope) ct_compute_nope<MODE, G>(xrow + j * 128, o);
+                else if (MODE == 2) ct_compute_rope2(a, xrow + j * 128, o);
+                ct_write<MODE, G, false>(a, row, j, rope, o, xrow + j * 128, aligned);
+            }
+        }
         __syncwarp();
-        if (pending >= 0 && lane == 0) mbar_arrive(&empty[pending]);
+        if (lane == 0) mbar_arrive(&empty[st]);
     }
 }
 

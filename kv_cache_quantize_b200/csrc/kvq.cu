@@ -341,18 +341,24 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
     // pipelined kernel when x rows are 16-byte aligned and a ring of at least
     // two 32-row stages fits in shared memory (d <= 1728); else the direct one
     const size_t smem_limit = 227 * 1024;
+    const bool rows_aligned = (reinterpret_cast<uintptr_t>(cache->data) % 16 == 0) && rows.row_bytes % 16 == 0 &&
+                              rows.block_stride % 16 == 0;
+    // packed rows leave by bulk copy when the rows are aligned, kvCacheCol is a
+    // multiple of 16 and each consumer warp owns one segment (d <= 1024); two
+    // input stages and one output buffer then keep two CTAs on an SM
+    const bool bulk_out = rows_aligned && col % 16 == 0 && d / 64 <= CT_MAX_CONSUMER_WARPS;
     auto ct_smem = [&](int stages) {
-        return ct_header_bytes(stages) + (size_t)stages * CT_ROWS * ct_pitch((int)(d / 64));
+        return ct_header_bytes(stages) + (size_t)stages * CT_ROWS * ct_pitch((int)(d / 64)) +
+               (bulk_out ? (size_t)CT_ROWS * ct_out_pitch((int)col) : 0);
     };
-    const int ct_stages = ct_smem(3) <= smem_limit ? 3 : (ct_smem(2) <= smem_limit ? 2 : 0);
+    const int want = bulk_out ? 2 : 3;
+    const int ct_stages = ct_smem(want) <= smem_limit ? want : (ct_smem(2) <= smem_limit ? 2 : 0);
     if (a.x_vec && ct_stages > 0) {
         // pipelined kernel: rows arrive in shared memory by bulk copy
         a.ncw = a.nseg < CT_MAX_CONSUMER_WARPS ? a.nseg : CT_MAX_CONSUMER_WARPS;
         a.stages = ct_stages;
-        a.rows_aligned = (reinterpret_cast<uintptr_t>(cache->data) % 16 == 0) && rows.row_bytes % 16 == 0 &&
-                         rows.block_stride % 16 == 0;
-        a.bulk_out = a.rows_aligned && col % 16 == 0 && a.nseg <= CT_MAX_CONSUMER_WARPS &&
-                     (quant_mode == 2 || col <= 2 * (d - 64));
+        a.rows_aligned = rows_aligned;
+        a.bulk_out = bulk_out;
         const size_t smem = ct_smem(ct_stages);
         const int64_t tiles = (T + CT_ROWS - 1) / CT_ROWS;
         const int threads = (a.ncw + 1) * 32;

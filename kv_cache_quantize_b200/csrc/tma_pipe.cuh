@@ -101,6 +101,11 @@ __device__ __forceinline__ void named_barrier_sync(int threads) {
     asm volatile("bar.sync 1, %0;" ::"r"(threads) : "memory");
 }
 
+// arrive at named barrier 1 without waiting
+__device__ __forceinline__ void named_barrier_arrive(int threads) {
+    asm volatile("bar.arrive 1, %0;" ::"r"(threads) : "memory");
+}
+
 // the same barrier, returning whether `pred` holds in every participating thread
 __device__ __forceinline__ bool named_barrier_and(int threads, bool pred) {
     uint32_t out;
