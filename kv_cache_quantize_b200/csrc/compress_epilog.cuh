@@ -42,9 +42,9 @@ struct CompressArgs {
 };
 
 // Division of a code's numerator by the group scale: the one-step Markstein
-// form (kvq_device.cuh), whose E4M3 / E2M1 codes kvq_selftest shows equal to
-// those of IEEE division on its whole domain.
-#define KVQ_SCALE_DIV div_scale1
+// form on pairs (div_scale8 / div_scale1_x2 in kvq_device.cuh), whose E4M3 /
+// E2M1 codes kvq_selftest shows equal to those of IEEE division on its whole
+// domain.
 
 constexpr int CE_TILE = 8;
 constexpr int CE_UNROLL = 3;
@@ -68,8 +68,7 @@ __device__ __forceinline__ int64_t load_slot(const void* slots, int is64, int64_
 __device__ __forceinline__ void div_by_scale8(const float (&f)[8], float sf, float (&q)[8]) {
     if (scale_in_fast_range(sf)) {
         const float r = __frcp_rn(sf);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = KVQ_SCALE_DIV(f[i], sf, r);
+        div_scale8(f, sf, r, q);
     } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], sf);
@@ -269,8 +268,7 @@ __device__ __forceinline__ void ct_compute_nope(const uint8_t* seg, SegOut& o) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) q[i] = 0.0f;
             } else if (fast) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) q[i] = KVQ_SCALE_DIV(f[i], sf, r);
+                div_scale8(f, sf, r, q);
             } else {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], sf);
@@ -299,8 +297,7 @@ __device__ __forceinline__ void ct_compute_nope(const uint8_t* seg, SegOut& o) {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) q[i] = 0.0f;
                 } else if (fast) {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) q[i] = KVQ_SCALE_DIV(f[i], sf, r);
+                    div_scale8(f, sf, r, q);
                 } else {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], sf);
@@ -429,20 +426,25 @@ __global__ void __launch_bounds__(CT_MAX_THREADS, 1) compress_tma_kernel(const C
 
     if (warp == NCW) {
         // ---------------- producer ----------------
+        // the slot of the next tile's row is loaded while the current stage is
+        // being consumed, so a released stage is refilled at once
+        auto lane_slot = [&](int64_t tile) -> int64_t {
+            const int64_t r = tile * CT_ROWS + lane;
+            return (tile < ntiles && r < a.T) ? load_slot(a.slots, a.slots_i64, r) : -1;
+        };
         int it = 0;
+        int64_t next_slot = lane_slot(blockIdx.x);
         for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
             const int st = it % S;
             const uint32_t round = (uint32_t)(it / S);
+            const int64_t slot = next_slot;
+            next_slot = lane_slot(tile + gridDim.x);
             if (!__all_sync(FULL_MASK, mbar_wait(&empty[st], (round & 1u) ^ 1u))) break;
             const int64_t row0 = tile * CT_ROWS;
-            const int rows = (int)(a.T - row0 < CT_ROWS ? a.T - row0 : CT_ROWS);
             uint8_t* p = nullptr;
-            if (lane < rows) {
-                const int64_t slot = load_slot(a.slots, a.slots_i64, row0 + lane);
-                if (slot != -1) {
-                    if (slot_ok(slot, a.cache.num_slots)) p = slot_row(a.cache, slot);
-                    else raise_fault(FAULT_SLOT_RANGE);
-                }
+            if (slot != -1) {
+                if (slot_ok(slot, a.cache.num_slots)) p = slot_row(a.cache, slot);
+                else raise_fault(FAULT_SLOT_RANGE);
             }
             rowptr[st * CT_ROWS + lane] = p;
             const unsigned valid = __ballot_sync(FULL_MASK, p != nullptr);

@@ -195,7 +195,11 @@ __global__ void selftest_div_kernel(int32_t which) {
         if (fabsf(a) > 512.0f * s) continue;
         const float r = __frcp_rn(s);
         const float ref = __fdiv_rn(a, s);
-        const float q1 = div_scale1(a, s, r);
+        float q1, q1b;
+        div_scale1_x2(a, -a, s, r, q1, q1b);    // the packed form the kernels use
+        if (__float_as_uint(q1b) != (__float_as_uint(q1) ^ 0x80000000u)) {
+            atomicAdd(&g_selftest_count, 1ull);  // the two halves must agree up to sign
+        }
         bool diff;
         switch (which) {
             case 0: diff = __float_as_uint(q1) != __float_as_uint(ref); break;

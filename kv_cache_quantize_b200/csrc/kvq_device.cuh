@@ -161,6 +161,30 @@ __device__ __forceinline__ float div_scale2(float a, float s, float r) {
     return with_sign_of(__fmaf_rn(rem1, r, q1), a);
 }
 
+// div_scale1 on two numerators at once with the packed binary32 pipe
+// (mul.rn.f32x2 / fma.rn.f32x2: each half is the same RN operation as the
+// scalar form, so the results are bit-identical to div_scale1).
+__device__ __forceinline__ void div_scale1_x2(float a0, float a1, float s, float r, float& q0, float& q1) {
+    asm("{\n\t.reg .b64 a, q, rem, rr, ns;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 rr, {%4, %4};\n\t"
+        "mov.b64 ns, {%5, %5};\n\t"
+        "mul.rn.f32x2 q, a, rr;\n\t"
+        "fma.rn.f32x2 rem, q, ns, a;\n\t"
+        "fma.rn.f32x2 q, rem, rr, q;\n\t"
+        "mov.b64 {%0, %1}, q;\n\t}"
+        : "=f"(q0), "=f"(q1)
+        : "f"(a0), "f"(a1), "f"(r), "f"(-s));
+    q0 = with_sign_of(q0, a0);
+    q1 = with_sign_of(q1, a1);
+}
+
+// eight quotients f[i] / s through div_scale1_x2
+__device__ __forceinline__ void div_scale8(const float (&f)[8], float s, float r, float (&q)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) div_scale1_x2(f[i], f[i + 1], s, r, q[i], q[i + 1]);
+}
+
 // amax / c for the format maxima c = 448, 57344, 6 (amax >= 0, a bf16 value):
 // the one-step form with the constant RN(1/c).
 __device__ __forceinline__ float div_by_fmax(float amax, float c) {
