@@ -37,6 +37,7 @@ struct DrqArgs {
     const float* activation_scale;  // [B*S] nullable
     const void* bias;               // [H] nullable
     int32_t bias_kind;              // 0 f32, 1 f16, 2 bf16, 3 int32
+    int32_t params_vec;             // all f32 parameter tensors are 16-byte aligned
     int32_t Nq, Nkv, D;
     uint16_t* q_out;        // [B*S, Nq*D]
     uint16_t* k_out;        // [B*S, Nkv*D] or null
@@ -91,14 +92,45 @@ __device__ __forceinline__ float dq_bias(const DrqArgs& a, int64_t i) {
     }
 }
 
+// E consecutive binary32 parameters starting at p (16-byte vectors when E % 4 == 0
+// and p is 16-byte aligned, which holds for the kernels' channel offsets when the
+// parameter tensors are 16-byte aligned: params_vec).
+template <int E>
+__device__ __forceinline__ void dq_param(const float* p, bool vec, float (&v)[E]) {
+    if (E % 4 == 0 && vec) {
+#pragma unroll
+        for (int k = 0; k < E; k += 4) {
+            const float4 w = __ldg(reinterpret_cast<const float4*>(p + k));
+            v[k] = w.x; v[k + 1] = w.y; v[k + 2] = w.z; v[k + 3] = w.w;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < E; ++k) v[k] = __ldg(p + k);
+    }
+}
+
 __device__ __forceinline__ uint32_t dq_round16(const DrqArgs& a, float v) {
     return a.cos_f16 ? to_f16_bits(v) : to_bf16_bits(v);
 }
 
+// E 16-bit outputs, packed into 4- or 8-byte stores
 template <int E>
 __device__ __forceinline__ void dq_store16(uint16_t* p, const DrqArgs& a, const float (&o)[E]) {
+    if (E % 4 == 0) {
 #pragma unroll
-    for (int k = 0; k < E; ++k) p[k] = (uint16_t)dq_round16(a, o[k]);
+        for (int k = 0; k < E; k += 4) {
+            const uint2 w = make_uint2(dq_round16(a, o[k]) | (dq_round16(a, o[k + 1]) << 16),
+                                       dq_round16(a, o[k + 2]) | (dq_round16(a, o[k + 3]) << 16));
+            st_b64(reinterpret_cast<uint8_t*>(p + k), w);
+        }
+    } else if (E % 2 == 0) {
+#pragma unroll
+        for (int k = 0; k < E; k += 2)
+            st_b32(reinterpret_cast<uint8_t*>(p + k), dq_round16(a, o[k]) | (dq_round16(a, o[k + 1]) << 16));
+    } else {
+#pragma unroll
+        for (int k = 0; k < E; ++k) p[k] = (uint16_t)dq_round16(a, o[k]);
+    }
 }
 
 // One head of one token: dequant, RoPE (q and k heads), outputs, int8 quant
@@ -108,13 +140,23 @@ __device__ __forceinline__ void dq_head(const DrqArgs& a, int64_t t, int hd, flo
                                         const float (&sn)[E], float act, int64_t slot, int pos, bool second_half) {
     const int D = a.D;
     const int ch0 = hd * D + pos;    // channel index within H
+    const bool pv = a.params_vec != 0;
     // 1 dequant: ((float)x * weight_scale) * activation_scale + bias
     if (a.x_kind == 0) {
+        float ws[E];
+        dq_param<E>(a.weight_scale + ch0, pv, ws);
+        float bs[E];
+        if (a.bias && a.bias_kind == 0) {
+            dq_param<E>(reinterpret_cast<const float*>(a.bias) + ch0, pv, bs);
+        } else if (a.bias) {
+#pragma unroll
+            for (int k = 0; k < E; ++k) bs[k] = dq_bias(a, ch0 + k);
+        }
 #pragma unroll
         for (int k = 0; k < E; ++k) {
-            float v = __fmul_rn(u[k], a.weight_scale[ch0 + k]);
+            float v = __fmul_rn(u[k], ws[k]);
             if (a.activation_scale) v = __fmul_rn(v, act);
-            if (a.bias) v = __fadd_rn(v, dq_bias(a, ch0 + k));
+            if (a.bias) v = __fadd_rn(v, bs[k]);
             u[k] = v;
         }
     }
@@ -140,15 +182,17 @@ __device__ __forceinline__ void dq_head(const DrqArgs& a, int64_t t, int hd, flo
     if (a.k_out) dq_store16<E>((is_k ? a.k_out : a.v_out) + t * (int64_t)(a.Nkv * D) + c0, a, o);
     if (slot < 0) return;
     // 4 quant: int8(rint(w / scale + offset)), saturating
-    const float* sc = is_k ? a.scale_k : a.scale_v;
-    const float* of = is_k ? a.offset_k : a.offset_v;
+    float sc[E], of[E];
+    dq_param<E>((is_k ? a.scale_k : a.scale_v) + c0, pv, sc);
+    const float* ofp = is_k ? a.offset_k : a.offset_v;
+    if (ofp) dq_param<E>(ofp + c0, pv, of);
     uint32_t packed[(E + 3) / 4];
 #pragma unroll
     for (int k = 0; k < (E + 3) / 4; ++k) packed[k] = 0u;
 #pragma unroll
     for (int k = 0; k < E; ++k) {
-        float q = __fdiv_rn(o[k], sc[c0 + k]);
-        if (of) q = __fadd_rn(q, of[c0 + k]);
+        float q = __fdiv_rn(o[k], sc[k]);
+        if (ofp) q = __fadd_rn(q, of[k]);
         packed[k / 4] |= ((uint32_t)int8_rne_sat(q) & 0xffu) << (8 * (k % 4));
     }
     // 5 cache write
@@ -322,10 +366,22 @@ __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(cons
             const uint16_t* cw = reinterpret_cast<const uint16_t*>(base + x_span) + k * D + pos;
             const uint16_t* sw = reinterpret_cast<const uint16_t*>(base + x_span + cs_span) + k * D + pos;
             float cs[E], sn[E];
+            if (E % 4 == 0) {
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                cs[e] = half_bits_to_f32(cw[e], f16);
-                sn[e] = half_bits_to_f32(sw[e], f16);
+                for (int e = 0; e < E; e += 4) {
+                    const uint2 c2 = *reinterpret_cast<const uint2*>(cw + e);
+                    const uint2 s2 = *reinterpret_cast<const uint2*>(sw + e);
+                    cs[e] = half_bits_to_f32(c2.x & 0xffffu, f16); cs[e + 1] = half_bits_to_f32(c2.x >> 16, f16);
+                    cs[e + 2] = half_bits_to_f32(c2.y & 0xffffu, f16); cs[e + 3] = half_bits_to_f32(c2.y >> 16, f16);
+                    sn[e] = half_bits_to_f32(s2.x & 0xffffu, f16); sn[e + 1] = half_bits_to_f32(s2.x >> 16, f16);
+                    sn[e + 2] = half_bits_to_f32(s2.y & 0xffffu, f16); sn[e + 3] = half_bits_to_f32(s2.y >> 16, f16);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    cs[e] = half_bits_to_f32(cw[e], f16);
+                    sn[e] = half_bits_to_f32(sw[e], f16);
+                }
             }
             const float act = (a.x_kind == 0 && a.activation_scale) ? a.activation_scale[t] : 1.0f;
             for (int i = 0; i < nh; ++i) {

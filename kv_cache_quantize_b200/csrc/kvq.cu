@@ -722,6 +722,10 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
     a.activation_scale = as;
     a.bias = bias_ptr;
     a.bias_kind = bias_kind;
+    {
+        auto al = [](const void* p) { return p == nullptr || reinterpret_cast<uintptr_t>(p) % 16 == 0; };
+        a.params_vec = al(sk) && al(sv) && al(ok) && al(ov) && al(ws) && (bias_kind != 0 || al(bias_ptr));
+    }
     a.Nq = (int32_t)Nq;
     a.Nkv = (int32_t)Nkv;
     a.D = (int32_t)D;
