@@ -41,6 +41,11 @@ WORKLOAD = ("kv_compress_epilog large sweep: T=262144 tokens, d=576 bf16 N(0,1) 
             "bf16 scale, rope FP8 E4M3 static x_scale=0.1, 352-B rows); cache blockSize=128, 4096 blocks; "
             "2% slot_mapping -1")
 FALLBACK_HBM_GBS = 6650.0
+# A single timed launch is preceded by a device-side wait of this many SM
+# cycles (~100 us), so that the host has enqueued the start event, the launch
+# and the stop event before the GPU reaches the start event: the events then
+# bracket device time only, not the host's call overhead.
+HOST_LEAD_CYCLES = 200_000
 
 
 # ---------------------------------------------------------------------------
@@ -267,6 +272,7 @@ def run_profile_workload(args):
     times = []
     for i in range(args.profile_reps):
         flush.fill_(i & 0xFF)
+        torch.cuda._sleep(HOST_LEAD_CYCLES)       # the host enqueues the launch before the GPU reaches e0
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         call(stream)
@@ -436,6 +442,7 @@ def main():
             times = []
             for i in range(reps + 3):
                 flush.fill_(i & 0xFF)                 # evict the previous launch's data from L2
+                torch.cuda._sleep(HOST_LEAD_CYCLES)   # the launch is enqueued before the GPU reaches e0
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
                 call(stream)

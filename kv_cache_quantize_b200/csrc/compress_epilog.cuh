@@ -57,10 +57,6 @@ __device__ __forceinline__ uint4 ld_scalar8(const uint16_t* p) {
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__device__ __forceinline__ int64_t load_slot(const void* slots, int is64, int64_t i) {
-    return is64 ? reinterpret_cast<const int64_t*>(slots)[i] : (int64_t) reinterpret_cast<const int32_t*>(slots)[i];
-}
-
 // One segment.  All lanes call this (the shuffles need the whole warp); lanes
 // whose segment is inactive or skipped carry live == false.
 // x_i / sf for the eight values of a lane: Markstein-corrected multiply by the
@@ -215,15 +211,32 @@ __host__ __device__ inline uint32_t ct_pitch(int nseg) { return (uint32_t)nseg *
 
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
 
-// |x| maximum of the 64 bf16 values of one segment (as bits)
+// |x| maximum of the bf16 values of nchunks 16-byte chunks (as bits)
 __device__ __forceinline__ uint32_t seg_absmax_bits(const uint8_t* seg, int nchunks) {
     uint32_t m2 = 0u;
     for (int k = 0; k < nchunks; ++k) {
         const uint4 v = lds128(seg + 16 * k);
-        const uint32_t msk = 0x7fff7fffu;
-        m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(v.x & msk, v.y & msk), __vmaxu2(v.z & msk, v.w & msk)));
+        m2 = absmax_bf16x2(m2, absmax_bf16x2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w)));
     }
+    m2 &= 0x7fff7fffu;
     return max(m2 & 0xffffu, m2 >> 16);
+}
+
+// Codes of eight values divided by the scale sf through the negated one-step
+// quotient (div_scale1_neg_x2): FP8 E4M3 as two words, or FP4 E2M1 as one.
+__device__ __forceinline__ uint2 e4m3x8_div(const float (&f)[8], float sf, float r) {
+    float t[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) div_scale1_neg_x2(f[i], f[i + 1], sf, r, t[i], t[i + 1]);
+    const uint2 c = fp8x8<false>(t);
+    return make_uint2(c.x ^ 0x80808080u, c.y ^ 0x80808080u);
+}
+
+__device__ __forceinline__ uint32_t e2m1x8_div(const float (&f)[8], float sf, float r) {
+    float t[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) div_scale1_neg_x2(f[i], f[i + 1], sf, r, t[i], t[i + 1]);
+    return e2m1x8(t) ^ 0x88888888u;
 }
 
 // Outputs of one 64-value segment held in registers: the code bytes packed
@@ -268,7 +281,10 @@ __device__ __forceinline__ void ct_compute_nope(const uint8_t* seg, SegOut& o) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) q[i] = 0.0f;
             } else if (fast) {
-                div_scale8(f, sf, r, q);
+                const uint2 c = e4m3x8_div(f, sf, r);
+                o.w[2 * k] = c.x;
+                o.w[2 * k + 1] = c.y;
+                continue;
             } else {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], sf);
@@ -297,7 +313,8 @@ __device__ __forceinline__ void ct_compute_nope(const uint8_t* seg, SegOut& o) {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) q[i] = 0.0f;
                 } else if (fast) {
-                    div_scale8(f, sf, r, q);
+                    o.w[g * GC + k] = e2m1x8_div(f, sf, r);
+                    continue;
                 } else {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(f[i], sf);

@@ -271,33 +271,181 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) dequant_rope_quant_kernel(const
 }
 
 // ---------------------------------------------------------------------------
-// Pipelined kernel (16-byte aligned x, cos and sin).  CTA = DQ_WARPS consumer
-// warps + 1 producer warp.  A stage holds TPS consecutive tokens: their x rows,
-// cos rows and sin rows arrive by three bulk copies (each a contiguous span),
-// and the producer stores their destination slots next to them.  Consumers
-// keep the head mapping of the direct kernel and read x, cos and sin from
-// shared memory.
+// Pipelined kernel (16-byte aligned x, cos and sin; D = 32 E with E = 2, 4 or
+// 8).  CTA = DT_CONSUMERS consumer warps + 1 producer warp.  A stage holds TPS
+// consecutive tokens: their x rows, cos rows and sin rows arrive by three bulk
+// copies (each a contiguous span); the producer resolves the tokens'
+// destination slots and activation scales one stage ahead and stores them
+// next to the stage.  Consumers: the warps are split evenly over the stage's
+// tokens, and the warps of one token split its Nq + 2 Nkv heads into
+// contiguous ranges, which they walk two heads per pass (lane l holds values
+// [E l, E l + E) of both heads, so a value's half-rotation partner is
+// __shfl_xor(16) away and both heads share the lane's cos / sin values).
 // ---------------------------------------------------------------------------
-constexpr int DT_THREADS = (DQ_WARPS + 1) * 32;
+constexpr int DT_CONSUMERS = 8;
+constexpr int DT_THREADS = (DT_CONSUMERS + 1) * 32;
 
 __host__ __device__ inline uint32_t dt_header_bytes(int stages, int tps) {
-    return ((uint32_t)(16 * stages + 8 * stages * tps) + 127u) & ~127u;
+    return ((uint32_t)(16 * stages + 12 * stages * tps) + 127u) & ~127u;
 }
 
 __host__ __device__ inline uint32_t dt_stage_bytes(int tps, int64_t H, int x_bytes, int D) {
     return (uint32_t)(((tps * H * x_bytes + 127) & ~127) + 2 * ((tps * D * 2 + 127) & ~127));
 }
 
+// Raw index entry of token t (page mode: its slot; contiguous mode: the start
+// position of its batch).
+__device__ __forceinline__ int64_t dq_index_raw(const DrqArgs& a, int64_t t) {
+    return load_slot(a.indices, a.indices_i64, a.cache_mode == 1 ? t : t / a.S);
+}
+
+// Destination row of token t from its raw index entry: >= 0 a cache slot,
+// -1 skip, -2 bad index (the rules of dq_slot).
+__device__ __forceinline__ int64_t dq_resolve(const DrqArgs& a, int64_t t, int64_t raw) {
+    if (a.cache_mode == 1) {
+        if (raw != -1 && !slot_ok(raw, a.kc.num_slots)) return -2;
+        return raw;
+    }
+    const int64_t b = t / a.S, s = t - b * a.S;
+    const int64_t c1 = a.kc.block_size;
+    if (raw == -1) return -1;
+    if (raw < 0 || raw + s >= c1 || b * c1 >= a.kc.num_slots) return -2;
+    return b * c1 + raw + s;
+}
+
+// E consecutive 16-bit floats from shared memory, widened
+template <int E, bool F16>
+__device__ __forceinline__ void dt_lds16(const uint16_t* p, float (&v)[E]) {
+    uint32_t w[E / 2];
+    if (E % 8 == 0) {
+#pragma unroll
+        for (int k = 0; k < E / 8; ++k) {
+            const uint4 q = *reinterpret_cast<const uint4*>(p + 8 * k);
+            w[4 * k] = q.x; w[4 * k + 1] = q.y; w[4 * k + 2] = q.z; w[4 * k + 3] = q.w;
+        }
+    } else if (E % 4 == 0) {
+        const uint2 q = *reinterpret_cast<const uint2*>(p);
+        w[0] = q.x; w[1] = q.y;
+    } else {
+#pragma unroll
+        for (int k = 0; k < E / 2; ++k) w[k] = reinterpret_cast<const uint32_t*>(p)[k];
+    }
+#pragma unroll
+    for (int k = 0; k < E / 2; ++k) {
+        v[2 * k] = F16 ? f16_lo(w[k]) : bf16_lo(w[k]);
+        v[2 * k + 1] = F16 ? f16_hi(w[k]) : bf16_hi(w[k]);
+    }
+}
+
+// E consecutive int32 values from shared memory, converted to binary32
 template <int E>
+__device__ __forceinline__ void dt_lds_i32(const int32_t* p, float (&v)[E]) {
+    if (E % 4 == 0) {
+#pragma unroll
+        for (int k = 0; k < E; k += 4) {
+            const int4 q = *reinterpret_cast<const int4*>(p + k);
+            v[k] = __int2float_rn(q.x); v[k + 1] = __int2float_rn(q.y);
+            v[k + 2] = __int2float_rn(q.z); v[k + 3] = __int2float_rn(q.w);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < E; k += 2) {
+            const int2 q = *reinterpret_cast<const int2*>(p + k);
+            v[k] = __int2float_rn(q.x); v[k + 1] = __int2float_rn(q.y);
+        }
+    }
+}
+
+// E binary32 parameters at p (16-byte vectors when vec and E % 4 == 0)
+template <int E>
+__device__ __forceinline__ void dt_param(const float* p, bool vec, float (&v)[E]) {
+    if (E % 4 == 0 && vec) {
+#pragma unroll
+        for (int k = 0; k < E; k += 4) {
+            const float4 q = __ldg(reinterpret_cast<const float4*>(p + k));
+            v[k] = q.x; v[k + 1] = q.y; v[k + 2] = q.z; v[k + 3] = q.w;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < E; ++k) v[k] = __ldg(p + k);
+    }
+}
+
+// E values rounded to 16-bit floats, packed two per word, stored at p
+template <int E, bool F16>
+__device__ __forceinline__ void dt_store16(uint16_t* p, const float (&o)[E]) {
+    uint32_t w[E / 2];
+#pragma unroll
+    for (int k = 0; k < E / 2; ++k) {
+        if (F16) {
+            asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w[k]) : "f"(o[2 * k + 1]), "f"(o[2 * k]));
+        } else {
+            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[k]) : "f"(o[2 * k + 1]), "f"(o[2 * k]));
+        }
+    }
+    uint8_t* b = reinterpret_cast<uint8_t*>(p);
+    if (E % 8 == 0) {
+#pragma unroll
+        for (int k = 0; k < E / 8; ++k) st_b128(b + 16 * k, make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]));
+    } else if (E % 4 == 0) {
+        st_b64(b, make_uint2(w[0], w[1]));
+    } else {
+#pragma unroll
+        for (int k = 0; k < E / 2; ++k) st_b32(b + 4 * k, w[k]);
+    }
+}
+
+// Output stage of one head (o: the head's values after dequant and RoPE):
+// q heads -> qOut; k / v heads -> kOut / vOut when requested, then static
+// int8 quantisation (Div -> Add offset -> round half to even, saturate) into
+// the cache row.
+template <int E, bool F16>
+__device__ __forceinline__ void dt_head_out(const DrqArgs& a, int64_t t, int hd, int pos, const float (&o)[E],
+                                            uint8_t* krow, uint8_t* vrow, bool pv) {
+    const int D = a.D;
+    if (hd < a.Nq) {
+        dt_store16<E, F16>(a.q_out + t * (int64_t)(a.Nq * D) + hd * D + pos, o);
+        return;
+    }
+    const bool is_k = hd < a.Nq + a.Nkv;
+    const int c0 = (is_k ? hd - a.Nq : hd - a.Nq - a.Nkv) * D + pos;   // channel in [0, Nkv*D)
+    if (a.k_out) dt_store16<E, F16>((is_k ? a.k_out : a.v_out) + t * (int64_t)(a.Nkv * D) + c0, o);
+    uint8_t* row = is_k ? krow : vrow;
+    if (row == nullptr) return;
+    float sc[E], of[E];
+    dt_param<E>((is_k ? a.scale_k : a.scale_v) + c0, pv, sc);
+    const float* ofp = is_k ? a.offset_k : a.offset_v;
+    if (ofp) dt_param<E>(ofp + c0, pv, of);
+    uint32_t packed[E / 4 > 0 ? E / 4 : 1];
+#pragma unroll
+    for (int k = 0; k < (E + 3) / 4; ++k) packed[k] = 0u;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        float q = __fdiv_rn(o[k], sc[k]);
+        if (ofp) q = __fadd_rn(q, of[k]);
+        packed[k / 4] |= ((uint32_t)int8_rne_sat(q) & 0xffu) << (8 * (k % 4));
+    }
+    if (E % 4 == 0) {
+#pragma unroll
+        for (int k = 0; k < E / 4; ++k) st_b32(row + c0 + 4 * k, packed[k]);
+    } else {
+        st_b16(row + c0, packed[0]);
+    }
+}
+
+// XK: 0 int32 x (dequantised), 1 bf16 x, 2 f16 x.  F16: cos / sin and the
+// 16-bit outputs are f16 (else bf16).
+template <int E, int XK, bool F16>
 __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(const DrqArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int S = a.stages, TPS = a.tps, D = a.D;
-    const int xb = a.x_kind == 0 ? 4 : 2;
+    constexpr int XB = XK == 0 ? 4 : 2;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + S;
     int64_t* slots = reinterpret_cast<int64_t*>(empty + S);
+    float* acts = reinterpret_cast<float*>(slots + S * TPS);
     uint8_t* stages = smem + dt_header_bytes(S, TPS);
-    const uint32_t x_span = (uint32_t)((TPS * a.H * xb + 127) & ~127);
+    const uint32_t x_span = (uint32_t)((TPS * a.H * XB + 127) & ~127);
     const uint32_t cs_span = (uint32_t)((TPS * D * 2 + 127) & ~127);
     const uint32_t stage_bytes = x_span + 2 * cs_span;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -307,35 +455,53 @@ __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(cons
     if (threadIdx.x == 0) {
         for (int st = 0; st < S; ++st) {
             mbar_init(&full[st], 1);
-            mbar_init(&empty[st], DQ_WARPS);
+            mbar_init(&empty[st], DT_CONSUMERS);
         }
         mbar_init_fence();
     }
     __syncthreads();
 
-    if (warp == DQ_WARPS) {
+    if (warp == DT_CONSUMERS) {
         // ---------------- producer ----------------
+        // lane k < TPS holds token k's raw index entry and activation scale
+        // for the next tile, loaded while the current tile is being issued
+        auto fetch = [&](int64_t tile, int64_t& raw, float& act) {
+            const int64_t t = tile * TPS + lane;
+            raw = -1;
+            act = 1.0f;
+            if (lane < TPS && tile < ntiles && t < ntok) {
+                raw = dq_index_raw(a, t);
+                if (XK == 0 && a.activation_scale) act = a.activation_scale[t];
+            }
+        };
         int it = 0;
+        int64_t raw_next;
+        float act_next;
+        fetch(blockIdx.x, raw_next, act_next);
         for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
             const int st = it % S;
             const uint32_t round = (uint32_t)(it / S);
+            const int64_t raw = raw_next;
+            const float act = act_next;
+            fetch(tile + gridDim.x, raw_next, act_next);
             if (!__all_sync(FULL_MASK, mbar_wait(&empty[st], (round & 1u) ^ 1u))) break;
             const int64_t t0 = tile * TPS;
             const int toks = (int)(ntok - t0 < TPS ? ntok - t0 : TPS);
-            for (int k = lane; k < toks; k += 32) {
-                int64_t slot = dq_slot(a, t0 + k);
+            if (lane < toks) {
+                int64_t slot = dq_resolve(a, t0 + lane, raw);
                 if (slot == -2) {
                     raise_fault(FAULT_SLOT_RANGE);
                     slot = -1;
                 }
-                slots[st * TPS + k] = slot;
+                slots[st * TPS + lane] = slot;
+                acts[st * TPS + lane] = act;
             }
             __syncwarp();
             if (lane == 0) {
                 uint8_t* base = stages + (size_t)st * stage_bytes;
-                const uint32_t xbytes = (uint32_t)(toks * a.H * xb), cbytes = (uint32_t)(toks * D * 2);
+                const uint32_t xbytes = (uint32_t)(toks * a.H * XB), cbytes = (uint32_t)(toks * D * 2);
                 mbar_arrive_expect_tx(&full[st], xbytes + 2 * cbytes);
-                bulk_copy_g2s(base, reinterpret_cast<const uint8_t*>(a.x) + (size_t)t0 * a.H * xb, xbytes, &full[st]);
+                bulk_copy_g2s(base, reinterpret_cast<const uint8_t*>(a.x) + (size_t)t0 * a.H * XB, xbytes, &full[st]);
                 bulk_copy_g2s(base + x_span, a.cos + (size_t)t0 * D, cbytes, &full[st]);
                 bulk_copy_g2s(base + x_span + cs_span, a.sin + (size_t)t0 * D, cbytes, &full[st]);
             }
@@ -348,10 +514,12 @@ __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(cons
 
     // ---------------- consumers ----------------
     const int NH = a.Nq + 2 * a.Nkv;
+    const int WPT = DT_CONSUMERS / TPS;               // warps per token
+    const int my_tok = warp / WPT, wt = warp - my_tok * WPT;
+    const int h_begin = (NH * wt) / WPT, h_end = (NH * (wt + 1)) / WPT;
     const int pos = lane * E;
-    const bool second_half = lane >= 16;
-    const bool f16 = a.cos_f16 != 0;
-    const int nh = (NH - warp + DQ_WARPS - 1) / DQ_WARPS;
+    const bool first_half = lane < 16;
+    const bool pv = a.params_vec != 0;
     int it = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
         const int st = it % S;
@@ -359,54 +527,72 @@ __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(cons
         if (!__all_sync(FULL_MASK, mbar_wait(&full[st], round & 1u))) break;
         const int64_t t0 = tile * TPS;
         const int toks = (int)(ntok - t0 < TPS ? ntok - t0 : TPS);
-        const uint8_t* base = stages + (size_t)st * stage_bytes;
-        for (int k = 0; k < toks; ++k) {
-            const int64_t t = t0 + k;
-            const int64_t slot = slots[st * TPS + k];
-            const uint16_t* cw = reinterpret_cast<const uint16_t*>(base + x_span) + k * D + pos;
-            const uint16_t* sw = reinterpret_cast<const uint16_t*>(base + x_span + cs_span) + k * D + pos;
+        if (my_tok < toks) {
+            const int64_t t = t0 + my_tok;
+            const uint8_t* base = stages + (size_t)st * stage_bytes;
+            const int64_t slot = slots[st * TPS + my_tok];
+            const float act = acts[st * TPS + my_tok];
+            uint8_t* krow = slot >= 0 ? slot_row(a.kc, slot) : nullptr;
+            uint8_t* vrow = slot >= 0 ? slot_row(a.vc, slot) : nullptr;
+            // cos, and sin carrying the sign of the lane's half of the rotation
             float cs[E], sn[E];
-            if (E % 4 == 0) {
+            dt_lds16<E, F16>(reinterpret_cast<const uint16_t*>(base + x_span) + my_tok * D + pos, cs);
+            dt_lds16<E, F16>(reinterpret_cast<const uint16_t*>(base + x_span + cs_span) + my_tok * D + pos, sn);
+            if (first_half) {
 #pragma unroll
-                for (int e = 0; e < E; e += 4) {
-                    const uint2 c2 = *reinterpret_cast<const uint2*>(cw + e);
-                    const uint2 s2 = *reinterpret_cast<const uint2*>(sw + e);
-                    cs[e] = half_bits_to_f32(c2.x & 0xffffu, f16); cs[e + 1] = half_bits_to_f32(c2.x >> 16, f16);
-                    cs[e + 2] = half_bits_to_f32(c2.y & 0xffffu, f16); cs[e + 3] = half_bits_to_f32(c2.y >> 16, f16);
-                    sn[e] = half_bits_to_f32(s2.x & 0xffffu, f16); sn[e + 1] = half_bits_to_f32(s2.x >> 16, f16);
-                    sn[e + 2] = half_bits_to_f32(s2.y & 0xffffu, f16); sn[e + 3] = half_bits_to_f32(s2.y >> 16, f16);
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    cs[e] = half_bits_to_f32(cw[e], f16);
-                    sn[e] = half_bits_to_f32(sw[e], f16);
-                }
+                for (int k = 0; k < E; ++k) sn[k] = -sn[k];
             }
-            const float act = (a.x_kind == 0 && a.activation_scale) ? a.activation_scale[t] : 1.0f;
-            for (int i = 0; i < nh; ++i) {
-                const int hd = warp + i * DQ_WARPS;
-                float u[E];
-                const int64_t e0 = (int64_t)k * a.H + (int64_t)hd * D + pos;
-                if (a.x_kind == 0) {
-                    const int32_t* xi = reinterpret_cast<const int32_t*>(base) + e0;
-                    if (E % 4 == 0) {
+            for (int h0 = h_begin; h0 < h_end; h0 += 2) {
+                const bool two = h0 + 1 < h_end;
+                float u[2][E];
 #pragma unroll
-                        for (int e = 0; e < E; e += 4) {
-                            const int4 w = *reinterpret_cast<const int4*>(xi + e);
-                            u[e] = __int2float_rn(w.x); u[e + 1] = __int2float_rn(w.y);
-                            u[e + 2] = __int2float_rn(w.z); u[e + 3] = __int2float_rn(w.w);
+                for (int j = 0; j < 2; ++j) {
+                    if (j == 1 && !two) break;
+                    const int64_t e0 = (int64_t)my_tok * a.H + (int64_t)(h0 + j) * D + pos;
+                    if (XK == 0) dt_lds_i32<E>(reinterpret_cast<const int32_t*>(base) + e0, u[j]);
+                    else dt_lds16<E, XK == 2>(reinterpret_cast<const uint16_t*>(base) + e0, u[j]);
+                }
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    if (j == 1 && !two) break;
+                    const int hd = h0 + j;
+                    if (XK == 0) {
+                        // dequant: ((float)x * weight_scale) * activation_scale + bias
+                        float ws[E], bs[E];
+                        dt_param<E>(a.weight_scale + hd * D + pos, pv, ws);
+                        if (a.bias && a.bias_kind == 0) {
+                            dt_param<E>(reinterpret_cast<const float*>(a.bias) + hd * D + pos, pv, bs);
+                        } else if (a.bias) {
+#pragma unroll
+                            for (int k = 0; k < E; ++k) bs[k] = dq_bias(a, hd * D + pos + k);
+                        }
+#pragma unroll
+                        for (int k = 0; k < E; ++k) {
+                            float v = __fmul_rn(u[j][k], ws[k]);
+                            if (a.activation_scale) v = __fmul_rn(v, act);
+                            if (a.bias) v = __fadd_rn(v, bs[k]);
+                            u[j][k] = v;
+                        }
+                    }
+                }
+                // RoPE on q and k heads (the whole warp shuffles)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    if (j == 1 && !two) break;
+                    const int hd = h0 + j;
+                    float o[E];
+                    if (hd < a.Nq + a.Nkv) {
+#pragma unroll
+                        for (int k = 0; k < E; ++k) {
+                            const float p = __shfl_xor_sync(FULL_MASK, u[j][k], 16);
+                            o[k] = __fadd_rn(__fmul_rn(u[j][k], cs[k]), __fmul_rn(p, sn[k]));
                         }
                     } else {
 #pragma unroll
-                        for (int e = 0; e < E; ++e) u[e] = __int2float_rn(xi[e]);
+                        for (int k = 0; k < E; ++k) o[k] = u[j][k];
                     }
-                } else {
-                    const uint16_t* xh = reinterpret_cast<const uint16_t*>(base) + e0;
-#pragma unroll
-                    for (int e = 0; e < E; ++e) u[e] = half_bits_to_f32(xh[e], a.x_kind == 2);
+                    dt_head_out<E, F16>(a, t, hd, pos, o, krow, vrow, pv);
                 }
-                dq_head<E>(a, t, hd, u, cs, sn, act, slot, pos, second_half);
             }
         }
         __syncwarp();

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "kvq.h"
 #include "compress_epilog.cuh"
@@ -122,6 +123,9 @@ kvq_status paged_from(const kvq_tensor* c, int64_t inner, PagedRows* out, int64_
     out->block_size = bs;
     out->row_bytes = row * eb;
     out->block_stride = (nb > 1 ? c->stride[0] : bs * row) * eb;
+    out->bs_shift = -1;
+    for (int k = 0; k < 62; ++k)
+        if (bs == (int64_t(1) << k)) out->bs_shift = k;
     *head_dim = hd;
     return KVQ_OK;
 }
@@ -143,10 +147,39 @@ int sm_count() {
     return cached[dev];
 }
 
-template <typename K>
-int64_t persistent_grid(K kernel, int threads, int64_t needed_blocks) {
+// Resident blocks per SM of a kernel at a launch shape, asked of the runtime
+// once per (kernel, device, threads, shared memory) and remembered: the
+// query costs host time on every call otherwise.  Kernels with dynamic shared
+// memory get their opt-in limit raised to the device maximum on first use.
+int resident_blocks(const void* fn, int threads, size_t smem) {
+    struct Entry { const void* fn; int dev, threads; size_t smem; int occ; };
+    static std::mutex mu;
+    static Entry table[128];
+    static int used = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+        if (table[i].fn == fn && table[i].dev == dev && table[i].threads == threads && table[i].smem == smem)
+            return table[i].occ;
+    bool attr_set = false;
+    for (int i = 0; i < used; ++i)
+        if (table[i].fn == fn && table[i].dev == dev) attr_set = true;
+    if (smem > 0 && !attr_set) {
+        int optin = 0;
+        if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess || optin <= 0)
+            optin = 227 * 1024;
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    }
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, 0) != cudaSuccess || occ < 1) occ = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, smem) != cudaSuccess || occ < 1) occ = 1;
+    if (used < 128) table[used++] = Entry{fn, dev, threads, smem, occ};
+    return occ;
+}
+
+template <typename K>
+int64_t persistent_grid(K kernel, int threads, int64_t needed_blocks, size_t smem = 0) {
+    const int occ = resident_blocks(reinterpret_cast<const void*>(kernel), threads, smem);
     const int64_t cap = (int64_t)sm_count() * occ;
     int64_t g = needed_blocks < cap ? needed_blocks : cap;
     return g < 1 ? 1 : g;
@@ -195,21 +228,29 @@ __global__ void selftest_div_kernel(int32_t which) {
         if (fabsf(a) > 512.0f * s) continue;
         const float r = __frcp_rn(s);
         const float ref = __fdiv_rn(a, s);
-        float q1, q1b;
-        div_scale1_x2(a, -a, s, r, q1, q1b);    // the packed form the kernels use
-        if (__float_as_uint(q1b) != (__float_as_uint(q1) ^ 0x80000000u)) {
-            atomicAdd(&g_selftest_count, 1ull);  // the two halves must agree up to sign
+        float q1, q1b, t1, t1b;
+        div_scale1_x2(a, -a, s, r, q1, q1b);        // the packed forms the kernels use
+        div_scale1_neg_x2(a, -a, s, r, t1, t1b);
+        if (__float_as_uint(q1b) != (__float_as_uint(q1) ^ 0x80000000u) ||
+            __float_as_uint(t1) != (__float_as_uint(q1) ^ 0x80000000u) ||
+            __float_as_uint(t1b) != (__float_as_uint(q1b) ^ 0x80000000u)) {
+            atomicAdd(&g_selftest_count, 1ull);  // both halves and both forms must agree up to sign
         }
         bool diff;
         switch (which) {
             case 0: diff = __float_as_uint(q1) != __float_as_uint(ref); break;
             case 5: diff = fabsf(ref) >= 1.17549435e-38f && __float_as_uint(q1) != __float_as_uint(ref); break;
             case 1: diff = __float_as_uint(div_scale2(a, s, r)) != __float_as_uint(ref); break;
-            case 2: diff = e4m3x2(q1, 0.0f) != e4m3x2(ref, 0.0f); break;
+            case 2: {
+                const uint32_t c = e4m3x2(ref, 0.0f);
+                diff = e4m3x2(q1, 0.0f) != c || (e4m3x2(t1, 0.0f) ^ 0x80u) != c;
+                break;
+            }
             default: {
-                const float v1[8] = {q1, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                const float v1[8] = {q1, t1, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
                 const float v2[8] = {ref, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                diff = (e2m1x8(v1) & 0xfu) != (e2m1x8(v2) & 0xfu);
+                const uint32_t c1 = e2m1x8(v1), c2 = e2m1x8(v2) & 0xfu;
+                diff = (c1 & 0xfu) != c2 || (((c1 >> 4) & 0xfu) ^ 0x8u) != c2;
             }
         }
         bad += diff ? 1ull : 0ull;
@@ -369,13 +410,7 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
 #define KVQ_LAUNCH_CT(M, GG)                                                                   \
     do {                                                                                       \
         auto k = compress_tma_kernel<M, GG>;                                                   \
-        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
-            return KVQ_ERR_CUDA;                                                               \
-        int occ = 0;                                                                           \
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, threads, smem) != cudaSuccess || occ < 1) \
-            occ = 1;                                                                           \
-        const int64_t cap = (int64_t)sm_count() * occ;                                         \
-        k<<<(unsigned)(tiles < cap ? tiles : cap), threads, smem, s>>>(a);                    \
+        k<<<(unsigned)persistent_grid(k, threads, tiles, smem), threads, smem, s>>>(a);        \
     } while (0)
         if (quant_mode == 0) KVQ_LAUNCH_CT(0, 64);
         else if (quant_mode == 1) KVQ_LAUNCH_CT(1, 64);
@@ -447,39 +482,41 @@ kvq_status kvq_indexer_quant_cache(const kvq_tensor* x, kvq_tensor* cache, kvq_t
     a.x_row_stride = rs;
     a.T = T;
     a.d = (int32_t)d;
-    a.nchunks = (int32_t)((d + 7) / 8);
-    a.x_f16 = x->dtype == KVQ_F16;
-    a.x_vec = (reinterpret_cast<uintptr_t>(x->data) % 16 == 0) && ((rs * 2) % 16 == 0);
+    a.ngroups = (int32_t)((d + 31) / 32);
+    a.team_shift = 0;
+    while ((1 << a.team_shift) < a.ngroups && a.team_shift < 5) ++a.team_shift;
+    const uintptr_t xa = reinterpret_cast<uintptr_t>(x->data);
+    a.x_vec = (xa % 32 == 0 && (rs * 2) % 32 == 0) ? 2 : ((xa % 16 == 0 && (rs * 2) % 16 == 0) ? 1 : 0);
     a.slots = slot_mapping->data;
     a.slots_i64 = slot_mapping->dtype == KVQ_I64;
     a.cache = crow;
     a.scale = srow;
-    a.e5m2 = cache->dtype == KVQ_F8E5M2;
-
-    int team = 32;
-    if (a.nchunks <= 4) team = 4;
-    else if (a.nchunks <= 8) team = 8;
-    else if (a.nchunks <= 16) team = 16;
+    a.code_vec32 = (reinterpret_cast<uintptr_t>(cache->data) % 32 == 0) && crow.row_bytes % 32 == 0 &&
+                   crow.block_stride % 32 == 0;
+    const bool f16 = x->dtype == KVQ_F16, e5m2 = cache->dtype == KVQ_F8E5M2;
+    const int64_t passes = (T + (32 >> a.team_shift) - 1) / (32 >> a.team_shift);
+    const int64_t need = (passes + (IX_THREADS / 32) - 1) / (IX_THREADS / 32);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-#define KVQ_LAUNCH_IX(M, TM)                                                                   \
+#define KVQ_LAUNCH_IX(M, F, E)                                                                 \
     do {                                                                                       \
-        constexpr int rps = 32 / TM, u = (32 / rps) < 8 ? (32 / rps) : 8;                      \
-        const int64_t tiles = (T + rps * u - 1) / (rps * u);                                   \
-        const int64_t need = (tiles + (IX_THREADS / 32) - 1) / (IX_THREADS / 32);              \
-        auto k = indexer_quant_kernel<M, TM>;                                                  \
+        auto k = indexer_quant_kernel<M, F, E>;                                                \
         k<<<(unsigned)persistent_grid(k, IX_THREADS, need), IX_THREADS, 0, s>>>(a);             \
     } while (0)
-#define KVQ_LAUNCH_IX_TEAM(M)                                                                  \
+#define KVQ_LAUNCH_IX_FE(M)                                                                    \
     do {                                                                                       \
-        if (team == 4) KVQ_LAUNCH_IX(M, 4);                                                    \
-        else if (team == 8) KVQ_LAUNCH_IX(M, 8);                                               \
-        else if (team == 16) KVQ_LAUNCH_IX(M, 16);                                             \
-        else KVQ_LAUNCH_IX(M, 32);                                                             \
+        if (f16) {                                                                             \
+            if (e5m2) KVQ_LAUNCH_IX(M, true, true);                                            \
+            else KVQ_LAUNCH_IX(M, true, false);                                                \
+        } else {                                                                               \
+            if (e5m2) KVQ_LAUNCH_IX(M, false, true);                                           \
+            else KVQ_LAUNCH_IX(M, false, false);                                               \
+        }                                                                                      \
     } while (0)
-    if (quant_mode == 0) KVQ_LAUNCH_IX_TEAM(0);
-    else if (quant_mode == 1) KVQ_LAUNCH_IX_TEAM(1);
-    else KVQ_LAUNCH_IX_TEAM(3);
-#undef KVQ_LAUNCH_IX_TEAM
+    if (quant_mode == 0) KVQ_LAUNCH_IX_FE(0);
+    else if (quant_mode == 1) KVQ_LAUNCH_IX_FE(1);
+    else if (f16) KVQ_LAUNCH_IX(3, true, false);
+    else KVQ_LAUNCH_IX(3, false, false);
+#undef KVQ_LAUNCH_IX_FE
 #undef KVQ_LAUNCH_IX
     return launched();
 }
@@ -738,33 +775,42 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
     const bool aligned = reinterpret_cast<uintptr_t>(x->data) % 16 == 0 &&
                          reinterpret_cast<uintptr_t>(cos->data) % 16 == 0 &&
                          reinterpret_cast<uintptr_t>(sin->data) % 16 == 0 && (D * 2) % 16 == 0;
-    if (aligned) {
-        // pipelined kernel: token rows, cos and sin arrive in shared memory by bulk copy
-        a.tps = (int32_t)(H * xb <= 8192 ? 2 : 1);
+    const int E = (int)(D / 32);
+    if (aligned && (E == 2 || E == 4 || E == 8)) {
+        // pipelined kernel: token rows, cos and sin arrive in shared memory by
+        // bulk copy; TPS tokens per stage (a divisor of the consumer warps,
+        // x span at most 32 KB), as many stages (2..4) as keep two CTAs on an SM
+        int tps = 1;
+        while (tps < DT_CONSUMERS && 2 * tps * H * xb <= 32768) tps *= 2;
+        a.tps = tps;
+        auto dt_smem = [&](int stages) {
+            return (size_t)dt_header_bytes(stages, tps) + (size_t)stages * dt_stage_bytes(tps, H, xb, (int)D);
+        };
         a.stages = 4;
-        const size_t smem = dt_header_bytes(a.stages, a.tps) + (size_t)a.stages * dt_stage_bytes(a.tps, H, xb, (int)D);
+        while (a.stages > 2 && dt_smem(a.stages) > 112 * 1024) --a.stages;
+        const size_t smem = dt_smem(a.stages);
         const int64_t tiles = (need + a.tps - 1) / a.tps;
-#define KVQ_LAUNCH_DT(E)                                                                       \
+        const bool f16 = a.cos_f16 != 0;
+#define KVQ_LAUNCH_DT(EE, XK, F)                                                               \
     do {                                                                                       \
-        auto k = dequant_rope_quant_tma_kernel<E>;                                             \
-        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
-            return KVQ_ERR_CUDA;                                                               \
-        int occ = 0;                                                                           \
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, DT_THREADS, smem) != cudaSuccess || occ < 1) \
-            occ = 1;                                                                           \
-        const int64_t cap = (int64_t)sm_count() * occ;                                         \
-        k<<<(unsigned)(tiles < cap ? tiles : cap), DT_THREADS, smem, s>>>(a);                 \
+        auto k = dequant_rope_quant_tma_kernel<EE, XK, F>;                                     \
+        k<<<(unsigned)persistent_grid(k, DT_THREADS, tiles, smem), DT_THREADS, smem, s>>>(a);  \
     } while (0)
-        switch (D / 32) {
-            case 1: KVQ_LAUNCH_DT(1); break;
-            case 2: KVQ_LAUNCH_DT(2); break;
-            case 3: KVQ_LAUNCH_DT(3); break;
-            case 4: KVQ_LAUNCH_DT(4); break;
-            case 5: KVQ_LAUNCH_DT(5); break;
-            case 6: KVQ_LAUNCH_DT(6); break;
-            case 7: KVQ_LAUNCH_DT(7); break;
-            default: KVQ_LAUNCH_DT(8); break;
+#define KVQ_LAUNCH_DT_E(XK, F)                                                                 \
+    do {                                                                                       \
+        if (E == 2) KVQ_LAUNCH_DT(2, XK, F);                                                   \
+        else if (E == 4) KVQ_LAUNCH_DT(4, XK, F);                                              \
+        else KVQ_LAUNCH_DT(8, XK, F);                                                          \
+    } while (0)
+        if (a.x_kind == 0) {
+            if (f16) KVQ_LAUNCH_DT_E(0, true);
+            else KVQ_LAUNCH_DT_E(0, false);
+        } else if (a.x_kind == 1) {
+            KVQ_LAUNCH_DT_E(1, false);
+        } else {
+            KVQ_LAUNCH_DT_E(2, true);
         }
+#undef KVQ_LAUNCH_DT_E
 #undef KVQ_LAUNCH_DT
         return launched();
     }

@@ -179,6 +179,34 @@ __device__ __forceinline__ void div_scale1_x2(float a0, float a1, float s, float
     q1 = with_sign_of(q1, a1);
 }
 
+// The same one-step quotient, negated, on a pair: nq = RN(a * -r) = -q0,
+// rem = RN(a + s nq) = a - s q0 (exact under the fused operation), and
+// t = RN(rem * -r + nq) = -RN(q0 + rem r).  t is exactly -(div_scale1(a)),
+// signed zeros included (a zero numerator gives t = -0 for a = +0 and +0 for
+// a = -0), so the sign fix of div_scale1 is not needed: callers encode t and
+// flip the code's sign bit, which for the symmetric round-to-nearest-even,
+// saturating FP8 / FP4 encodings equals encoding -t.
+__device__ __forceinline__ void div_scale1_neg_x2(float a0, float a1, float s, float r, float& t0, float& t1) {
+    asm("{\n\t.reg .b64 a, nq, rem, nr, ss;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 nr, {%4, %4};\n\t"
+        "mov.b64 ss, {%5, %5};\n\t"
+        "mul.rn.f32x2 nq, a, nr;\n\t"
+        "fma.rn.f32x2 rem, nq, ss, a;\n\t"
+        "fma.rn.f32x2 nq, rem, nr, nq;\n\t"
+        "mov.b64 {%0, %1}, nq;\n\t}"
+        : "=f"(t0), "=f"(t1)
+        : "f"(a0), "f"(a1), "f"(-r), "f"(s));
+}
+
+// Largest magnitude of the two bf16 halves of a and b, per half (max of the
+// absolute values; the sign bits of the result are not meaningful).
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 // eight quotients f[i] / s through div_scale1_x2
 __device__ __forceinline__ void div_scale8(const float (&f)[8], float s, float r, float (&q)[8]) {
 #pragma unroll
@@ -271,6 +299,53 @@ __device__ __forceinline__ void st_partial(uint8_t* p, uint4 v, int nbytes) {
         if (k < nbytes) p[k] = (uint8_t)(w[k >> 2] >> (8 * (k & 3)));
 }
 
+// 32 16-bit values (64 bytes) at p as 16 words (value 2i in the low half of word i).
+__device__ __forceinline__ void ld_slice(const uint16_t* p, int vec, uint32_t (&w)[16]) {
+    if (vec == 2) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            asm("ld.global.nc.L1::no_allocate.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                : "=r"(w[8 * h]), "=r"(w[8 * h + 1]), "=r"(w[8 * h + 2]), "=r"(w[8 * h + 3]), "=r"(w[8 * h + 4]),
+                  "=r"(w[8 * h + 5]), "=r"(w[8 * h + 6]), "=r"(w[8 * h + 7])
+                : "l"(p + 16 * h));
+    } else if (vec == 1) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint4 v = ld_stream16(p + 8 * k);
+            w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = (uint32_t)__ldcs(p + 2 * i) | ((uint32_t)__ldcs(p + 2 * i + 1) << 16);
+    }
+}
+
+// 32 bytes at p (8 words, little-endian).
+__device__ __forceinline__ void st_32B(uint8_t* p, const uint32_t* w, bool vec32) {
+    if (vec32) {
+        asm volatile("st.global.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+                     "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                     : "memory");
+    } else {
+        st_b128(p, make_uint4(w[0], w[1], w[2], w[3]));
+        st_b128(p + 16, make_uint4(w[4], w[5], w[6], w[7]));
+    }
+}
+
+// |x| maximum (as bf16 bits) of the 2*N values in words w[i0 .. i0+N)
+template <int N>
+__device__ __forceinline__ uint32_t absmax_words(const uint32_t (&w)[16], int i0) {
+    const uint32_t msk = 0x7fff7fffu;
+    uint32_t m = w[i0] & msk;
+#pragma unroll
+    for (int i = 1; i < N; ++i) m = __vmaxu2(m, w[i0 + i] & msk);
+    return max(m & 0xffffu, m >> 16);
+}
+
+__device__ __forceinline__ int64_t load_slot(const void* slots, int is64, int64_t i) {
+    return is64 ? reinterpret_cast<const int64_t*>(slots)[i] : (int64_t) reinterpret_cast<const int32_t*>(slots)[i];
+}
+
 // ---------------------------------------------------------------------------
 // Paged cache rows: slot s -> block s / block_size, row s % block_size.
 // ---------------------------------------------------------------------------
@@ -280,9 +355,14 @@ struct PagedRows {
     int64_t block_size;
     int64_t row_bytes;
     int64_t block_stride;  // bytes
+    int32_t bs_shift;      // log2(block_size) when block_size is a power of two, else -1
 };
 
 __device__ __forceinline__ uint8_t* slot_row(const PagedRows& c, int64_t s) {
+    if (c.bs_shift >= 0) {
+        const int64_t blk = s >> c.bs_shift;
+        return c.base + blk * c.block_stride + (s & (c.block_size - 1)) * c.row_bytes;
+    }
     if (c.num_slots <= 0x7fffffff) {
         const uint32_t us = (uint32_t)s, bs = (uint32_t)c.block_size;
         const uint32_t blk = us / bs;
