@@ -11,8 +11,10 @@ reads 604 MB of input -- more than the 126 MB L2 -- and needs no L2 flush.
 
 value = token rows quantised per second over all ranks (2 x 262144 per step and
 GPU); the roofline object reports the dominant kernel's algorithmic HBM bytes
-per launch over its CUDA-event duration.  The other four workloads are timed
-once each (L2 flushed before every launch) and reported under "per_config".
+per launch over its CUDA-event duration.  Every workload is also timed on its
+own under "per_config": back-to-back launches cycling through enough input
+copies that their bytes exceed twice the L2 size (one copy, L2-resident, for
+the latency-bound decode-sized workloads).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -41,11 +43,6 @@ WORKLOAD = ("kv_compress_epilog large sweep: T=262144 tokens, d=576 bf16 N(0,1) 
             "bf16 scale, rope FP8 E4M3 static x_scale=0.1, 352-B rows); cache blockSize=128, 4096 blocks; "
             "2% slot_mapping -1")
 FALLBACK_HBM_GBS = 6650.0
-# A single timed launch is preceded by a device-side wait of this many SM
-# cycles (~100 us), so that the host has enqueued the start event, the launch
-# and the stop event before the GPU reaches the start event: the events then
-# bracket device time only, not the host's call overhead.
-HOST_LEAD_CYCLES = 200_000
 
 
 # ---------------------------------------------------------------------------
@@ -260,30 +257,55 @@ def run_reference(args):
     return 0
 
 
+def rotation(case, make, l2_bytes: int):
+    """Device copies of a workload to cycle through so that consecutive launches
+    find their inputs out of L2: enough copies that their algorithmic bytes add
+    up to twice the L2 size (at most 16).  Workloads under 4 MB are latency-
+    bound and run on one copy (L2-resident)."""
+    from kv_cache_quantize_b200 import workloads as W
+    nb = algorithmic_bytes(case)
+    k = 1 if nb < (4 << 20) else min(16, max(1, -(-2 * l2_bytes // nb)))
+    calls = [W.build_call(case)[0]]
+    for _ in range(k - 1):
+        calls.append(W.build_call(make())[0])
+    return calls
+
+
+def device_us_per_launch(calls, stream, reps: int) -> float:
+    """Mean device time of one launch over `reps` back-to-back launches that
+    cycle through `calls`.  A device-side wait long enough for the host to
+    enqueue every launch precedes the start event, so the events bracket
+    device time only (no host call overhead, no idle gaps)."""
+    import torch
+    t0 = time.perf_counter()
+    for i in range(3 * len(calls)):
+        calls[i % len(calls)](stream)
+    host_s = (time.perf_counter() - t0) / (3 * len(calls))
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(2.0e9 * (2.0 * host_s * reps + 50e-6)))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(reps):
+        calls[i % len(calls)](stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return 1e3 * e0.elapsed_time(e1) / reps
+
+
 def run_profile_workload(args):
     """Run one named workload a few times (for ncu captures of a single kernel)."""
     import torch
     import kv_cache_quantize_b200 as kvq
     from kv_cache_quantize_b200 import workloads as W
-    case = W.CONFIGS[args.profile_workload]()
-    call, _, _ = W.build_call(case)
+    make = W.CONFIGS[args.profile_workload]
+    case = make()
+    calls = rotation(case, make, torch.cuda.get_device_properties(0).L2_cache_size)
     stream = torch.cuda.current_stream()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    times = []
-    for i in range(args.profile_reps):
-        flush.fill_(i & 0xFF)
-        torch.cuda._sleep(HOST_LEAD_CYCLES)       # the host enqueues the launch before the GPU reaches e0
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        call(stream)
-        e1.record(stream)
-        times.append((e0, e1))
-    torch.cuda.synchronize()
+    us = device_us_per_launch(calls, stream, args.profile_reps)
     if kvq.get_error(stream) != 0:
         raise RuntimeError("device fault bits set")
-    us = [1e3 * a.elapsed_time(b) for a, b in times]
-    print(f"{args.profile_workload}: {len(us)} launches, median {statistics.median(us):.1f} us, "
-          f"{algorithmic_bytes(case) / statistics.median(us) / 1e3:.0f} GB/s algorithmic")
+    print(f"{args.profile_workload}: {args.profile_reps} launches over {len(calls)} input copies, "
+          f"{us:.1f} us per launch, {algorithmic_bytes(case) / us / 1e3:.0f} GB/s algorithmic")
     return 0
 
 
@@ -297,8 +319,8 @@ def main():
     ap.add_argument("--no-per-config", action="store_true", help="skip the per-workload breakdown")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing for cpu_baseline")
     ap.add_argument("--profile-workload", default=None,
-                    help="profiling mode: run only this named workload --profile-reps times (L2 flushed "
-                         "before each launch) and print its median launch time; no JSON line")
+                    help="profiling mode: run only this named workload --profile-reps times (back to back, "
+                         "cycling input copies larger than L2) and print its time per launch; no JSON line")
     ap.add_argument("--profile-reps", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -434,31 +456,19 @@ def main():
     per_config = None
     if rank == 0 and not args.no_per_config:
         per_config = {}
-        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         for name, make in W.CONFIGS.items():
             case = {"cfg5a_compress_mode0": case_a, "cfg5b_compress_mode2": case_b}.get(name) or make()
-            call, _, _ = W.build_call(case)
-            reps = 50
-            times = []
-            for i in range(reps + 3):
-                flush.fill_(i & 0xFF)                 # evict the previous launch's data from L2
-                torch.cuda._sleep(HOST_LEAD_CYCLES)   # the launch is enqueued before the GPU reaches e0
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                call(stream)
-                e1.record(stream)
-                if i >= 3:
-                    times.append((e0, e1))
-            torch.cuda.synchronize(dev)
-            us = sorted(1e3 * a.elapsed_time(b) for a, b in times)
-            med = statistics.median(us) / 1e6
+            calls = rotation(case, make, l2)
+            us = device_us_per_launch(calls, stream, 200)
             nb = algorithmic_bytes(case)
-            per_config[name] = {"tokens": token_rows(case), "alg_bytes": nb, "median_us": med * 1e6,
-                                "tokens_per_s": token_rows(case) / med, "alg_GBps": nb / med / 1e9,
-                                "frac_of_peak": nb / med / 1e9 / peak}
-            del call, case
+            per_config[name] = {"tokens": token_rows(case), "alg_bytes": nb, "us_per_launch": us,
+                                "tokens_per_s": token_rows(case) / us * 1e6, "alg_GBps": nb / us / 1e3,
+                                "frac_of_peak": nb / us / 1e3 / peak, "input_copies": len(calls),
+                                "l2": ("L2-resident (latency-bound)" if nb < (4 << 20) else
+                                       f"{len(calls)} input copies cycled, {len(calls) * nb >> 20} MB > L2")}
+            del calls, case
             torch.cuda.empty_cache()
-        del flush
 
     # ---------------- CPU oracle baseline (rank 0, N = 1) ----------------
     cpu = None

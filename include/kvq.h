@@ -254,8 +254,12 @@ KVQ_API kvq_status kvq_convert(int32_t fmt, const float* in, int64_t n, void* ou
  * differs from the code of the IEEE quotient; 4: the number of positive
  * finite bf16 and f16 values a for which the constant-divisor form of a / 448,
  * a / 57344 or a / 6 differs from IEEE division; 5: as 0 but counting only
- * pairs whose IEEE quotient is a normal binary32 number.  Blocks until done;
- * *result receives the count (0 means the shortcut is exact on the domain). */
+ * pairs whose IEEE quotient is a normal binary32 number; 6: the number of
+ * groups of four, among 2^28 random (value, scale, offset) triples (half of
+ * them within a few ulps of a rounding tie), whose static int8 codes from the
+ * dequant kernel's reciprocal-based quotient differ from those of IEEE
+ * division.  Blocks until done; *result receives the count (0 means the
+ * shortcut is exact on the domain). */
 KVQ_API kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream);
 
 /* Static description of a status code. */

@@ -271,22 +271,33 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) dequant_rope_quant_kernel(const
 }
 
 // ---------------------------------------------------------------------------
-// Pipelined kernel (16-byte aligned x, cos and sin; D = 32 E with E = 2, 4 or
-// 8).  CTA = DT_CONSUMERS consumer warps + 1 producer warp.  A stage holds TPS
-// consecutive tokens: their x rows, cos rows and sin rows arrive by three bulk
-// copies (each a contiguous span); the producer resolves the tokens'
-// destination slots and activation scales one stage ahead and stores them
-// next to the stage.  Consumers: the warps are split evenly over the stage's
-// tokens, and the warps of one token split its Nq + 2 Nkv heads into
-// contiguous ranges, which they walk two heads per pass (lane l holds values
-// [E l, E l + E) of both heads, so a value's half-rotation partner is
-// __shfl_xor(16) away and both heads share the lane's cos / sin values).
+// Pipelined kernel (16-byte aligned x, cos and sin).  CTA = DT_CONSUMERS
+// consumer warps + 1 producer warp.  A stage holds TPS consecutive tokens:
+// their x rows, cos rows and sin rows arrive by three bulk copies (each a
+// contiguous span); the producer resolves the tokens' destination slots and
+// activation scales one stage ahead and stores them next to the stage.  The
+// per-channel parameters (weight scale, bias, the k / v scales and offsets)
+// are staged in shared memory once per CTA as binary32.
+//
+// Lane layout: a head of D values is L = D/8 lanes; lane l of a head holds the
+// four values [4l, 4l + 4) and their half-rotation partners [D/2 + 4l,
+// D/2 + 4l + 4), so RoPE needs no shuffle, and a warp holds 32/L heads side by
+// side (a PASS).  The stage's passes (TPS tokens x ceil(NH / (32/L)) passes,
+// token-major) are dealt to the consumer warps round-robin, which spreads the
+// costlier k / v passes (int8 quantisation) evenly; a warp widens a token's
+// cos / sin when it moves to that token.
 // ---------------------------------------------------------------------------
 constexpr int DT_CONSUMERS = 8;
 constexpr int DT_THREADS = (DT_CONSUMERS + 1) * 32;
 
 __host__ __device__ inline uint32_t dt_header_bytes(int stages, int tps) {
     return ((uint32_t)(16 * stages + 12 * stages * tps) + 127u) & ~127u;
+}
+
+// binary32 parameters: weight scale and bias [H] (int32 x only), then the k and
+// v scales, offsets and scale reciprocals [C = Nkv * D]
+__host__ __device__ inline uint32_t dt_param_bytes(int64_t H, int64_t C, bool dq) {
+    return (uint32_t)(((dq ? 8 * H : 0) + 24 * C + 127) & ~127);
 }
 
 __host__ __device__ inline uint32_t dt_stage_bytes(int tps, int64_t H, int x_bytes, int D) {
@@ -313,139 +324,109 @@ __device__ __forceinline__ int64_t dq_resolve(const DrqArgs& a, int64_t t, int64
     return b * c1 + raw + s;
 }
 
-// E consecutive 16-bit floats from shared memory, widened
-template <int E, bool F16>
-__device__ __forceinline__ void dt_lds16(const uint16_t* p, float (&v)[E]) {
-    uint32_t w[E / 2];
-    if (E % 8 == 0) {
-#pragma unroll
-        for (int k = 0; k < E / 8; ++k) {
-            const uint4 q = *reinterpret_cast<const uint4*>(p + 8 * k);
-            w[4 * k] = q.x; w[4 * k + 1] = q.y; w[4 * k + 2] = q.z; w[4 * k + 3] = q.w;
-        }
-    } else if (E % 4 == 0) {
-        const uint2 q = *reinterpret_cast<const uint2*>(p);
-        w[0] = q.x; w[1] = q.y;
-    } else {
-#pragma unroll
-        for (int k = 0; k < E / 2; ++k) w[k] = reinterpret_cast<const uint32_t*>(p)[k];
-    }
-#pragma unroll
-    for (int k = 0; k < E / 2; ++k) {
-        v[2 * k] = F16 ? f16_lo(w[k]) : bf16_lo(w[k]);
-        v[2 * k + 1] = F16 ? f16_hi(w[k]) : bf16_hi(w[k]);
-    }
+// four 16-bit floats from shared memory, widened
+template <bool F16>
+__device__ __forceinline__ void dt_lds4h(const uint16_t* p, float (&v)[4]) {
+    const uint2 q = *reinterpret_cast<const uint2*>(p);
+    v[0] = F16 ? f16_lo(q.x) : bf16_lo(q.x);
+    v[1] = F16 ? f16_hi(q.x) : bf16_hi(q.x);
+    v[2] = F16 ? f16_lo(q.y) : bf16_lo(q.y);
+    v[3] = F16 ? f16_hi(q.y) : bf16_hi(q.y);
 }
 
-// E consecutive int32 values from shared memory, converted to binary32
-template <int E>
-__device__ __forceinline__ void dt_lds_i32(const int32_t* p, float (&v)[E]) {
-    if (E % 4 == 0) {
-#pragma unroll
-        for (int k = 0; k < E; k += 4) {
-            const int4 q = *reinterpret_cast<const int4*>(p + k);
-            v[k] = __int2float_rn(q.x); v[k + 1] = __int2float_rn(q.y);
-            v[k + 2] = __int2float_rn(q.z); v[k + 3] = __int2float_rn(q.w);
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < E; k += 2) {
-            const int2 q = *reinterpret_cast<const int2*>(p + k);
-            v[k] = __int2float_rn(q.x); v[k + 1] = __int2float_rn(q.y);
-        }
-    }
+__device__ __forceinline__ void dt_lds4i(const int32_t* p, float (&v)[4]) {
+    const int4 q = *reinterpret_cast<const int4*>(p);
+    v[0] = __int2float_rn(q.x); v[1] = __int2float_rn(q.y);
+    v[2] = __int2float_rn(q.z); v[3] = __int2float_rn(q.w);
 }
 
-// E binary32 parameters at p (16-byte vectors when vec and E % 4 == 0)
-template <int E>
-__device__ __forceinline__ void dt_param(const float* p, bool vec, float (&v)[E]) {
-    if (E % 4 == 0 && vec) {
-#pragma unroll
-        for (int k = 0; k < E; k += 4) {
-            const float4 q = __ldg(reinterpret_cast<const float4*>(p + k));
-            v[k] = q.x; v[k + 1] = q.y; v[k + 2] = q.z; v[k + 3] = q.w;
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < E; ++k) v[k] = __ldg(p + k);
-    }
+__device__ __forceinline__ void dt_lds4f(const float* p, float (&v)[4]) {
+    const float4 q = *reinterpret_cast<const float4*>(p);
+    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
 }
 
-// E values rounded to 16-bit floats, packed two per word, stored at p
-template <int E, bool F16>
-__device__ __forceinline__ void dt_store16(uint16_t* p, const float (&o)[E]) {
-    uint32_t w[E / 2];
-#pragma unroll
-    for (int k = 0; k < E / 2; ++k) {
-        if (F16) {
-            asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w[k]) : "f"(o[2 * k + 1]), "f"(o[2 * k]));
-        } else {
-            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[k]) : "f"(o[2 * k + 1]), "f"(o[2 * k]));
-        }
-    }
-    uint8_t* b = reinterpret_cast<uint8_t*>(p);
-    if (E % 8 == 0) {
-#pragma unroll
-        for (int k = 0; k < E / 8; ++k) st_b128(b + 16 * k, make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]));
-    } else if (E % 4 == 0) {
-        st_b64(b, make_uint2(w[0], w[1]));
+// four values rounded to 16-bit floats, stored (8 bytes) at p
+template <bool F16>
+__device__ __forceinline__ void dt_store4h(uint16_t* p, const float (&o)[4]) {
+    uint32_t w0, w1;
+    if (F16) {
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w0) : "f"(o[1]), "f"(o[0]));
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w1) : "f"(o[3]), "f"(o[2]));
     } else {
-#pragma unroll
-        for (int k = 0; k < E / 2; ++k) st_b32(b + 4 * k, w[k]);
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w0) : "f"(o[1]), "f"(o[0]));
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w1) : "f"(o[3]), "f"(o[2]));
     }
+    st_b64(reinterpret_cast<uint8_t*>(p), make_uint2(w0, w1));
 }
 
-// Output stage of one head (o: the head's values after dequant and RoPE):
-// q heads -> qOut; k / v heads -> kOut / vOut when requested, then static
-// int8 quantisation (Div -> Add offset -> round half to even, saturate) into
-// the cache row.
-template <int E, bool F16>
-__device__ __forceinline__ void dt_head_out(const DrqArgs& a, int64_t t, int hd, int pos, const float (&o)[E],
-                                            uint8_t* krow, uint8_t* vrow, bool pv) {
-    const int D = a.D;
-    if (hd < a.Nq) {
-        dt_store16<E, F16>(a.q_out + t * (int64_t)(a.Nq * D) + hd * D + pos, o);
-        return;
-    }
-    const bool is_k = hd < a.Nq + a.Nkv;
-    const int c0 = (is_k ? hd - a.Nq : hd - a.Nq - a.Nkv) * D + pos;   // channel in [0, Nkv*D)
-    if (a.k_out) dt_store16<E, F16>((is_k ? a.k_out : a.v_out) + t * (int64_t)(a.Nkv * D) + c0, o);
-    uint8_t* row = is_k ? krow : vrow;
-    if (row == nullptr) return;
-    float sc[E], of[E];
-    dt_param<E>((is_k ? a.scale_k : a.scale_v) + c0, pv, sc);
-    const float* ofp = is_k ? a.offset_k : a.offset_v;
-    if (ofp) dt_param<E>(ofp + c0, pv, of);
-    uint32_t packed[E / 4 > 0 ? E / 4 : 1];
-#pragma unroll
-    for (int k = 0; k < (E + 3) / 4; ++k) packed[k] = 0u;
-#pragma unroll
-    for (int k = 0; k < E; ++k) {
-        float q = __fdiv_rn(o[k], sc[k]);
-        if (ofp) q = __fadd_rn(q, of[k]);
-        packed[k / 4] |= ((uint32_t)int8_rne_sat(q) & 0xffu) << (8 * (k % 4));
-    }
-    if (E % 4 == 0) {
-#pragma unroll
-        for (int k = 0; k < E / 4; ++k) st_b32(row + c0 + 4 * k, packed[k]);
+// Static int8 of four values: round half to even of o / scale + offset,
+// saturated (offset 0 when absent), packed little-endian.  r holds RN(1/scale)
+// for channels whose scale lies in [2^-60, 2^60] and whose |offset| <= 2^16,
+// else 0.  When every r is set and every |o| <= 2^60 the quotient comes
+// from the two-step Markstein form, which is then exact wherever the result
+// depends on it: a quotient in [2^-30, 2^20] has normal operands, residuals
+// and result, so it equals the IEEE quotient; below 2^-30 the rounded sum
+// with any binary32 offset, hence the integer, does not depend on the
+// quotient's last bits; above 2^20 the integer saturates either way.  Other
+// lanes divide with IEEE division.  kvq_selftest checks the two paths against
+// each other on random and near-tie triples.
+__device__ __forceinline__ uint32_t int8x4_quant(const float (&o)[4], const float (&s)[4], const float (&f)[4],
+                                                 const float (&r)[4]) {
+    float q[4];
+    const uint32_t lim = 0x5d800000u;     // 2^60
+    const bool fast = r[0] != 0.0f && r[1] != 0.0f && r[2] != 0.0f && r[3] != 0.0f &&
+                      (__float_as_uint(o[0]) & 0x7fffffffu) <= lim && (__float_as_uint(o[1]) & 0x7fffffffu) <= lim &&
+                      (__float_as_uint(o[2]) & 0x7fffffffu) <= lim && (__float_as_uint(o[3]) & 0x7fffffffu) <= lim;
+    if (fast) {
+        div2_add_x2(o[0], o[1], s[0], s[1], r[0], r[1], f[0], f[1], q[0], q[1]);
+        div2_add_x2(o[2], o[3], s[2], s[3], r[2], r[3], f[2], f[3], q[2], q[3]);
     } else {
-        st_b16(row + c0, packed[0]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) q[k] = __fadd_rn(__fdiv_rn(o[k], s[k]), f[k]);
     }
+    return int8x4_rne_sat(q[0], q[1], q[2], q[3]);
+}
+
+// RN(1/scale) where the fast quotient of int8x4_quant applies, else 0
+__device__ __forceinline__ float int8_quant_rcp(float sc, float of) {
+    const uint32_t e = (__float_as_uint(sc) >> 23) & 0xffu;
+    const bool ok = sc > 0.0f && e >= 67u && e <= 187u && fabsf(of) <= 65536.0f;
+    return ok ? __frcp_rn(sc) : 0.0f;
+}
+
+__device__ __forceinline__ uint32_t dt_int8x4(const float (&o)[4], const float* sc, const float* of, const float* rc) {
+    float s[4], f[4], r[4];
+    dt_lds4f(sc, s);
+    dt_lds4f(of, f);
+    dt_lds4f(rc, r);
+    return int8x4_quant(o, s, f, r);
 }
 
 // XK: 0 int32 x (dequantised), 1 bf16 x, 2 f16 x.  F16: cos / sin and the
 // 16-bit outputs are f16 (else bf16).
-template <int E, int XK, bool F16>
+template <int XK, bool F16>
 __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(const DrqArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     const int S = a.stages, TPS = a.tps, D = a.D;
     constexpr int XB = XK == 0 ? 4 : 2;
+    constexpr bool DQ = XK == 0;
+    const int64_t H = a.H;
+    const int C = a.Nkv * D;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + S;
     int64_t* slots = reinterpret_cast<int64_t*>(empty + S);
     float* acts = reinterpret_cast<float*>(slots + S * TPS);
-    uint8_t* stages = smem + dt_header_bytes(S, TPS);
-    const uint32_t x_span = (uint32_t)((TPS * a.H * XB + 127) & ~127);
+    float* prm = reinterpret_cast<float*>(smem + dt_header_bytes(S, TPS));
+    float* p_ws = prm;                      // [H]  (int32 x)
+    float* p_bias = prm + H;                // [H]  (int32 x; -0.0, the exact additive identity, when absent)
+    float* p_sk = prm + (DQ ? 2 * H : 0);   // [C]
+    float* p_sv = p_sk + C;
+    float* p_ok = p_sv + C;                 // [C] (0 when absent)
+    float* p_ov = p_ok + C;
+    float* p_rk = p_ov + C;                 // [C] RN(1/scale) where the fast quotient applies, else 0
+    float* p_rv = p_rk + C;
+    uint8_t* stages = smem + dt_header_bytes(S, TPS) + dt_param_bytes(H, C, DQ);
+    const uint32_t x_span = (uint32_t)((TPS * H * XB + 127) & ~127);
     const uint32_t cs_span = (uint32_t)((TPS * D * 2 + 127) & ~127);
     const uint32_t stage_bytes = x_span + 2 * cs_span;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -459,6 +440,20 @@ __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(cons
         }
         mbar_init_fence();
     }
+    if (DQ) {
+        for (int64_t i = threadIdx.x; i < H; i += blockDim.x) {
+            p_ws[i] = a.weight_scale[i];
+            p_bias[i] = a.bias ? dq_bias(a, i) : -0.0f;
+        }
+    }
+    for (int i = threadIdx.x; i < C; i += blockDim.x) {
+        p_sk[i] = a.scale_k[i];
+        p_sv[i] = a.scale_v[i];
+        p_ok[i] = a.offset_k ? a.offset_k[i] : 0.0f;
+        p_ov[i] = a.offset_v ? a.offset_v[i] : 0.0f;
+        p_rk[i] = int8_quant_rcp(p_sk[i], p_ok[i]);
+        p_rv[i] = int8_quant_rcp(p_sv[i], p_ov[i]);
+    }
     __syncthreads();
 
     if (warp == DT_CONSUMERS) {
@@ -471,7 +466,7 @@ __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(cons
             act = 1.0f;
             if (lane < TPS && tile < ntiles && t < ntok) {
                 raw = dq_index_raw(a, t);
-                if (XK == 0 && a.activation_scale) act = a.activation_scale[t];
+                if (DQ && a.activation_scale) act = a.activation_scale[t];
             }
         };
         int it = 0;
@@ -499,9 +494,9 @@ __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(cons
             __syncwarp();
             if (lane == 0) {
                 uint8_t* base = stages + (size_t)st * stage_bytes;
-                const uint32_t xbytes = (uint32_t)(toks * a.H * XB), cbytes = (uint32_t)(toks * D * 2);
+                const uint32_t xbytes = (uint32_t)(toks * H * XB), cbytes = (uint32_t)(toks * D * 2);
                 mbar_arrive_expect_tx(&full[st], xbytes + 2 * cbytes);
-                bulk_copy_g2s(base, reinterpret_cast<const uint8_t*>(a.x) + (size_t)t0 * a.H * XB, xbytes, &full[st]);
+                bulk_copy_g2s(base, reinterpret_cast<const uint8_t*>(a.x) + (size_t)t0 * H * XB, xbytes, &full[st]);
                 bulk_copy_g2s(base + x_span, a.cos + (size_t)t0 * D, cbytes, &full[st]);
                 bulk_copy_g2s(base + x_span + cs_span, a.sin + (size_t)t0 * D, cbytes, &full[st]);
             }
@@ -514,12 +509,12 @@ __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(cons
 
     // ---------------- consumers ----------------
     const int NH = a.Nq + 2 * a.Nkv;
-    const int WPT = DT_CONSUMERS / TPS;               // warps per token
-    const int my_tok = warp / WPT, wt = warp - my_tok * WPT;
-    const int h_begin = (NH * wt) / WPT, h_end = (NH * (wt + 1)) / WPT;
-    const int pos = lane * E;
-    const bool first_half = lane < 16;
-    const bool pv = a.params_vec != 0;
+    const int L = D >> 3;                     // lanes per head
+    const int HPW = 32 / L;                   // heads per pass
+    const int hl = lane / L, l = lane - hl * L;
+    const bool lane_on = hl < HPW;
+    const int NP = (NH + HPW - 1) / HPW;      // passes per token
+    const int j0 = 4 * l, j1 = (D >> 1) + 4 * l;
     int it = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
         const int st = it % S;
@@ -527,73 +522,88 @@ __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(cons
         if (!__all_sync(FULL_MASK, mbar_wait(&full[st], round & 1u))) break;
         const int64_t t0 = tile * TPS;
         const int toks = (int)(ntok - t0 < TPS ? ntok - t0 : TPS);
-        if (my_tok < toks) {
-            const int64_t t = t0 + my_tok;
-            const uint8_t* base = stages + (size_t)st * stage_bytes;
-            const int64_t slot = slots[st * TPS + my_tok];
-            const float act = acts[st * TPS + my_tok];
-            uint8_t* krow = slot >= 0 ? slot_row(a.kc, slot) : nullptr;
-            uint8_t* vrow = slot >= 0 ? slot_row(a.vc, slot) : nullptr;
-            // cos, and sin carrying the sign of the lane's half of the rotation
-            float cs[E], sn[E];
-            dt_lds16<E, F16>(reinterpret_cast<const uint16_t*>(base + x_span) + my_tok * D + pos, cs);
-            dt_lds16<E, F16>(reinterpret_cast<const uint16_t*>(base + x_span + cs_span) + my_tok * D + pos, sn);
-            if (first_half) {
+        const uint8_t* base = stages + (size_t)st * stage_bytes;
+        const int ntask = toks * NP;
+        int tok = -1;
+        int64_t t = 0;
+        float act = 1.0f;
+        uint8_t *krow = nullptr, *vrow = nullptr;
+        float ca[4], cb[4], nsa[4], sb[4];     // cos / sin at j0 (a) and j1 (b); nsa = -sin at j0
+        for (int task = warp; task < ntask; task += DT_CONSUMERS) {
+            const int tk = task / NP, p = task - tk * NP;
+            if (tk != tok) {
+                tok = tk;
+                t = t0 + tok;
+                const int64_t slot = slots[st * TPS + tok];
+                act = acts[st * TPS + tok];
+                krow = slot >= 0 ? slot_row(a.kc, slot) : nullptr;
+                vrow = slot >= 0 ? slot_row(a.vc, slot) : nullptr;
+                const uint16_t* cp = reinterpret_cast<const uint16_t*>(base + x_span) + tok * D;
+                const uint16_t* sp = reinterpret_cast<const uint16_t*>(base + x_span + cs_span) + tok * D;
+                dt_lds4h<F16>(cp + j0, ca);
+                dt_lds4h<F16>(cp + j1, cb);
+                dt_lds4h<F16>(sp + j0, nsa);
+                dt_lds4h<F16>(sp + j1, sb);
 #pragma unroll
-                for (int k = 0; k < E; ++k) sn[k] = -sn[k];
+                for (int k = 0; k < 4; ++k) nsa[k] = -nsa[k];
             }
-            for (int h0 = h_begin; h0 < h_end; h0 += 2) {
-                const bool two = h0 + 1 < h_end;
-                float u[2][E];
+            const int hd = p * HPW + hl;
+            if (!lane_on || hd >= NH) continue;
+            float ua[4], ub[4];
+            const int64_t e0 = (int64_t)tok * H + (int64_t)hd * D;
+            if (DQ) {
+                dt_lds4i(reinterpret_cast<const int32_t*>(base) + e0 + j0, ua);
+                dt_lds4i(reinterpret_cast<const int32_t*>(base) + e0 + j1, ub);
+                // dequant: ((float)x * weight_scale) * activation_scale + bias
+                float wa[4], wb[4], ba[4], bb[4];
+                dt_lds4f(p_ws + hd * D + j0, wa);
+                dt_lds4f(p_ws + hd * D + j1, wb);
+                dt_lds4f(p_bias + hd * D + j0, ba);
+                dt_lds4f(p_bias + hd * D + j1, bb);
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    if (j == 1 && !two) break;
-                    const int64_t e0 = (int64_t)my_tok * a.H + (int64_t)(h0 + j) * D + pos;
-                    if (XK == 0) dt_lds_i32<E>(reinterpret_cast<const int32_t*>(base) + e0, u[j]);
-                    else dt_lds16<E, XK == 2>(reinterpret_cast<const uint16_t*>(base) + e0, u[j]);
+                for (int k = 0; k < 4; ++k) {
+                    ua[k] = __fadd_rn(__fmul_rn(__fmul_rn(ua[k], wa[k]), act), ba[k]);
+                    ub[k] = __fadd_rn(__fmul_rn(__fmul_rn(ub[k], wb[k]), act), bb[k]);
                 }
+            } else {
+                dt_lds4h<XK == 2>(reinterpret_cast<const uint16_t*>(base) + e0 + j0, ua);
+                dt_lds4h<XK == 2>(reinterpret_cast<const uint16_t*>(base) + e0 + j1, ub);
+            }
+            float oa[4], ob[4];
+            if (hd < a.Nq + a.Nkv) {
+                // RoPE, half rotation: o_j = u_j c_j - u_{j+D/2} s_j, o_{j+D/2} = u_{j+D/2} c_{j+D/2} + u_j s_{j+D/2}
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    if (j == 1 && !two) break;
-                    const int hd = h0 + j;
-                    if (XK == 0) {
-                        // dequant: ((float)x * weight_scale) * activation_scale + bias
-                        float ws[E], bs[E];
-                        dt_param<E>(a.weight_scale + hd * D + pos, pv, ws);
-                        if (a.bias && a.bias_kind == 0) {
-                            dt_param<E>(reinterpret_cast<const float*>(a.bias) + hd * D + pos, pv, bs);
-                        } else if (a.bias) {
-#pragma unroll
-                            for (int k = 0; k < E; ++k) bs[k] = dq_bias(a, hd * D + pos + k);
-                        }
-#pragma unroll
-                        for (int k = 0; k < E; ++k) {
-                            float v = __fmul_rn(u[j][k], ws[k]);
-                            if (a.activation_scale) v = __fmul_rn(v, act);
-                            if (a.bias) v = __fadd_rn(v, bs[k]);
-                            u[j][k] = v;
-                        }
-                    }
+                for (int k = 0; k < 4; ++k) {
+                    oa[k] = __fadd_rn(__fmul_rn(ua[k], ca[k]), __fmul_rn(ub[k], nsa[k]));
+                    ob[k] = __fadd_rn(__fmul_rn(ub[k], cb[k]), __fmul_rn(ua[k], sb[k]));
                 }
-                // RoPE on q and k heads (the whole warp shuffles)
+            } else {
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    if (j == 1 && !two) break;
-                    const int hd = h0 + j;
-                    float o[E];
-                    if (hd < a.Nq + a.Nkv) {
-#pragma unroll
-                        for (int k = 0; k < E; ++k) {
-                            const float p = __shfl_xor_sync(FULL_MASK, u[j][k], 16);
-                            o[k] = __fadd_rn(__fmul_rn(u[j][k], cs[k]), __fmul_rn(p, sn[k]));
-                        }
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < E; ++k) o[k] = u[j][k];
-                    }
-                    dt_head_out<E, F16>(a, t, hd, pos, o, krow, vrow, pv);
+                for (int k = 0; k < 4; ++k) {
+                    oa[k] = ua[k];
+                    ob[k] = ub[k];
                 }
             }
+            if (hd < a.Nq) {
+                uint16_t* q = a.q_out + t * (int64_t)(a.Nq * D) + hd * D;
+                dt_store4h<F16>(q + j0, oa);
+                dt_store4h<F16>(q + j1, ob);
+                continue;
+            }
+            const bool is_k = hd < a.Nq + a.Nkv;
+            const int c0 = (is_k ? hd - a.Nq : hd - a.Nq - a.Nkv) * D;   // channel base in [0, Nkv*D)
+            if (a.k_out) {
+                uint16_t* kv = (is_k ? a.k_out : a.v_out) + t * (int64_t)C + c0;
+                dt_store4h<F16>(kv + j0, oa);
+                dt_store4h<F16>(kv + j1, ob);
+            }
+            uint8_t* row = is_k ? krow : vrow;
+            if (row == nullptr) continue;
+            const float* sc = (is_k ? p_sk : p_sv) + c0;
+            const float* of = (is_k ? p_ok : p_ov) + c0;
+            const float* rc = (is_k ? p_rk : p_rv) + c0;
+            st_b32(row + c0 + j0, dt_int8x4(oa, sc + j0, of + j0, rc + j0));
+            st_b32(row + c0 + j1, dt_int8x4(ob, sc + j1, of + j1, rc + j1));
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[st]);

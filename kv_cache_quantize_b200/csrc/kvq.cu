@@ -258,6 +258,59 @@ __global__ void selftest_div_kernel(int32_t which) {
     if (bad) atomicAdd(&g_selftest_count, bad);
 }
 
+// The fast int8 quantisation of the dequant kernel (int8x4_quant) against
+// IEEE division on 2^28 random (o, scale, offset) triples per call: o of random
+// sign and binade in [2^-70, 2^70], scale in [2^-70, 2^70], offset 0, a small
+// integer, or a random value up to 2^17; half of the o values are placed within
+// a few ulps of a rounding tie (o = (k + 1/2 - offset) * scale, k in
+// [-140, 140]).  Counter-based hash (SplitMix64 finaliser) for the draws.
+__device__ __forceinline__ uint64_t st_mix(uint64_t z) {
+    z += 0x9e3779b97f4a7c15ull;
+    z = (z ^ (z >> 30)) * 0xbf58476d1ce4e5b9ull;
+    z = (z ^ (z >> 27)) * 0x94d049bb133111ebull;
+    return z ^ (z >> 31);
+}
+
+__device__ __forceinline__ float st_float(uint64_t h, int emin, int emax) {
+    const int e = emin + (int)((h >> 40) % (uint64_t)(emax - emin + 1));
+    const uint32_t m = (uint32_t)h & 0x7fffffu;
+    return __uint_as_float(((uint32_t)(e + 127) << 23) | m);
+}
+
+__global__ void selftest_int8_kernel() {
+    const uint64_t i0 = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) * 16u;
+    unsigned long long bad = 0;
+    for (uint64_t i = i0; i < i0 + 16u; i += 4u) {
+        float o[4], sc[4], of[4], r[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint64_t h1 = st_mix(4 * (i + k)), h2 = st_mix(4 * (i + k) + 1), h3 = st_mix(4 * (i + k) + 2),
+                           h4 = st_mix(4 * (i + k) + 3);
+            sc[k] = st_float(h2, -70, 70);
+            const uint32_t kind = (uint32_t)(h3 & 3u);
+            of[k] = kind == 0 ? 0.0f : (kind == 1 ? (float)((int)((h3 >> 8) % 17u) - 8)
+                                                  : st_float(h3 >> 2, -20, 17) * ((h3 >> 60) & 1u ? -1.0f : 1.0f));
+            if (h4 & 1u) {
+                const float tk = (float)((int)((h4 >> 8) % 281u) - 140);
+                float v = __fmul_rn(__fadd_rn(__fadd_rn(tk, 0.5f), -of[k]), sc[k]);
+                const int nudge = (int)((h4 >> 20) % 5u) - 2;
+                v = __uint_as_float(__float_as_uint(v) + nudge);
+                o[k] = v;
+            } else {
+                o[k] = st_float(h1, -70, 70) * ((h1 >> 63) ? -1.0f : 1.0f);
+            }
+            r[k] = int8_quant_rcp(sc[k], of[k]);
+        }
+        const uint32_t fast = int8x4_quant(o, sc, of, r);
+        uint32_t ref = 0u;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            ref |= ((uint32_t)int8_rne_sat(__fadd_rn(__fdiv_rn(o[k], sc[k]), of[k])) & 0xffu) << (8 * k);
+        bad += fast != ref ? 1ull : 0ull;
+    }
+    if (bad) atomicAdd(&g_selftest_count, bad);
+}
+
 // every positive finite bf16 amax (bits < 0x7f80) and every positive finite
 // f16 amax (bits < 0x7c00) over the three format maxima
 __global__ void selftest_fmax_kernel() {
@@ -280,13 +333,14 @@ extern "C" {
 
 kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream) {
     if (!result) return KVQ_ERR_NULL;
-    if (which < 0 || which > 5) return KVQ_ERR_ATTR;
+    if (which < 0 || which > 6) return KVQ_ERR_ATTR;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const unsigned long long zero = 0ull;
     unsigned long long h = 0ull;
     if (cudaMemcpyToSymbolAsync(g_selftest_count, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
         return KVQ_ERR_CUDA;
     if (which == 4) selftest_fmax_kernel<<<256, 256, 0, s>>>();
+    else if (which == 6) selftest_int8_kernel<<<65536, 256, 0, s>>>();
     else selftest_div_kernel<<<65536, 256, 0, s>>>(which);
     if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
     if (cudaMemcpyFromSymbolAsync(&h, g_selftest_count, sizeof(h), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -398,7 +452,10 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
     };
     const int want = bulk_out ? 2 : 3;
     const int ct_stages = ct_smem(want) <= smem_limit ? want : (ct_smem(2) <= smem_limit ? 2 : 0);
-    if (a.x_vec && ct_stages > 0) {
+    // decode-sized batches (fewer rows than one 32-row tile per SM) take the
+    // direct kernel: no pipeline to fill, one load-compute-store round trip
+    const bool small = T < 32 * (int64_t)sm_count();
+    if (a.x_vec && ct_stages > 0 && !small) {
         // pipelined kernel: rows arrive in shared memory by bulk copy
         a.ncw = a.nseg < CT_MAX_CONSUMER_WARPS ? a.nseg : CT_MAX_CONSUMER_WARPS;
         a.stages = ct_stages;
@@ -775,42 +832,35 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
     const bool aligned = reinterpret_cast<uintptr_t>(x->data) % 16 == 0 &&
                          reinterpret_cast<uintptr_t>(cos->data) % 16 == 0 &&
                          reinterpret_cast<uintptr_t>(sin->data) % 16 == 0 && (D * 2) % 16 == 0;
-    const int E = (int)(D / 32);
-    if (aligned && (E == 2 || E == 4 || E == 8)) {
+    const size_t prm = dt_param_bytes(H, Nkv * D, dq);
+    if (aligned && D % 8 == 0 && D <= 256 && prm <= 64 * 1024) {
         // pipelined kernel: token rows, cos and sin arrive in shared memory by
-        // bulk copy; TPS tokens per stage (a divisor of the consumer warps,
-        // x span at most 32 KB), as many stages (2..4) as keep two CTAs on an SM
+        // bulk copy; TPS tokens per stage (a divisor of the consumer warps, x
+        // span at most 32 KB), as many stages (2..4) as keep two CTAs on an SM
         int tps = 1;
         while (tps < DT_CONSUMERS && 2 * tps * H * xb <= 32768) tps *= 2;
         a.tps = tps;
         auto dt_smem = [&](int stages) {
-            return (size_t)dt_header_bytes(stages, tps) + (size_t)stages * dt_stage_bytes(tps, H, xb, (int)D);
+            return (size_t)dt_header_bytes(stages, tps) + prm + (size_t)stages * dt_stage_bytes(tps, H, xb, (int)D);
         };
         a.stages = 4;
         while (a.stages > 2 && dt_smem(a.stages) > 112 * 1024) --a.stages;
         const size_t smem = dt_smem(a.stages);
         const int64_t tiles = (need + a.tps - 1) / a.tps;
         const bool f16 = a.cos_f16 != 0;
-#define KVQ_LAUNCH_DT(EE, XK, F)                                                               \
+#define KVQ_LAUNCH_DT(XK, F)                                                                   \
     do {                                                                                       \
-        auto k = dequant_rope_quant_tma_kernel<EE, XK, F>;                                     \
+        auto k = dequant_rope_quant_tma_kernel<XK, F>;                                         \
         k<<<(unsigned)persistent_grid(k, DT_THREADS, tiles, smem), DT_THREADS, smem, s>>>(a);  \
     } while (0)
-#define KVQ_LAUNCH_DT_E(XK, F)                                                                 \
-    do {                                                                                       \
-        if (E == 2) KVQ_LAUNCH_DT(2, XK, F);                                                   \
-        else if (E == 4) KVQ_LAUNCH_DT(4, XK, F);                                              \
-        else KVQ_LAUNCH_DT(8, XK, F);                                                          \
-    } while (0)
         if (a.x_kind == 0) {
-            if (f16) KVQ_LAUNCH_DT_E(0, true);
-            else KVQ_LAUNCH_DT_E(0, false);
+            if (f16) KVQ_LAUNCH_DT(0, true);
+            else KVQ_LAUNCH_DT(0, false);
         } else if (a.x_kind == 1) {
-            KVQ_LAUNCH_DT_E(1, false);
+            KVQ_LAUNCH_DT(1, false);
         } else {
-            KVQ_LAUNCH_DT_E(2, true);
+            KVQ_LAUNCH_DT(2, true);
         }
-#undef KVQ_LAUNCH_DT_E
 #undef KVQ_LAUNCH_DT
         return launched();
     }

@@ -199,6 +199,52 @@ __device__ __forceinline__ void div_scale1_neg_x2(float a0, float a1, float s, f
         : "f"(a0), "f"(a1), "f"(-r), "f"(s));
 }
 
+// ---------------------------------------------------------------------------
+// Packed binary32 pairs (mul/add/fma .rn.f32x2: each half is exactly the IEEE
+// round-to-nearest-even scalar operation, subnormals kept).  The compiler may
+// fuse a packed multiply into a following packed add, so a packed product is
+// only ever fed to the addend of a fused multiply-add here, never to an add:
+// plain products-then-sums stay on the scalar __fmul_rn / __fadd_rn.
+// ---------------------------------------------------------------------------
+// The quotient a / s of a pair by the two-step Markstein form with r = RN(1/s)
+// (P. Markstein, IBM J. Res. Dev. 34(1), 1990): q0 = RN(a r); each step forms
+// the exact residual a - s q under a fused multiply-add and sets
+// q = RN(q + residual r).  After the first step q is faithful, so the second
+// returns the correctly rounded quotient RN(a / s) whenever a, s, r and the
+// quotient stay inside the normal range (the caller's guard); then the
+// offset is added: (q0 + f0, q1 + f1).
+__device__ __forceinline__ void div2_add_x2(float a0, float a1, float s0, float s1, float r0, float r1, float f0,
+                                            float f1, float& y0, float& y1) {
+    asm("{\n\t.reg .b64 a, ns, r, f, q, e;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 ns, {%4, %5};\n\t"
+        "mov.b64 r, {%6, %7};\n\t"
+        "mov.b64 f, {%8, %9};\n\t"
+        "mul.rn.f32x2 q, a, r;\n\t"
+        "fma.rn.f32x2 e, q, ns, a;\n\t"
+        "fma.rn.f32x2 q, e, r, q;\n\t"
+        "fma.rn.f32x2 e, q, ns, a;\n\t"
+        "fma.rn.f32x2 q, e, r, q;\n\t"
+        "add.rn.f32x2 q, q, f;\n\t"
+        "mov.b64 {%0, %1}, q;\n\t}"
+        : "=f"(y0), "=f"(y1)
+        : "f"(a0), "f"(a1), "f"(-s0), "f"(-s1), "f"(r0), "f"(r1), "f"(f0), "f"(f1));
+}
+
+// Four binary32 values rounded half to even to integers and saturated to
+// int8, packed little-endian (value 0 in byte 0).  NaN gives 0.
+__device__ __forceinline__ uint32_t int8x4_rne_sat(float v0, float v1, float v2, float v3) {
+    int32_t i0, i1, i2, i3;
+    asm("cvt.rni.s32.f32 %0, %1;" : "=r"(i0) : "f"(v0));
+    asm("cvt.rni.s32.f32 %0, %1;" : "=r"(i1) : "f"(v1));
+    asm("cvt.rni.s32.f32 %0, %1;" : "=r"(i2) : "f"(v2));
+    asm("cvt.rni.s32.f32 %0, %1;" : "=r"(i3) : "f"(v3));
+    uint32_t hi, r;
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(hi) : "r"(i3), "r"(i2));
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(i1), "r"(i0), "r"(hi));
+    return r;
+}
+
 // Largest magnitude of the two bf16 halves of a and b, per half (max of the
 // absolute values; the sign bits of the result are not meaningful).
 __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {

@@ -67,6 +67,29 @@ def test_compress_ragged_counts(T):
     _same(_ce(T, 576, 0, seed=7))
 
 
+# Batches of at least one 32-row tile per SM take the pipelined (bulk-copy)
+# kernel; smaller ones the direct kernel.  T_PIPE is above that threshold on
+# any GPU with up to 188 SMs and leaves a ragged last tile.
+T_PIPE = 6037
+
+
+@pytest.mark.parametrize("mode,G", [(0, 64), (1, 64), (2, 16), (2, 32), (2, 64)])
+@pytest.mark.parametrize("d", [128, 576, 1024])
+def test_compress_pipelined(mode, G, d):
+    _same(_ce(T_PIPE, d, mode, G, kind="wide" if d == 576 else "normal", seed=21))
+
+
+@pytest.mark.parametrize("mode,G", [(0, 64), (1, 64), (2, 32)])
+@pytest.mark.parametrize("extra,pad", [(0, 0), (1, 0), (3, 40), (16, 1000)])
+def test_compress_pipelined_row_alignments(mode, G, extra, pad):
+    _same(_ce(T_PIPE, 320, mode, G, extra=extra, pad=pad, seed=23))
+
+
+@pytest.mark.parametrize("T", [6016, 6017, 6047])
+def test_compress_pipelined_ragged_counts(T):
+    _same(_ce(T, 576, 2, 32, seed=25))
+
+
 def test_compress_max_width_and_int64_slots():
     _same(_ce(40, 8192, 0, seed=9, slot_dtype=np.int64))
     _same(_ce(40, 8192, 2, 16, seed=9, slot_dtype=np.int64))

@@ -6,7 +6,11 @@ whole input domain against IEEE division:
     quotient itself may differ in its last bits for a small share of pairs,
     which is reported, not required);
   * amax / 448, amax / 57344, amax / 6 with constant reciprocals: bit-identical
-    for every positive finite bf16 and f16 amax."""
+    for every positive finite bf16 and f16 amax;
+  * the dequant kernel's static int8 quantisation through a per-channel
+    reciprocal (two-step Markstein form, IEEE division outside its guard):
+    the same int8 codes as IEEE division on 2^28 random and near-tie
+    (value, scale, offset) triples."""
 import pytest
 
 import kv_cache_quantize_b200 as kvq
@@ -16,7 +20,8 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("which,what", [(2, "E4M3 codes of the one-step quotient"),
                                         (3, "E2M1 codes of the one-step quotient"),
-                                        (4, "constant-divisor scale quotients")])
+                                        (4, "constant-divisor scale quotients"),
+                                        (6, "int8 codes of the reciprocal-based quotient")])
 def test_shortcut_is_exact(which, what):
     assert kvq.selftest(which) == 0, what
 
