@@ -38,6 +38,8 @@ struct DrqArgs {
     const void* bias;               // [H] nullable
     int32_t bias_kind;              // 0 f32, 1 f16, 2 bf16, 3 int32
     int32_t params_vec;             // all f32 parameter tensors are 16-byte aligned
+    int32_t out_vec8;               // q_out, k_out, v_out are 8-byte aligned
+    int32_t rows_vec4;              // k / v cache rows start on 4-byte boundaries
     int32_t Nq, Nkv, D;
     uint16_t* q_out;        // [B*S, Nq*D]
     uint16_t* k_out;        // [B*S, Nkv*D] or null
@@ -221,9 +223,6 @@ __device__ __forceinline__ int64_t dq_slot(const DrqArgs& a, int64_t t) {
     return b * c1 + start + s;
 }
 
-__device__ __forceinline__ float half_bits_to_f32(uint32_t h, bool f16) {
-    return f16 ? __half2float(__ushort_as_half((unsigned short)h)) : __uint_as_float(h << 16);
-}
 
 template <int E>
 __global__ void __launch_bounds__(DQ_WARPS * 32) dequant_rope_quant_kernel(const DrqArgs a) {
@@ -282,10 +281,9 @@ __global__ void __launch_bounds__(DQ_WARPS * 32) dequant_rope_quant_kernel(const
 // Lane layout: a head of D values is L = D/8 lanes; lane l of a head holds the
 // four values [4l, 4l + 4) and their half-rotation partners [D/2 + 4l,
 // D/2 + 4l + 4), so RoPE needs no shuffle, and a warp holds 32/L heads side by
-// side (a PASS).  The stage's passes (TPS tokens x ceil(NH / (32/L)) passes,
-// token-major) are dealt to the consumer warps round-robin, which spreads the
-// costlier k / v passes (int8 quantisation) evenly; a warp widens a token's
-// cos / sin when it moves to that token.
+// side (a PASS).  Each token of a stage has 8/TPS consumer warps, which take
+// its passes round-robin (spreading the costlier k / v passes with their int8
+// quantisation evenly) and widen its cos / sin once.
 // ---------------------------------------------------------------------------
 constexpr int DT_CONSUMERS = 8;
 constexpr int DT_THREADS = (DT_CONSUMERS + 1) * 32;
@@ -345,20 +343,6 @@ __device__ __forceinline__ void dt_lds4f(const float* p, float (&v)[4]) {
     v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
 }
 
-// four values rounded to 16-bit floats, stored (8 bytes) at p
-template <bool F16>
-__device__ __forceinline__ void dt_store4h(uint16_t* p, const float (&o)[4]) {
-    uint32_t w0, w1;
-    if (F16) {
-        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w0) : "f"(o[1]), "f"(o[0]));
-        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w1) : "f"(o[3]), "f"(o[2]));
-    } else {
-        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w0) : "f"(o[1]), "f"(o[0]));
-        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w1) : "f"(o[3]), "f"(o[2]));
-    }
-    st_b64(reinterpret_cast<uint8_t*>(p), make_uint2(w0, w1));
-}
-
 // Static int8 of four values: round half to even of o / scale + offset,
 // saturated (offset 0 when absent), packed little-endian.  r holds RN(1/scale)
 // for channels whose scale lies in [2^-60, 2^60] and whose |offset| <= 2^16,
@@ -370,16 +354,21 @@ __device__ __forceinline__ void dt_store4h(uint16_t* p, const float (&o)[4]) {
 // quotient's last bits; above 2^20 the integer saturates either way.  Other
 // lanes divide with IEEE division.  kvq_selftest checks the two paths against
 // each other on random and near-tie triples.
+__device__ __forceinline__ float div2_add(float a, float s, float r, float f) {
+    const float q0 = __fmul_rn(a, r);
+    const float q1 = __fmaf_rn(__fmaf_rn(-q0, s, a), r, q0);
+    const float q2 = __fmaf_rn(__fmaf_rn(-q1, s, a), r, q1);
+    return __fadd_rn(q2, f);
+}
+
 __device__ __forceinline__ uint32_t int8x4_quant(const float (&o)[4], const float (&s)[4], const float (&f)[4],
                                                  const float (&r)[4]) {
     float q[4];
-    const uint32_t lim = 0x5d800000u;     // 2^60
-    const bool fast = r[0] != 0.0f && r[1] != 0.0f && r[2] != 0.0f && r[3] != 0.0f &&
-                      (__float_as_uint(o[0]) & 0x7fffffffu) <= lim && (__float_as_uint(o[1]) & 0x7fffffffu) <= lim &&
-                      (__float_as_uint(o[2]) & 0x7fffffffu) <= lim && (__float_as_uint(o[3]) & 0x7fffffffu) <= lim;
-    if (fast) {
-        div2_add_x2(o[0], o[1], s[0], s[1], r[0], r[1], f[0], f[1], q[0], q[1]);
-        div2_add_x2(o[2], o[3], s[2], s[3], r[2], r[3], f[2], f[3], q[2], q[3]);
+    const float m = fmaxf(fmaxf(fabsf(o[0]), fabsf(o[1])), fmaxf(fabsf(o[2]), fabsf(o[3])));
+    const float rmin = fminf(fminf(r[0], r[1]), fminf(r[2], r[3]));
+    if (m <= 1.152921504606846976e18f && rmin > 0.0f) {      // |o| <= 2^60, every channel eligible
+#pragma unroll
+        for (int k = 0; k < 4; ++k) q[k] = div2_add(o[k], s[k], r[k], f[k]);
     } else {
 #pragma unroll
         for (int k = 0; k < 4; ++k) q[k] = __fadd_rn(__fdiv_rn(o[k], s[k]), f[k]);
@@ -508,6 +497,9 @@ __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(cons
     }
 
     // ---------------- consumers ----------------
+    // warp w serves token w / WPT of each stage and takes that token's passes
+    // wt, wt + WPT, ... (wt = w mod WPT): each warp stays on one token, and the
+    // stride mixes the costlier k / v passes evenly over the token's warps
     const int NH = a.Nq + 2 * a.Nkv;
     const int L = D >> 3;                     // lanes per head
     const int HPW = 32 / L;                   // heads per pass
@@ -515,6 +507,21 @@ __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(cons
     const bool lane_on = hl < HPW;
     const int NP = (NH + HPW - 1) / HPW;      // passes per token
     const int j0 = 4 * l, j1 = (D >> 1) + 4 * l;
+    const int WPT = DT_CONSUMERS / TPS;
+    const int my_tok = warp / WPT, wt = warp - my_tok * WPT;
+    const bool v8 = a.out_vec8 != 0, r4 = a.rows_vec4 != 0;
+    auto store4h = [&](uint16_t* p, const float (&o)[4]) {
+        uint32_t w0, w1;
+        if (F16) {
+            asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w0) : "f"(o[1]), "f"(o[0]));
+            asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w1) : "f"(o[3]), "f"(o[2]));
+        } else {
+            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w0) : "f"(o[1]), "f"(o[0]));
+            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w1) : "f"(o[3]), "f"(o[2]));
+        }
+        if (v8) *reinterpret_cast<uint2*>(p) = make_uint2(w0, w1);
+        else st_b64(reinterpret_cast<uint8_t*>(p), make_uint2(w0, w1));
+    };
     int it = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
         const int st = it % S;
@@ -523,87 +530,89 @@ __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(cons
         const int64_t t0 = tile * TPS;
         const int toks = (int)(ntok - t0 < TPS ? ntok - t0 : TPS);
         const uint8_t* base = stages + (size_t)st * stage_bytes;
-        const int ntask = toks * NP;
-        int tok = -1;
-        int64_t t = 0;
-        float act = 1.0f;
-        uint8_t *krow = nullptr, *vrow = nullptr;
-        float ca[4], cb[4], nsa[4], sb[4];     // cos / sin at j0 (a) and j1 (b); nsa = -sin at j0
-        for (int task = warp; task < ntask; task += DT_CONSUMERS) {
-            const int tk = task / NP, p = task - tk * NP;
-            if (tk != tok) {
-                tok = tk;
-                t = t0 + tok;
-                const int64_t slot = slots[st * TPS + tok];
-                act = acts[st * TPS + tok];
-                krow = slot >= 0 ? slot_row(a.kc, slot) : nullptr;
-                vrow = slot >= 0 ? slot_row(a.vc, slot) : nullptr;
-                const uint16_t* cp = reinterpret_cast<const uint16_t*>(base + x_span) + tok * D;
-                const uint16_t* sp = reinterpret_cast<const uint16_t*>(base + x_span + cs_span) + tok * D;
-                dt_lds4h<F16>(cp + j0, ca);
-                dt_lds4h<F16>(cp + j1, cb);
-                dt_lds4h<F16>(sp + j0, nsa);
-                dt_lds4h<F16>(sp + j1, sb);
+        if (my_tok < toks && lane_on) {
+            const int64_t t = t0 + my_tok;
+            const int64_t slot = slots[st * TPS + my_tok];
+            const float act = acts[st * TPS + my_tok];
+            uint8_t* krow = slot >= 0 ? slot_row(a.kc, slot) : nullptr;
+            uint8_t* vrow = slot >= 0 ? slot_row(a.vc, slot) : nullptr;
+            // cos / sin at j0 (a) and j1 (b); nsa = -sin at j0
+            float ca[4], cb[4], nsa[4], sb[4];
+            const uint16_t* cp = reinterpret_cast<const uint16_t*>(base + x_span) + my_tok * D;
+            const uint16_t* sp = reinterpret_cast<const uint16_t*>(base + x_span + cs_span) + my_tok * D;
+            dt_lds4h<F16>(cp + j0, ca);
+            dt_lds4h<F16>(cp + j1, cb);
+            dt_lds4h<F16>(sp + j0, nsa);
+            dt_lds4h<F16>(sp + j1, sb);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) nsa[k] = -nsa[k];
-            }
-            const int hd = p * HPW + hl;
-            if (!lane_on || hd >= NH) continue;
-            float ua[4], ub[4];
-            const int64_t e0 = (int64_t)tok * H + (int64_t)hd * D;
-            if (DQ) {
-                dt_lds4i(reinterpret_cast<const int32_t*>(base) + e0 + j0, ua);
-                dt_lds4i(reinterpret_cast<const int32_t*>(base) + e0 + j1, ub);
-                // dequant: ((float)x * weight_scale) * activation_scale + bias
-                float wa[4], wb[4], ba[4], bb[4];
-                dt_lds4f(p_ws + hd * D + j0, wa);
-                dt_lds4f(p_ws + hd * D + j1, wb);
-                dt_lds4f(p_bias + hd * D + j0, ba);
-                dt_lds4f(p_bias + hd * D + j1, bb);
+            for (int k = 0; k < 4; ++k) nsa[k] = -nsa[k];
+            const uint8_t* xt = base + (size_t)my_tok * H * XB;
+            for (int p = wt; p < NP; p += WPT) {
+                const int hd = p * HPW + hl;
+                if (hd >= NH) continue;
+                float ua[4], ub[4];
+                const int e0 = hd * D;
+                if (DQ) {
+                    dt_lds4i(reinterpret_cast<const int32_t*>(xt) + e0 + j0, ua);
+                    dt_lds4i(reinterpret_cast<const int32_t*>(xt) + e0 + j1, ub);
+                    // dequant: ((float)x * weight_scale) * activation_scale + bias
+                    float wa[4], wb[4], ba[4], bb[4];
+                    dt_lds4f(p_ws + e0 + j0, wa);
+                    dt_lds4f(p_ws + e0 + j1, wb);
+                    dt_lds4f(p_bias + e0 + j0, ba);
+                    dt_lds4f(p_bias + e0 + j1, bb);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    ua[k] = __fadd_rn(__fmul_rn(__fmul_rn(ua[k], wa[k]), act), ba[k]);
-                    ub[k] = __fadd_rn(__fmul_rn(__fmul_rn(ub[k], wb[k]), act), bb[k]);
+                    for (int k = 0; k < 4; ++k) {
+                        ua[k] = __fadd_rn(__fmul_rn(__fmul_rn(ua[k], wa[k]), act), ba[k]);
+                        ub[k] = __fadd_rn(__fmul_rn(__fmul_rn(ub[k], wb[k]), act), bb[k]);
+                    }
+                } else {
+                    dt_lds4h<XK == 2>(reinterpret_cast<const uint16_t*>(xt) + e0 + j0, ua);
+                    dt_lds4h<XK == 2>(reinterpret_cast<const uint16_t*>(xt) + e0 + j1, ub);
                 }
-            } else {
-                dt_lds4h<XK == 2>(reinterpret_cast<const uint16_t*>(base) + e0 + j0, ua);
-                dt_lds4h<XK == 2>(reinterpret_cast<const uint16_t*>(base) + e0 + j1, ub);
-            }
-            float oa[4], ob[4];
-            if (hd < a.Nq + a.Nkv) {
-                // RoPE, half rotation: o_j = u_j c_j - u_{j+D/2} s_j, o_{j+D/2} = u_{j+D/2} c_{j+D/2} + u_j s_{j+D/2}
+                float oa[4], ob[4];
+                if (hd < a.Nq + a.Nkv) {
+                    // RoPE, half rotation: o_j = u_j c_j - u_{j+D/2} s_j, o_{j+D/2} = u_{j+D/2} c_{j+D/2} + u_j s_{j+D/2}
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    oa[k] = __fadd_rn(__fmul_rn(ua[k], ca[k]), __fmul_rn(ub[k], nsa[k]));
-                    ob[k] = __fadd_rn(__fmul_rn(ub[k], cb[k]), __fmul_rn(ua[k], sb[k]));
-                }
-            } else {
+                    for (int k = 0; k < 4; ++k) {
+                        oa[k] = __fadd_rn(__fmul_rn(ua[k], ca[k]), __fmul_rn(ub[k], nsa[k]));
+                        ob[k] = __fadd_rn(__fmul_rn(ub[k], cb[k]), __fmul_rn(ua[k], sb[k]));
+                    }
+                } else {
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    oa[k] = ua[k];
-                    ob[k] = ub[k];
+                    for (int k = 0; k < 4; ++k) {
+                        oa[k] = ua[k];
+                        ob[k] = ub[k];
+                    }
+                }
+                if (hd < a.Nq) {
+                    uint16_t* q = a.q_out + t * (int64_t)(a.Nq * D) + e0;
+                    store4h(q + j0, oa);
+                    store4h(q + j1, ob);
+                    continue;
+                }
+                const bool is_k = hd < a.Nq + a.Nkv;
+                const int c0 = (is_k ? hd - a.Nq : hd - a.Nq - a.Nkv) * D;   // channel base in [0, Nkv*D)
+                if (a.k_out) {
+                    uint16_t* kv = (is_k ? a.k_out : a.v_out) + t * (int64_t)C + c0;
+                    store4h(kv + j0, oa);
+                    store4h(kv + j1, ob);
+                }
+                uint8_t* row = is_k ? krow : vrow;
+                if (row == nullptr) continue;
+                const float* sc = (is_k ? p_sk : p_sv) + c0;
+                const float* of = (is_k ? p_ok : p_ov) + c0;
+                const float* rc = (is_k ? p_rk : p_rv) + c0;
+                const uint32_t q0 = dt_int8x4(oa, sc + j0, of + j0, rc + j0);
+                const uint32_t q1 = dt_int8x4(ob, sc + j1, of + j1, rc + j1);
+                if (r4) {
+                    *reinterpret_cast<uint32_t*>(row + c0 + j0) = q0;
+                    *reinterpret_cast<uint32_t*>(row + c0 + j1) = q1;
+                } else {
+                    st_b32(row + c0 + j0, q0);
+                    st_b32(row + c0 + j1, q1);
                 }
             }
-            if (hd < a.Nq) {
-                uint16_t* q = a.q_out + t * (int64_t)(a.Nq * D) + hd * D;
-                dt_store4h<F16>(q + j0, oa);
-                dt_store4h<F16>(q + j1, ob);
-                continue;
-            }
-            const bool is_k = hd < a.Nq + a.Nkv;
-            const int c0 = (is_k ? hd - a.Nq : hd - a.Nq - a.Nkv) * D;   // channel base in [0, Nkv*D)
-            if (a.k_out) {
-                uint16_t* kv = (is_k ? a.k_out : a.v_out) + t * (int64_t)C + c0;
-                dt_store4h<F16>(kv + j0, oa);
-                dt_store4h<F16>(kv + j1, ob);
-            }
-            uint8_t* row = is_k ? krow : vrow;
-            if (row == nullptr) continue;
-            const float* sc = (is_k ? p_sk : p_sv) + c0;
-            const float* of = (is_k ? p_ok : p_ov) + c0;
-            const float* rc = (is_k ? p_rk : p_rv) + c0;
-            st_b32(row + c0 + j0, dt_int8x4(oa, sc + j0, of + j0, rc + j0));
-            st_b32(row + c0 + j1, dt_int8x4(ob, sc + j1, of + j1, rc + j1));
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[st]);

@@ -819,6 +819,12 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
     {
         auto al = [](const void* p) { return p == nullptr || reinterpret_cast<uintptr_t>(p) % 16 == 0; };
         a.params_vec = al(sk) && al(sv) && al(ok) && al(ov) && al(ws) && (bias_kind != 0 || al(bias_ptr));
+        auto al8 = [](const void* p) { return p == nullptr || reinterpret_cast<uintptr_t>(p) % 8 == 0; };
+        a.out_vec8 = al8(q_out->data) && al8(kop) && al8(vop);
+        auto r4 = [](const PagedRows& r) {
+            return reinterpret_cast<uintptr_t>(r.base) % 4 == 0 && r.row_bytes % 4 == 0 && r.block_stride % 4 == 0;
+        };
+        a.rows_vec4 = r4(kr) && r4(vr);
     }
     a.Nq = (int32_t)Nq;
     a.Nkv = (int32_t)Nkv;
