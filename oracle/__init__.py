@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
                                                  _vp, _vp, ctypes.c_int, ctypes.POINTER(_CacheOut),
                                                  ctypes.POINTER(_CacheOut), ctypes.c_float, _vp]
         L.kvqo_dequant_rope_quant_kvcache.argtypes = [ctypes.POINTER(_DrqArgs), _vp]
+        L.kvqo_kv_decompress.argtypes = [ctypes.POINTER(_Paged), _vp, _i64, _i64, ctypes.c_int, _i64,
+                                         ctypes.c_float, _vp, _i64, _vp]
         _LIB = L
     return _LIB
 
@@ -197,6 +199,28 @@ def kv_compress_epilog(x_bits: np.ndarray, slot_mapping, cache: Paged, quant_mod
         _check(rc, "kv_compress_epilog")
         return int(faults[0])
     return _parallel_rows(T, threads, run)
+
+
+def kv_decompress(cache: Paged, slot_mapping, d: int, quant_mode: int, quant_group_size: int = 64,
+                  x_scale: float = 1.0, y: Optional[np.ndarray] = None, threads: int = 1):
+    """Decode the packed rows named by slot_mapping into bf16 bit patterns y [T, d]
+    (rows of skipped tokens keep y's initial contents, zeros by default).
+    Returns (y, fault bits)."""
+    s = _slots(slot_mapping)
+    T = s.size
+    if y is None:
+        y = np.zeros((T, d), dtype=np.uint16)
+    assert y.dtype == np.uint16 and y.shape == (T, d) and y.flags["C_CONTIGUOUS"]
+    pc = cache.c()
+
+    def run(lo, hi):
+        faults = np.zeros(1, dtype=np.uint32)
+        rc = lib().kvqo_kv_decompress(ctypes.byref(pc), s[lo:].ctypes.data, hi - lo, d, quant_mode,
+                                      quant_group_size, ctypes.c_float(x_scale), y[lo:].ctypes.data, d,
+                                      _ptr(faults))
+        _check(rc, "kv_decompress")
+        return int(faults[0])
+    return y, _parallel_rows(T, threads, run)
 
 
 def indexer_quant_cache(x_bits: np.ndarray, x_dtype: str, slot_mapping, cache: Paged, cache_fp8: str,

@@ -404,6 +404,80 @@ int kvqo_kv_compress_epilog(const uint16_t* x, int64_t T, int64_t d, int64_t x_r
     return KVQO_OK;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Packed-row decoder: the inverse of compress_row, as the attention side   */
+/* reads the cache ([DRQ] 两种 KV Cache 更新模式: the cache rows are what    */
+/* attention consumes).  Each code is decoded exactly (decode_bits), scaled */
+/* by its group's stored scale with one binary32 multiply and rounded to    */
+/* bf16 (round to nearest even):                                            */
+/*   modes 0/1: nope y_i = bf16(fp8(q_i) * scale_g)  (scale_g: the bf16      */
+/*              value, or 2^(b-127) for the E8M0 byte b); rope: the stored   */
+/*              bf16 values;                                                 */
+/*   mode 2:    nope y_i = bf16(e2m1(q_i) * scale_g); rope                   */
+/*              y_j = bf16(fp8(r_j) / xScale), one IEEE division (the        */
+/*              inverse of the static multiply).                             */
+/* Readings: the pages define only the encoding; decoding with the stored   */
+/* scale and one rounding to bf16 is the plain inverse.                     */
+/* ------------------------------------------------------------------------ */
+static void decompress_row(const uint8_t* row, int64_t d, int quant_mode, int64_t G, float x_scale, uint16_t* y)
+{
+    const int64_t n = d - 64;
+    if (quant_mode == 0 || quant_mode == 1) {
+        const uint8_t* scales = row + n + 128;
+        for (int64_t g = 0; g < n / 64; ++g) {
+            float sf;
+            if (quant_mode == 0) {
+                uint16_t sb = (uint16_t)(scales[2 * g] | (scales[2 * g + 1] << 8));
+                sf = bf16_to_f32(sb);
+            } else {
+                sf = (float)ldexp(1.0, (int)scales[g] - 127);   /* exact: 2^-127 .. 2^127 */
+            }
+            for (int64_t i = 0; i < 64; ++i) {
+                float v = decode_bits(&FMT_E4M3, row[64 * g + i]);
+                y[64 * g + i] = f32_to_bf16(v * sf);
+            }
+        }
+        for (int64_t j = 0; j < 64; ++j) y[n + j] = (uint16_t)(row[n + 2 * j] | (row[n + 2 * j + 1] << 8));
+    } else {
+        const uint8_t* rope = row + n / 2;
+        const uint8_t* scales = row + n / 2 + 64;
+        for (int64_t g = 0; g < n / G; ++g) {
+            uint16_t sb = (uint16_t)(scales[2 * g] | (scales[2 * g + 1] << 8));
+            float sf = bf16_to_f32(sb);
+            for (int64_t i = 0; i < G; ++i) {
+                int64_t e = G * g + i;
+                uint32_t c = (row[e / 2] >> (4 * (e % 2))) & 0xFu;
+                y[e] = f32_to_bf16(decode_bits(&FMT_E2M1, c) * sf);
+            }
+        }
+        for (int64_t j = 0; j < 64; ++j) y[n + j] = f32_to_bf16(decode_bits(&FMT_E4M3, rope[j]) / x_scale);
+    }
+}
+
+/* Decode the rows of slot_mapping into y [T, d] (row stride y_row_stride   */
+/* elements).  Tokens whose slot is -1 leave their y row untouched; other   */
+/* slots outside the cache also leave it and raise the fault bit.           */
+int kvqo_kv_decompress(const kvqo_paged* cache, const int64_t* slot_mapping, int64_t T, int64_t d,
+                       int quant_mode, int64_t quant_group_size, float x_scale, uint16_t* y,
+                       int64_t y_row_stride, uint32_t* faults)
+{
+    if (d <= 64 || d % 64 != 0 || d > 8192) return KVQO_EINVAL;
+    if (quant_mode < 0 || quant_mode > 2) return KVQO_EINVAL;
+    if (quant_mode == 2) {
+        if (quant_group_size != 16 && quant_group_size != 32 && quant_group_size != 64) return KVQO_EINVAL;
+        if ((d - 64) % quant_group_size != 0) return KVQO_EINVAL;
+    }
+    int64_t col = kvqo_kv_cache_col(d, quant_mode, quant_group_size);
+    if (col < 0 || col > cache->row_bytes) return KVQO_EINVAL;
+    for (int64_t t = 0; t < T; ++t) {
+        int64_t s = slot_mapping[t];
+        if (s == -1) continue;
+        if (s < 0 || s >= num_slots(cache)) { *faults |= KVQO_FAULT_SLOT_RANGE; continue; }
+        decompress_row(slot_row(cache, s), d, quant_mode, quant_group_size, x_scale, y + t * y_row_stride);
+    }
+    return KVQO_OK;
+}
+
 /* ======================================================================== */
 /* [IDX] indexer_quant_cache                                                */
 /* ======================================================================== */
