@@ -469,6 +469,29 @@ def main():
                                        f"{len(calls)} input copies cycled, {len(calls) * nb >> 20} MB > L2")}
             del calls, case
             torch.cuda.empty_cache()
+        # the packed-row decoder on the headline caches (written by the timed encoder)
+        for name, case in (("cfg5a_decompress_mode0", case_a), ("cfg5b_decompress_mode2", case_b)):
+            call, st, _ = W.build_call(case)
+            call(stream)
+            cb, at = case.caches["cache"], case.attrs
+            view = st["cache"][cb.offset:].as_strided((cb.num_blocks, cb.block_size, 1, cb.head_dim),
+                                                      (cb.block_stride, cb.head_dim, cb.head_dim, 1))
+            slots = torch.from_numpy(np.ascontiguousarray(case.arrays["slot_mapping"])).to(dev)
+            T, d = case.arrays["x"].shape
+            y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+
+            def dcall(strm, view=view, slots=slots, y=y, at=at):
+                kvq.kv_decompress(view, slots, y, at["quant_mode"], at["quant_group_size"], at["x_scale"],
+                                  stream=strm)
+            us = device_us_per_launch([dcall], stream, 200)
+            valid = int((case.arrays["slot_mapping"] != -1).sum())
+            col = kvq.kv_cache_col(d, at["quant_mode"], at["quant_group_size"])
+            nb = valid * (col + 2 * d) + T * case.arrays["slot_mapping"].itemsize
+            per_config[name] = {"tokens": T, "alg_bytes": nb, "us_per_launch": us, "tokens_per_s": T / us * 1e6,
+                                "alg_GBps": nb / us / 1e3, "frac_of_peak": nb / us / 1e3 / peak,
+                                "input_copies": 1, "l2": f"{nb >> 20} MB > L2"}
+            del call, st, view, slots, y
+            torch.cuda.empty_cache()
 
     # ---------------- CPU oracle baseline (rank 0, N = 1) ----------------
     cpu = None

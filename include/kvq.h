@@ -127,6 +127,32 @@ KVQ_API kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor*
                                   int32_t quant_mode, int32_t quant_group_size, float x_scale,
                                   kvq_stream stream);
 
+/* ------------------------------------------------------------------------ */
+/* kv_decompress: the packed-row decoder, the inverse of kv_compress_epilog  */
+/* as the attention side reads the cache.  Source: the row layout and the    */
+/* formulas of aclnnKvCompressEpilog (计算公式, 约束说明), read backwards;   */
+/* the pages define only the encoding, so the decode is their plain inverse. */
+/*                                                                           */
+/* cache        uint8 [blockNum, blockSize, 1, headDim] written by            */
+/*              kv_compress_epilog with the same quant_mode,                  */
+/*              quant_group_size and x_scale (headDim >= kvCacheCol).         */
+/* slot_mapping int32 or int64, T elements, contiguous: the slot of each     */
+/*              output row; -1 leaves the row untouched.                      */
+/* y            bf16 [..., d] (the last dimension contiguous, the leading     */
+/*              dimensions flattenable to T rows with one row stride),        */
+/*              written row by row:                                           */
+/*   modes 0/1: nope y = bf16_rn(code value * group scale) (the bf16 scale,  */
+/*              or 2^(b-127) for the E8M0 byte b); rope = the stored bf16;   */
+/*   mode 2:    nope y = bf16_rn(E2M1 value * group scale); rope =           */
+/*              bf16_rn(E4M3 value / x_scale) (IEEE division).                */
+/* Validation as kv_compress_epilog; a slot outside the cache leaves its row */
+/* untouched and sets KVQ_FAULT_SLOT_RANGE (kvq_get_error).  The caller owns */
+/* y; the call allocates nothing and enqueues one kernel on `stream`.        */
+/* ------------------------------------------------------------------------ */
+KVQ_API kvq_status kvq_kv_decompress(const kvq_tensor* cache, const kvq_tensor* slot_mapping, kvq_tensor* y,
+                                     int32_t quant_mode, int32_t quant_group_size, float x_scale,
+                                     kvq_stream stream);
+
 /* Bytes of one packed row (kvCacheCol) for kv_compress_epilog, or -1 for an
  * invalid (d, quant_mode, quant_group_size).  Closed form of
  * aclnnKvCompressEpilog 约束说明 (headDim constraint); d=256, mode 1 -> 323. */

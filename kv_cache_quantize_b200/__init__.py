@@ -7,8 +7,8 @@ first call raises.
 
 Operations (same names as the C ABI without the ``kvq_`` prefix):
   kv_compress_epilog, indexer_quant_cache, kv_rmsnorm_rope_cache,
-  dequant_rope_quant_kvcache; utilities get_error, kv_cache_col,
-  indexer_scale_col, convert.
+  dequant_rope_quant_kvcache; the packed-row decoder kv_decompress;
+  utilities get_error, kv_cache_col, indexer_scale_col, convert.
 """
 from __future__ import annotations
 
@@ -19,7 +19,8 @@ from typing import Optional, Sequence, Tuple
 import torch
 
 __all__ = [
-    "KvqError", "lib", "library_path", "kv_compress_epilog", "indexer_quant_cache", "kv_rmsnorm_rope_cache",
+    "KvqError", "lib", "library_path", "kv_compress_epilog", "kv_decompress", "indexer_quant_cache",
+    "kv_rmsnorm_rope_cache",
     "dequant_rope_quant_kvcache", "get_error", "kv_cache_col", "indexer_scale_col", "convert", "selftest",
     "FAULT_SLOT_RANGE", "STATUS",
 ]
@@ -68,6 +69,7 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(library_path)
         i32, i64, vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p
         L.kvq_kv_compress_epilog.argtypes = [_P, _P, _P, i32, i32, ctypes.c_float, vp]
+        L.kvq_kv_decompress.argtypes = [_P, _P, _P, i32, i32, ctypes.c_float, vp]
         L.kvq_indexer_quant_cache.argtypes = [_P, _P, _P, _P, i32, vp]
         L.kvq_kv_rmsnorm_rope_cache.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float, i32, vp]
         L.kvq_dequant_rope_quant_kvcache.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -82,7 +84,8 @@ def lib() -> ctypes.CDLL:
         L.kvq_status_string.argtypes = [i32]
         L.kvq_status_string.restype = ctypes.c_char_p
         L.kvq_version.restype = i32
-        for name in ("kvq_kv_compress_epilog", "kvq_indexer_quant_cache", "kvq_kv_rmsnorm_rope_cache",
+        for name in ("kvq_kv_compress_epilog", "kvq_kv_decompress", "kvq_indexer_quant_cache",
+                     "kvq_kv_rmsnorm_rope_cache",
                      "kvq_dequant_rope_quant_kvcache", "kvq_get_error", "kvq_convert", "kvq_selftest"):
             getattr(L, name).restype = i32
         _LIB = L
@@ -134,6 +137,16 @@ def kv_compress_epilog(x: torch.Tensor, slot_mapping: torch.Tensor, cache: torch
     _check("kv_compress_epilog", lib().kvq_kv_compress_epilog(
         _ref(desc(x)), _ref(desc(slot_mapping)), _ref(desc(cache)), int(quant_mode), int(quant_group_size),
         float(x_scale), _stream(stream, x)))
+
+
+def kv_decompress(cache: torch.Tensor, slot_mapping: torch.Tensor, y: torch.Tensor, quant_mode: int,
+                  quant_group_size: int = 64, x_scale: float = 1.0, stream=None) -> torch.Tensor:
+    """Decode the packed rows named by slot_mapping into the bf16 rows of y (see kvq_kv_decompress);
+    rows whose slot is -1 keep their contents.  Returns y."""
+    _check("kv_decompress", lib().kvq_kv_decompress(
+        _ref(desc(cache)), _ref(desc(slot_mapping)), _ref(desc(y)), int(quant_mode), int(quant_group_size),
+        float(x_scale), _stream(stream, y)))
+    return y
 
 
 def indexer_quant_cache(x: torch.Tensor, cache: torch.Tensor, cache_scale: torch.Tensor,

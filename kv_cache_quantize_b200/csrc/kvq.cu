@@ -12,6 +12,7 @@
 #include "compress_epilog.cuh"
 #include "dequant_rope_quant.cuh"
 #include "indexer_quant.cuh"
+#include "kv_decompress.cuh"
 #include "rmsnorm_rope.cuh"
 
 namespace {
@@ -494,6 +495,63 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
 }
 
 // ---------------------------------------------------------------------------
+kvq_status kvq_kv_decompress(const kvq_tensor* cache, const kvq_tensor* slot_mapping, kvq_tensor* y,
+                             int32_t quant_mode, int32_t quant_group_size, float x_scale, kvq_stream stream) {
+    if (!cache || !slot_mapping || !y) return KVQ_ERR_NULL;
+    if (!valid_desc(cache) || !valid_desc(slot_mapping) || !valid_desc(y)) return KVQ_ERR_DTYPE;
+    if (y->dtype != KVQ_BF16) return KVQ_ERR_DTYPE;
+    if (y->ndim < 1) return KVQ_ERR_NDIM;
+    int64_t T, ys;
+    if (!flatten_rows(y, &T, &ys)) return KVQ_ERR_LAYOUT;
+    const int64_t d = y->shape[y->ndim - 1];
+    if (d <= 64 || d % 64 != 0 || d > 8192) return KVQ_ERR_SHAPE;
+    if (quant_mode < 0 || quant_mode > 2) return KVQ_ERR_ATTR;
+    const int32_t G = quant_mode == 2 ? quant_group_size : 64;
+    if (quant_mode == 2 && ((G != 16 && G != 32 && G != 64) || (d - 64) % G != 0)) return KVQ_ERR_ATTR;
+    if (!is_index_dtype(slot_mapping->dtype)) return KVQ_ERR_DTYPE;
+    if (numel(slot_mapping) != T) return KVQ_ERR_SHAPE;
+    if (!contiguous(slot_mapping)) return KVQ_ERR_LAYOUT;
+    if (cache->dtype != KVQ_U8 && cache->dtype != KVQ_I8) return KVQ_ERR_DTYPE;
+    if (cache->ndim != 4) return KVQ_ERR_NDIM;
+    if (cache->shape[2] != 1) return KVQ_ERR_SHAPE;
+    PagedRows rows;
+    int64_t head_dim;
+    kvq_status st = paged_from(cache, 1, &rows, &head_dim);
+    if (st != KVQ_OK) return st;
+    if (head_dim < kvq_kv_cache_col(d, quant_mode, G)) return KVQ_ERR_CAPACITY;
+    if (T == 0) return KVQ_OK;
+    if (!y->data || !slot_mapping->data || (!cache->data && rows.num_slots > 0)) return KVQ_ERR_NULL;
+
+    DecompressArgs a;
+    a.cache = rows;
+    a.slots = slot_mapping->data;
+    a.slots_i64 = slot_mapping->dtype == KVQ_I64;
+    a.T = T;
+    a.y = static_cast<uint16_t*>(y->data);
+    a.y_row_stride = ys;
+    a.nslice = (int32_t)(d / 32);
+    a.n = (int32_t)(d - 64);
+    a.x_scale = x_scale;
+    a.rows_vec16 = (reinterpret_cast<uintptr_t>(cache->data) % 16 == 0) && rows.row_bytes % 16 == 0 &&
+                   rows.block_stride % 16 == 0;
+    a.y_vec32 = (reinterpret_cast<uintptr_t>(y->data) % 32 == 0) && (ys * 2) % 32 == 0;
+    const int64_t nchunks = (T * a.nslice + 31) / 32;
+    const int64_t need = (nchunks + (DC_THREADS / 32) - 1) / (DC_THREADS / 32);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+#define KVQ_LAUNCH_DC(M, GG)                                                                   \
+    do {                                                                                       \
+        auto k = kv_decompress_kernel<M, GG>;                                                  \
+        k<<<(unsigned)persistent_grid(k, DC_THREADS, need), DC_THREADS, 0, s>>>(a);             \
+    } while (0)
+    if (quant_mode == 0) KVQ_LAUNCH_DC(0, 64);
+    else if (quant_mode == 1) KVQ_LAUNCH_DC(1, 64);
+    else if (G == 16) KVQ_LAUNCH_DC(2, 16);
+    else if (G == 32) KVQ_LAUNCH_DC(2, 32);
+    else KVQ_LAUNCH_DC(2, 64);
+#undef KVQ_LAUNCH_DC
+    return launched();
+}
+
 kvq_status kvq_indexer_quant_cache(const kvq_tensor* x, kvq_tensor* cache, kvq_tensor* cache_scale,
                                    const kvq_tensor* slot_mapping, int32_t quant_mode, kvq_stream stream) {
     if (!x || !cache || !cache_scale || !slot_mapping) return KVQ_ERR_NULL;

@@ -129,6 +129,28 @@ def test_compress_validation(L):
     assert ce(L, D([0, 576], "bf16"), D([0], "i32"), c) == OK                       # nothing to do
 
 
+def kd(L, c, s, y, mode=0, G=64):
+    return L.kvq_kv_decompress(R(c), R(s), R(y), mode, G, ctypes.c_float(1.0), None)
+
+
+def test_decompress_validation(L):
+    y, s, c = D([64, 576], "bf16"), D([64], "i32"), D([8, 16, 1, 672], "u8")
+    assert kd(L, c, s, y) == ENULL                        # valid up to the (absent) data
+    assert L.kvq_kv_decompress(R(c), R(s), None, 0, 64, ctypes.c_float(1), None) == ENULL
+    assert kd(L, c, s, D([64, 576], "f16")) == EDTYPE
+    assert kd(L, c, s, D([64, 600], "bf16")) == ESHAPE    # d % 64
+    assert kd(L, c, s, D([64, 64], "bf16")) == ESHAPE
+    assert kd(L, c, D([63], "i32"), y) == ESHAPE
+    assert kd(L, c, D([64], "f32"), y) == EDTYPE
+    assert kd(L, c, s, y, mode=3) == EATTR
+    assert kd(L, D([8, 16, 1, 1024], "u8"), s, y, mode=2, G=48) == EATTR
+    assert kd(L, D([8, 16, 1, 671], "u8"), s, y) == ECAP  # headDim < kvCacheCol (672)
+    assert kd(L, D([8, 16, 1, 672], "e4m3"), s, y) == EDTYPE
+    assert kd(L, D([8, 16, 672], "u8"), s, y) == ENDIM
+    assert kd(L, c, s, D([64, 576], "bf16", [1, 64])) == ELAYOUT
+    assert kd(L, c, D([0], "i32"), D([0, 576], "bf16")) == OK
+
+
 def test_indexer_validation(L):
     x, s = D([64, 128], "bf16"), D([64], "i32")
     c8, c4, sc = D([16, 8, 1, 128], "e4m3"), D([16, 8, 1, 64], "u8"), D([16, 8, 1, 4], "e8m0")
