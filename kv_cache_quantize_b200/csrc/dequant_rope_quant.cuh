@@ -3,13 +3,10 @@
 // Cache 更新模式, Kernel 实现要点: dequant Cast -> Mul -> Muls -> Add, RoPE with
 // the sine negated first, quant Div -> Add offset -> round to int8).
 //
-// A CTA walks tokens (grid-stride); its DQ_WARPS warps split the token's
-// Nq + 2*Nkv heads (warp w takes heads w, w + DQ_WARPS, ...).  Within a head of
-// D values each lane holds E = D/32 consecutive values, so the first half of
-// the head sits in lanes 0-15 and the second half in lanes 16-31 at the same
-// register positions: the half-rotation partner of every value is one
-// __shfl_xor(16) away.  Up to DQ_PASS of a warp's heads are loaded before
-// any of them is processed.
+// Two kernels: the pipelined one (aligned inputs, D a multiple of 8 up to
+// 256; see its comment below) and a general one for every other shape and
+// alignment the pages allow (one CTA per token, one thread per RoPE pair or
+// per value).
 #pragma once
 
 #include "kvq_device.cuh"
@@ -49,162 +46,12 @@ struct DrqArgs {
     int32_t stages;
 };
 
-constexpr int DQ_WARPS = 8;
-constexpr int DQ_MAX_HEADS_PER_WARP = 8;
-constexpr int DQ_PASS = 4;
-
-template <int E>
-__device__ __forceinline__ void dq_load(const DrqArgs& a, int64_t e0, float (&u)[E], const int32_t* xi) {
-    if (a.x_kind == 0) {
-        int32_t v[E];
-        if (E % 4 == 0 && a.x_vec) {
-#pragma unroll
-            for (int k = 0; k < E; k += 4) {
-                const int4 w = __ldcs(reinterpret_cast<const int4*>(xi + e0 + k));
-                v[k] = w.x; v[k + 1] = w.y; v[k + 2] = w.z; v[k + 3] = w.w;
-            }
-        } else if (E % 2 == 0 && a.x_vec) {
-#pragma unroll
-            for (int k = 0; k < E; k += 2) {
-                const int2 w = __ldcs(reinterpret_cast<const int2*>(xi + e0 + k));
-                v[k] = w.x; v[k + 1] = w.y;
-            }
-        } else {
-#pragma unroll
-            for (int k = 0; k < E; ++k) v[k] = __ldcs(xi + e0 + k);
-        }
-#pragma unroll
-        for (int k = 0; k < E; ++k) u[k] = __int2float_rn(v[k]);
-    } else {
-        const uint16_t* xh = reinterpret_cast<const uint16_t*>(a.x);
-#pragma unroll
-        for (int k = 0; k < E; ++k) {
-            const uint32_t hb = __ldcs(xh + e0 + k);
-            u[k] = a.x_kind == 2 ? __half2float(__ushort_as_half((unsigned short)hb)) : __uint_as_float(hb << 16);
-        }
-    }
-}
-
 __device__ __forceinline__ float dq_bias(const DrqArgs& a, int64_t i) {
     switch (a.bias_kind) {
         case 0: return reinterpret_cast<const float*>(a.bias)[i];
         case 1: return __half2float(__ushort_as_half(reinterpret_cast<const unsigned short*>(a.bias)[i]));
         case 2: return __uint_as_float((uint32_t) reinterpret_cast<const uint16_t*>(a.bias)[i] << 16);
         default: return __int2float_rn(reinterpret_cast<const int32_t*>(a.bias)[i]);
-    }
-}
-
-// E consecutive binary32 parameters starting at p (16-byte vectors when E % 4 == 0
-// and p is 16-byte aligned, which holds for the kernels' channel offsets when the
-// parameter tensors are 16-byte aligned: params_vec).
-template <int E>
-__device__ __forceinline__ void dq_param(const float* p, bool vec, float (&v)[E]) {
-    if (E % 4 == 0 && vec) {
-#pragma unroll
-        for (int k = 0; k < E; k += 4) {
-            const float4 w = __ldg(reinterpret_cast<const float4*>(p + k));
-            v[k] = w.x; v[k + 1] = w.y; v[k + 2] = w.z; v[k + 3] = w.w;
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < E; ++k) v[k] = __ldg(p + k);
-    }
-}
-
-__device__ __forceinline__ uint32_t dq_round16(const DrqArgs& a, float v) {
-    return a.cos_f16 ? to_f16_bits(v) : to_bf16_bits(v);
-}
-
-// E 16-bit outputs, packed into 4- or 8-byte stores
-template <int E>
-__device__ __forceinline__ void dq_store16(uint16_t* p, const DrqArgs& a, const float (&o)[E]) {
-    if (E % 4 == 0) {
-#pragma unroll
-        for (int k = 0; k < E; k += 4) {
-            const uint2 w = make_uint2(dq_round16(a, o[k]) | (dq_round16(a, o[k + 1]) << 16),
-                                       dq_round16(a, o[k + 2]) | (dq_round16(a, o[k + 3]) << 16));
-            st_b64(reinterpret_cast<uint8_t*>(p + k), w);
-        }
-    } else if (E % 2 == 0) {
-#pragma unroll
-        for (int k = 0; k < E; k += 2)
-            st_b32(reinterpret_cast<uint8_t*>(p + k), dq_round16(a, o[k]) | (dq_round16(a, o[k + 1]) << 16));
-    } else {
-#pragma unroll
-        for (int k = 0; k < E; ++k) p[k] = (uint16_t)dq_round16(a, o[k]);
-    }
-}
-
-// One head of one token: dequant, RoPE (q and k heads), outputs, int8 quant
-// and the cache write.  Called with the whole warp (the RoPE shuffle).
-template <int E>
-__device__ __forceinline__ void dq_head(const DrqArgs& a, int64_t t, int hd, float (&u)[E], const float (&cs)[E],
-                                        const float (&sn)[E], float act, int64_t slot, int pos, bool second_half) {
-    const int D = a.D;
-    const int ch0 = hd * D + pos;    // channel index within H
-    const bool pv = a.params_vec != 0;
-    // 1 dequant: ((float)x * weight_scale) * activation_scale + bias
-    if (a.x_kind == 0) {
-        float ws[E];
-        dq_param<E>(a.weight_scale + ch0, pv, ws);
-        float bs[E];
-        if (a.bias && a.bias_kind == 0) {
-            dq_param<E>(reinterpret_cast<const float*>(a.bias) + ch0, pv, bs);
-        } else if (a.bias) {
-#pragma unroll
-            for (int k = 0; k < E; ++k) bs[k] = dq_bias(a, ch0 + k);
-        }
-#pragma unroll
-        for (int k = 0; k < E; ++k) {
-            float v = __fmul_rn(u[k], ws[k]);
-            if (a.activation_scale) v = __fmul_rn(v, act);
-            if (a.bias) v = __fadd_rn(v, bs[k]);
-            u[k] = v;
-        }
-    }
-    float o[E];
-    if (hd < a.Nq + a.Nkv) {
-        // 3 RoPE, half rotation: the partner value is 16 lanes away
-#pragma unroll
-        for (int k = 0; k < E; ++k) {
-            const float p = __shfl_xor_sync(FULL_MASK, u[k], 16);
-            const float sgn_s = second_half ? sn[k] : -sn[k];
-            o[k] = __fadd_rn(__fmul_rn(u[k], cs[k]), __fmul_rn(p, sgn_s));
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < E; ++k) o[k] = u[k];
-    }
-    if (hd < a.Nq) {
-        dq_store16<E>(a.q_out + t * (int64_t)(a.Nq * D) + ch0, a, o);
-        return;
-    }
-    const bool is_k = hd < a.Nq + a.Nkv;
-    const int c0 = (is_k ? hd - a.Nq : hd - a.Nq - a.Nkv) * D + pos;   // channel in [0, Nkv*D)
-    if (a.k_out) dq_store16<E>((is_k ? a.k_out : a.v_out) + t * (int64_t)(a.Nkv * D) + c0, a, o);
-    if (slot < 0) return;
-    // 4 quant: int8(rint(w / scale + offset)), saturating
-    float sc[E], of[E];
-    dq_param<E>((is_k ? a.scale_k : a.scale_v) + c0, pv, sc);
-    const float* ofp = is_k ? a.offset_k : a.offset_v;
-    if (ofp) dq_param<E>(ofp + c0, pv, of);
-    uint32_t packed[(E + 3) / 4];
-#pragma unroll
-    for (int k = 0; k < (E + 3) / 4; ++k) packed[k] = 0u;
-#pragma unroll
-    for (int k = 0; k < E; ++k) {
-        float q = __fdiv_rn(o[k], sc[k]);
-        if (ofp) q = __fadd_rn(q, of[k]);
-        packed[k / 4] |= ((uint32_t)int8_rne_sat(q) & 0xffu) << (8 * (k % 4));
-    }
-    // 5 cache write
-    uint8_t* row = slot_row(is_k ? a.kc : a.vc, slot) + c0;
-    if (E % 4 == 0) {
-#pragma unroll
-        for (int k = 0; k < E / 4; ++k) st_b32(row + 4 * k, packed[k]);
-    } else {
-#pragma unroll
-        for (int k = 0; k < E; ++k) row[k] = (uint8_t)(packed[k / 4] >> (8 * (k % 4)));
     }
 }
 
@@ -223,48 +70,86 @@ __device__ __forceinline__ int64_t dq_slot(const DrqArgs& a, int64_t t) {
     return b * c1 + start + s;
 }
 
+// ---------------------------------------------------------------------------
+// General kernel: one CTA per token (grid-stride over tokens).  Thread i
+// takes RoPE pairs i, i + blockDim, ... of the q and k heads -- value j of a
+// head and its half-rotation partner j + D/2 together -- then values i,
+// i + blockDim, ... of the v heads.  Element loads and stores are 16-bit or
+// 8-bit and coalesced across the CTA; any alignment, any even D.
+// ---------------------------------------------------------------------------
+constexpr int DG_THREADS = 256;
 
-template <int E>
-__global__ void __launch_bounds__(DQ_WARPS * 32) dequant_rope_quant_kernel(const DrqArgs a) {
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int NH = a.Nq + 2 * a.Nkv;
+// element i of the token's x row, dequantised: ((float)x * ws) * act + bias
+__device__ __forceinline__ float dg_value(const DrqArgs& a, int64_t t, int64_t i, float act) {
+    if (a.x_kind == 0) {
+        float v = __fmul_rn(__int2float_rn(reinterpret_cast<const int32_t*>(a.x)[t * a.H + i]), a.weight_scale[i]);
+        if (a.activation_scale) v = __fmul_rn(v, act);
+        if (a.bias) v = __fadd_rn(v, dq_bias(a, i));
+        return v;
+    }
+    const uint32_t h = reinterpret_cast<const uint16_t*>(a.x)[t * a.H + i];
+    return a.x_kind == 2 ? __half2float(__ushort_as_half((unsigned short)h)) : __uint_as_float(h << 16);
+}
+
+__device__ __forceinline__ float dg_half(const uint16_t* p, int64_t i, bool f16) {
+    const uint32_t h = p[i];
+    return f16 ? __half2float(__ushort_as_half((unsigned short)h)) : __uint_as_float(h << 16);
+}
+
+__device__ __forceinline__ uint16_t dg_round16(float v, bool f16) {
+    return (uint16_t)(f16 ? to_f16_bits(v) : to_bf16_bits(v));
+}
+
+// static int8 of channel c: round half to even of o / scale + offset, saturated
+__device__ __forceinline__ uint8_t dg_int8(const float* sc, const float* of, int64_t c, float o) {
+    float q = __fdiv_rn(o, sc[c]);
+    if (of) q = __fadd_rn(q, of[c]);
+    return (uint8_t)int8_rne_sat(q);
+}
+
+__global__ void __launch_bounds__(DG_THREADS) dequant_rope_quant_general_kernel(const DrqArgs a) {
     const int64_t ntok = a.B * a.S;
-    const int D = a.D;
-    const int pos = lane * E;                // first position of this lane inside a head
-    const bool second_half = lane >= 16;
-    const int32_t* xi = reinterpret_cast<const int32_t*>(a.x);
-
+    const int D = a.D, h = a.D / 2;
+    const int64_t C = (int64_t)a.Nkv * D;
+    const bool f16 = a.cos_f16 != 0;
     for (int64_t t = blockIdx.x; t < ntok; t += gridDim.x) {
-        // destination row of this token (or -1 skip / -2 fault)
         const int64_t slot = dq_slot(a, t);
         if (slot == -2 && threadIdx.x == 0) raise_fault(FAULT_SLOT_RANGE);
-
-        float cs[E], sn[E];
-#pragma unroll
-        for (int k = 0; k < E; ++k) {
-            const uint32_t cb = a.cos[t * D + pos + k], sb = a.sin[t * D + pos + k];
-            cs[k] = a.cos_f16 ? __half2float(__ushort_as_half((unsigned short)cb)) : __uint_as_float(cb << 16);
-            sn[k] = a.cos_f16 ? __half2float(__ushort_as_half((unsigned short)sb)) : __uint_as_float(sb << 16);
-        }
+        uint8_t* krow = slot >= 0 ? slot_row(a.kc, slot) : nullptr;
+        uint8_t* vrow = slot >= 0 ? slot_row(a.vc, slot) : nullptr;
         const float act = (a.x_kind == 0 && a.activation_scale) ? a.activation_scale[t] : 1.0f;
-
-        // the warp's heads are hd = warp + i * DQ_WARPS; DQ_PASS of them are
-        // loaded before any is processed
-        const int nh = (NH - warp + DQ_WARPS - 1) / DQ_WARPS;
-        for (int i0 = 0; i0 < nh; i0 += DQ_PASS) {
-            float u[DQ_PASS][E];
-#pragma unroll
-            for (int i = 0; i < DQ_PASS; ++i) {
-                const int hd = warp + (i0 + i) * DQ_WARPS;
-                if (i0 + i < nh) dq_load<E>(a, t * a.H + (int64_t)hd * D + pos, u[i], xi);
+        const uint16_t* cs = a.cos + t * D;
+        const uint16_t* sn = a.sin + t * D;
+        // q and k heads: RoPE pairs (j, j + D/2)
+        const int64_t npairs = (int64_t)(a.Nq + a.Nkv) * h;
+        for (int64_t p = threadIdx.x; p < npairs; p += blockDim.x) {
+            const int hd = (int)(p / h), j = (int)(p - (int64_t)hd * h);
+            const int64_t e0 = (int64_t)hd * D + j;
+            const float u0 = dg_value(a, t, e0, act), u1 = dg_value(a, t, e0 + h, act);
+            // o_j = u_j c_j - u_{j+h} s_j,  o_{j+h} = u_{j+h} c_{j+h} + u_j s_{j+h}
+            const float o0 = __fadd_rn(__fmul_rn(u0, dg_half(cs, j, f16)), __fmul_rn(u1, -dg_half(sn, j, f16)));
+            const float o1 = __fadd_rn(__fmul_rn(u1, dg_half(cs, j + h, f16)), __fmul_rn(u0, dg_half(sn, j + h, f16)));
+            if (hd < a.Nq) {
+                uint16_t* q = a.q_out + t * (int64_t)a.Nq * D + e0;
+                q[0] = dg_round16(o0, f16);
+                q[h] = dg_round16(o1, f16);
+                continue;
             }
-#pragma unroll
-            for (int i = 0; i < DQ_PASS; ++i) {
-                if (i0 + i >= nh) break;
-                const int hd = warp + (i0 + i) * DQ_WARPS;
-                dq_head<E>(a, t, hd, u[i], cs, sn, act, slot, pos, second_half);
+            const int64_t c = (int64_t)(hd - a.Nq) * D + j;
+            if (a.k_out) {
+                a.k_out[t * C + c] = dg_round16(o0, f16);
+                a.k_out[t * C + c + h] = dg_round16(o1, f16);
             }
+            if (krow) {
+                krow[c] = dg_int8(a.scale_k, a.offset_k, c, o0);
+                krow[c + h] = dg_int8(a.scale_k, a.offset_k, c + h, o1);
+            }
+        }
+        // v heads: no RoPE
+        for (int64_t c = threadIdx.x; c < C; c += blockDim.x) {
+            const float o = dg_value(a, t, (int64_t)(a.Nq + a.Nkv) * D + c, act);
+            if (a.v_out) a.v_out[t * C + c] = dg_round16(o, f16);
+            if (vrow) vrow[c] = dg_int8(a.scale_v, a.offset_v, c, o);
         }
     }
 }

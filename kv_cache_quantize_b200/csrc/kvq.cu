@@ -792,7 +792,6 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
     if (st != KVQ_OK) return st;
     st = paged_from(v_cache, Nkv, &vr, &hd);
     if (st != KVQ_OK) return st;
-    if (D % 32 != 0 || D > 256 || Nq + 2 * Nkv > DQ_WARPS * DQ_MAX_HEADS_PER_WARP) return KVQ_ERR_UNSUPPORTED;
     if (!contiguous(x) || !contiguous(cos) || !contiguous(sin) || !contiguous(indices) || !contiguous(q_out))
         return KVQ_ERR_LAYOUT;
     if (numel(cos) != B * S * D || numel(sin) != B * S * D) return KVQ_ERR_SHAPE;
@@ -928,22 +927,10 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
 #undef KVQ_LAUNCH_DT
         return launched();
     }
-#define KVQ_LAUNCH_DQ(E)                                                                       \
-    do {                                                                                       \
-        auto k = dequant_rope_quant_kernel<E>;                                                 \
-        k<<<(unsigned)persistent_grid(k, DQ_WARPS * 32, need), DQ_WARPS * 32, 0, s>>>(a);       \
-    } while (0)
-    switch (D / 32) {
-        case 1: KVQ_LAUNCH_DQ(1); break;
-        case 2: KVQ_LAUNCH_DQ(2); break;
-        case 3: KVQ_LAUNCH_DQ(3); break;
-        case 4: KVQ_LAUNCH_DQ(4); break;
-        case 5: KVQ_LAUNCH_DQ(5); break;
-        case 6: KVQ_LAUNCH_DQ(6); break;
-        case 7: KVQ_LAUNCH_DQ(7); break;
-        default: KVQ_LAUNCH_DQ(8); break;
-    }
-#undef KVQ_LAUNCH_DQ
+    // every other shape and alignment: one CTA per token
+    dequant_rope_quant_general_kernel<<<(unsigned)persistent_grid(dequant_rope_quant_general_kernel, DG_THREADS,
+                                                                  need),
+                                        DG_THREADS, 0, s>>>(a);
     return launched();
 }
 

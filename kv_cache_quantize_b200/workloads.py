@@ -347,12 +347,22 @@ def idx(a) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
 
 
-def build_call(case: Case):
+def shifted(t: torch.Tensor) -> torch.Tensor:
+    """The same values in a view that starts one element into a larger buffer
+    (so no longer 16-byte aligned), for tests of the unaligned paths."""
+    buf = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+    buf[1:].copy_(t.reshape(-1))
+    return buf[1:].view(t.shape)
+
+
+def build_call(case: Case, misalign: bool = False):
     """Device tensors for a case and a closure that runs the library call once.
 
     Returns (call, storages, outputs): call(stream=None) enqueues the operation;
     storages maps each cache name to the device copy of its whole byte buffer;
     outputs collects the dense outputs (q_out, k_out, v_out) after a call.
+    misalign: dequant_rope_quant_kvcache's x, cos and sin start one element
+    past a 16-byte boundary.
     """
     import kv_cache_quantize_b200 as kvq
     a, at = case.arrays, case.attrs
@@ -394,6 +404,8 @@ def build_call(case: Case):
         else:
             x = half_tensor(a["x"], at["x_dtype"])
         cos, sin = half_tensor(a["cos"], at["cos_dtype"]), half_tensor(a["sin"], at["cos_dtype"])
+        if misalign:
+            x, cos, sin = shifted(x), shifted(cos), shifted(sin)
         bias = None
         if "bias" in a:
             bdt = at["bias_dtype"]

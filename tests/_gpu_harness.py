@@ -13,9 +13,9 @@ import kv_cache_quantize_b200 as kvq
 from kv_cache_quantize_b200.workloads import Case, build_call, dev_cache, half_tensor  # noqa: F401
 
 
-def run_gpu(case: Case):
+def run_gpu(case: Case, misalign: bool = False):
     """Returns (storages as numpy, 16-bit outputs as uint16 numpy, fault bits)."""
-    call, st, outs = build_call(case)
+    call, st, outs = build_call(case, misalign)
     kvq.get_error()            # clear stale bits
     call()
     torch.cuda.synchronize()

@@ -227,9 +227,13 @@ def test_dequant_rope_quant_validation(L):
     assert f(kvo=1) == ENULL                                # kv_output needs k_out / v_out
     assert f(bias=D([3072], "i8")) == EDTYPE
     assert f(bias=D([3072], "bf16")) == ENULL
-    kc48 = D([512, 128, 4, 48], "i8")
+    kc48, s48 = D([512, 128, 4, 48], "i8"), D([4, 48], "f32")
     assert f(kc=kc48, vc=kc48, c=D([16, 1024, 1, 48], "bf16"), x=D([16, 1024, 1152], "i32"),
-             splits=(768, 192, 192), q=D([16, 1024, 16, 48], "bf16")) == EUNSUP   # D % 32 != 0
+             splits=(768, 192, 192), q=D([16, 1024, 16, 48], "bf16"), sk=s48,
+             ws=D([1152], "f32")) == ENULL   # D % 32 != 0 is supported
+    kc24 = D([512, 128, 4, 24], "i8")
+    assert f(kc=kc24, vc=kc24, c=D([16, 1024, 1, 24], "bf16"), x=D([16, 1024, 576], "i32"),
+             splits=(288, 144, 144), q=D([16, 1024, 12, 24], "bf16")) == ESHAPE   # D % 16 != 0
 
 
 def test_empty_inputs_are_accepted_whatever_their_strides(L):

@@ -18,9 +18,9 @@ pytestmark = pytest.mark.gpu
 THREADS = 16
 
 
-def _same(case, check_outputs=True):
+def _same(case, check_outputs=True, misalign=False):
     st_o, out_o, f_o = run_oracle(case, threads=THREADS)
-    st_g, out_g, f_g = run_gpu(case)
+    st_g, out_g, f_g = run_gpu(case, misalign)
     assert f_g == f_o, f"fault bits gpu={f_g} oracle={f_o}"
     for k in st_o:
         a, b = st_g[k], st_o[k]
@@ -241,6 +241,29 @@ def test_drq_modes(cache_mode, kv_output):
 @pytest.mark.parametrize("D", [32, 64, 96, 256])
 def test_drq_head_dims(D):
     _same(_dq(D=D, Nq=4, Nkv=1, kv_output=True))   # H = 6*D, a multiple of 64
+
+
+# head sizes a multiple of 16 but not of 32 (pipelined kernel, D/8 lanes per
+# head), and heads wider than 256 (general kernel); H = 4 D a multiple of 64
+@pytest.mark.parametrize("D", [16, 48, 80, 512, 1024])
+def test_drq_other_head_dims(D):
+    _same(_dq(D=D, Nq=2, Nkv=1, kv_output=True, S=12))
+
+
+# inputs off 16-byte alignment take the general kernel
+@pytest.mark.parametrize("D,x_dtype", [(128, "i32"), (64, "bf16"), (16, "i32"), (512, "f16")])
+@pytest.mark.parametrize("cache_mode", ["page", "contiguous"])
+def test_drq_unaligned_inputs(D, x_dtype, cache_mode):
+    _same(_dq(D=D, Nq=2, Nkv=1, S=12, x_dtype=x_dtype, cos_dtype="bf16" if x_dtype != "f16" else "f16",
+              kv_output=True, cache_mode=cache_mode, skip_frac=0.1 if cache_mode == "page" else 0.0),
+          misalign=True)
+
+
+def test_drq_unaligned_bias_kinds_and_named_shape():
+    for bias_dtype in ("bf16", "i32", None):
+        _same(_dq(bias_dtype=bias_dtype, with_offsets=bias_dtype is not None,
+                  with_activation_scale=bias_dtype is not None), misalign=True)
+    _same(W.cfg4_dequant_rope_quant(x_range=1 << 12), misalign=True)
 
 
 @pytest.mark.parametrize("bias_dtype", ["f32", "bf16", "f16", "i32", None])
