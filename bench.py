@@ -17,10 +17,13 @@ copies that their bytes exceed twice the L2 size (one copy, L2-resident, for
 the latency-bound decode-sized workloads).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--scaling weak|strong]
 
 With N > 1 the script runs under torchrun, one process per GPU; tokens are
-independent, so every rank runs its own copy of the workload (weak scaling, no
-collective on the data path) and the step time is the maximum over ranks.
+independent and each rank owns its caches, so there is no collective on the
+data path: by default every rank runs its own copy of the workload (weak
+scaling); --scaling strong splits the rows of one workload over the ranks.
+The step time is the maximum over ranks.
 """
 from __future__ import annotations
 
@@ -132,6 +135,52 @@ def profiled_traffic(kernel: str):
         if len(parts) >= 3 and parts[0] == kernel and parts[1] == src:
             return float(parts[2])
     return None
+
+
+# ---------------------------------------------------------------------------
+# ranks.  Every token row is independent and each rank owns its caches (its
+# own sequences' blocks), so ranks exchange nothing on the data path; the
+# process group carries only barriers and the max-over-ranks timing.
+# ---------------------------------------------------------------------------
+def shard_range(n: int, rank: int, world: int):
+    """Contiguous share [lo, hi) of n units for rank; shares differ by at most one."""
+    q, r = divmod(n, world)
+    lo = rank * q + min(rank, r)
+    return lo, lo + q + (1 if rank < r else 0)
+
+
+def rank_workload(make, rank: int, world: int, scaling: str):
+    """This rank's part of a compress workload.  weak: a whole copy with the rank's
+    own seed (per-GPU work fixed as ranks are added); strong: rows
+    shard_range(T, rank, world) of the one seed-0 workload, written into the
+    rank's own copy of the cache."""
+    if scaling == "weak":
+        return make(seed=rank)
+    case = make(seed=0)
+    T = case.arrays["x"].shape[0]
+    lo, hi = shard_range(T, rank, world)
+    case.arrays = {"x": case.arrays["x"][lo:hi], "slot_mapping": case.arrays["slot_mapping"][lo:hi]}
+    case.name = f"{case.name}[{lo}:{hi}]"
+    return case
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest x over the ranks of the default process group (x itself alone)."""
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(n: int, dist, device) -> int:
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return n
+    t = torch.tensor([n], dtype=torch.int64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return int(t.item())
 
 
 # ---------------------------------------------------------------------------
@@ -316,6 +365,8 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--scaling", default="weak", choices=["weak", "strong"],
+                    help="weak: each rank a whole copy of the workload; strong: its rows split over the ranks")
     ap.add_argument("--no-per-config", action="store_true", help="skip the per-workload breakdown")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing for cpu_baseline")
     ap.add_argument("--profile-workload", default=None,
@@ -348,8 +399,8 @@ def main():
     kvq.lib()
 
     # ---------------- headline workload ----------------
-    case_a = W.cfg5a_compress_mode0(seed=rank)
-    case_b = W.cfg5b_compress_mode2(seed=rank)
+    case_a = rank_workload(W.cfg5a_compress_mode0, rank, world, args.scaling)
+    case_b = rank_workload(W.cfg5b_compress_mode2, rank, world, args.scaling)
     call_a, st_a, _ = W.build_call(case_a)
     call_b, st_b, _ = W.build_call(case_b)
     stream = torch.cuda.current_stream(dev)
@@ -379,17 +430,15 @@ def main():
             e2.record(stream)
         stop.record(stream)
         torch.cuda.synchronize(dev)
-    elapsed = start.elapsed_time(stop) / 1e3
+    elapsed = max_over_ranks(start.elapsed_time(stop) / 1e3, dist, dev)
+    tokens_all_ranks = sum_over_ranks(tokens_per_step, dist, dev)
     if world > 1:
-        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
         dist.barrier()
     ms_a = [e0.elapsed_time(e1) for e0, e1, _ in ev]
     ms_b = [e1.elapsed_time(e2) for _, e1, e2 in ev]
     faults = kvq.get_error(stream)
 
-    value = world * tokens_per_step * args.steps / elapsed
+    value = tokens_all_ranks * args.steps / elapsed
     peak, peak_kind = hbm_peak()
     avg_a, avg_b = statistics.mean(ms_a) / 1e3, statistics.mean(ms_b) / 1e3
     kernels = {
@@ -505,12 +554,14 @@ def main():
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "scaling": args.scaling, "vs_baseline": None, "dtype": "f32", "data": "synthetic",
                 "config": {"workload": WORKLOAD, "tokens_per_step_per_gpu": tokens_per_step,
                            "alg_bytes_per_step_per_gpu": bytes_a + bytes_b,
                            "alg_GBps_per_gpu": (bytes_a + bytes_b) * args.steps / elapsed / 1e9,
                            "l2": "inputs larger than L2 (two 302 MB x buffers per step), no flush",
-                           "parallelism": f"replicas x{world} (independent token batches, no collective)"},
+                           "parallelism": (f"replicas x{world} (independent token batches, no collective)"
+                                           if args.scaling == "weak" else
+                                           f"rows split over {world} ranks (own caches, no collective)")},
                 "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": 2 * args.steps, "clocks": clocks.summary(), "fault_bits": faults,
                 "per_config": per_config}
