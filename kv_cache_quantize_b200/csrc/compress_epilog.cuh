@@ -144,6 +144,8 @@ __device__ __forceinline__ void ce_segment(const CompressArgs& a, const uint4& v
 
 template <int MODE, int G>
 __global__ void __launch_bounds__(CE_THREADS) compress_epilog_kernel(const CompressArgs a) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int team = lane >> 3;
     const int sub = lane & 7;
@@ -415,6 +417,8 @@ __host__ __device__ inline uint32_t ct_out_pitch(int col) { return (uint32_t)(((
 
 template <int MODE, int G>
 __global__ void __launch_bounds__(CT_MAX_THREADS, 1) compress_tma_kernel(const CompressArgs a) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ __align__(128) uint8_t smem[];
     const int S = a.stages;
     const int NCW = a.ncw;                         // consumer warps

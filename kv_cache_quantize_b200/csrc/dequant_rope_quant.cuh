@@ -108,6 +108,8 @@ __device__ __forceinline__ uint8_t dg_int8(const float* sc, const float* of, int
 }
 
 __global__ void __launch_bounds__(DG_THREADS) dequant_rope_quant_general_kernel(const DrqArgs a) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t ntok = a.B * a.S;
     const int D = a.D, h = a.D / 2;
     const int64_t C = (int64_t)a.Nkv * D;
@@ -280,6 +282,8 @@ __device__ __forceinline__ uint32_t dt_int8x4(const float (&o)[4], const float* 
 // 16-bit outputs are f16 (else bf16).
 template <int XK, bool F16>
 __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(const DrqArgs a) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ __align__(128) uint8_t smem[];
     const int S = a.stages, TPS = a.tps, D = a.D;
     constexpr int XB = XK == 0 ? 4 : 2;

@@ -84,6 +84,8 @@ __device__ __forceinline__ void ix_store_codes(uint8_t* p, const uint32_t (&c)[8
 
 template <int MODE, bool F16, bool E5M2>
 __global__ void __launch_bounds__(IX_THREADS) indexer_quant_kernel(const IndexerArgs a) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int ts = a.team_shift;
     const int TG = 1 << ts;

@@ -170,6 +170,8 @@ __device__ __forceinline__ const uint8_t* dc_row(const DecompressArgs& a, int64_
 
 template <int MODE, int G>
 __global__ void __launch_bounds__(DC_THREADS) kv_decompress_kernel(const DecompressArgs a) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;

@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "kvq.h"
 #include "compress_epilog.cuh"
@@ -186,6 +187,24 @@ int64_t persistent_grid(K kernel, int threads, int64_t needed_blocks, size_t sme
     return g < 1 ? 1 : g;
 }
 
+// Launch with programmatic stream serialization (see pdl_wait in
+// kvq_device.cuh): the kernel may be scheduled before the previous kernel of
+// the stream completes and waits for it on the device.
+template <typename... P, typename... A>
+void launch(void (*kernel)(P...), unsigned grid, unsigned block, size_t smem, cudaStream_t s, A&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
+
 kvq_status launched() {
     return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
@@ -194,6 +213,8 @@ kvq_status launched() {
 // conversion kernel (kvq_convert)
 // ---------------------------------------------------------------------------
 __global__ void convert_kernel(int32_t fmt, const float* in, int64_t n, uint8_t* out) {
+    pdl_wait();
+    pdl_trigger();
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         const float v = in[i];
         switch (fmt) {
@@ -468,7 +489,7 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
 #define KVQ_LAUNCH_CT(M, GG)                                                                   \
     do {                                                                                       \
         auto k = compress_tma_kernel<M, GG>;                                                   \
-        k<<<(unsigned)persistent_grid(k, threads, tiles, smem), threads, smem, s>>>(a);        \
+        launch(k, (unsigned)persistent_grid(k, threads, tiles, smem), threads, smem, s, a);     \
     } while (0)
         if (quant_mode == 0) KVQ_LAUNCH_CT(0, 64);
         else if (quant_mode == 1) KVQ_LAUNCH_CT(1, 64);
@@ -483,7 +504,7 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
 #define KVQ_LAUNCH_CE(M, GG)                                                                   \
     do {                                                                                       \
         auto k = compress_epilog_kernel<M, GG>;                                                \
-        k<<<(unsigned)persistent_grid(k, CE_THREADS, need), CE_THREADS, 0, s>>>(a);             \
+        launch(k, (unsigned)persistent_grid(k, CE_THREADS, need), CE_THREADS, 0, s, a);          \
     } while (0)
     if (quant_mode == 0) KVQ_LAUNCH_CE(0, 64);
     else if (quant_mode == 1) KVQ_LAUNCH_CE(1, 64);
@@ -541,7 +562,7 @@ kvq_status kvq_kv_decompress(const kvq_tensor* cache, const kvq_tensor* slot_map
 #define KVQ_LAUNCH_DC(M, GG)                                                                   \
     do {                                                                                       \
         auto k = kv_decompress_kernel<M, GG>;                                                  \
-        k<<<(unsigned)persistent_grid(k, DC_THREADS, need), DC_THREADS, 0, s>>>(a);             \
+        launch(k, (unsigned)persistent_grid(k, DC_THREADS, need), DC_THREADS, 0, s, a);          \
     } while (0)
     if (quant_mode == 0) KVQ_LAUNCH_DC(0, 64);
     else if (quant_mode == 1) KVQ_LAUNCH_DC(1, 64);
@@ -615,7 +636,7 @@ kvq_status kvq_indexer_quant_cache(const kvq_tensor* x, kvq_tensor* cache, kvq_t
 #define KVQ_LAUNCH_IX(M, F, E)                                                                 \
     do {                                                                                       \
         auto k = indexer_quant_kernel<M, F, E>;                                                \
-        k<<<(unsigned)persistent_grid(k, IX_THREADS, need), IX_THREADS, 0, s>>>(a);             \
+        launch(k, (unsigned)persistent_grid(k, IX_THREADS, need), IX_THREADS, 0, s, a);          \
     } while (0)
 #define KVQ_LAUNCH_IX_FE(M)                                                                    \
     do {                                                                                       \
@@ -744,8 +765,8 @@ kvq_status kvq_kv_rmsnorm_rope_cache(const kvq_tensor* kv, const kvq_tensor* gam
     a.eps = epsilon;
     const int64_t warps_per_block = RR_THREADS / 32;
     const int64_t need = (B * S + warps_per_block - 1) / warps_per_block;
-    rmsnorm_rope_kernel<<<(unsigned)persistent_grid(rmsnorm_rope_kernel, RR_THREADS, need), RR_THREADS, 0,
-                          reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    launch(rmsnorm_rope_kernel, (unsigned)persistent_grid(rmsnorm_rope_kernel, RR_THREADS, need), RR_THREADS, 0,
+           reinterpret_cast<cudaStream_t>(stream), a);
     return launched();
 }
 
@@ -914,7 +935,7 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
 #define KVQ_LAUNCH_DT(XK, F)                                                                   \
     do {                                                                                       \
         auto k = dequant_rope_quant_tma_kernel<XK, F>;                                         \
-        k<<<(unsigned)persistent_grid(k, DT_THREADS, tiles, smem), DT_THREADS, smem, s>>>(a);  \
+        launch(k, (unsigned)persistent_grid(k, DT_THREADS, tiles, smem), DT_THREADS, smem, s, a); \
     } while (0)
         if (a.x_kind == 0) {
             if (f16) KVQ_LAUNCH_DT(0, true);
@@ -928,9 +949,8 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
         return launched();
     }
     // every other shape and alignment: one CTA per token
-    dequant_rope_quant_general_kernel<<<(unsigned)persistent_grid(dequant_rope_quant_general_kernel, DG_THREADS,
-                                                                  need),
-                                        DG_THREADS, 0, s>>>(a);
+    launch(dequant_rope_quant_general_kernel,
+           (unsigned)persistent_grid(dequant_rope_quant_general_kernel, DG_THREADS, need), DG_THREADS, 0, s, a);
     return launched();
 }
 
@@ -956,8 +976,8 @@ kvq_status kvq_convert(int32_t fmt, const float* in, int64_t n, void* out, kvq_s
     if (n == 0) return KVQ_OK;
     if (!in || !out) return KVQ_ERR_NULL;
     const int64_t need = (n + 255) / 256;
-    convert_kernel<<<(unsigned)persistent_grid(convert_kernel, 256, need), 256, 0,
-                     reinterpret_cast<cudaStream_t>(stream)>>>(fmt, in, n, static_cast<uint8_t*>(out));
+    launch(convert_kernel, (unsigned)persistent_grid(convert_kernel, 256, need), 256, 0,
+           reinterpret_cast<cudaStream_t>(stream), fmt, in, n, static_cast<uint8_t*>(out));
     return launched();
 }
 

@@ -27,6 +27,19 @@ constexpr unsigned FAULT_SLOT_RANGE = 0x1u;
 __device__ __forceinline__ void raise_fault(unsigned bits) { atomicOr(&g_fault_word, bits); }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  The library launches its kernels so that a
+// kernel may be scheduled while the previous kernel of the stream is still
+// finishing; every kernel calls pdl_wait() before its first global-memory
+// access (reads and writes: the previous kernel may still read what this one
+// overwrites), which returns once the previous kernel has completed and its
+// writes are visible (at once for a kernel launched without the attribute),
+// and then pdl_trigger(), which lets the next kernel's CTAs start as soon as
+// this grid's CTAs leave room for them.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // 16-bit float widening (exact) and narrowing (round to nearest even)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -96,6 +96,8 @@ __device__ __forceinline__ int64_t rr_slot(const RmsRopeArgs& a, int64_t b, int6
 }
 
 __global__ void __launch_bounds__(RR_THREADS) rmsnorm_rope_kernel(const RmsRopeArgs a) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
