@@ -284,8 +284,11 @@ KVQ_API kvq_status kvq_convert(int32_t fmt, const float* in, int64_t n, void* ou
  * groups of four, among 2^28 random (value, scale, offset) triples (half of
  * them within a few ulps of a rounding tie), whose static int8 codes from the
  * dequant kernel's reciprocal-based quotient differ from those of IEEE
- * division.  Blocks until done; *result receives the count (0 means the
- * shortcut is exact on the domain). */
+ * division; 7: the bounded wait of the pipelined kernels, run out on purpose
+ * (a shared-memory barrier that nothing completes, a short limit): 1 when the
+ * wait gave up as designed -- it also sets KVQ_FAULT_TIMEOUT, which
+ * kvq_get_error returns and clears.  Blocks until done; *result receives the
+ * count (0 means the shortcut is exact on the domain). */
 KVQ_API kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream);
 
 /* Static description of a status code. */

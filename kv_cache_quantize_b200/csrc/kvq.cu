@@ -9,6 +9,8 @@
 #include <mutex>
 #include <utility>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kvq.h"
 #include "compress_epilog.cuh"
 #include "dequant_rope_quant.cuh"
@@ -133,6 +135,13 @@ kvq_status paged_from(const kvq_tensor* c, int64_t inner, PagedRows* out, int64_
 }
 
 bool is_index_dtype(int32_t dt) { return dt == KVQ_I32 || dt == KVQ_I64; }
+
+// A named NVTX range over one C-ABI call (visible in profilers; a no-op
+// unless a tool is attached).
+struct Trace {
+    explicit Trace(const char* name) { nvtxRangePushA(name); }
+    ~Trace() { nvtxRangePop(); }
+};
 
 // ---------------------------------------------------------------------------
 // launch sizing: a grid of (SMs x resident blocks) persistent blocks at most
@@ -333,6 +342,21 @@ __global__ void selftest_int8_kernel() {
     if (bad) atomicAdd(&g_selftest_count, bad);
 }
 
+// The bounded wait of the pipelined kernels running out: one warp waits on
+// an mbarrier that nothing arrives on, with a short limit; the wait must
+// return false (counted) and set FAULT_TIMEOUT in the fault word.  The CTA
+// then exits normally -- no GPU fault, hang or trap is involved.
+__global__ void selftest_timeout_kernel() {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    const bool done = __all_sync(FULL_MASK, mbar_wait(&bar, 0u, 4096u));
+    if (threadIdx.x == 0 && !done) atomicAdd(&g_selftest_count, 1ull);
+}
+
 // every positive finite bf16 amax (bits < 0x7f80) and every positive finite
 // f16 amax (bits < 0x7c00) over the three format maxima
 __global__ void selftest_fmax_kernel() {
@@ -355,7 +379,7 @@ extern "C" {
 
 kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream) {
     if (!result) return KVQ_ERR_NULL;
-    if (which < 0 || which > 6) return KVQ_ERR_ATTR;
+    if (which < 0 || which > 7) return KVQ_ERR_ATTR;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const unsigned long long zero = 0ull;
     unsigned long long h = 0ull;
@@ -363,6 +387,7 @@ kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream) {
         return KVQ_ERR_CUDA;
     if (which == 4) selftest_fmax_kernel<<<256, 256, 0, s>>>();
     else if (which == 6) selftest_int8_kernel<<<65536, 256, 0, s>>>();
+    else if (which == 7) selftest_timeout_kernel<<<1, 32, 0, s>>>();
     else selftest_div_kernel<<<65536, 256, 0, s>>>(which);
     if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
     if (cudaMemcpyFromSymbolAsync(&h, g_selftest_count, sizeof(h), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -417,6 +442,7 @@ int64_t kvq_indexer_scale_col(int64_t d, int32_t quant_mode) {
 kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_mapping, kvq_tensor* cache,
                                   int32_t quant_mode, int32_t quant_group_size, float x_scale,
                                   kvq_stream stream) {
+    Trace trace("kvq_kv_compress_epilog");
     if (!x || !slot_mapping || !cache) return KVQ_ERR_NULL;
     if (!valid_desc(x) || !valid_desc(slot_mapping) || !valid_desc(cache)) return KVQ_ERR_DTYPE;
     if (x->dtype != KVQ_BF16) return KVQ_ERR_DTYPE;
@@ -518,6 +544,7 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
 // ---------------------------------------------------------------------------
 kvq_status kvq_kv_decompress(const kvq_tensor* cache, const kvq_tensor* slot_mapping, kvq_tensor* y,
                              int32_t quant_mode, int32_t quant_group_size, float x_scale, kvq_stream stream) {
+    Trace trace("kvq_kv_decompress");
     if (!cache || !slot_mapping || !y) return KVQ_ERR_NULL;
     if (!valid_desc(cache) || !valid_desc(slot_mapping) || !valid_desc(y)) return KVQ_ERR_DTYPE;
     if (y->dtype != KVQ_BF16) return KVQ_ERR_DTYPE;
@@ -575,6 +602,7 @@ kvq_status kvq_kv_decompress(const kvq_tensor* cache, const kvq_tensor* slot_map
 
 kvq_status kvq_indexer_quant_cache(const kvq_tensor* x, kvq_tensor* cache, kvq_tensor* cache_scale,
                                    const kvq_tensor* slot_mapping, int32_t quant_mode, kvq_stream stream) {
+    Trace trace("kvq_indexer_quant_cache");
     if (!x || !cache || !cache_scale || !slot_mapping) return KVQ_ERR_NULL;
     if (!valid_desc(x) || !valid_desc(cache) || !valid_desc(cache_scale) || !valid_desc(slot_mapping))
         return KVQ_ERR_DTYPE;
@@ -708,6 +736,7 @@ kvq_status kvq_kv_rmsnorm_rope_cache(const kvq_tensor* kv, const kvq_tensor* gam
                                      const kvq_tensor* ckv_scale, const kvq_tensor* k_offset,
                                      const kvq_tensor* ckv_offset, float epsilon, int32_t cache_mode,
                                      kvq_stream stream) {
+    Trace trace("kvq_kv_rmsnorm_rope_cache");
     if (!kv || !gamma || !cos || !sin || !index || !k_cache || !ckv_cache) return KVQ_ERR_NULL;
     if (!valid_desc(kv) || !valid_desc(gamma) || !valid_desc(cos) || !valid_desc(sin) || !valid_desc(index))
         return KVQ_ERR_DTYPE;
@@ -780,6 +809,7 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
                                           int32_t quant_mode, int32_t layout, int32_t kv_output,
                                           int32_t cache_mode, kvq_tensor* q_out, kvq_tensor* k_out,
                                           kvq_tensor* v_out, kvq_stream stream) {
+    Trace trace("kvq_dequant_rope_quant_kvcache");
     if (!x || !cos || !sin || !k_cache || !v_cache || !indices || !scale_k || !scale_v || !q_out || !size_splits)
         return KVQ_ERR_NULL;
     if (!valid_desc(x) || !valid_desc(cos) || !valid_desc(sin) || !valid_desc(k_cache) || !valid_desc(v_cache) ||

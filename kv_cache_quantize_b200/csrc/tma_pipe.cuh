@@ -54,9 +54,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
-// Wait until the phase of the given parity has completed; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    for (uint32_t i = 0; i < PIPE_WAIT_LIMIT; ++i)
+// Wait until the phase of the given parity has completed; false (and the
+// FAULT_TIMEOUT bit) after `limit` unsuccessful tries.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit = PIPE_WAIT_LIMIT) {
+    for (uint32_t i = 0; i < limit; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     raise_fault(FAULT_TIMEOUT);
     return false;

@@ -10,7 +10,10 @@ whole input domain against IEEE division:
   * the dequant kernel's static int8 quantisation through a per-channel
     reciprocal (two-step Markstein form, IEEE division outside its guard):
     the same int8 codes as IEEE division on 2^28 random and near-tie
-    (value, scale, offset) triples."""
+    (value, scale, offset) triples.
+Also the failure path of the pipelined kernels' bounded waits: a wait on a
+barrier that nothing completes gives up after its limit and reports
+FAULT_TIMEOUT through the fault word (no GPU fault, hang or trap)."""
 import pytest
 
 import kv_cache_quantize_b200 as kvq
@@ -29,3 +32,10 @@ def test_shortcut_is_exact(which, what):
 def test_report_quotient_bit_differences():
     one, two, normal = kvq.selftest(0), kvq.selftest(1), kvq.selftest(5)
     print(f"quotient bit differences from IEEE: one-step {one} (normal range {normal}), two-step {two}")
+
+
+def test_bounded_wait_reports_timeout():
+    kvq.get_error()                         # clear
+    assert kvq.selftest(7) == 1             # the wait gave up, as designed
+    assert kvq.get_error() == 0x2           # FAULT_TIMEOUT, then cleared
+    assert kvq.get_error() == 0
