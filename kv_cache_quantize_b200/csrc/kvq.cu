@@ -794,8 +794,18 @@ kvq_status kvq_kv_rmsnorm_rope_cache(const kvq_tensor* kv, const kvq_tensor* gam
     a.eps = epsilon;
     const int64_t warps_per_block = RR_THREADS / 32;
     const int64_t need = (B * S + warps_per_block - 1) / warps_per_block;
-    launch(rmsnorm_rope_kernel, (unsigned)persistent_grid(rmsnorm_rope_kernel, RR_THREADS, need), RR_THREADS, 0,
-           reinterpret_cast<cudaStream_t>(stream), a);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool vec = reinterpret_cast<uintptr_t>(kv->data) % 16 == 0 &&
+                     reinterpret_cast<uintptr_t>(gamma->data) % 16 == 0 && D % 8 == 0 && Dv % 8 == 0;
+    const int64_t nch = Dv / 8;
+    if (vec && nch <= 32) launch(rmsnorm_rope_kernel<1>, (unsigned)persistent_grid(rmsnorm_rope_kernel<1>, RR_THREADS, need),
+                                 RR_THREADS, 0, s, a);
+    else if (vec && nch <= 64) launch(rmsnorm_rope_kernel<2>, (unsigned)persistent_grid(rmsnorm_rope_kernel<2>, RR_THREADS, need),
+                                      RR_THREADS, 0, s, a);
+    else if (vec && nch <= 128) launch(rmsnorm_rope_kernel<4>, (unsigned)persistent_grid(rmsnorm_rope_kernel<4>, RR_THREADS, need),
+                                       RR_THREADS, 0, s, a);
+    else launch(rmsnorm_rope_kernel<0>, (unsigned)persistent_grid(rmsnorm_rope_kernel<0>, RR_THREADS, need),
+                RR_THREADS, 0, s, a);
     return launched();
 }
 

@@ -4,11 +4,13 @@
 //
 // One warp per token.  The sum of squares follows the library's fixed order:
 // value i of the RMSNorm segment belongs to 8-value chunk i/8, chunk c to lane
-// c % 32; each lane adds x*x of its values in index order (x*x is exact for
-// 16-bit inputs), then the lanes combine by the butterfly p += p[lane ^ k],
-// k = 16, 8, 4, 2, 1.  The row is read a second time (from L1) to write the
-// normalised values.  The rope segment is handled one interleaved pair per
-// lane.  gamma, cos and sin are small and stay in L1/L2 across tokens.
+// c % 32; each lane adds x*x of its values in index order, then the lanes
+// combine by the butterfly p += p[lane ^ k], k = 16, 8, 4, 2, 1.  Aligned rows
+// are read as 16-byte chunks kept in registers for the normalisation and
+// written back as 8- or 16-byte chunks; other rows element by element (the
+// row read twice, the second time from L1).  The rope segment is handled one
+// interleaved pair per lane.  gamma, cos and sin are small and stay in L1/L2
+// across tokens.
 #pragma once
 
 #include "kvq_device.cuh"
@@ -95,6 +97,51 @@ __device__ __forceinline__ int64_t rr_slot(const RmsRopeArgs& a, int64_t b, int6
     return v;
 }
 
+// y[0..7] = chunk c of the RMSNorm segment normalised and scaled, stored as
+// the ckv cache's dtype (8 values at row element 8c)
+__device__ __forceinline__ void rr_store_chunk(const CacheOut& c, uint8_t* row, int ch, const float (&y)[8]) {
+    const int j0 = 8 * ch;
+    switch (c.dt) {
+        case CDT_BF16:
+        case CDT_F16: {
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t lo = c.dt == CDT_BF16 ? to_bf16_bits(y[2 * k]) : to_f16_bits(y[2 * k]);
+                const uint32_t hi = c.dt == CDT_BF16 ? to_bf16_bits(y[2 * k + 1]) : to_f16_bits(y[2 * k + 1]);
+                w[k] = lo | (hi << 16);
+            }
+            st_b128(row + 2 * j0, make_uint4(w[0], w[1], w[2], w[3]));
+            break;
+        }
+        case CDT_E4M3:
+        case CDT_E5M2: {
+            float q[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) q[k] = __fdiv_rn(y[k], c.scale[c.scale_n == 1 ? 0 : j0 + k]);
+            st_b64(row + j0, c.dt == CDT_E4M3 ? fp8x8<false>(q) : fp8x8<true>(q));
+            break;
+        }
+        case CDT_I8: {
+            uint32_t w[2] = {0u, 0u};
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                float q = __fdiv_rn(y[k], c.scale[c.scale_n == 1 ? 0 : j0 + k]);
+                if (c.offset) q = __fadd_rn(q, c.offset[c.offset_n == 1 ? 0 : j0 + k]);
+                w[k >> 2] |= ((uint32_t)int8_rne_sat(q) & 0xffu) << (8 * (k & 3));
+            }
+            st_b64(row + j0, make_uint2(w[0], w[1]));
+            break;
+        }
+        default: break;
+    }
+}
+
+// NCH == 0: element-wise loads (any alignment, any Dv).  NCH > 0: 16-byte
+// rows (kv, gamma 16-byte aligned, D and Dv multiples of 8) with at most
+// 32 * NCH chunks: each lane keeps its chunks c = lane, lane + 32, ... in
+// registers between the sum of squares and the normalisation.
+template <int NCH>
 __global__ void __launch_bounds__(RR_THREADS) rmsnorm_rope_kernel(const RmsRopeArgs a) {
     pdl_wait();
     pdl_trigger();
@@ -105,7 +152,26 @@ __global__ void __launch_bounds__(RR_THREADS) rmsnorm_rope_kernel(const RmsRopeA
     const int nch = (a.Dv + 7) / 8;
     const int h = a.Dk / 2;
 
+    // register kernel: the next token's RMSNorm chunks are loaded while the
+    // current token is normalised (a token's row is read whether or not it is
+    // skipped)
+    uint4 xn[NCH > 0 ? NCH : 1];
+    auto load_chunks = [&](int64_t t, uint4 (&v)[NCH > 0 ? NCH : 1]) {
+#pragma unroll
+        for (int m = 0; m < NCH; ++m) {
+            const int c = lane + 32 * m;
+            v[m] = (t < ntok && c < nch) ? __ldg(reinterpret_cast<const uint4*>(a.kv + t * a.D) + c)
+                                         : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    if (NCH > 0) load_chunks(gwarp, xn);
     for (int64_t t = gwarp; t < ntok; t += nwarps) {
+        uint4 xv[NCH > 0 ? NCH : 1];
+        if (NCH > 0) {
+#pragma unroll
+            for (int m = 0; m < NCH; ++m) xv[m] = xn[m];
+            load_chunks(t + nwarps, xn);
+        }
         const int64_t b = t / a.S, s = t - (t / a.S) * a.S;
         const int64_t slot = rr_slot(a, b, s);     // warp-uniform
         if (slot == -2) {
@@ -114,26 +180,60 @@ __global__ void __launch_bounds__(RR_THREADS) rmsnorm_rope_kernel(const RmsRopeA
         }
         if (slot < 0) continue;
         const uint16_t* x = a.kv + t * a.D;
-
-        // RMSNorm: sum of squares in the fixed lane order
-        float acc = 0.0f;
-        for (int c = lane; c < nch; c += 32) {
-            for (int i = 8 * c; i < 8 * c + 8 && i < a.Dv; ++i) {
-                const float v = half_at(x, i, a.kv_f16);
-                acc = __fadd_rn(acc, __fmul_rn(v, v));
-            }
-        }
-#pragma unroll
-        for (int k = 16; k >= 1; k >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(FULL_MASK, acc, k));
-        const float mean = __fdiv_rn(acc, (float)a.Dv);
-        const float rms = __fsqrt_rn(__fadd_rn(mean, a.eps));
-
         uint8_t* crow = slot_row(a.ckv.rows, slot);
-        for (int c = lane; c < nch; c += 32) {
-            for (int i = 8 * c; i < 8 * c + 8 && i < a.Dv; ++i) {
-                const float v = half_at(x, i, a.kv_f16);
-                const float y = __fmul_rn(__fdiv_rn(v, rms), half_at(a.gamma, i, a.kv_f16));
-                store_elem(a.ckv, crow, i, y);
+
+        if (NCH > 0) {
+            // RMSNorm: sum of squares in the fixed lane order, chunks from registers
+            float acc = 0.0f;
+#pragma unroll
+            for (int m = 0; m < NCH; ++m) {
+                if (lane + 32 * m >= nch) break;
+                float f[8];
+                if (a.kv_f16) widen8<true>(xv[m], f);
+                else widen8<false>(xv[m], f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc = __fadd_rn(acc, __fmul_rn(f[i], f[i]));
+            }
+#pragma unroll
+            for (int k = 16; k >= 1; k >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(FULL_MASK, acc, k));
+            const float mean = __fdiv_rn(acc, (float)a.Dv);
+            const float rms = __fsqrt_rn(__fadd_rn(mean, a.eps));
+#pragma unroll
+            for (int m = 0; m < NCH; ++m) {
+                const int c = lane + 32 * m;
+                if (c >= nch) break;
+                float f[8], g[8], y[8];
+                const uint4 gv = __ldg(reinterpret_cast<const uint4*>(a.gamma) + c);
+                if (a.kv_f16) {
+                    widen8<true>(xv[m], f);
+                    widen8<true>(gv, g);
+                } else {
+                    widen8<false>(xv[m], f);
+                    widen8<false>(gv, g);
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fdiv_rn(f[i], rms), g[i]);
+                rr_store_chunk(a.ckv, crow, c, y);
+            }
+        } else {
+            // RMSNorm: sum of squares in the fixed lane order
+            float acc = 0.0f;
+            for (int c = lane; c < nch; c += 32) {
+                for (int i = 8 * c; i < 8 * c + 8 && i < a.Dv; ++i) {
+                    const float v = half_at(x, i, a.kv_f16);
+                    acc = __fadd_rn(acc, __fmul_rn(v, v));
+                }
+            }
+#pragma unroll
+            for (int k = 16; k >= 1; k >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(FULL_MASK, acc, k));
+            const float mean = __fdiv_rn(acc, (float)a.Dv);
+            const float rms = __fsqrt_rn(__fadd_rn(mean, a.eps));
+            for (int c = lane; c < nch; c += 32) {
+                for (int i = 8 * c; i < 8 * c + 8 && i < a.Dv; ++i) {
+                    const float v = half_at(x, i, a.kv_f16);
+                    const float y = __fmul_rn(__fdiv_rn(v, rms), half_at(a.gamma, i, a.kv_f16));
+                    store_elem(a.ckv, crow, i, y);
+                }
             }
         }
 

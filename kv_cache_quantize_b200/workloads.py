@@ -303,9 +303,19 @@ def cfg5b_compress_mode2(seed: int = 0) -> Case:
                         seed=seed)
 
 
+def prefill_rmsnorm_rope(seed: int = 0) -> Case:
+    """The DeepSeek-V3 shape of cfg2 at prefill size: 65536 tokens (not one of
+    the five published workloads; it measures the kernel where bandwidth, not
+    latency, bounds it)."""
+    return gen_rmsnorm_rope("prefill_rmsnorm_rope", B=65536, S=1, D=576, Dv=512, num_blocks=1024, block_size=128,
+                            k_dtype="bf16", ckv_dtype="e4m3", ckv_scale=[1.0 / 64.0], epsilon=1e-6,
+                            cache_mode="PA_BNSD", skip_frac=0.05, seed=seed)
+
+
 CONFIGS = {
     "cfg1_compress_mode1": cfg1_compress_mode1,
     "cfg2_rmsnorm_rope": cfg2_rmsnorm_rope,
+    "prefill_rmsnorm_rope": prefill_rmsnorm_rope,
     "cfg3a_indexer_mxfp8": cfg3a_indexer_mxfp8,
     "cfg3b_indexer_mxfp4": cfg3b_indexer_mxfp4,
     "cfg4_dequant_rope_quant": cfg4_dequant_rope_quant,

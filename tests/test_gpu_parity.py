@@ -222,6 +222,17 @@ def test_rmsnorm_rope_named_workload_full_size():
     _same(W.cfg2_rmsnorm_rope())
 
 
+def test_rmsnorm_rope_prefill_size():
+    _same(W.prefill_rmsnorm_rope())
+
+
+@pytest.mark.parametrize("ckv_dtype,k_dtype", [("i8", "bf16"), ("bf16", "bf16"), ("e5m2", "f16"), ("i8", "i8")])
+def test_rmsnorm_rope_vector_path_dtypes(ckv_dtype, k_dtype):
+    """Aligned rows with Dv = 256 / 512 / 1024 take the register-chunk kernel for every ckv dtype."""
+    for D, Dv in ((320, 256), (576, 512), (1088, 1024)):
+        _same(_rr(D=D, Dv=Dv, k_dtype=k_dtype, ckv_dtype=ckv_dtype))
+
+
 # ---------------------------------------------------------------------------
 # dequant_rope_quant_kvcache
 # ---------------------------------------------------------------------------
