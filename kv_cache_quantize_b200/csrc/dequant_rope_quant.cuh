@@ -171,6 +171,14 @@ __global__ void __launch_bounds__(DG_THREADS) dequant_rope_quant_general_kernel(
 // side (a PASS).  Each token of a stage has 8/TPS consumer warps, which take
 // its passes round-robin (spreading the costlier k / v passes with their int8
 // quantisation evenly) and widen its cos / sin once.
+//
+// The stage count S, TPS and (for the common head size 128) D are template
+// parameters (S in 2..4, TPS in 2, 4, 8: every pair the launch rule picks for
+// H <= 4096; DC = 0 reads D from the arguments): with the ring's shape and the
+// lane layout known at compile time the consumers' index and address
+// arithmetic folds to constants, which measured 11 % faster (61.9 -> 55.3 us
+// on x int32 [16, 1024, 3072]) than the same kernel reading all three from its
+// arguments.
 // ---------------------------------------------------------------------------
 constexpr int DT_CONSUMERS = 8;
 constexpr int DT_THREADS = (DT_CONSUMERS + 1) * 32;
@@ -279,13 +287,16 @@ __device__ __forceinline__ uint32_t dt_int8x4(const float (&o)[4], const float* 
 }
 
 // XK: 0 int32 x (dequantised), 1 bf16 x, 2 f16 x.  F16: cos / sin and the
-// 16-bit outputs are f16 (else bf16).
-template <int XK, bool F16>
+// 16-bit outputs are f16 (else bf16).  S stages of TPS tokens (a.stages and
+// a.tps hold the same values); head size DC, or a.D when DC is 0.
+template <int XK, bool F16, int S, int TPS, int DC>
 __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(const DrqArgs a) {
+    static_assert(S >= 2 && S <= 4 && (TPS == 2 || TPS == 4 || TPS == 8), "ring shape");
+    static_assert(DC == 0 || (DC % 8 == 0 && DC <= 256), "head size");
     pdl_wait();
     pdl_trigger();
     extern __shared__ __align__(128) uint8_t smem[];
-    const int S = a.stages, TPS = a.tps, D = a.D;
+    const int D = DC ? DC : a.D;
     constexpr int XB = XK == 0 ? 4 : 2;
     constexpr bool DQ = XK == 0;
     const int64_t H = a.H;
@@ -396,7 +407,7 @@ __global__ void __launch_bounds__(DT_THREADS) dequant_rope_quant_tma_kernel(cons
     const bool lane_on = hl < HPW;
     const int NP = (NH + HPW - 1) / HPW;      // passes per token
     const int j0 = 4 * l, j1 = (D >> 1) + 4 * l;
-    const int WPT = DT_CONSUMERS / TPS;
+    constexpr int WPT = DT_CONSUMERS / TPS;
     const int my_tok = warp / WPT, wt = warp - my_tok * WPT;
     const bool v8 = a.out_vec8 != 0, r4 = a.rows_vec4 != 0;
     auto store4h = [&](uint16_t* p, const float (&o)[4]) {

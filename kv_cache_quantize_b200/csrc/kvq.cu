@@ -373,6 +373,29 @@ __global__ void selftest_fmax_kernel() {
     if (bad) atomicAdd(&g_selftest_count, bad);
 }
 
+// The pipelined dequant kernel instantiated for the ring shape (a.stages,
+// a.tps) that the host picked, and for D = 128 or any other head size.
+template <int XK, bool F16, int S, int TPS>
+void launch_drq_tma(const DrqArgs& a, int64_t tiles, size_t smem, cudaStream_t s) {
+    auto k = a.D == 128 ? dequant_rope_quant_tma_kernel<XK, F16, S, TPS, 128>
+                        : dequant_rope_quant_tma_kernel<XK, F16, S, TPS, 0>;
+    launch(k, (unsigned)persistent_grid(k, DT_THREADS, tiles, smem), DT_THREADS, smem, s, a);
+}
+
+template <int XK, bool F16, int S>
+void launch_drq_tps(const DrqArgs& a, int64_t tiles, size_t smem, cudaStream_t s) {
+    if (a.tps == 2) launch_drq_tma<XK, F16, S, 2>(a, tiles, smem, s);
+    else if (a.tps == 4) launch_drq_tma<XK, F16, S, 4>(a, tiles, smem, s);
+    else launch_drq_tma<XK, F16, S, 8>(a, tiles, smem, s);
+}
+
+template <int XK, bool F16>
+void launch_drq_ring(const DrqArgs& a, int64_t tiles, size_t smem, cudaStream_t s) {
+    if (a.stages == 2) launch_drq_tps<XK, F16, 2>(a, tiles, smem, s);
+    else if (a.stages == 3) launch_drq_tps<XK, F16, 3>(a, tiles, smem, s);
+    else launch_drq_tps<XK, F16, 4>(a, tiles, smem, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -962,7 +985,7 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
         // bulk copy; TPS tokens per stage (a divisor of the consumer warps, x
         // span at most 32 KB), as many stages (2..4) as keep two CTAs on an SM
         int tps = 1;
-        while (tps < DT_CONSUMERS && 2 * tps * H * xb <= 32768) tps *= 2;
+        while (tps < DT_CONSUMERS && 2 * tps * H * xb <= 32768) tps *= 2;     // 2, 4 or 8 (H <= 4096)
         a.tps = tps;
         auto dt_smem = [&](int stages) {
             return (size_t)dt_header_bytes(stages, tps) + prm + (size_t)stages * dt_stage_bytes(tps, H, xb, (int)D);
@@ -972,20 +995,14 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
         const size_t smem = dt_smem(a.stages);
         const int64_t tiles = (need + a.tps - 1) / a.tps;
         const bool f16 = a.cos_f16 != 0;
-#define KVQ_LAUNCH_DT(XK, F)                                                                   \
-    do {                                                                                       \
-        auto k = dequant_rope_quant_tma_kernel<XK, F>;                                         \
-        launch(k, (unsigned)persistent_grid(k, DT_THREADS, tiles, smem), DT_THREADS, smem, s, a); \
-    } while (0)
         if (a.x_kind == 0) {
-            if (f16) KVQ_LAUNCH_DT(0, true);
-            else KVQ_LAUNCH_DT(0, false);
+            if (f16) launch_drq_ring<0, true>(a, tiles, smem, s);
+            else launch_drq_ring<0, false>(a, tiles, smem, s);
         } else if (a.x_kind == 1) {
-            KVQ_LAUNCH_DT(1, false);
+            launch_drq_ring<1, false>(a, tiles, smem, s);
         } else {
-            KVQ_LAUNCH_DT(2, true);
+            launch_drq_ring<2, true>(a, tiles, smem, s);
         }
-#undef KVQ_LAUNCH_DT
         return launched();
     }
     // every other shape and alignment: one CTA per token

@@ -292,6 +292,19 @@ def test_drq_two_dim_x():
     _same(_dq(S=1, x_2d=True, kv_output=True, cache_mode="contiguous"))
 
 
+@pytest.mark.parametrize("B", [1, 97])
+def test_drq_operator_test_suite_shapes(B):
+    """The two end-to-end cases of the operator's own test suite
+    (aclnnDequantRopeQuantKvcache, 测试与验证): 2-D x [1, 2304] float16 split
+    1536/384/384, and 2-D x [1, 3584] int32 split 1792/896/896 with a bf16
+    bias, both in page mode.  The page gives the splits, not the head size:
+    D = 128 (so Nq, Nkv = 12, 3 and 14, 7).  B = 97 repeats each shape over
+    more rows."""
+    _same(_dq(B=B, S=1, x_2d=True, Nq=12, Nkv=3, D=128, x_dtype="f16", cos_dtype="f16", cache_mode="page",
+              c0=4, c1=64, kv_output=True))
+    _same(_dq(B=B, S=1, x_2d=True, Nq=14, Nkv=7, D=128, bias_dtype="bf16", cache_mode="page", c0=4, c1=64))
+
+
 def test_drq_many_heads():
     _same(_dq(Nq=40, Nkv=8, D=32, S=8))
 
