@@ -537,7 +537,7 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
         const int threads = (a.ncw + 1) * 32;
 #define KVQ_LAUNCH_CT(M, GG)                                                                   \
     do {                                                                                       \
-        auto k = compress_tma_kernel<M, GG>;                                                   \
+        auto k = ct_stages == 2 ? compress_tma_kernel<M, GG, 2> : compress_tma_kernel<M, GG, 3>; \
         launch(k, (unsigned)persistent_grid(k, threads, tiles, smem), threads, smem, s, a);     \
     } while (0)
         if (quant_mode == 0) KVQ_LAUNCH_CT(0, 64);
