@@ -442,17 +442,17 @@ def main():
     peak, peak_kind = hbm_peak()
     avg_a, avg_b = statistics.mean(ms_a) / 1e3, statistics.mean(ms_b) / 1e3
     kernels = {
-        "compress_tma_kernel<0,64> (quantMode 0)": {
+        "compress_tma_kernel<0,64,2> (quantMode 0)": {
             "alg_bytes_per_launch": bytes_a, "avg_us": 1e6 * avg_a, "median_us": 1e6 * statistics.median(ms_a) / 1e3,
             "alg_GBps": bytes_a / avg_a / 1e9, "frac_of_peak": bytes_a / avg_a / 1e9 / peak,
             "share_of_step": avg_a / (avg_a + avg_b)},
-        "compress_tma_kernel<2,32> (quantMode 2)": {
+        "compress_tma_kernel<2,32,2> (quantMode 2)": {
             "alg_bytes_per_launch": bytes_b, "avg_us": 1e6 * avg_b, "median_us": 1e6 * statistics.median(ms_b) / 1e3,
             "alg_GBps": bytes_b / avg_b / 1e9, "frac_of_peak": bytes_b / avg_b / 1e9 / peak,
             "share_of_step": avg_b / (avg_a + avg_b)},
     }
-    dom_name, dom_bytes, dom_avg = ("compress_tma_kernel<0,64>", bytes_a, avg_a) if avg_a >= avg_b else \
-        ("compress_tma_kernel<2,32>", bytes_b, avg_b)
+    dom_name, dom_bytes, dom_avg = ("compress_tma_kernel<0,64,2>", bytes_a, avg_a) if avg_a >= avg_b else \
+        ("compress_tma_kernel<2,32,2>", bytes_b, avg_b)
     achieved = dom_bytes / dom_avg / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "traffic": profiled_traffic(dom_name), "kernel": dom_name,
