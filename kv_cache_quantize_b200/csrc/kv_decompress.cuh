@@ -87,9 +87,8 @@ __device__ __forceinline__ float e8m0_value(uint32_t b) {
 // one slice of a live row: decode w (codes, or the stored rope) with scale bits sc
 // rope_tab (mode 2): bf16_rn(E4M3 value / xScale) for each of the 256 codes
 template <int MODE, int G>
-__device__ __forceinline__ void dc_slice(const DecompressArgs& a, const uint32_t (&w)[16], uint32_t sc, int j,
-                                         uint16_t* yrow, const uint16_t* rope_tab) {
-    const int nn = a.nslice - 2;
+__device__ __forceinline__ void dc_slice(const DecompressArgs& a, int nn, const uint32_t (&w)[16], uint32_t sc,
+                                         int j, uint16_t* yrow, const uint16_t* rope_tab) {
     uint32_t out[16];
     if (j >= nn) {
         if (MODE != 2) {
@@ -127,11 +126,10 @@ __device__ __forceinline__ void dc_slice(const DecompressArgs& a, const uint32_t
 }
 
 // packed bytes a slice needs: its codes (or the 64 bytes of a bf16 rope) in w,
-// its group scale bits in sc
+// its group scale bits in sc (nn: the number of nope slices)
 template <int MODE, int G>
-__device__ __forceinline__ void dc_fetch(const DecompressArgs& a, const uint8_t* row, int j, uint32_t (&w)[16],
-                                         uint32_t& sc) {
-    const int nn = a.nslice - 2;
+__device__ __forceinline__ void dc_fetch(const DecompressArgs& a, int nn, const uint8_t* row, int j,
+                                         uint32_t (&w)[16], uint32_t& sc) {
     const bool v16 = a.rows_vec16 != 0;
     sc = 0u;
     if (j >= nn) {
@@ -168,14 +166,18 @@ __device__ __forceinline__ const uint8_t* dc_row(const DecompressArgs& a, int64_
     return slot_row(a.cache, s);
 }
 
-template <int MODE, int G>
+// NS: slices per row (d / 32) when known at compile time (18: d = 576), else 0
+// and a.nslice; the constant form measured 11 % faster in mode 0 at d = 576.
+template <int MODE, int G, int NS>
 __global__ void __launch_bounds__(DC_THREADS) kv_decompress_kernel(const DecompressArgs a) {
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const int64_t nchunks = (a.T * a.nslice + 31) / 32;
+    const int ns = NS ? NS : a.nslice;
+    const int nn = ns - 2;
+    const int64_t nchunks = (a.T * ns + 31) / 32;
     // mode 2: the decoded rope value of every E4M3 code, one IEEE division each
     __shared__ uint16_t rope_tab[MODE == 2 ? 256 : 1];
     if (MODE == 2) {
@@ -187,7 +189,6 @@ __global__ void __launch_bounds__(DC_THREADS) kv_decompress_kernel(const Decompr
         __syncthreads();
     }
     if (gwarp >= nchunks) return;
-    const int ns = a.nslice;
     // the lane's slice (row, j) in chunk c, and its step from chunk c to c + nwarps
     const int64_t hs = gwarp * 32 + lane;
     int64_t row0 = hs / ns;
@@ -210,15 +211,15 @@ __global__ void __launch_bounds__(DC_THREADS) kv_decompress_kernel(const Decompr
     int64_t s1 = dc_slot(a, row1, row1 < a.T && gwarp + nwarps < nchunks);
     const uint8_t* p0 = dc_row(a, s0, j0);
     uint32_t w0[16], w1[16], sc0 = 0u, sc1 = 0u;
-    if (p0) dc_fetch<MODE, G>(a, p0, j0, w0, sc0);
+    if (p0) dc_fetch<MODE, G>(a, nn, p0, j0, w0, sc0);
     for (int64_t c = gwarp; c < nchunks; c += nwarps) {
         int64_t row2 = row1;
         int j2 = j1;
         advance(row2, j2);
         const int64_t s2 = dc_slot(a, row2, row2 < a.T && c + 2 * nwarps < nchunks);
         const uint8_t* p1 = dc_row(a, s1, j1);
-        if (p1) dc_fetch<MODE, G>(a, p1, j1, w1, sc1);
-        if (p0) dc_slice<MODE, G>(a, w0, sc0, j0, a.y + row0 * a.y_row_stride, rope_tab);
+        if (p1) dc_fetch<MODE, G>(a, nn, p1, j1, w1, sc1);
+        if (p0) dc_slice<MODE, G>(a, nn, w0, sc0, j0, a.y + row0 * a.y_row_stride, rope_tab);
 #pragma unroll
         for (int i = 0; i < 16; ++i) w0[i] = w1[i];
         sc0 = sc1;

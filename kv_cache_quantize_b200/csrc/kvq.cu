@@ -611,7 +611,7 @@ kvq_status kvq_kv_decompress(const kvq_tensor* cache, const kvq_tensor* slot_map
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 #define KVQ_LAUNCH_DC(M, GG)                                                                   \
     do {                                                                                       \
-        auto k = kv_decompress_kernel<M, GG>;                                                  \
+        auto k = a.nslice == 18 ? kv_decompress_kernel<M, GG, 18> : kv_decompress_kernel<M, GG, 0>; \
         launch(k, (unsigned)persistent_grid(k, DC_THREADS, need), DC_THREADS, 0, s, a);          \
     } while (0)
     if (quant_mode == 0) KVQ_LAUNCH_DC(0, 64);
