@@ -46,9 +46,12 @@ struct RmsRopeArgs {
 
 constexpr int RR_THREADS = 128;
 
-__device__ __forceinline__ float half_at(const uint16_t* p, int64_t i, int f16) {
-    const uint32_t h = p[i];
+__device__ __forceinline__ float half_bits(uint32_t h, int f16) {
     return f16 ? __half2float(__ushort_as_half((unsigned short)h)) : __uint_as_float(h << 16);
+}
+
+__device__ __forceinline__ float half_at(const uint16_t* p, int64_t i, int f16) {
+    return half_bits(p[i], f16);
 }
 
 // Store y as element j of a cache row (unquantised: rounded to the dtype;
@@ -75,26 +78,31 @@ __device__ __forceinline__ void store_elem(const CacheOut& c, uint8_t* row, int 
     }
 }
 
-__device__ __forceinline__ int64_t rr_slot(const RmsRopeArgs& a, int64_t b, int64_t s) {
-    const int64_t t = b * a.S + s;
+// Token t's batch b and position s (needed by the Norm and PA_BLK_BNSD modes
+// only; 0 otherwise) and the position of its entry in the index tensor.
+__device__ __forceinline__ int64_t rr_index_pos(const RmsRopeArgs& a, int64_t t, int64_t& b, int64_t& s) {
+    b = 0;
+    s = 0;
+    if (a.cache_mode != 0 && a.cache_mode != 3) return t;  // PA, PA_BNSD: one entry per token
+    b = t / a.S;
+    s = t - b * a.S;
+    if (a.cache_mode == 0) return t;
     const int64_t bs = a.k.rows.block_size;
+    return b * ((a.S + bs - 1) / bs) + s / bs;               // PA_BLK_BNSD: one entry per block of tokens
+}
+
+// Destination slot of token (b, s) from its index entry v: >= 0 a slot, -1
+// skip, -2 out of range.
+__device__ __forceinline__ int64_t rr_resolve(const RmsRopeArgs& a, int64_t b, int64_t s, int64_t v) {
+    const int64_t bs = a.k.rows.block_size;
+    if (v == -1) return -1;
     if (a.cache_mode == 0) {                       // Norm: [B, S] positions, one block per batch
-        const int64_t v = load_slot(a.index, a.index_i64, t);
-        if (v == -1) return -1;
         if (v < 0 || v >= bs || b * bs >= a.k.rows.num_slots) return -2;
         return b * bs + v;
     }
-    if (a.cache_mode == 3) {                       // PA_BLK_BNSD: one entry per block of tokens
-        const int64_t nb = (a.S + bs - 1) / bs;
-        const int64_t v = load_slot(a.index, a.index_i64, b * nb + s / bs);
-        if (v == -1) return -1;
-        if (v < 0 || v >= a.k.rows.num_slots) return -2;
-        return (v / bs) * bs + s % bs;
-    }
-    const int64_t v = load_slot(a.index, a.index_i64, t);   // PA, PA_BNSD
-    if (v == -1) return -1;
     if (v < 0 || v >= a.k.rows.num_slots) return -2;
-    return v;
+    if (a.cache_mode == 3) return (v / bs) * bs + s % bs;
+    return v;                                      // PA, PA_BNSD
 }
 
 // y[0..7] = chunk c of the RMSNorm segment normalised and scaled, stored as
@@ -141,8 +149,11 @@ __device__ __forceinline__ void rr_store_chunk(const CacheOut& c, uint8_t* row, 
 // rows (kv, gamma 16-byte aligned, D and Dv multiples of 8) with at most
 // 32 * NCH chunks: each lane keeps its chunks c = lane, lane + 32, ... in
 // registers between the sum of squares and the normalisation.
+// Eight CTAs of four warps per SM (at most 64 registers): the kernel is bound
+// by latency and the two IEEE divisions per value, and runs faster with more
+// warps resident (79 us at 8 CTAs per SM vs 93 us at 5 for 65,536 tokens).
 template <int NCH>
-__global__ void __launch_bounds__(RR_THREADS) rmsnorm_rope_kernel(const RmsRopeArgs a) {
+__global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRopeArgs a) {
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
@@ -164,7 +175,23 @@ __global__ void __launch_bounds__(RR_THREADS) rmsnorm_rope_kernel(const RmsRopeA
                                          : make_uint4(0u, 0u, 0u, 0u);
         }
     };
+    // the next token's index entry (and, with at most 32 RoPE pairs, each
+    // lane's RoPE inputs) are loaded while the current token is processed
+    const bool rope_pf = NCH > 0 && h <= 32;
+    int64_t v_next = -1, b_next = 0, s_next = 0;
+    uint32_t zn = 0u, cn = 0u, sn = 0u;
+    auto prefetch = [&](int64_t t) {
+        if (t >= ntok) return;
+        v_next = load_slot(a.index, a.index_i64, rr_index_pos(a, t, b_next, s_next));
+        if (rope_pf && lane < h) {
+            const uint16_t* z = a.kv + t * a.D + a.Dv;
+            zn = (uint32_t)z[2 * lane] | ((uint32_t)z[2 * lane + 1] << 16);
+            cn = (uint32_t)a.cos[t * a.Dk + lane] | ((uint32_t)a.cos[t * a.Dk + h + lane] << 16);
+            sn = (uint32_t)a.sin[t * a.Dk + lane] | ((uint32_t)a.sin[t * a.Dk + h + lane] << 16);
+        }
+    };
     if (NCH > 0) load_chunks(gwarp, xn);
+    prefetch(gwarp);
     for (int64_t t = gwarp; t < ntok; t += nwarps) {
         uint4 xv[NCH > 0 ? NCH : 1];
         if (NCH > 0) {
@@ -172,8 +199,9 @@ __global__ void __launch_bounds__(RR_THREADS) rmsnorm_rope_kernel(const RmsRopeA
             for (int m = 0; m < NCH; ++m) xv[m] = xn[m];
             load_chunks(t + nwarps, xn);
         }
-        const int64_t b = t / a.S, s = t - (t / a.S) * a.S;
-        const int64_t slot = rr_slot(a, b, s);     // warp-uniform
+        const int64_t slot = rr_resolve(a, b_next, s_next, v_next);     // warp-uniform
+        const uint32_t zr = zn, cr = cn, sr = sn;
+        prefetch(t + nwarps);
         if (slot == -2) {
             if (lane == 0) raise_fault(FAULT_SLOT_RANGE);
             continue;
@@ -237,8 +265,19 @@ __global__ void __launch_bounds__(RR_THREADS) rmsnorm_rope_kernel(const RmsRopeA
             }
         }
 
-        // interleaved RoPE: y_j = z_2j c_j - z_2j+1 s_j, y_h+j = z_2j+1 c_h+j + z_2j s_h+j
         uint8_t* krow = slot_row(a.k.rows, slot);
+        if (rope_pf) {
+            // interleaved RoPE on the prefetched pair of this lane
+            if (lane < h) {
+                const float z0 = half_bits(zr & 0xffffu, a.kv_f16), z1 = half_bits(zr >> 16, a.kv_f16);
+                const float c0 = half_bits(cr & 0xffffu, a.kv_f16), c1 = half_bits(cr >> 16, a.kv_f16);
+                const float s0 = half_bits(sr & 0xffffu, a.kv_f16), s1 = half_bits(sr >> 16, a.kv_f16);
+                store_elem(a.k, krow, lane, __fadd_rn(__fmul_rn(z0, c0), __fmul_rn(-z1, s0)));
+                store_elem(a.k, krow, h + lane, __fadd_rn(__fmul_rn(z1, c1), __fmul_rn(z0, s1)));
+            }
+            continue;
+        }
+        // interleaved RoPE: y_j = z_2j c_j - z_2j+1 s_j, y_h+j = z_2j+1 c_h+j + z_2j s_h+j
         const uint16_t* z = x + a.Dv;
         const uint16_t* cs = a.cos + t * a.Dk;
         const uint16_t* sn = a.sin + t * a.Dk;
