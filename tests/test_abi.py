@@ -242,3 +242,22 @@ def test_empty_inputs_are_accepted_whatever_their_strides(L):
     xi, si = D([0, 128], "f16", [0, 0]), D([0], "i64", [0])
     assert L.kvq_indexer_quant_cache(R(xi), R(D([16, 8, 1, 128], "e4m3")), R(D([16, 8, 1, 4], "e8m0")), R(si), 0,
                                      None) == OK
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """No CPU or library fallback: with libkvq.so absent the first call raises."""
+    import subprocess
+    import sys
+    code = ("import kv_cache_quantize_b200 as kvq, torch\n"
+            f"kvq.library_path = {str(tmp_path / 'absent.so')!r}\n"
+            "x = torch.zeros((4, 128), dtype=torch.bfloat16)\n"
+            "s = torch.zeros(4, dtype=torch.int32)\n"
+            "c = torch.zeros((1, 16, 1, 224), dtype=torch.uint8)\n"
+            "try:\n"
+            "    kvq.kv_compress_epilog(x, s, c, 0)\n"
+            "except RuntimeError as e:\n"
+            "    print('raised:', e)\n"
+            "else:\n"
+            "    print('no error')\n")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT, timeout=300)
+    assert "raised:" in out.stdout and "not built" in out.stdout, out.stdout + out.stderr
