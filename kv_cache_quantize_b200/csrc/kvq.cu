@@ -165,7 +165,7 @@ int sm_count() {
 int resident_blocks(const void* fn, int threads, size_t smem) {
     struct Entry { const void* fn; int dev, threads; size_t smem; int occ; };
     static std::mutex mu;
-    static Entry table[128];
+    static Entry table[512];
     static int used = 0;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
@@ -173,9 +173,9 @@ int resident_blocks(const void* fn, int threads, size_t smem) {
     for (int i = 0; i < used; ++i)
         if (table[i].fn == fn && table[i].dev == dev && table[i].threads == threads && table[i].smem == smem)
             return table[i].occ;
-    bool attr_set = false;
+    bool attr_set = false;          // the shared-memory limit was raised by an earlier entry
     for (int i = 0; i < used; ++i)
-        if (table[i].fn == fn && table[i].dev == dev) attr_set = true;
+        if (table[i].fn == fn && table[i].dev == dev && table[i].smem > 0) attr_set = true;
     if (smem > 0 && !attr_set) {
         int optin = 0;
         if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess || optin <= 0)
@@ -184,7 +184,7 @@ int resident_blocks(const void* fn, int threads, size_t smem) {
     }
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, smem) != cudaSuccess || occ < 1) occ = 1;
-    if (used < 128) table[used++] = Entry{fn, dev, threads, smem, occ};
+    if (used < 512) table[used++] = Entry{fn, dev, threads, smem, occ};
     return occ;
 }
 
