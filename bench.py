@@ -85,13 +85,16 @@ def algorithmic_bytes(case) -> int:
         T = B * S
         H = a["x"].shape[-1]
         D, Nq, Nkv = at["D"], at["Nq"], at["Nkv"]
+        dq = at["x_dtype"] == "i32"          # the dequant inputs take effect for int32 x only
         per_tok = H * a["x"].itemsize + 2 * 2 * D + Nq * D * 2 + 2 * Nkv * D
         if at["kv_output"]:
             per_tok += 2 * Nkv * D * 2
         per_tok += a["indices"].itemsize if at["cache_mode"] == "page" else 0
-        per_tok += 4 if "activation_scale" in a else 0
-        params = sum(a[k].nbytes for k in ("weight_scale", "bias", "scale_k", "scale_v", "offset_k", "offset_v")
-                     if k in a)
+        per_tok += 4 if dq and "activation_scale" in a else 0
+        used = ("scale_k", "scale_v", "offset_k", "offset_v") + (("weight_scale", "bias") if dq else ())
+        params = sum(a[k].nbytes for k in used if k in a)
+        if at["cache_mode"] != "page":
+            params += a["indices"].nbytes       # one start position per batch
         return T * per_tok + params
     raise ValueError(case.op)
 

@@ -312,6 +312,46 @@ def prefill_rmsnorm_rope(seed: int = 0) -> Case:
                             cache_mode="PA_BNSD", skip_frac=0.05, seed=seed)
 
 
+# ---------------------------------------------------------------------------
+# the further modes of the four operations at the named workloads' sizes
+# ---------------------------------------------------------------------------
+def cfg3c_indexer_fp8(seed: int = 0) -> Case:
+    """cfg3a's rows in the fp8 mode: one binary32 scale per row."""
+    return gen_indexer("cfg3c_indexer_fp8", T=65536, d=128, quant_mode=1, num_blocks=2048, block_size=64,
+                       cache_head_dim=128, scale_head_dim=1, cache_dtype="e4m3", skip_frac=0.05, seed=seed)
+
+
+def cfg3d_indexer_mxfp8_e5m2(seed: int = 0) -> Case:
+    """cfg3a with an E5M2 code cache."""
+    return gen_indexer("cfg3d_indexer_mxfp8_e5m2", T=65536, d=128, quant_mode=0, num_blocks=2048, block_size=64,
+                       cache_head_dim=128, scale_head_dim=4, cache_dtype="e5m2", skip_frac=0.05, seed=seed)
+
+
+def prefill_rmsnorm_rope_int8(seed: int = 0) -> Case:
+    """The prefill shape with both caches static int8: per-channel scales
+    U(1/48, 1/24) and integer offsets in [-4, 4] for ckv, a per-tensor scale
+    1/64 and offset 0 for k."""
+    r = _rng(seed, 20)
+    return gen_rmsnorm_rope("prefill_rmsnorm_rope_int8", B=65536, S=1, D=576, Dv=512, num_blocks=1024,
+                            block_size=128, k_dtype="i8", ckv_dtype="i8", k_scale=[1.0 / 64.0], k_offset=[0.0],
+                            ckv_scale=r.uniform(1.0 / 48.0, 1.0 / 24.0, size=512),
+                            ckv_offset=r.integers(-4, 4, size=512, endpoint=True).astype(np.float32),
+                            epsilon=1e-6, cache_mode="PA_BNSD", skip_frac=0.05, seed=seed)
+
+
+def cfg4b_dequant_contiguous_kv_output(seed: int = 0) -> Case:
+    """cfg4 in contiguous cache mode ([16, 2048, 4, 128] caches, each batch's
+    1024 tokens written from its start position) with kOut / vOut."""
+    return gen_dequant_rope_quant("cfg4b_dequant_contiguous_kv_output", B=16, S=1024, Nq=16, Nkv=4, D=128, c0=16,
+                                  c1=2048, cache_mode="contiguous", kv_output=True, seed=seed)
+
+
+def cfg4c_dequant_bf16_x(seed: int = 0) -> Case:
+    """cfg4's shapes with bf16 x (no dequantisation) in page mode."""
+    return gen_dequant_rope_quant("cfg4c_dequant_bf16_x", B=16, S=1024, Nq=16, Nkv=4, D=128, c0=512, c1=128,
+                                  x_dtype="bf16", cos_dtype="bf16", cache_mode="page", seed=seed)
+
+
 CONFIGS = {
     "cfg1_compress_mode1": cfg1_compress_mode1,
     "cfg2_rmsnorm_rope": cfg2_rmsnorm_rope,
@@ -321,6 +361,11 @@ CONFIGS = {
     "cfg4_dequant_rope_quant": cfg4_dequant_rope_quant,
     "cfg5a_compress_mode0": cfg5a_compress_mode0,
     "cfg5b_compress_mode2": cfg5b_compress_mode2,
+    "cfg3c_indexer_fp8": cfg3c_indexer_fp8,
+    "cfg3d_indexer_mxfp8_e5m2": cfg3d_indexer_mxfp8_e5m2,
+    "prefill_rmsnorm_rope_int8": prefill_rmsnorm_rope_int8,
+    "cfg4b_dequant_contiguous_kv_output": cfg4b_dequant_contiguous_kv_output,
+    "cfg4c_dequant_bf16_x": cfg4c_dequant_bf16_x,
 }
 
 

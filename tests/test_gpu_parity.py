@@ -170,7 +170,8 @@ def test_indexer_wide_values_and_padding(mode, cdt):
     _same(_ix(97, 128, mode, cdt, kind="wide", pad=24, extra=0, seed=3))
 
 
-@pytest.mark.parametrize("name", ["cfg3a_indexer_mxfp8", "cfg3b_indexer_mxfp4"])
+@pytest.mark.parametrize("name", ["cfg3a_indexer_mxfp8", "cfg3b_indexer_mxfp4", "cfg3c_indexer_fp8",
+                                  "cfg3d_indexer_mxfp8_e5m2"])
 def test_indexer_named_workloads_full_size(name):
     _same(W.CONFIGS[name]())
 
@@ -222,8 +223,9 @@ def test_rmsnorm_rope_named_workload_full_size():
     _same(W.cfg2_rmsnorm_rope())
 
 
-def test_rmsnorm_rope_prefill_size():
-    _same(W.prefill_rmsnorm_rope())
+@pytest.mark.parametrize("name", ["prefill_rmsnorm_rope", "prefill_rmsnorm_rope_int8"])
+def test_rmsnorm_rope_prefill_size(name):
+    _same(W.CONFIGS[name]())
 
 
 @pytest.mark.parametrize("ckv_dtype,k_dtype", [("i8", "bf16"), ("bf16", "bf16"), ("e5m2", "f16"), ("i8", "i8")])
@@ -315,8 +317,10 @@ def test_drq_bad_index_fault():
     _same(case)
 
 
-def test_drq_named_workload_full_size():
-    _same(W.cfg4_dequant_rope_quant())
+@pytest.mark.parametrize("name", ["cfg4_dequant_rope_quant", "cfg4b_dequant_contiguous_kv_output",
+                                  "cfg4c_dequant_bf16_x"])
+def test_drq_named_workload_full_size(name):
+    _same(W.CONFIGS[name]())
 
 
 def test_drq_named_workload_narrow_range():
