@@ -287,8 +287,12 @@ KVQ_API kvq_status kvq_convert(int32_t fmt, const float* in, int64_t n, void* ou
  * division; 7: the bounded wait of the pipelined kernels, run out on purpose
  * (a shared-memory barrier that nothing completes, a short limit): 1 when the
  * wait gave up as designed -- it also sets KVQ_FAULT_TIMEOUT, which
- * kvq_get_error returns and clears.  Blocks until done; *result receives the
- * count (0 means the shortcut is exact on the domain). */
+ * kvq_get_error returns and clears; 8: the number of (value, row maximum,
+ * format) cases, among 2^28 random bf16 / f16 pairs with |value| <= maximum,
+ * each encoded as E4M3 and as E5M2, whose code from the indexer fp8 mode's
+ * two-step quotient by maximum / FP8_MAX differs from the code of the IEEE
+ * quotient.  Blocks until done; *result receives the count (0 means the
+ * shortcut is exact on the domain). */
 KVQ_API kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream);
 
 /* Static description of a status code. */

@@ -71,6 +71,30 @@ __device__ __forceinline__ void ix_fp8_codes(const uint32_t (&w)[16], float s, u
     }
 }
 
+// fp8 mode: whether the row's codes may come from the two-step quotient
+// (div_scale2 with r = RN(1/scale)) instead of IEEE division.  For a finite
+// amax >= 2^-60, scale = RN(amax / FMAX) and r are normal; a value with
+// |x| >= 2^-100 has a normal quotient and normal residuals, so the two-step
+// form returns exactly the IEEE quotient (Markstein, IBM J. Res. Dev. 34(1),
+// 1990); a smaller |x| has a quotient below 2^-23 in magnitude either way,
+// whose code is the signed zero of x's sign either way.  kvq_selftest 8
+// checks the codes of both paths against each other.
+__device__ __forceinline__ bool ix_fp8_fast(float amax) {
+    return amax >= 8.673617379884035e-19f && amax <= 3.4028234663852886e38f;   // [2^-60, FLT_MAX]
+}
+
+// FP8 codes of the 32 values of w divided by s through the two-step quotient
+template <bool F16, bool E5M2>
+__device__ __forceinline__ void ix_fp8_codes_q2(const uint32_t (&w)[16], float s, float r, uint32_t (&c)[8]) {
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        float q[4] = {ix_lo<F16>(w[i]), ix_hi<F16>(w[i]), ix_lo<F16>(w[i + 1]), ix_hi<F16>(w[i + 1])};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) q[k] = div_scale2(q[k], s, r);
+        c[i / 2] = fp8x2<E5M2>(q[0], q[1]) | (fp8x2<E5M2>(q[2], q[3]) << 16);
+    }
+}
+
 // The first nbytes (<= 32) of the 8 code words at p
 __device__ __forceinline__ void ix_store_codes(uint8_t* p, const uint32_t (&c)[8], int nbytes, bool vec32) {
     if (nbytes >= 32) {
@@ -129,11 +153,15 @@ __global__ void __launch_bounds__(IX_THREADS) indexer_quant_kernel(const Indexer
             }
             for (int k = TG >> 1; k >= 1; k >>= 1) m = max(m, __shfl_xor_sync(FULL_MASK, m, k));
             if (!live) continue;
-            const float scale = div_by_fmax(ix_amax<F16>(m), FMAX);
+            const float amax = ix_amax<F16>(m);
+            const float scale = div_by_fmax(amax, FMAX);
+            const bool fast = ix_fp8_fast(amax);
+            const float r = fast ? __frcp_rn(scale) : 0.0f;
             for (int g = gl; g < a.ngroups; g += TG) {
                 if (!keep) ix_load_group(a, xrow, g, w);
                 uint32_t c[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-                if (scale != 0.0f) ix_fp8_codes<F16, E5M2, true>(w, scale, c);
+                if (fast) ix_fp8_codes_q2<F16, E5M2>(w, scale, r, c);
+                else if (scale != 0.0f) ix_fp8_codes<F16, E5M2, true>(w, scale, c);
                 ix_store_codes(crow + 32 * g, c, a.d - 32 * g, v32);
             }
             if (gl == 0) st_b32(srow, __float_as_uint(scale));

@@ -357,6 +357,46 @@ __global__ void selftest_timeout_kernel() {
     if (threadIdx.x == 0 && !done) atomicAdd(&g_selftest_count, 1ull);
 }
 
+// The indexer's fp8 mode: codes from the two-step quotient (where
+// ix_fp8_fast admits the row maximum) against codes from IEEE division, for
+// 2^28 random (x, amax) pairs per call: amax a random finite bf16 (as bits)
+// of binade 2^-70 .. 2^127 or f16 (alternating calls' halves), x a random
+// value of the same type with |x| <= amax (every binade down to the
+// subnormals, zeros of both signs included), E4M3 and E5M2 codes; counts the
+// pairs whose codes differ.
+__global__ void selftest_fp8_row_kernel() {
+    const uint64_t i0 = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) * 16u;
+    unsigned long long bad = 0;
+    for (uint64_t i = i0; i < i0 + 16u; ++i) {
+        const uint64_t h1 = st_mix(2 * i), h2 = st_mix(2 * i + 1);
+        const bool f16 = (i >> 20) & 1u;
+        float amax, x;
+        if (f16) {
+            const uint32_t ab = 1u + (uint32_t)(h1 % 0x7bffu);                      // (0, 65504]
+            amax = __half2float(__ushort_as_half((unsigned short)ab));
+            const uint32_t xb = (uint32_t)((h2 >> 8) % (ab + 1u)) | ((uint32_t)(h2 & 1u) << 15);
+            x = __half2float(__ushort_as_half((unsigned short)xb));
+        } else {
+            const uint32_t ab = 0x0880u + (uint32_t)(h1 % (0x7f80u - 0x0880u));    // [~2^-111, max bf16]
+            amax = __uint_as_float(ab << 16);
+            const uint32_t xb = (uint32_t)((h2 >> 8) % (ab + 1u)) | ((uint32_t)(h2 & 1u) << 15);
+            x = __uint_as_float(xb << 16);
+        }
+        if (!kvq::ix_fp8_fast(amax)) continue;
+#pragma unroll
+        for (int e5 = 0; e5 < 2; ++e5) {
+            const float fmax = e5 ? 57344.0f : 448.0f;
+            const float s = div_by_fmax(amax, fmax);
+            const float q2 = div_scale2(x, s, __frcp_rn(s));
+            const float qi = __fdiv_rn(x, s);
+            const uint32_t c2 = e5 ? fp8x2<true>(q2, 0.0f) : fp8x2<false>(q2, 0.0f);
+            const uint32_t ci = e5 ? fp8x2<true>(qi, 0.0f) : fp8x2<false>(qi, 0.0f);
+            bad += c2 != ci ? 1ull : 0ull;
+        }
+    }
+    if (bad) atomicAdd(&g_selftest_count, bad);
+}
+
 // every positive finite bf16 amax (bits < 0x7f80) and every positive finite
 // f16 amax (bits < 0x7c00) over the three format maxima
 __global__ void selftest_fmax_kernel() {
@@ -402,7 +442,7 @@ extern "C" {
 
 kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream) {
     if (!result) return KVQ_ERR_NULL;
-    if (which < 0 || which > 7) return KVQ_ERR_ATTR;
+    if (which < 0 || which > 8) return KVQ_ERR_ATTR;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const unsigned long long zero = 0ull;
     unsigned long long h = 0ull;
@@ -411,6 +451,7 @@ kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream) {
     if (which == 4) selftest_fmax_kernel<<<256, 256, 0, s>>>();
     else if (which == 6) selftest_int8_kernel<<<65536, 256, 0, s>>>();
     else if (which == 7) selftest_timeout_kernel<<<1, 32, 0, s>>>();
+    else if (which == 8) selftest_fp8_row_kernel<<<65536, 256, 0, s>>>();
     else selftest_div_kernel<<<65536, 256, 0, s>>>(which);
     if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
     if (cudaMemcpyFromSymbolAsync(&h, g_selftest_count, sizeof(h), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)

@@ -10,7 +10,10 @@ whole input domain against IEEE division:
   * the dequant kernel's static int8 quantisation through a per-channel
     reciprocal (two-step Markstein form, IEEE division outside its guard):
     the same int8 codes as IEEE division on 2^28 random and near-tie
-    (value, scale, offset) triples.
+    (value, scale, offset) triples;
+  * the indexer fp8 mode's division by the row scale (two-step Markstein form
+    where the row maximum is a finite value >= 2^-60): the same E4M3 and E5M2
+    codes as IEEE division on 2^28 random bf16 / f16 (value, maximum) pairs.
 Also the failure path of the pipelined kernels' bounded waits: a wait on a
 barrier that nothing completes gives up after its limit and reports
 FAULT_TIMEOUT through the fault word (no GPU fault, hang or trap)."""
@@ -24,7 +27,8 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("which,what", [(2, "E4M3 codes of the one-step quotient"),
                                         (3, "E2M1 codes of the one-step quotient"),
                                         (4, "constant-divisor scale quotients"),
-                                        (6, "int8 codes of the reciprocal-based quotient")])
+                                        (6, "int8 codes of the reciprocal-based quotient"),
+                                        (8, "fp8 row-scale codes of the two-step quotient")])
 def test_shortcut_is_exact(which, what):
     assert kvq.selftest(which) == 0, what
 
