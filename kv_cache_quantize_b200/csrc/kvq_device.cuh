@@ -244,6 +244,26 @@ __device__ __forceinline__ void div2_add_x2(float a0, float a1, float s0, float 
         : "f"(a0), "f"(a1), "f"(-s0), "f"(-s1), "f"(r0), "f"(r1), "f"(f0), "f"(f1));
 }
 
+// The two-step quotient of div2_add_x2 without the offset, one common divisor
+// s with r = RN(1/s), signed zeros kept (a zero numerator gives a zero of its
+// sign): (RN(a0 / s), RN(a1 / s)) under the same range conditions.
+__device__ __forceinline__ void div2_x2(float a0, float a1, float s, float r, float& q0, float& q1) {
+    asm("{\n\t.reg .b64 a, ns, rr, q, e;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 ns, {%4, %4};\n\t"
+        "mov.b64 rr, {%5, %5};\n\t"
+        "mul.rn.f32x2 q, a, rr;\n\t"
+        "fma.rn.f32x2 e, q, ns, a;\n\t"
+        "fma.rn.f32x2 q, e, rr, q;\n\t"
+        "fma.rn.f32x2 e, q, ns, a;\n\t"
+        "fma.rn.f32x2 q, e, rr, q;\n\t"
+        "mov.b64 {%0, %1}, q;\n\t}"
+        : "=f"(q0), "=f"(q1)
+        : "f"(a0), "f"(a1), "f"(-s), "f"(r));
+    q0 = with_sign_of(q0, a0);
+    q1 = with_sign_of(q1, a1);
+}
+
 // Four binary32 values rounded half to even to integers and saturated to
 // int8, packed little-endian (value 0 in byte 0).  NaN gives 0.
 __device__ __forceinline__ uint32_t int8x4_rne_sat(float v0, float v1, float v2, float v3) {

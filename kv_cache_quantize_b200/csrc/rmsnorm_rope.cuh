@@ -105,9 +105,21 @@ __device__ __forceinline__ int64_t rr_resolve(const RmsRopeArgs& a, int64_t b, i
     return v;                                      // PA, PA_BNSD
 }
 
+// A per-tensor ckv scale s in [2^-40, 2^40] and r = RN(1/s): the FP8 codes of
+// y / s come from the two-step quotient (div2_x2) for chunks with every
+// |y| <= 2^60.  It is exact for |y| >= 2^-103 (the residual is then a
+// multiple of 2^-149, so the fused operations form it exactly, and the
+// quotient stays normal); a smaller |y| has |y / s| < 2^-63, whose code is
+// the zero of y's sign either way.
+struct CkvDiv {
+    float s, r;
+    bool fast;
+};
+
 // y[0..7] = chunk c of the RMSNorm segment normalised and scaled, stored as
 // the ckv cache's dtype (8 values at row element 8c)
-__device__ __forceinline__ void rr_store_chunk(const CacheOut& c, uint8_t* row, int ch, const float (&y)[8]) {
+__device__ __forceinline__ void rr_store_chunk(const CacheOut& c, uint8_t* row, int ch, const float (&y)[8],
+                                               const CkvDiv& dv) {
     const int j0 = 8 * ch;
     switch (c.dt) {
         case CDT_BF16:
@@ -125,8 +137,16 @@ __device__ __forceinline__ void rr_store_chunk(const CacheOut& c, uint8_t* row, 
         case CDT_E4M3:
         case CDT_E5M2: {
             float q[8];
+            float ym = 0.0f;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) q[k] = __fdiv_rn(y[k], c.scale[c.scale_n == 1 ? 0 : j0 + k]);
+            for (int k = 0; k < 8; ++k) ym = fmaxf(ym, fabsf(y[k]));
+            if (dv.fast && ym <= 1.152921504606846976e18f) {            // 2^60
+#pragma unroll
+                for (int k = 0; k < 8; k += 2) div2_x2(y[k], y[k + 1], dv.s, dv.r, q[k], q[k + 1]);
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) q[k] = __fdiv_rn(y[k], c.scale[c.scale_n == 1 ? 0 : j0 + k]);
+            }
             st_b64(row + j0, c.dt == CDT_E4M3 ? fp8x8<false>(q) : fp8x8<true>(q));
             break;
         }
@@ -190,6 +210,12 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
             sn = (uint32_t)a.sin[t * a.Dk + lane] | ((uint32_t)a.sin[t * a.Dk + h + lane] << 16);
         }
     };
+    CkvDiv dv{0.0f, 0.0f, false};
+    if (NCH > 0 && (a.ckv.dt == CDT_E4M3 || a.ckv.dt == CDT_E5M2) && a.ckv.scale_n == 1) {
+        dv.s = a.ckv.scale[0];
+        dv.fast = dv.s >= 9.094947017729282e-13f && dv.s <= 1.099511627776e12f;   // [2^-40, 2^40]
+        dv.r = dv.fast ? __frcp_rn(dv.s) : 0.0f;
+    }
     if (NCH > 0) load_chunks(gwarp, xn);
     prefetch(gwarp);
     for (int64_t t = gwarp; t < ntok; t += nwarps) {
@@ -211,8 +237,11 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
         uint8_t* crow = slot_row(a.ckv.rows, slot);
 
         if (NCH > 0) {
-            // RMSNorm: sum of squares in the fixed lane order, chunks from registers
+            // RMSNorm: sum of squares in the fixed lane order, chunks from registers;
+            // also the lane's smallest nonzero |x|, as 2 |x|bits - 2 (zeros wrap
+            // to the largest value)
             float acc = 0.0f;
+            uint32_t xmin2 = 0xffffffffu;
 #pragma unroll
             for (int m = 0; m < NCH; ++m) {
                 if (lane + 32 * m >= nch) break;
@@ -220,12 +249,29 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
                 if (a.kv_f16) widen8<true>(xv[m], f);
                 else widen8<false>(xv[m], f);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc = __fadd_rn(acc, __fmul_rn(f[i], f[i]));
+                for (int i = 0; i < 8; ++i) {
+                    acc = __fadd_rn(acc, __fmul_rn(f[i], f[i]));
+                    xmin2 = min(xmin2, 2u * __float_as_uint(f[i]) - 2u);
+                }
             }
 #pragma unroll
             for (int k = 16; k >= 1; k >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(FULL_MASK, acc, k));
             const float mean = __fdiv_rn(acc, (float)a.Dv);
             const float rms = __fsqrt_rn(__fadd_rn(mean, a.eps));
+            // x / rms as (x 2^64) / (rms 2^64), the same real quotient, by the
+            // two-step form.  For rms in [2^-60, 2^50] every |x| is below
+            // rms sqrt(Dv) < 2^56, so the scaled numerators (bf16 / f16: at
+            // least 2^-133 unscaled), divisor, reciprocal and residuals are
+            // normal; the lane also needs every nonzero |x| >= RN(rms 2^-125)
+            // (a normal quotient, with a factor 2 for the rounding of the
+            // bound: a subnormal quotient can be an exact rounding tie, which
+            // the two-step form may break the wrong way).  Then the quotient
+            // is RN(x / rms).
+            const float thr = __fmul_rn(rms, 2.350988701644575e-38f);            // rms 2^-125
+            const bool nfast = rms >= 8.673617379884035e-19f && rms <= 1.125899906842624e15f &&
+                               xmin2 >= 2u * __float_as_uint(thr) - 2u;
+            const float rs64 = __fmul_rn(rms, 1.8446744073709552e19f);
+            const float rr64 = nfast ? __frcp_rn(rs64) : 0.0f;
 #pragma unroll
             for (int m = 0; m < NCH; ++m) {
                 const int c = lane + 32 * m;
@@ -239,9 +285,18 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
                     widen8<false>(xv[m], f);
                     widen8<false>(gv, g);
                 }
+                if (nfast) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fdiv_rn(f[i], rms), g[i]);
-                rr_store_chunk(a.ckv, crow, c, y);
+                    for (int i = 0; i < 8; i += 2)
+                        div2_x2(__fmul_rn(f[i], 1.8446744073709552e19f), __fmul_rn(f[i + 1], 1.8446744073709552e19f),
+                                rs64, rr64, y[i], y[i + 1]);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(y[i], g[i]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fdiv_rn(f[i], rms), g[i]);
+                }
+                rr_store_chunk(a.ckv, crow, c, y, dv);
             }
         } else {
             // RMSNorm: sum of squares in the fixed lane order

@@ -228,6 +228,34 @@ def test_rmsnorm_rope_prefill_size(name):
     _same(W.CONFIGS[name]())
 
 
+@pytest.mark.parametrize("ckv_dtype", ["bf16", "e4m3"])
+def test_rmsnorm_rope_subnormal_and_tie_quotients(ckv_dtype):
+    """Rows whose x / rms quotients are subnormal, two of them exact rounding
+    ties (epsilon 0): rms = 2^17 with x = 3 * 2^-133 (quotient 3 * 2^-150,
+    which rounds to the even 2^-148) and rms = 3 * 2^17 with the same x
+    (quotient 2^-150, which rounds to 0); other rows mix bf16 subnormals, zeros
+    and large values into random rows."""
+    case = _rr(B=48, ckv_dtype=ckv_dtype, k_dtype="bf16", seed=41, epsilon=0.0)
+    kv = case.arrays["kv"].reshape(48, 576)
+    live = np.nonzero(case.arrays["index"].reshape(-1) != -1)[0]
+    bits = lambda v: W.to_bf16_bits(np.array([v], dtype=np.float32))[0]
+    for r, big in ((live[0], 2.0 ** 21), (live[1], 3.0 * 2.0 ** 21)):
+        kv[r, :512] = 0
+        kv[r, 10] = kv[r, 300] = bits(big)
+        kv[r, 77] = 3                                 # 3 * 2^-133, a bf16 subnormal
+        kv[r, 78] = 3 | 0x8000                        # its negative
+    # a gamma of 2^100 on those two channels carries the quotients' last bits
+    # into the output (2^-148 * 2^100 = 2^-48 is a normal bf16 value)
+    case.arrays["gamma"][77] = case.arrays["gamma"][78] = bits(2.0 ** 100)
+    rng = np.random.default_rng(43)
+    for r in live[2::3]:
+        cols = rng.choice(512, size=12, replace=False)
+        kv[r, cols[:6]] = rng.integers(1, 128, size=6).astype(np.uint16) | (rng.integers(0, 2, size=6) << 15).astype(np.uint16)
+        kv[r, cols[6:9]] = 0
+        kv[r, cols[9:]] = bits(2.0 ** 40)
+    _same(case)
+
+
 @pytest.mark.parametrize("ckv_dtype,k_dtype", [("i8", "bf16"), ("bf16", "bf16"), ("e5m2", "f16"), ("i8", "i8")])
 def test_rmsnorm_rope_vector_path_dtypes(ckv_dtype, k_dtype):
     """Aligned rows with Dv = 256 / 512 / 1024 take the register-chunk kernel for every ckv dtype."""
