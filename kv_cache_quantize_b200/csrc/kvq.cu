@@ -862,12 +862,15 @@ kvq_status kvq_kv_rmsnorm_rope_cache(const kvq_tensor* kv, const kvq_tensor* gam
     const bool vec = reinterpret_cast<uintptr_t>(kv->data) % 16 == 0 &&
                      reinterpret_cast<uintptr_t>(gamma->data) % 16 == 0 && D % 8 == 0 && Dv % 8 == 0;
     const int64_t nch = Dv / 8;
-    if (vec && nch <= 32) launch(rmsnorm_rope_kernel<1>, (unsigned)persistent_grid(rmsnorm_rope_kernel<1>, RR_THREADS, need),
-                                 RR_THREADS, 0, s, a);
-    else if (vec && nch <= 64) launch(rmsnorm_rope_kernel<2>, (unsigned)persistent_grid(rmsnorm_rope_kernel<2>, RR_THREADS, need),
-                                      RR_THREADS, 0, s, a);
-    else if (vec && nch <= 128) launch(rmsnorm_rope_kernel<4>, (unsigned)persistent_grid(rmsnorm_rope_kernel<4>, RR_THREADS, need),
-                                       RR_THREADS, 0, s, a);
+    // the register-chunk kernels stage an int8 ckv cache's parameters in shared memory
+    a.ckv_stage = vec && nch <= 128 && cc.dt == CDT_I8;
+    const size_t smem = a.ckv_stage ? (size_t)3 * Dv * sizeof(float) : 0;
+    if (vec && nch <= 32) launch(rmsnorm_rope_kernel<1>, (unsigned)persistent_grid(rmsnorm_rope_kernel<1>, RR_THREADS, need, smem),
+                                 RR_THREADS, smem, s, a);
+    else if (vec && nch <= 64) launch(rmsnorm_rope_kernel<2>, (unsigned)persistent_grid(rmsnorm_rope_kernel<2>, RR_THREADS, need, smem),
+                                      RR_THREADS, smem, s, a);
+    else if (vec && nch <= 128) launch(rmsnorm_rope_kernel<4>, (unsigned)persistent_grid(rmsnorm_rope_kernel<4>, RR_THREADS, need, smem),
+                                       RR_THREADS, smem, s, a);
     else launch(rmsnorm_rope_kernel<0>, (unsigned)persistent_grid(rmsnorm_rope_kernel<0>, RR_THREADS, need),
                 RR_THREADS, 0, s, a);
     return launched();

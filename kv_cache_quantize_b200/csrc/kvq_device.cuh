@@ -278,6 +278,46 @@ __device__ __forceinline__ uint32_t int8x4_rne_sat(float v0, float v1, float v2,
     return r;
 }
 
+// Static int8 of four values: round half to even of o / scale + offset,
+// saturated (offset 0 when absent), packed little-endian.  r holds RN(1/scale)
+// for channels whose scale lies in [2^-60, 2^60] and whose |offset| <= 2^16,
+// else 0.  When every r is set and every |o| <= 2^60 the quotient comes
+// from the two-step Markstein form, which is then exact wherever the result
+// depends on it: a quotient in [2^-30, 2^20] has normal operands, residuals
+// and result, so it equals the IEEE quotient; below 2^-30 the rounded sum
+// with any binary32 offset, hence the integer, does not depend on the
+// quotient's last bits; above 2^20 the integer saturates either way.  Other
+// lanes divide with IEEE division.  kvq_selftest checks the two paths against
+// each other on random and near-tie triples.
+__device__ __forceinline__ float div2_add(float a, float s, float r, float f) {
+    const float q0 = __fmul_rn(a, r);
+    const float q1 = __fmaf_rn(__fmaf_rn(-q0, s, a), r, q0);
+    const float q2 = __fmaf_rn(__fmaf_rn(-q1, s, a), r, q1);
+    return __fadd_rn(q2, f);
+}
+
+__device__ __forceinline__ uint32_t int8x4_quant(const float (&o)[4], const float (&s)[4], const float (&f)[4],
+                                                 const float (&r)[4]) {
+    float q[4];
+    const float m = fmaxf(fmaxf(fabsf(o[0]), fabsf(o[1])), fmaxf(fabsf(o[2]), fabsf(o[3])));
+    const float rmin = fminf(fminf(r[0], r[1]), fminf(r[2], r[3]));
+    if (m <= 1.152921504606846976e18f && rmin > 0.0f) {      // |o| <= 2^60, every channel eligible
+#pragma unroll
+        for (int k = 0; k < 4; ++k) q[k] = div2_add(o[k], s[k], r[k], f[k]);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) q[k] = __fadd_rn(__fdiv_rn(o[k], s[k]), f[k]);
+    }
+    return int8x4_rne_sat(q[0], q[1], q[2], q[3]);
+}
+
+// RN(1/scale) where the fast quotient of int8x4_quant applies, else 0
+__device__ __forceinline__ float int8_quant_rcp(float sc, float of) {
+    const uint32_t e = (__float_as_uint(sc) >> 23) & 0xffu;
+    const bool ok = sc > 0.0f && e >= 67u && e <= 187u && fabsf(of) <= 65536.0f;
+    return ok ? __frcp_rn(sc) : 0.0f;
+}
+
 // Largest magnitude of the two bf16 halves of a and b, per half (max of the
 // absolute values; the sign bits of the result are not meaningful).
 __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {

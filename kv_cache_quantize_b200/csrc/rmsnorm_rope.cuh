@@ -42,6 +42,7 @@ struct RmsRopeArgs {
     CacheOut k;             // Dk values per row
     CacheOut ckv;           // Dv values per row
     float eps;
+    int32_t ckv_stage;      // int8 ckv: scales, offsets and reciprocals staged in shared memory ([3][Dv])
 };
 
 constexpr int RR_THREADS = 128;
@@ -119,7 +120,7 @@ struct CkvDiv {
 // y[0..7] = chunk c of the RMSNorm segment normalised and scaled, stored as
 // the ckv cache's dtype (8 values at row element 8c)
 __device__ __forceinline__ void rr_store_chunk(const CacheOut& c, uint8_t* row, int ch, const float (&y)[8],
-                                               const CkvDiv& dv) {
+                                               const CkvDiv& dv, const float* stg, int Dv) {
     const int j0 = 8 * ch;
     switch (c.dt) {
         case CDT_BF16:
@@ -151,6 +152,22 @@ __device__ __forceinline__ void rr_store_chunk(const CacheOut& c, uint8_t* row, 
             break;
         }
         case CDT_I8: {
+            if (stg) {
+                // the staged per-channel scale, offset and RN(1/scale): int8x4_quant
+                uint32_t w[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float4 sv = *reinterpret_cast<const float4*>(stg + j0 + 4 * h);
+                    const float4 fv = *reinterpret_cast<const float4*>(stg + Dv + j0 + 4 * h);
+                    const float4 rv = *reinterpret_cast<const float4*>(stg + 2 * Dv + j0 + 4 * h);
+                    const float o4[4] = {y[4 * h], y[4 * h + 1], y[4 * h + 2], y[4 * h + 3]};
+                    const float s4[4] = {sv.x, sv.y, sv.z, sv.w}, f4[4] = {fv.x, fv.y, fv.z, fv.w};
+                    const float r4[4] = {rv.x, rv.y, rv.z, rv.w};
+                    w[h] = int8x4_quant(o4, s4, f4, r4);
+                }
+                st_b64(row + j0, make_uint2(w[0], w[1]));
+                break;
+            }
             uint32_t w[2] = {0u, 0u};
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
@@ -210,6 +227,21 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
             sn = (uint32_t)a.sin[t * a.Dk + lane] | ((uint32_t)a.sin[t * a.Dk + h + lane] << 16);
         }
     };
+    // int8 ckv: per-channel scale, offset (0 when absent) and the reciprocal
+    // of int8x4_quant, staged once per CTA
+    extern __shared__ __align__(16) float rr_stage[];
+    const float* stg = nullptr;
+    if (NCH > 0 && a.ckv_stage) {
+        for (int i = threadIdx.x; i < a.Dv; i += blockDim.x) {
+            const float sc = a.ckv.scale[a.ckv.scale_n == 1 ? 0 : i];
+            const float of = a.ckv.offset ? a.ckv.offset[a.ckv.offset_n == 1 ? 0 : i] : 0.0f;
+            rr_stage[i] = sc;
+            rr_stage[a.Dv + i] = of;
+            rr_stage[2 * a.Dv + i] = int8_quant_rcp(sc, of);
+        }
+        __syncthreads();
+        stg = rr_stage;
+    }
     CkvDiv dv{0.0f, 0.0f, false};
     if (NCH > 0 && (a.ckv.dt == CDT_E4M3 || a.ckv.dt == CDT_E5M2) && a.ckv.scale_n == 1) {
         dv.s = a.ckv.scale[0];
@@ -296,7 +328,7 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
 #pragma unroll
                     for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fdiv_rn(f[i], rms), g[i]);
                 }
-                rr_store_chunk(a.ckv, crow, c, y, dv);
+                rr_store_chunk(a.ckv, crow, c, y, dv, stg, a.Dv);
             }
         } else {
             // RMSNorm: sum of squares in the fixed lane order
