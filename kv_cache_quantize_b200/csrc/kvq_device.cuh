@@ -410,14 +410,6 @@ __device__ __forceinline__ void st_b128(uint8_t* p, uint4 v) {
     }
 }
 
-// Store the first nbytes (0..16) of v at p, byte by byte.
-__device__ __forceinline__ void st_partial(uint8_t* p, uint4 v, int nbytes) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int k = 0; k < 16; ++k)
-        if (k < nbytes) p[k] = (uint8_t)(w[k >> 2] >> (8 * (k & 3)));
-}
-
 // 32 16-bit values (64 bytes) at p as 16 words (value 2i in the low half of word i).
 __device__ __forceinline__ void ld_slice(const uint16_t* p, int vec, uint32_t (&w)[16]) {
     if (vec == 2) {

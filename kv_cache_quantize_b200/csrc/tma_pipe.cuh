@@ -107,18 +107,4 @@ __device__ __forceinline__ void named_barrier_arrive(int threads) {
     asm volatile("bar.arrive 1, %0;" ::"r"(threads) : "memory");
 }
 
-// the same barrier, returning whether `pred` holds in every participating thread
-__device__ __forceinline__ bool named_barrier_and(int threads, bool pred) {
-    uint32_t out;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, 1, %2, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(out)
-        : "r"((uint32_t)pred), "r"(threads)
-        : "memory");
-    return out != 0;
-}
-
 }  // namespace kvq
