@@ -32,6 +32,8 @@ struct CompressArgs {
     int32_t col;            // kvCacheCol
     float x_scale;          // mode 2 rope multiplier
     int32_t x_vec;          // every row chunk is 16-byte aligned
+    // direct kernel only
+    int32_t ce_rows;        // rows per warp tile, 1 .. CE_TILE
     // pipelined kernel only
     int32_t stages;         // ring depth
     int32_t ncw;            // consumer warps
@@ -46,6 +48,11 @@ struct CompressArgs {
 // E2M1 codes kvq_selftest shows equal to those of IEEE division on its whole
 // domain.
 
+// Direct kernel: a warp takes tiles of ce_rows rows (at most CE_TILE), loading
+// CE_UNROLL 16-byte chunks per lane per round; the host picks the smallest
+// tile whose segments still fill one round, so that a decode-sized batch is
+// spread over as many warps as it has rows and each warp makes one
+// load-compute-store round trip.
 constexpr int CE_TILE = 8;
 constexpr int CE_UNROLL = 3;
 constexpr int CE_THREADS = 256;
@@ -151,11 +158,12 @@ __global__ void __launch_bounds__(CE_THREADS) compress_epilog_kernel(const Compr
     const int sub = lane & 7;
     const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const int64_t ntiles = (a.T + CE_TILE - 1) / CE_TILE;
+    const int tr = a.ce_rows;
+    const int64_t ntiles = (a.T + tr - 1) / tr;
 
     for (int64_t tile = gwarp; tile < ntiles; tile += nwarps) {
-        const int64_t row0 = tile * CE_TILE;
-        const int rows = (int)(a.T - row0 < CE_TILE ? a.T - row0 : CE_TILE);
+        const int64_t row0 = tile * tr;
+        const int rows = (int)(a.T - row0 < tr ? a.T - row0 : tr);
         int64_t my_slot = -1;
         if (lane < rows) {
             my_slot = load_slot(a.slots, a.slots_i64, row0 + lane);

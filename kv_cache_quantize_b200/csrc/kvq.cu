@@ -589,7 +589,11 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
 #undef KVQ_LAUNCH_CT
         return launched();
     }
-    const int64_t tiles = (T + CE_TILE - 1) / CE_TILE;
+    {
+        const int64_t r = (4 * CE_UNROLL) / a.nseg;       // rows whose segments fill one round
+        a.ce_rows = (int32_t)(r < 1 ? 1 : (r > CE_TILE ? CE_TILE : r));
+    }
+    const int64_t tiles = (T + a.ce_rows - 1) / a.ce_rows;
     const int64_t need = (tiles + (CE_THREADS / 32) - 1) / (CE_THREADS / 32);
 #define KVQ_LAUNCH_CE(M, GG)                                                                   \
     do {                                                                                       \
