@@ -163,7 +163,7 @@ KVQ_API int64_t kvq_kv_cache_col(int64_t d, int32_t quant_mode, int32_t quant_gr
 /* Source: indexer_quant_cache, 接口功能 / 语义说明 / 约束说明.                 */
 /*                                                                           */
 /* x            bf16 or f16 [..., d], last dimension contiguous, leading dims */
-/*              flattenable to T rows.                                        */
+/*              flattenable to T rows; 1 <= d <= 2^24 (else KVQ_ERR_SHAPE).   */
 /* cache        [blockNum, blockSize, 1, headDim]: FLOAT8 E4M3 or E5M2 for    */
 /*              mxfp8/fp8 (headDim >= d), uint8 for mxfp4 (headDim >=         */
 /*              ceil(d/2) bytes, two E2M1 codes per byte, even element low).  */
@@ -189,7 +189,8 @@ KVQ_API int64_t kvq_indexer_scale_col(int64_t d, int32_t quant_mode);
 /* Source: aclnnKvRmsNormRopeCache, 接口功能 / 计算公式 / 约束说明.             */
 /*                                                                           */
 /* kv        bf16 or f16 [B, 1, S, D] contiguous (N = 1).  D = Dv + Dk with   */
-/*           Dv = ckv_cache's last dim, Dk = k_cache's last dim, Dk even.     */
+/*           Dv = ckv_cache's last dim, Dk = k_cache's last dim, Dk even,    */
+/*           D <= 2^24 (else KVQ_ERR_SHAPE).                                   */
 /* gamma     [Dv], same dtype as kv.                                          */
 /* cos, sin  [B, 1, S, Dk], same dtype as kv, contiguous.                     */
 /* index     int32/int64.  cache_mode 0 Norm: [B, S], values in [-1, Scache), */

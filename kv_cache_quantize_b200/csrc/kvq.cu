@@ -679,7 +679,7 @@ kvq_status kvq_indexer_quant_cache(const kvq_tensor* x, kvq_tensor* cache, kvq_t
     int64_t T, rs;
     if (!flatten_rows(x, &T, &rs)) return KVQ_ERR_LAYOUT;
     const int64_t d = x->shape[x->ndim - 1];
-    if (d < 1) return KVQ_ERR_SHAPE;
+    if (d < 1 || d > (1 << 24)) return KVQ_ERR_SHAPE;    // the kernel indexes a row with 32-bit integers
     if (quant_mode == 2) return KVQ_ERR_UNSUPPORTED;
     if (quant_mode != 0 && quant_mode != 1 && quant_mode != 3) return KVQ_ERR_ATTR;
     if (quant_mode == 3) {
@@ -824,6 +824,7 @@ kvq_status kvq_kv_rmsnorm_rope_cache(const kvq_tensor* kv, const kvq_tensor* gam
     st = setup_cache_out(ckv_cache, ckv_scale, ckv_offset, &cc, &Dv);
     if (st != KVQ_OK) return st;
     if (Dk + Dv != D || Dk % 2 != 0 || Dk < 2 || Dv < 1) return KVQ_ERR_SHAPE;
+    if (D > (1 << 24)) return KVQ_ERR_SHAPE;              // the kernel indexes a row with 32-bit integers
     const bool kq = kc.dt >= CDT_E4M3, cq = cc.dt >= CDT_E4M3;
     if (kq && cq && kc.dt != cc.dt) return KVQ_ERR_DTYPE;     // scenario 3 needs one dtype
     if (k_cache->shape[0] != ckv_cache->shape[0] || kc.rows.block_size != cc.rows.block_size) return KVQ_ERR_SHAPE;

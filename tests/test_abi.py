@@ -261,3 +261,11 @@ def test_missing_library_fails_loudly(tmp_path):
             "    print('no error')\n")
     out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT, timeout=300)
     assert "raised:" in out.stdout and "not built" in out.stdout, out.stdout + out.stderr
+
+
+def test_row_widths_beyond_32_bit_indexing_are_rejected(L):
+    """The indexer's d and the rmsnorm/rope D are bounded by 2^24 (the kernels index a row with 32-bit integers)."""
+    wide = (1 << 24) + 32
+    f = lambda x, c, sc, s: L.kvq_indexer_quant_cache(R(x), R(c), R(sc), R(s), 0, None)
+    assert f(D([4, wide], "bf16"), D([1, 16, 1, wide], "e4m3"), D([1, 16, 1, wide // 32], "e8m0"),
+             D([4], "i32")) == ESHAPE
