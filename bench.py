@@ -272,7 +272,7 @@ def run_reference(args):
         return 0
     from kv_cache_quantize_b200 import workloads as W
     threads = os.cpu_count() or 1
-    cases = [W.cfg5a_compress_mode0(), W.cfg5b_compress_mode2()]
+    cases = [W.compress_mode0_T262144_d576(), W.compress_mode2_G32_T262144_d576()]
     # size each step so that warmup + steps end within about two minutes
     rate, _, _ = oracle_rows_per_s(cases, 2.0, threads)
     per_step_s = min(10.0, 120.0 / max(1, args.steps + args.warmup))
@@ -402,8 +402,8 @@ def main():
     kvq.lib()
 
     # ---------------- headline workload ----------------
-    case_a = rank_workload(W.cfg5a_compress_mode0, rank, world, args.scaling)
-    case_b = rank_workload(W.cfg5b_compress_mode2, rank, world, args.scaling)
+    case_a = rank_workload(W.compress_mode0_T262144_d576, rank, world, args.scaling)
+    case_b = rank_workload(W.compress_mode2_G32_T262144_d576, rank, world, args.scaling)
     call_a, st_a, _ = W.build_call(case_a)
     call_b, st_b, _ = W.build_call(case_b)
     stream = torch.cuda.current_stream(dev)
@@ -510,7 +510,8 @@ def main():
         per_config = {}
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         for name, make in W.CONFIGS.items():
-            case = {"cfg5a_compress_mode0": case_a, "cfg5b_compress_mode2": case_b}.get(name) or make()
+            case = {"compress_mode0_T262144_d576": case_a,
+                    "compress_mode2_G32_T262144_d576": case_b}.get(name) or make()
             calls = rotation(case, make, l2)
             us = device_us_per_launch(calls, stream, 200)
             nb = algorithmic_bytes(case)
@@ -522,7 +523,7 @@ def main():
             del calls, case
             torch.cuda.empty_cache()
         # the packed-row decoder on the headline caches (written by the timed encoder)
-        for name, case in (("cfg5a_decompress_mode0", case_a), ("cfg5b_decompress_mode2", case_b)):
+        for name, case in (("decompress_mode0_T262144_d576", case_a), ("decompress_mode2_G32_T262144_d576", case_b)):
             call, st, _ = W.build_call(case)
             call(stream)
             cb, at = case.caches["cache"], case.attrs

@@ -266,106 +266,108 @@ def gen_dequant_rope_quant(name: str, B: int, S: int, Nq: int, Nkv: int, D: int,
 # ---------------------------------------------------------------------------
 # the five named workloads (sizes and distributions as specified for them)
 # ---------------------------------------------------------------------------
-def cfg1_compress_mode1(seed: int = 0) -> Case:
-    return gen_compress("cfg1_compress_mode1", T=64, d=256, quant_mode=1, num_blocks=8, block_size=16,
+def compress_mode1_T64_d256(seed: int = 0) -> Case:
+    return gen_compress("compress_mode1_T64_d256", T=64, d=256, quant_mode=1, num_blocks=8, block_size=16,
                         head_dim=323, skip_frac=0.10, seed=seed)
 
 
-def cfg2_rmsnorm_rope(seed: int = 0) -> Case:
-    return gen_rmsnorm_rope("cfg2_rmsnorm_rope", B=64, S=1, D=576, Dv=512, num_blocks=4096, block_size=128,
+def rmsnorm_rope_decode_B64_D576(seed: int = 0) -> Case:
+    return gen_rmsnorm_rope("rmsnorm_rope_decode_B64_D576", B=64, S=1, D=576, Dv=512, num_blocks=4096, block_size=128,
                             k_dtype="bf16", ckv_dtype="e4m3", ckv_scale=[1.0 / 64.0], epsilon=1e-6,
                             cache_mode="PA_BNSD", skip_frac=0.05, seed=seed)
 
 
-def cfg3a_indexer_mxfp8(seed: int = 0) -> Case:
-    return gen_indexer("cfg3a_indexer_mxfp8", T=65536, d=128, quant_mode=0, num_blocks=2048, block_size=64,
+def indexer_mxfp8_T65536_d128(seed: int = 0) -> Case:
+    return gen_indexer("indexer_mxfp8_T65536_d128", T=65536, d=128, quant_mode=0, num_blocks=2048, block_size=64,
                        cache_head_dim=128, scale_head_dim=4, cache_dtype="e4m3", skip_frac=0.05, seed=seed)
 
 
-def cfg3b_indexer_mxfp4(seed: int = 0) -> Case:
-    return gen_indexer("cfg3b_indexer_mxfp4", T=65536, d=128, quant_mode=3, num_blocks=2048, block_size=64,
+def indexer_mxfp4_T65536_d128(seed: int = 0) -> Case:
+    return gen_indexer("indexer_mxfp4_T65536_d128", T=65536, d=128, quant_mode=3, num_blocks=2048, block_size=64,
                        cache_head_dim=64, scale_head_dim=4, cache_dtype="u8", skip_frac=0.05, seed=seed)
 
 
-def cfg4_dequant_rope_quant(seed: int = 0, x_range: int = 1 << 20) -> Case:
-    return gen_dequant_rope_quant("cfg4_dequant_rope_quant", B=16, S=1024, Nq=16, Nkv=4, D=128, c0=512,
+def dequant_rope_quant_page_B16_S1024_H3072(seed: int = 0, x_range: int = 1 << 20) -> Case:
+    return gen_dequant_rope_quant("dequant_rope_quant_page_B16_S1024_H3072", B=16, S=1024, Nq=16, Nkv=4, D=128, c0=512,
                                   c1=128, x_range=x_range, cache_mode="page", seed=seed)
 
 
-def cfg5a_compress_mode0(seed: int = 0) -> Case:
-    return gen_compress("cfg5a_compress_mode0", T=262144, d=576, quant_mode=0, num_blocks=4096,
+def compress_mode0_T262144_d576(seed: int = 0) -> Case:
+    return gen_compress("compress_mode0_T262144_d576", T=262144, d=576, quant_mode=0, num_blocks=4096,
                         block_size=128, head_dim=672, skip_frac=0.02, outlier_frac=0.01, seed=seed)
 
 
-def cfg5b_compress_mode2(seed: int = 0) -> Case:
-    return gen_compress("cfg5b_compress_mode2", T=262144, d=576, quant_mode=2, group_size=32, x_scale=0.1,
+def compress_mode2_G32_T262144_d576(seed: int = 0) -> Case:
+    return gen_compress("compress_mode2_G32_T262144_d576", T=262144, d=576, quant_mode=2, group_size=32, x_scale=0.1,
                         num_blocks=4096, block_size=128, head_dim=352, skip_frac=0.02, outlier_frac=0.01,
                         seed=seed)
 
 
-def prefill_rmsnorm_rope(seed: int = 0) -> Case:
-    """The DeepSeek-V3 shape of cfg2 at prefill size: 65536 tokens (not one of
-    the five published workloads; it measures the kernel where bandwidth, not
-    latency, bounds it)."""
-    return gen_rmsnorm_rope("prefill_rmsnorm_rope", B=65536, S=1, D=576, Dv=512, num_blocks=1024, block_size=128,
-                            k_dtype="bf16", ckv_dtype="e4m3", ckv_scale=[1.0 / 64.0], epsilon=1e-6,
+def rmsnorm_rope_prefill_B65536_D576(seed: int = 0) -> Case:
+    """The DeepSeek-V3 decode shape (576 = 512 RMSNorm + 64 RoPE columns) at
+    prefill size, 65536 tokens, where bandwidth rather than launch latency
+    should bound the kernel."""
+    return gen_rmsnorm_rope("rmsnorm_rope_prefill_B65536_D576", B=65536, S=1, D=576, Dv=512, num_blocks=1024,
+                            block_size=128, k_dtype="bf16", ckv_dtype="e4m3", ckv_scale=[1.0 / 64.0], epsilon=1e-6,
                             cache_mode="PA_BNSD", skip_frac=0.05, seed=seed)
 
 
 # ---------------------------------------------------------------------------
 # the further modes of the four operations at the named workloads' sizes
 # ---------------------------------------------------------------------------
-def cfg3c_indexer_fp8(seed: int = 0) -> Case:
-    """cfg3a's rows in the fp8 mode: one binary32 scale per row."""
-    return gen_indexer("cfg3c_indexer_fp8", T=65536, d=128, quant_mode=1, num_blocks=2048, block_size=64,
+def indexer_fp8_T65536_d128(seed: int = 0) -> Case:
+    """The mxfp8 indexer rows (65536 x 128) in the fp8 mode: one binary32 scale per row."""
+    return gen_indexer("indexer_fp8_T65536_d128", T=65536, d=128, quant_mode=1, num_blocks=2048, block_size=64,
                        cache_head_dim=128, scale_head_dim=1, cache_dtype="e4m3", skip_frac=0.05, seed=seed)
 
 
-def cfg3d_indexer_mxfp8_e5m2(seed: int = 0) -> Case:
-    """cfg3a with an E5M2 code cache."""
-    return gen_indexer("cfg3d_indexer_mxfp8_e5m2", T=65536, d=128, quant_mode=0, num_blocks=2048, block_size=64,
+def indexer_mxfp8_e5m2_T65536_d128(seed: int = 0) -> Case:
+    """The mxfp8 indexer rows (65536 x 128) into an E5M2 code cache."""
+    return gen_indexer("indexer_mxfp8_e5m2_T65536_d128", T=65536, d=128, quant_mode=0, num_blocks=2048, block_size=64,
                        cache_head_dim=128, scale_head_dim=4, cache_dtype="e5m2", skip_frac=0.05, seed=seed)
 
 
-def prefill_rmsnorm_rope_int8(seed: int = 0) -> Case:
+def rmsnorm_rope_int8_prefill_B65536_D576(seed: int = 0) -> Case:
     """The prefill shape with both caches static int8: per-channel scales
     U(1/48, 1/24) and integer offsets in [-4, 4] for ckv, a per-tensor scale
     1/64 and offset 0 for k."""
     r = _rng(seed, 20)
-    return gen_rmsnorm_rope("prefill_rmsnorm_rope_int8", B=65536, S=1, D=576, Dv=512, num_blocks=1024,
+    return gen_rmsnorm_rope("rmsnorm_rope_int8_prefill_B65536_D576", B=65536, S=1, D=576, Dv=512, num_blocks=1024,
                             block_size=128, k_dtype="i8", ckv_dtype="i8", k_scale=[1.0 / 64.0], k_offset=[0.0],
                             ckv_scale=r.uniform(1.0 / 48.0, 1.0 / 24.0, size=512),
                             ckv_offset=r.integers(-4, 4, size=512, endpoint=True).astype(np.float32),
                             epsilon=1e-6, cache_mode="PA_BNSD", skip_frac=0.05, seed=seed)
 
 
-def cfg4b_dequant_contiguous_kv_output(seed: int = 0) -> Case:
-    """cfg4 in contiguous cache mode ([16, 2048, 4, 128] caches, each batch's
-    1024 tokens written from its start position) with kOut / vOut."""
-    return gen_dequant_rope_quant("cfg4b_dequant_contiguous_kv_output", B=16, S=1024, Nq=16, Nkv=4, D=128, c0=16,
-                                  c1=2048, cache_mode="contiguous", kv_output=True, seed=seed)
+def dequant_rope_quant_contiguous_kvout_B16_S1024_H3072(seed: int = 0) -> Case:
+    """The page-mode dequant workload (x int32 [16, 1024, 3072]) in contiguous
+    cache mode ([16, 2048, 4, 128] caches, each batch's 1024 tokens written
+    from its start position) with kOut / vOut."""
+    return gen_dequant_rope_quant("dequant_rope_quant_contiguous_kvout_B16_S1024_H3072", B=16, S=1024, Nq=16,
+                                  Nkv=4, D=128, c0=16, c1=2048, cache_mode="contiguous", kv_output=True, seed=seed)
 
 
-def cfg4c_dequant_bf16_x(seed: int = 0) -> Case:
-    """cfg4's shapes with bf16 x (no dequantisation) in page mode."""
-    return gen_dequant_rope_quant("cfg4c_dequant_bf16_x", B=16, S=1024, Nq=16, Nkv=4, D=128, c0=512, c1=128,
-                                  x_dtype="bf16", cos_dtype="bf16", cache_mode="page", seed=seed)
+def dequant_rope_quant_bf16_page_B16_S1024_H3072(seed: int = 0) -> Case:
+    """The page-mode dequant workload's shapes with bf16 x (no dequantisation)."""
+    return gen_dequant_rope_quant("dequant_rope_quant_bf16_page_B16_S1024_H3072", B=16, S=1024, Nq=16, Nkv=4,
+                                  D=128, c0=512, c1=128, x_dtype="bf16", cos_dtype="bf16", cache_mode="page",
+                                  seed=seed)
 
 
 CONFIGS = {
-    "cfg1_compress_mode1": cfg1_compress_mode1,
-    "cfg2_rmsnorm_rope": cfg2_rmsnorm_rope,
-    "prefill_rmsnorm_rope": prefill_rmsnorm_rope,
-    "cfg3a_indexer_mxfp8": cfg3a_indexer_mxfp8,
-    "cfg3b_indexer_mxfp4": cfg3b_indexer_mxfp4,
-    "cfg4_dequant_rope_quant": cfg4_dequant_rope_quant,
-    "cfg5a_compress_mode0": cfg5a_compress_mode0,
-    "cfg5b_compress_mode2": cfg5b_compress_mode2,
-    "cfg3c_indexer_fp8": cfg3c_indexer_fp8,
-    "cfg3d_indexer_mxfp8_e5m2": cfg3d_indexer_mxfp8_e5m2,
-    "prefill_rmsnorm_rope_int8": prefill_rmsnorm_rope_int8,
-    "cfg4b_dequant_contiguous_kv_output": cfg4b_dequant_contiguous_kv_output,
-    "cfg4c_dequant_bf16_x": cfg4c_dequant_bf16_x,
+    "compress_mode1_T64_d256": compress_mode1_T64_d256,
+    "rmsnorm_rope_decode_B64_D576": rmsnorm_rope_decode_B64_D576,
+    "rmsnorm_rope_prefill_B65536_D576": rmsnorm_rope_prefill_B65536_D576,
+    "indexer_mxfp8_T65536_d128": indexer_mxfp8_T65536_d128,
+    "indexer_mxfp4_T65536_d128": indexer_mxfp4_T65536_d128,
+    "dequant_rope_quant_page_B16_S1024_H3072": dequant_rope_quant_page_B16_S1024_H3072,
+    "compress_mode0_T262144_d576": compress_mode0_T262144_d576,
+    "compress_mode2_G32_T262144_d576": compress_mode2_G32_T262144_d576,
+    "indexer_fp8_T65536_d128": indexer_fp8_T65536_d128,
+    "indexer_mxfp8_e5m2_T65536_d128": indexer_mxfp8_e5m2_T65536_d128,
+    "rmsnorm_rope_int8_prefill_B65536_D576": rmsnorm_rope_int8_prefill_B65536_D576,
+    "dequant_rope_quant_contiguous_kvout_B16_S1024_H3072": dequant_rope_quant_contiguous_kvout_B16_S1024_H3072,
+    "dequant_rope_quant_bf16_page_B16_S1024_H3072": dequant_rope_quant_bf16_page_B16_S1024_H3072,
 }
 
 

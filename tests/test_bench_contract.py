@@ -19,14 +19,14 @@ import bench  # noqa: E402
 from kv_cache_quantize_b200 import workloads as W  # noqa: E402
 
 EXPECTED_BYTES = {
-    "cfg1_compress_mode1": 58 * (512 + 323) + 64 * 4,
+    "compress_mode1_T64_d256": 58 * (512 + 323) + 64 * 4,
     # 61 valid tokens x (1152 kv + 256 cos/sin + 512 ckv + 128 k) + 64 x 4 index + 1024 gamma + 4 scale
-    "cfg2_rmsnorm_rope": 61 * 2048 + 64 * 4 + 1024 + 4,
-    "cfg3a_indexer_mxfp8": 62260 * (256 + 128 + 4) + 65536 * 4,
-    "cfg3b_indexer_mxfp4": 62260 * (256 + 64 + 4) + 65536 * 4,
-    "cfg4_dequant_rope_quant": 16384 * 17928 + 32768,
-    "cfg5a_compress_mode0": 256902 * (1152 + 672) + 262144 * 4,
-    "cfg5b_compress_mode2": 256902 * (1152 + 352) + 262144 * 4,
+    "rmsnorm_rope_decode_B64_D576": 61 * 2048 + 64 * 4 + 1024 + 4,
+    "indexer_mxfp8_T65536_d128": 62260 * (256 + 128 + 4) + 65536 * 4,
+    "indexer_mxfp4_T65536_d128": 62260 * (256 + 64 + 4) + 65536 * 4,
+    "dequant_rope_quant_page_B16_S1024_H3072": 16384 * 17928 + 32768,
+    "compress_mode0_T262144_d576": 256902 * (1152 + 672) + 262144 * 4,
+    "compress_mode2_G32_T262144_d576": 256902 * (1152 + 352) + 262144 * 4,
 }
 
 

@@ -100,6 +100,7 @@ def test_decompress_bad_slots_fault_and_int64():
     assert np.all(y[3] == MARK) and np.all(y[10] == MARK)
 
 
-@pytest.mark.parametrize("name", ["cfg5a_compress_mode0", "cfg5b_compress_mode2", "cfg1_compress_mode1"])
+@pytest.mark.parametrize("name", ["compress_mode0_T262144_d576", "compress_mode2_G32_T262144_d576",
+                                  "compress_mode1_T64_d256"])
 def test_decompress_named_workloads_full_size(name):
     _same(W.CONFIGS[name]())

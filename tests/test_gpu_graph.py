@@ -25,10 +25,10 @@ def _cases():
     return [
         W.gen_compress("g_ce0", T=5003, d=576, quant_mode=0, num_blocks=640, block_size=16,
                        head_dim=oracle.kv_cache_col(576, 0, 64) + 3, skip_frac=0.1, seed=71),
-        W.cfg1_compress_mode1(),
+        W.compress_mode1_T64_d256(),
         W.gen_indexer("g_ix", T=3001, d=128, quant_mode=3, num_blocks=128, block_size=64, cache_head_dim=64,
                       scale_head_dim=4, cache_dtype="u8", skip_frac=0.05, seed=72),
-        W.cfg2_rmsnorm_rope(),
+        W.rmsnorm_rope_decode_B64_D576(),
         W.gen_dequant_rope_quant("g_dq", B=3, S=40, Nq=4, Nkv=2, D=128, c0=8, c1=64, x_range=1 << 12, seed=73,
                                  skip_frac=0.1),
     ]

@@ -134,13 +134,14 @@ def test_compress_all_skipped():
     assert np.array_equal(st_g["cache"], case.caches["cache"].storage)
 
 
-@pytest.mark.parametrize("name", ["cfg1_compress_mode1", "cfg5a_compress_mode0", "cfg5b_compress_mode2"])
+@pytest.mark.parametrize("name", ["compress_mode1_T64_d256", "compress_mode0_T262144_d576",
+                                  "compress_mode2_G32_T262144_d576"])
 def test_compress_named_workloads_full_size(name):
     _same(W.CONFIGS[name]())
 
 
 def test_compress_is_deterministic():
-    case = W.cfg5b_compress_mode2()
+    case = W.compress_mode2_G32_T262144_d576()
     a, _, _ = run_gpu(case)
     b, _, _ = run_gpu(case)
     assert np.array_equal(a["cache"], b["cache"])
@@ -170,8 +171,8 @@ def test_indexer_wide_values_and_padding(mode, cdt):
     _same(_ix(97, 128, mode, cdt, kind="wide", pad=24, extra=0, seed=3))
 
 
-@pytest.mark.parametrize("name", ["cfg3a_indexer_mxfp8", "cfg3b_indexer_mxfp4", "cfg3c_indexer_fp8",
-                                  "cfg3d_indexer_mxfp8_e5m2"])
+@pytest.mark.parametrize("name", ["indexer_mxfp8_T65536_d128", "indexer_mxfp4_T65536_d128", "indexer_fp8_T65536_d128",
+                                  "indexer_mxfp8_e5m2_T65536_d128"])
 def test_indexer_named_workloads_full_size(name):
     _same(W.CONFIGS[name]())
 
@@ -220,10 +221,10 @@ def test_rmsnorm_rope_other_widths_and_f16(D, Dv):
 
 
 def test_rmsnorm_rope_named_workload_full_size():
-    _same(W.cfg2_rmsnorm_rope())
+    _same(W.rmsnorm_rope_decode_B64_D576())
 
 
-@pytest.mark.parametrize("name", ["prefill_rmsnorm_rope", "prefill_rmsnorm_rope_int8"])
+@pytest.mark.parametrize("name", ["rmsnorm_rope_prefill_B65536_D576", "rmsnorm_rope_int8_prefill_B65536_D576"])
 def test_rmsnorm_rope_prefill_size(name):
     _same(W.CONFIGS[name]())
 
@@ -250,7 +251,8 @@ def test_rmsnorm_rope_subnormal_and_tie_quotients(ckv_dtype):
     rng = np.random.default_rng(43)
     for r in live[2::3]:
         cols = rng.choice(512, size=12, replace=False)
-        kv[r, cols[:6]] = rng.integers(1, 128, size=6).astype(np.uint16) | (rng.integers(0, 2, size=6) << 15).astype(np.uint16)
+        sign = (rng.integers(0, 2, size=6) << 15).astype(np.uint16)
+        kv[r, cols[:6]] = rng.integers(1, 128, size=6).astype(np.uint16) | sign
         kv[r, cols[6:9]] = 0
         kv[r, cols[9:]] = bits(2.0 ** 40)
     _same(case)
@@ -304,7 +306,7 @@ def test_drq_unaligned_bias_kinds_and_named_shape():
     for bias_dtype in ("bf16", "i32", None):
         _same(_dq(bias_dtype=bias_dtype, with_offsets=bias_dtype is not None,
                   with_activation_scale=bias_dtype is not None), misalign=True)
-    _same(W.cfg4_dequant_rope_quant(x_range=1 << 12), misalign=True)
+    _same(W.dequant_rope_quant_page_B16_S1024_H3072(x_range=1 << 12), misalign=True)
 
 
 @pytest.mark.parametrize("bias_dtype", ["f32", "bf16", "f16", "i32", None])
@@ -345,12 +347,13 @@ def test_drq_bad_index_fault():
     _same(case)
 
 
-@pytest.mark.parametrize("name", ["cfg4_dequant_rope_quant", "cfg4b_dequant_contiguous_kv_output",
-                                  "cfg4c_dequant_bf16_x"])
+@pytest.mark.parametrize("name", ["dequant_rope_quant_page_B16_S1024_H3072",
+                                  "dequant_rope_quant_contiguous_kvout_B16_S1024_H3072",
+                                  "dequant_rope_quant_bf16_page_B16_S1024_H3072"])
 def test_drq_named_workload_full_size(name):
     _same(W.CONFIGS[name]())
 
 
 def test_drq_named_workload_narrow_range():
     """Same shapes with |x| <= 2^12, where few int8 codes saturate."""
-    _same(W.cfg4_dequant_rope_quant(x_range=1 << 12))
+    _same(W.dequant_rope_quant_page_B16_S1024_H3072(x_range=1 << 12))
