@@ -11,10 +11,10 @@ reads 604 MB of input -- more than the 126 MB L2 -- and needs no L2 flush.
 
 value = token rows quantised per second over all ranks (2 x 262144 per step and
 GPU); the roofline object reports the dominant kernel's algorithmic HBM bytes
-per launch over its CUDA-event duration.  Every workload is also timed on its
-own under "per_config": back-to-back launches cycling through enough input
-copies that their bytes exceed twice the L2 size (one copy, L2-resident, for
-the latency-bound decode-sized workloads).
+per launch over its CUDA-event duration.  On one GPU every workload is also
+timed on its own under "per_config": back-to-back launches cycling through
+enough input copies that their bytes exceed twice the L2 size (one copy,
+L2-resident, for the latency-bound decode-sized workloads).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--scaling weak|strong]
@@ -504,9 +504,10 @@ def main():
            "note": "pinned host x + slot_mapping copied in, both passes through the C ABI, fault word read back"}
     del xa_host, xb_host, xa_dev, xb_dev, cache_a, cache_b
 
-    # ---------------- per-workload breakdown (rank 0) ----------------
+    # ---------------- per-workload breakdown (single GPU only: with several
+    # ranks the others would wait for rank 0 at the final barrier) ----------------
     per_config = None
-    if rank == 0 and not args.no_per_config:
+    if rank == 0 and world == 1 and not args.no_per_config:
         per_config = {}
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         for name, make in W.CONFIGS.items():
