@@ -269,3 +269,11 @@ def test_row_widths_beyond_32_bit_indexing_are_rejected(L):
     f = lambda x, c, sc, s: L.kvq_indexer_quant_cache(R(x), R(c), R(sc), R(s), 0, None)
     assert f(D([4, wide], "bf16"), D([1, 16, 1, wide], "e4m3"), D([1, 16, 1, wide // 32], "e8m0"),
              D([4], "i32")) == ESHAPE
+
+
+def test_selftest_numbering(L):
+    """Self-tests 0..8 exist; other numbers and a NULL result are rejected before any device work."""
+    out = ctypes.c_uint64(0)
+    assert L.kvq_selftest(9, ctypes.byref(out), None) == EATTR
+    assert L.kvq_selftest(-1, ctypes.byref(out), None) == EATTR
+    assert L.kvq_selftest(0, None, None) == ENULL
