@@ -119,11 +119,18 @@ def hbm_peak():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the CUDA sources with comments and blank lines removed: it
+    changes with the code the counters depend on, not with its comments."""
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "kv_cache_quantize_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+        h.update(name.encode() + code.encode())
     return h.hexdigest()[:16]
 
 

@@ -5,10 +5,11 @@
 // the (d-64)/64 nope segments and the rope segment last.  A segment is handled
 // by a TEAM of 8 lanes, each lane one 16-byte chunk of 8 values, so a warp
 // works on 4 segments at a time and a 64-value quantisation group is one team
-// (FP4 groups of 32 / 16 are 4 / 2 lanes of it).  A warp owns a tile of 8
-// consecutive rows: lanes 0..7 load the tile's 8 slots once (coalesced), the
-// teams walk the tile's segments, and CE_UNROLL segments per team are loaded
-// before any is processed so each lane keeps several 16-byte loads in flight.
+// (FP4 groups of 32 / 16 are 4 / 2 lanes of it).  A warp owns a tile of up to
+// 8 consecutive rows (ce_rows, picked by the host): its first lanes load the
+// tile's slots once (coalesced), the teams walk the tile's segments, and
+// CE_UNROLL segments per team are loaded before any is processed so each lane
+// keeps several 16-byte loads in flight.
 // Group maxima are butterfly shuffles inside the team.  Every output byte of a
 // row has exactly one writer: codes by their chunk's lane, a group's scale by
 // the group's first lane, the rope and the zero padding by the rope team.
