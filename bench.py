@@ -351,15 +351,51 @@ def device_us_per_launch(calls, stream, reps: int) -> float:
     return 1e3 * e0.elapsed_time(e1) / reps
 
 
+# the packed-row decoder, timed on the caches of the two headline passes
+DECODER_WORKLOADS = {"decompress_mode0_T262144_d576": "compress_mode0_T262144_d576",
+                     "decompress_mode2_G32_T262144_d576": "compress_mode2_G32_T262144_d576"}
+
+
+def decoder_call(case, stream):
+    """Encode the case's rows into its cache once, then return (call, algorithmic
+    bytes) for decoding them back into a bf16 [T, d] buffer."""
+    import numpy as np
+    import torch
+    import kv_cache_quantize_b200 as kvq
+    from kv_cache_quantize_b200 import workloads as W
+    call, st, _ = W.build_call(case)
+    call(stream)
+    cb, at = case.caches["cache"], case.attrs
+    view = st["cache"][cb.offset:].as_strided((cb.num_blocks, cb.block_size, 1, cb.head_dim),
+                                              (cb.block_stride, cb.head_dim, cb.head_dim, 1))
+    slots = torch.from_numpy(np.ascontiguousarray(case.arrays["slot_mapping"])).to(st["cache"].device)
+    T, d = case.arrays["x"].shape
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=st["cache"].device)
+
+    def dcall(strm):
+        kvq.kv_decompress(view, slots, y, at["quant_mode"], at["quant_group_size"], at["x_scale"], stream=strm)
+    valid = int((case.arrays["slot_mapping"] != -1).sum())
+    col = kvq.kv_cache_col(d, at["quant_mode"], at["quant_group_size"])
+    return dcall, valid * (col + 2 * d) + T * case.arrays["slot_mapping"].itemsize
+
+
 def run_profile_workload(args):
     """Run one named workload a few times (for ncu captures of a single kernel)."""
     import torch
     import kv_cache_quantize_b200 as kvq
     from kv_cache_quantize_b200 import workloads as W
+    stream = torch.cuda.current_stream()
+    if args.profile_workload in DECODER_WORKLOADS:
+        dcall, nb = decoder_call(W.CONFIGS[DECODER_WORKLOADS[args.profile_workload]](), stream)
+        us = device_us_per_launch([dcall], stream, args.profile_reps)
+        if kvq.get_error(stream) != 0:
+            raise RuntimeError("device fault bits set")
+        print(f"{args.profile_workload}: {args.profile_reps} launches over 1 input copies, "
+              f"{us:.1f} us per launch, {nb / us / 1e3:.0f} GB/s algorithmic")
+        return 0
     make = W.CONFIGS[args.profile_workload]
     case = make()
     calls = rotation(case, make, torch.cuda.get_device_properties(0).L2_cache_size)
-    stream = torch.cuda.current_stream()
     us = device_us_per_launch(calls, stream, args.profile_reps)
     if kvq.get_error(stream) != 0:
         raise RuntimeError("device fault bits set")
@@ -380,8 +416,10 @@ def main():
     ap.add_argument("--no-per-config", action="store_true", help="skip the per-workload breakdown")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing for cpu_baseline")
     ap.add_argument("--profile-workload", default=None,
-                    help="profiling mode: run only this named workload --profile-reps times (back to back, "
-                         "cycling input copies larger than L2) and print its time per launch; no JSON line")
+                    help="profiling mode: run only this named workload (a workloads.CONFIGS name, or "
+                         "decompress_mode0_T262144_d576 / decompress_mode2_G32_T262144_d576 for the decoder) "
+                         "--profile-reps times (back to back, cycling input copies larger than L2) and print its "
+                         "time per launch; no JSON line")
     ap.add_argument("--profile-reps", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -532,26 +570,13 @@ def main():
             torch.cuda.empty_cache()
         # the packed-row decoder on the headline caches (written by the timed encoder)
         for name, case in (("decompress_mode0_T262144_d576", case_a), ("decompress_mode2_G32_T262144_d576", case_b)):
-            call, st, _ = W.build_call(case)
-            call(stream)
-            cb, at = case.caches["cache"], case.attrs
-            view = st["cache"][cb.offset:].as_strided((cb.num_blocks, cb.block_size, 1, cb.head_dim),
-                                                      (cb.block_stride, cb.head_dim, cb.head_dim, 1))
-            slots = torch.from_numpy(np.ascontiguousarray(case.arrays["slot_mapping"])).to(dev)
-            T, d = case.arrays["x"].shape
-            y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
-
-            def dcall(strm, view=view, slots=slots, y=y, at=at):
-                kvq.kv_decompress(view, slots, y, at["quant_mode"], at["quant_group_size"], at["x_scale"],
-                                  stream=strm)
+            dcall, nb = decoder_call(case, stream)
             us = device_us_per_launch([dcall], stream, 200)
-            valid = int((case.arrays["slot_mapping"] != -1).sum())
-            col = kvq.kv_cache_col(d, at["quant_mode"], at["quant_group_size"])
-            nb = valid * (col + 2 * d) + T * case.arrays["slot_mapping"].itemsize
+            T = case.arrays["x"].shape[0]
             per_config[name] = {"tokens": T, "alg_bytes": nb, "us_per_launch": us, "tokens_per_s": T / us * 1e6,
                                 "alg_GBps": nb / us / 1e3, "frac_of_peak": nb / us / 1e3 / peak,
                                 "input_copies": 1, "l2": f"{nb >> 20} MB > L2"}
-            del call, st, view, slots, y
+            del dcall
             torch.cuda.empty_cache()
 
     # ---------------- CPU oracle baseline (rank 0, N = 1) ----------------
