@@ -114,6 +114,22 @@ def _ref(d: Optional[KvqTensor]):
     return None if d is None else ctypes.byref(d)
 
 
+def _one_device(op: str, *tensors) -> None:
+    """Every non-empty tensor of a call must live on one CUDA device: the kernels
+    dereference the pointers on the device, and a host pointer or another
+    device's memory would fault there instead of failing here."""
+    dev = None
+    for t in tensors:
+        if t is None or t.numel() == 0:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{op}: tensors must be on a CUDA device, got one on {t.device}")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{op}: tensors on {dev} and {t.device}; all must be on one device")
+
+
 def _stream(stream, *tensors) -> int:
     if stream is None:
         dev = next((t.device for t in tensors if t is not None and t.is_cuda), None)
@@ -134,6 +150,7 @@ def _check(op: str, status: int) -> None:
 def kv_compress_epilog(x: torch.Tensor, slot_mapping: torch.Tensor, cache: torch.Tensor, quant_mode: int,
                        quant_group_size: int = 64, x_scale: float = 1.0, stream=None) -> None:
     """In-place group quantisation of x's rows into the paged cache (see kvq_kv_compress_epilog)."""
+    _one_device("kv_compress_epilog", x, slot_mapping, cache)
     _check("kv_compress_epilog", lib().kvq_kv_compress_epilog(
         _ref(desc(x)), _ref(desc(slot_mapping)), _ref(desc(cache)), int(quant_mode), int(quant_group_size),
         float(x_scale), _stream(stream, x)))
@@ -143,6 +160,7 @@ def kv_decompress(cache: torch.Tensor, slot_mapping: torch.Tensor, y: torch.Tens
                   quant_group_size: int = 64, x_scale: float = 1.0, stream=None) -> torch.Tensor:
     """Decode the packed rows named by slot_mapping into the bf16 rows of y (see kvq_kv_decompress);
     rows whose slot is -1 keep their contents.  Returns y."""
+    _one_device("kv_decompress", cache, slot_mapping, y)
     _check("kv_decompress", lib().kvq_kv_decompress(
         _ref(desc(cache)), _ref(desc(slot_mapping)), _ref(desc(y)), int(quant_mode), int(quant_group_size),
         float(x_scale), _stream(stream, y)))
@@ -152,6 +170,7 @@ def kv_decompress(cache: torch.Tensor, slot_mapping: torch.Tensor, y: torch.Tens
 def indexer_quant_cache(x: torch.Tensor, cache: torch.Tensor, cache_scale: torch.Tensor,
                         slot_mapping: torch.Tensor, quant_mode="mxfp8", stream=None) -> None:
     """In-place mxfp8 / fp8 / mxfp4 quantisation into cache and cache_scale (see kvq_indexer_quant_cache)."""
+    _one_device("indexer_quant_cache", x, cache, cache_scale, slot_mapping)
     mode = INDEXER_MODES[quant_mode] if isinstance(quant_mode, str) else int(quant_mode)
     _check("indexer_quant_cache", lib().kvq_indexer_quant_cache(
         _ref(desc(x)), _ref(desc(cache)), _ref(desc(cache_scale)), _ref(desc(slot_mapping)), mode,
@@ -164,6 +183,8 @@ def kv_rmsnorm_rope_cache(kv: torch.Tensor, gamma: torch.Tensor, cos: torch.Tens
                           k_offset: Optional[torch.Tensor] = None, ckv_offset: Optional[torch.Tensor] = None,
                           epsilon: float = 1e-5, cache_mode="PA_BNSD", stream=None) -> None:
     """RMSNorm of kv[..., :Dv] -> ckv_cache and interleaved RoPE of kv[..., Dv:] -> k_cache, in place."""
+    _one_device("kv_rmsnorm_rope_cache", kv, gamma, cos, sin, index, k_cache, ckv_cache, k_scale, ckv_scale,
+                k_offset, ckv_offset)
     mode = RMS_CACHE_MODES[cache_mode] if isinstance(cache_mode, str) else int(cache_mode)
     _check("kv_rmsnorm_rope_cache", lib().kvq_kv_rmsnorm_rope_cache(
         _ref(desc(kv)), _ref(desc(gamma)), _ref(desc(cos)), _ref(desc(sin)), _ref(desc(index)),
@@ -202,6 +223,8 @@ def dequant_rope_quant_kvcache(x: torch.Tensor, cos: torch.Tensor, sin: torch.Te
     if v_out is None:
         v_out = torch.empty(lead + (Nkv, D) if kv_output else (0,) + lead[1:] + (Nkv, D), dtype=odt,
                             device=x.device)
+    _one_device("dequant_rope_quant_kvcache", x, cos, sin, k_cache, v_cache, indices, scale_k, scale_v, offset_k,
+                offset_v, weight_scale, activation_scale, bias, q_out, k_out, v_out)
     arr = (ctypes.c_int64 * max(1, len(splits)))(*splits)
     qm = {"static": 0}.get(quant_mode, -1) if isinstance(quant_mode, str) else int(quant_mode)
     lo = {"BSND": 0}.get(layout, -1) if isinstance(layout, str) else int(layout)

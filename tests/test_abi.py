@@ -250,9 +250,9 @@ def test_missing_library_fails_loudly(tmp_path):
     import sys
     code = ("import kv_cache_quantize_b200 as kvq, torch\n"
             f"kvq.library_path = {str(tmp_path / 'absent.so')!r}\n"
-            "x = torch.zeros((4, 128), dtype=torch.bfloat16)\n"
-            "s = torch.zeros(4, dtype=torch.int32)\n"
-            "c = torch.zeros((1, 16, 1, 224), dtype=torch.uint8)\n"
+            "x = torch.zeros((0, 128), dtype=torch.bfloat16)\n"
+            "s = torch.zeros(0, dtype=torch.int32)\n"
+            "c = torch.zeros((0, 16, 1, 224), dtype=torch.uint8)\n"
             "try:\n"
             "    kvq.kv_compress_epilog(x, s, c, 0)\n"
             "except RuntimeError as e:\n"
@@ -277,3 +277,17 @@ def test_selftest_numbering(L):
     assert L.kvq_selftest(9, ctypes.byref(out), None) == EATTR
     assert L.kvq_selftest(-1, ctypes.byref(out), None) == EATTR
     assert L.kvq_selftest(0, None, None) == ENULL
+
+
+def test_host_tensors_are_rejected_before_any_launch():
+    """A host tensor (or tensors on two devices) would make a kernel dereference a
+    pointer it cannot use: the binding refuses the call instead."""
+    x = torch.zeros((4, 128), dtype=torch.bfloat16)
+    s = torch.zeros(4, dtype=torch.int32)
+    c = torch.zeros((1, 16, 1, 224), dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA device"):
+        kvq.kv_compress_epilog(x, s, c, 0)
+    with pytest.raises(ValueError, match="CUDA device"):
+        kvq.indexer_quant_cache(x, c, c, s, "mxfp8")
+    with pytest.raises(ValueError, match="CUDA device"):
+        kvq.kv_decompress(c, s, x, 0)
