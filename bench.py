@@ -197,21 +197,38 @@ def sum_over_ranks(n: int, dist, device) -> int:
 # clocks during the timed region (NVML: the same counters nvidia-smi reads)
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock and throttle reasons of THIS process's GPU, sampled in a thread.
+
+    NVML numbers GPUs by physical index and ignores CUDA_VISIBLE_DEVICES, so the
+    handle is opened by the CUDA device's UUID (or, failing that, its PCI bus
+    id), never by the CUDA ordinal; the UUID is recorded with the samples."""
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.period = period_s
         self.samples = []
         self.reasons = set()
         self.max_mhz = None
+        self.uuid = None
         self._stop = threading.Event()
         self._thr = None
         try:
             import pynvml
+            import torch
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            props = torch.cuda.get_device_properties(device_index)
+            uuid = str(props.uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+                self.uuid = uuid
+            except Exception:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+                u = pynvml.nvmlDeviceGetUUID(self.h)
+                self.uuid = u.decode() if isinstance(u, bytes) else str(u)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
         except Exception:
             self.nv = None
@@ -240,10 +257,9 @@ class ClockSampler:
             self._thr.join()
 
     def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "period_ms": 1e3 * self.period, "gpu_uuid": self.uuid}
 
 
 # ---------------------------------------------------------------------------
@@ -552,8 +568,10 @@ def main():
     # ---------------- per-workload breakdown (single GPU only: with several
     # ranks the others would wait for rank 0 at the final barrier) ----------------
     per_config = None
+    per_config_clocks = None
     if rank == 0 and world == 1 and not args.no_per_config:
         per_config = {}
+        pc_sampler = ClockSampler(local, 0.005).__enter__()
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         for name, make in W.CONFIGS.items():
             case = {"compress_mode0_T262144_d576": case_a,
@@ -578,6 +596,30 @@ def main():
                                 "input_copies": 1, "l2": f"{nb >> 20} MB > L2"}
             del dcall
             torch.cuda.empty_cache()
+        # the same access pattern without arithmetic (kvq_scatter_rows): the DRAM
+        # ceiling the two compress passes are compared with
+        from kv_cache_quantize_b200.workloads import dev_cache
+        for name, case in (("scatter_rows_as_mode0_T262144_d576", case_a),
+                           ("scatter_rows_as_mode2_G32_T262144_d576", case_b)):
+            at = case.attrs
+            xt = torch.from_numpy(case.arrays["x"].view(np.int16)).view(torch.bfloat16).to(dev)
+            sl = torch.from_numpy(case.arrays["slot_mapping"]).to(dev)
+            _, view = dev_cache(case.caches["cache"], torch.uint8)
+            col = kvq.kv_cache_col(xt.shape[1], at["quant_mode"], at["quant_group_size"])
+
+            def scall(strm, xt=xt, sl=sl, view=view, col=col):
+                kvq.scatter_rows(xt, sl, view, col, stream=strm)
+            us = device_us_per_launch([scall], stream, 200)
+            nb = algorithmic_bytes(case)
+            T = case.arrays["x"].shape[0]
+            per_config[name] = {"tokens": T, "alg_bytes": nb, "us_per_launch": us, "tokens_per_s": T / us * 1e6,
+                                "alg_GBps": nb / us / 1e3, "frac_of_peak": nb / us / 1e3 / peak,
+                                "input_copies": 1, "l2": f"{nb >> 20} MB > L2",
+                                "note": "compress access pattern, no arithmetic"}
+            del xt, sl, view, scall
+            torch.cuda.empty_cache()
+        pc_sampler.__exit__(None, None, None)
+        per_config_clocks = pc_sampler.summary()
 
     # ---------------- CPU oracle baseline (rank 0, N = 1) ----------------
     cpu = None
@@ -601,7 +643,7 @@ def main():
                                            f"rows split over {world} ranks (own caches, no collective)")},
                 "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": 2 * args.steps, "clocks": clocks.summary(), "fault_bits": faults,
-                "per_config": per_config}
+                "per_config": per_config, "per_config_clocks": per_config_clocks}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

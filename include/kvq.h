@@ -16,12 +16,15 @@
  *
  * Errors.  A host-detected problem (null pointer, wrong rank, shape, dtype,
  * attribute, layout or capacity) returns a nonzero kvq_status and launches
- * nothing.  After a launch the call returns KVQ_ERR_CUDA if the launch itself
- * failed (cudaGetLastError), else KVQ_OK.  Data faults the device can see --
- * a slot index outside [0, num_slots) that is not -1 -- skip the affected row
- * and set a bit in a per-device fault word that kvq_get_error() returns and
- * clears.  Duplicate slots are not detected (the pages declare the result
- * undefined); rows then have two writers and either may win.
+ * nothing.  After a launch the call returns KVQ_ERR_CUDA if that launch itself
+ * failed (the status of the launch call; errors left by unrelated earlier CUDA
+ * work are neither reported nor cleared), else KVQ_OK.  Data faults the
+ * device can see -- a slot index outside [0, num_slots) that is not -1 --
+ * skip the affected row and set a bit in a per-device fault word; a call's
+ * KVQ_OK does not say that no such fault happened: callers that need to know
+ * call kvq_get_error(), which returns and clears the bits.  Duplicate slots
+ * are not detected (the pages declare the result undefined); rows then have
+ * two writers and either may win.
  *
  * Sources (page title and section):
  *   aclnnKvCompressEpilog        -- 接口功能, 计算公式, 约束说明
@@ -259,9 +262,14 @@ KVQ_API kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq
 /* Utilities                                                                 */
 /* ------------------------------------------------------------------------ */
 
-/* Enqueue a read of this device's fault word, wait for `stream`, store the
- * bits in *fault_bits and clear the word.  Returns KVQ_ERR_CUDA if the stream
- * reported an error (the bits are then 0). */
+/* Read and clear the current device's fault word: enqueues on `stream` one
+ * kernel that atomically exchanges the word with 0 (after every earlier
+ * kernel of the stream has completed), copies that value back, waits for
+ * `stream` and stores the bits in *fault_bits.  Because the read and the
+ * clear are one atomic operation, a bit raised by a kernel on another stream
+ * is returned either by this call or by the next one, never lost.  Returns
+ * KVQ_ERR_CUDA if the launch, the copy or the stream reported an error (the
+ * bits are then 0). */
 KVQ_API kvq_status kvq_get_error(kvq_stream stream, uint32_t* fault_bits);
 
 /* Element-wise conversion of n binary32 values on the device with the same
@@ -295,6 +303,19 @@ KVQ_API kvq_status kvq_convert(int32_t fmt, const float* in, int64_t n, void* ou
  * quotient.  Blocks until done; *result receives the count (0 means the
  * shortcut is exact on the domain). */
 KVQ_API kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream);
+
+/* The memory access pattern of kv_compress_epilog without its arithmetic (no
+ * counterpart on the pages; a measuring stick for the compress kernels): for
+ * each token t with slot s = slot_mapping[t] != -1, read the whole row t of x
+ * (any dtype, [..., d] with the last dimension contiguous, d * element size a
+ * multiple of 16 and at most 2048 bytes, rows 16-byte aligned) and write its
+ * first out_bytes bytes (a multiple of 16, at most the row size) to the start
+ * of slot row s of cache (uint8 [blockNum, blockSize, 1, headDim], headDim >=
+ * out_bytes, rows 16-byte aligned; otherwise KVQ_ERR_LAYOUT).  Slots outside
+ * the cache skip the row and set KVQ_FAULT_SLOT_RANGE.  One kernel on `stream`;
+ * nothing is allocated. */
+KVQ_API kvq_status kvq_scatter_rows(const kvq_tensor* x, const kvq_tensor* slot_mapping, kvq_tensor* cache,
+                                    int64_t out_bytes, kvq_stream stream);
 
 /* Static description of a status code. */
 KVQ_API const char* kvq_status_string(kvq_status status);

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <utility>
 
@@ -17,6 +18,7 @@
 #include "indexer_quant.cuh"
 #include "kv_decompress.cuh"
 #include "rmsnorm_rope.cuh"
+#include "scatter_copy.cuh"
 
 namespace {
 
@@ -199,8 +201,10 @@ int64_t persistent_grid(K kernel, int threads, int64_t needed_blocks, size_t sme
 // Launch with programmatic stream serialization (see pdl_wait in
 // kvq_device.cuh): the kernel may be scheduled before the previous kernel of
 // the stream completes and waits for it on the device.
+// Returns the launch's own status (not cudaGetLastError, which would also
+// report -- and clear -- errors left by unrelated earlier CUDA work).
 template <typename... P, typename... A>
-void launch(void (*kernel)(P...), unsigned grid, unsigned block, size_t smem, cudaStream_t s, A&&... args) {
+cudaError_t launch(void (*kernel)(P...), unsigned grid, unsigned block, size_t smem, cudaStream_t s, A&&... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(block);
@@ -211,12 +215,19 @@ void launch(void (*kernel)(P...), unsigned grid, unsigned block, size_t smem, cu
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
 }
 
-kvq_status launched() {
-    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
-}
+kvq_status launched(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+// ---------------------------------------------------------------------------
+// fault word read-and-clear (kvq_get_error): one atomic exchange on the device
+// into a snapshot slot that the host then copies back
+// ---------------------------------------------------------------------------
+constexpr uint32_t FAULT_SNAPSHOTS = 64;
+__device__ unsigned int g_fault_snapshot[FAULT_SNAPSHOTS];
+
+__global__ void fault_exchange_kernel(uint32_t slot) { g_fault_snapshot[slot] = atomicExch(&g_fault_word, 0u); }
 
 // ---------------------------------------------------------------------------
 // conversion kernel (kvq_convert)
@@ -416,24 +427,24 @@ __global__ void selftest_fmax_kernel() {
 // The pipelined dequant kernel instantiated for the ring shape (a.stages,
 // a.tps) that the host picked, and for D = 128 or any other head size.
 template <int XK, bool F16, int S, int TPS>
-void launch_drq_tma(const DrqArgs& a, int64_t tiles, size_t smem, cudaStream_t s) {
+cudaError_t launch_drq_tma(const DrqArgs& a, int64_t tiles, size_t smem, cudaStream_t s) {
     auto k = a.D == 128 ? dequant_rope_quant_tma_kernel<XK, F16, S, TPS, 128>
                         : dequant_rope_quant_tma_kernel<XK, F16, S, TPS, 0>;
-    launch(k, (unsigned)persistent_grid(k, DT_THREADS, tiles, smem), DT_THREADS, smem, s, a);
+    return launch(k, (unsigned)persistent_grid(k, DT_THREADS, tiles, smem), DT_THREADS, smem, s, a);
 }
 
 template <int XK, bool F16, int S>
-void launch_drq_tps(const DrqArgs& a, int64_t tiles, size_t smem, cudaStream_t s) {
-    if (a.tps == 2) launch_drq_tma<XK, F16, S, 2>(a, tiles, smem, s);
-    else if (a.tps == 4) launch_drq_tma<XK, F16, S, 4>(a, tiles, smem, s);
-    else launch_drq_tma<XK, F16, S, 8>(a, tiles, smem, s);
+cudaError_t launch_drq_tps(const DrqArgs& a, int64_t tiles, size_t smem, cudaStream_t s) {
+    if (a.tps == 2) return launch_drq_tma<XK, F16, S, 2>(a, tiles, smem, s);
+    if (a.tps == 4) return launch_drq_tma<XK, F16, S, 4>(a, tiles, smem, s);
+    return launch_drq_tma<XK, F16, S, 8>(a, tiles, smem, s);
 }
 
 template <int XK, bool F16>
-void launch_drq_ring(const DrqArgs& a, int64_t tiles, size_t smem, cudaStream_t s) {
-    if (a.stages == 2) launch_drq_tps<XK, F16, 2>(a, tiles, smem, s);
-    else if (a.stages == 3) launch_drq_tps<XK, F16, 3>(a, tiles, smem, s);
-    else launch_drq_tps<XK, F16, 4>(a, tiles, smem, s);
+cudaError_t launch_drq_ring(const DrqArgs& a, int64_t tiles, size_t smem, cudaStream_t s) {
+    if (a.stages == 2) return launch_drq_tps<XK, F16, 2>(a, tiles, smem, s);
+    if (a.stages == 3) return launch_drq_tps<XK, F16, 3>(a, tiles, smem, s);
+    return launch_drq_tps<XK, F16, 4>(a, tiles, smem, s);
 }
 
 }  // namespace
@@ -576,10 +587,11 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
         const size_t smem = ct_smem(ct_stages);
         const int64_t tiles = (T + CT_ROWS - 1) / CT_ROWS;
         const int threads = (a.ncw + 1) * 32;
+        cudaError_t err = cudaSuccess;
 #define KVQ_LAUNCH_CT(M, GG)                                                                   \
     do {                                                                                       \
         auto k = ct_stages == 2 ? compress_tma_kernel<M, GG, 2> : compress_tma_kernel<M, GG, 3>; \
-        launch(k, (unsigned)persistent_grid(k, threads, tiles, smem), threads, smem, s, a);     \
+        err = launch(k, (unsigned)persistent_grid(k, threads, tiles, smem), threads, smem, s, a); \
     } while (0)
         if (quant_mode == 0) KVQ_LAUNCH_CT(0, 64);
         else if (quant_mode == 1) KVQ_LAUNCH_CT(1, 64);
@@ -587,7 +599,7 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
         else if (G == 32) KVQ_LAUNCH_CT(2, 32);
         else KVQ_LAUNCH_CT(2, 64);
 #undef KVQ_LAUNCH_CT
-        return launched();
+        return launched(err);
     }
     {
         const int64_t r = (4 * CE_UNROLL) / a.nseg;       // rows whose segments fill one round
@@ -595,10 +607,11 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
     }
     const int64_t tiles = (T + a.ce_rows - 1) / a.ce_rows;
     const int64_t need = (tiles + (CE_THREADS / 32) - 1) / (CE_THREADS / 32);
+    cudaError_t err = cudaSuccess;
 #define KVQ_LAUNCH_CE(M, GG)                                                                   \
     do {                                                                                       \
         auto k = compress_epilog_kernel<M, GG>;                                                \
-        launch(k, (unsigned)persistent_grid(k, CE_THREADS, need), CE_THREADS, 0, s, a);          \
+        err = launch(k, (unsigned)persistent_grid(k, CE_THREADS, need), CE_THREADS, 0, s, a);    \
     } while (0)
     if (quant_mode == 0) KVQ_LAUNCH_CE(0, 64);
     else if (quant_mode == 1) KVQ_LAUNCH_CE(1, 64);
@@ -606,7 +619,7 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
     else if (G == 32) KVQ_LAUNCH_CE(2, 32);
     else KVQ_LAUNCH_CE(2, 64);
 #undef KVQ_LAUNCH_CE
-    return launched();
+    return launched(err);
 }
 
 // ---------------------------------------------------------------------------
@@ -654,10 +667,11 @@ kvq_status kvq_kv_decompress(const kvq_tensor* cache, const kvq_tensor* slot_map
     const int64_t nchunks = (T * a.nslice + 31) / 32;
     const int64_t need = (nchunks + (DC_THREADS / 32) - 1) / (DC_THREADS / 32);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err = cudaSuccess;
 #define KVQ_LAUNCH_DC(M, GG)                                                                   \
     do {                                                                                       \
         auto k = a.nslice == 18 ? kv_decompress_kernel<M, GG, 18> : kv_decompress_kernel<M, GG, 0>; \
-        launch(k, (unsigned)persistent_grid(k, DC_THREADS, need), DC_THREADS, 0, s, a);          \
+        err = launch(k, (unsigned)persistent_grid(k, DC_THREADS, need), DC_THREADS, 0, s, a);    \
     } while (0)
     if (quant_mode == 0) KVQ_LAUNCH_DC(0, 64);
     else if (quant_mode == 1) KVQ_LAUNCH_DC(1, 64);
@@ -665,7 +679,7 @@ kvq_status kvq_kv_decompress(const kvq_tensor* cache, const kvq_tensor* slot_map
     else if (G == 32) KVQ_LAUNCH_DC(2, 32);
     else KVQ_LAUNCH_DC(2, 64);
 #undef KVQ_LAUNCH_DC
-    return launched();
+    return launched(err);
 }
 
 kvq_status kvq_indexer_quant_cache(const kvq_tensor* x, kvq_tensor* cache, kvq_tensor* cache_scale,
@@ -729,10 +743,11 @@ kvq_status kvq_indexer_quant_cache(const kvq_tensor* x, kvq_tensor* cache, kvq_t
     const int64_t passes = (T + (32 >> a.team_shift) - 1) / (32 >> a.team_shift);
     const int64_t need = (passes + (IX_THREADS / 32) - 1) / (IX_THREADS / 32);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t err = cudaSuccess;
 #define KVQ_LAUNCH_IX(M, F, E)                                                                 \
     do {                                                                                       \
         auto k = indexer_quant_kernel<M, F, E>;                                                \
-        launch(k, (unsigned)persistent_grid(k, IX_THREADS, need), IX_THREADS, 0, s, a);          \
+        err = launch(k, (unsigned)persistent_grid(k, IX_THREADS, need), IX_THREADS, 0, s, a);    \
     } while (0)
 #define KVQ_LAUNCH_IX_FE(M)                                                                    \
     do {                                                                                       \
@@ -750,7 +765,7 @@ kvq_status kvq_indexer_quant_cache(const kvq_tensor* x, kvq_tensor* cache, kvq_t
     else KVQ_LAUNCH_IX(3, false, false);
 #undef KVQ_LAUNCH_IX_FE
 #undef KVQ_LAUNCH_IX
-    return launched();
+    return launched(err);
 }
 
 // ---------------------------------------------------------------------------
@@ -870,15 +885,13 @@ kvq_status kvq_kv_rmsnorm_rope_cache(const kvq_tensor* kv, const kvq_tensor* gam
     // the register-chunk kernels stage an int8 ckv cache's parameters in shared memory
     a.ckv_stage = vec && nch <= 128 && cc.dt == CDT_I8;
     const size_t smem = a.ckv_stage ? (size_t)3 * Dv * sizeof(float) : 0;
-    if (vec && nch <= 32) launch(rmsnorm_rope_kernel<1>, (unsigned)persistent_grid(rmsnorm_rope_kernel<1>, RR_THREADS, need, smem),
-                                 RR_THREADS, smem, s, a);
-    else if (vec && nch <= 64) launch(rmsnorm_rope_kernel<2>, (unsigned)persistent_grid(rmsnorm_rope_kernel<2>, RR_THREADS, need, smem),
-                                      RR_THREADS, smem, s, a);
-    else if (vec && nch <= 128) launch(rmsnorm_rope_kernel<4>, (unsigned)persistent_grid(rmsnorm_rope_kernel<4>, RR_THREADS, need, smem),
-                                       RR_THREADS, smem, s, a);
-    else launch(rmsnorm_rope_kernel<0>, (unsigned)persistent_grid(rmsnorm_rope_kernel<0>, RR_THREADS, need),
-                RR_THREADS, 0, s, a);
-    return launched();
+    auto run = [&](auto kernel, size_t sm) {
+        return launched(launch(kernel, (unsigned)persistent_grid(kernel, RR_THREADS, need, sm), RR_THREADS, sm, s, a));
+    };
+    if (vec && nch <= 32) return run(rmsnorm_rope_kernel<1>, smem);
+    if (vec && nch <= 64) return run(rmsnorm_rope_kernel<2>, smem);
+    if (vec && nch <= 128) return run(rmsnorm_rope_kernel<4>, smem);
+    return run(rmsnorm_rope_kernel<0>, (size_t)0);
 }
 
 // ---------------------------------------------------------------------------
@@ -1044,20 +1057,15 @@ kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq_tensor*
         const size_t smem = dt_smem(a.stages);
         const int64_t tiles = (need + a.tps - 1) / a.tps;
         const bool f16 = a.cos_f16 != 0;
-        if (a.x_kind == 0) {
-            if (f16) launch_drq_ring<0, true>(a, tiles, smem, s);
-            else launch_drq_ring<0, false>(a, tiles, smem, s);
-        } else if (a.x_kind == 1) {
-            launch_drq_ring<1, false>(a, tiles, smem, s);
-        } else {
-            launch_drq_ring<2, true>(a, tiles, smem, s);
-        }
-        return launched();
+        if (a.x_kind == 0) return launched(f16 ? launch_drq_ring<0, true>(a, tiles, smem, s)
+                                               : launch_drq_ring<0, false>(a, tiles, smem, s));
+        if (a.x_kind == 1) return launched(launch_drq_ring<1, false>(a, tiles, smem, s));
+        return launched(launch_drq_ring<2, true>(a, tiles, smem, s));
     }
     // every other shape and alignment: one CTA per token
-    launch(dequant_rope_quant_general_kernel,
-           (unsigned)persistent_grid(dequant_rope_quant_general_kernel, DG_THREADS, need), DG_THREADS, 0, s, a);
-    return launched();
+    return launched(launch(dequant_rope_quant_general_kernel,
+                           (unsigned)persistent_grid(dequant_rope_quant_general_kernel, DG_THREADS, need),
+                           DG_THREADS, 0, s, a));
 }
 
 // ---------------------------------------------------------------------------
@@ -1065,15 +1073,76 @@ kvq_status kvq_get_error(kvq_stream stream, uint32_t* fault_bits) {
     if (!fault_bits) return KVQ_ERR_NULL;
     *fault_bits = 0u;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // one device-side atomic exchange reads and clears the word, so a bit
+    // raised by a kernel on another stream is either returned by this call or
+    // left for the next one; concurrent callers take different snapshot slots
+    static std::atomic<uint32_t> ticket{0};
+    const uint32_t slot = ticket.fetch_add(1u, std::memory_order_relaxed) % FAULT_SNAPSHOTS;
     unsigned int h = 0u;
-    const unsigned int zero = 0u;
-    if (cudaMemcpyFromSymbolAsync(&h, g_fault_word, sizeof(h), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    // a plain launch (no programmatic serialization): the exchange runs after
+    // every earlier kernel of the stream has completed
+    uint32_t slot_arg = slot;
+    void* args[] = {&slot_arg};
+    if (cudaLaunchKernel(reinterpret_cast<const void*>(fault_exchange_kernel), dim3(1), dim3(1), args, 0, s) !=
+        cudaSuccess)
         return KVQ_ERR_CUDA;
-    if (cudaMemcpyToSymbolAsync(g_fault_word, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    if (cudaMemcpyFromSymbolAsync(&h, g_fault_snapshot, sizeof(h), slot * sizeof(h), cudaMemcpyDeviceToHost, s) !=
+        cudaSuccess)
         return KVQ_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return KVQ_ERR_CUDA;
     *fault_bits = h;
     return KVQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+kvq_status kvq_scatter_rows(const kvq_tensor* x, const kvq_tensor* slot_mapping, kvq_tensor* cache,
+                            int64_t out_bytes, kvq_stream stream) {
+    Trace trace("kvq_scatter_rows");
+    if (!x || !slot_mapping || !cache) return KVQ_ERR_NULL;
+    if (!valid_desc(x) || !valid_desc(slot_mapping) || !valid_desc(cache)) return KVQ_ERR_DTYPE;
+    if (x->ndim < 1) return KVQ_ERR_NDIM;
+    int64_t T, rs;
+    if (!flatten_rows(x, &T, &rs)) return KVQ_ERR_LAYOUT;
+    const int64_t eb = elem_bytes(x->dtype);
+    const int64_t in_bytes = x->shape[x->ndim - 1] * eb;
+    if (in_bytes % 16 != 0 || in_bytes < 16 || in_bytes > 16 * 32 * SC_MAX_CHUNKS_PER_LANE) return KVQ_ERR_SHAPE;
+    if (out_bytes < 16 || out_bytes % 16 != 0 || out_bytes > in_bytes) return KVQ_ERR_ATTR;
+    if (!is_index_dtype(slot_mapping->dtype)) return KVQ_ERR_DTYPE;
+    if (numel(slot_mapping) != T) return KVQ_ERR_SHAPE;
+    if (!contiguous(slot_mapping)) return KVQ_ERR_LAYOUT;
+    if (cache->dtype != KVQ_U8 && cache->dtype != KVQ_I8) return KVQ_ERR_DTYPE;
+    if (cache->ndim != 4) return KVQ_ERR_NDIM;
+    if (cache->shape[2] != 1) return KVQ_ERR_SHAPE;
+    PagedRows rows;
+    int64_t head_dim;
+    kvq_status st = paged_from(cache, 1, &rows, &head_dim);
+    if (st != KVQ_OK) return st;
+    if (head_dim < out_bytes) return KVQ_ERR_CAPACITY;
+    if (T == 0) return KVQ_OK;
+    if (!x->data || !slot_mapping->data || !cache->data) return KVQ_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(x->data) % 16 != 0 || (rs * eb) % 16 != 0 ||
+        reinterpret_cast<uintptr_t>(cache->data) % 16 != 0 || rows.row_bytes % 16 != 0 ||
+        rows.block_stride % 16 != 0)
+        return KVQ_ERR_LAYOUT;
+    ScatterCopyArgs a;
+    a.x = static_cast<const uint8_t*>(x->data);
+    a.x_row_bytes = rs * eb;
+    a.T = T;
+    a.slots = slot_mapping->data;
+    a.slots_i64 = slot_mapping->dtype == KVQ_I64;
+    a.cache = rows;
+    a.in_chunks = (int32_t)(in_bytes / 16);
+    a.out_chunks = (int32_t)(out_bytes / 16);
+    const int ncl = (a.in_chunks + 31) / 32;
+    const int64_t need = ((T + 1) / 2 + (SC_THREADS / 32) - 1) / (SC_THREADS / 32);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    auto run = [&](auto kernel) {
+        return launched(launch(kernel, (unsigned)persistent_grid(kernel, SC_THREADS, need), SC_THREADS, 0, s, a));
+    };
+    if (ncl == 1) return run(scatter_copy_kernel<1>);
+    if (ncl == 2) return run(scatter_copy_kernel<2>);
+    if (ncl == 3) return run(scatter_copy_kernel<3>);
+    return run(scatter_copy_kernel<4>);
 }
 
 kvq_status kvq_convert(int32_t fmt, const float* in, int64_t n, void* out, kvq_stream stream) {
@@ -1082,9 +1151,8 @@ kvq_status kvq_convert(int32_t fmt, const float* in, int64_t n, void* out, kvq_s
     if (n == 0) return KVQ_OK;
     if (!in || !out) return KVQ_ERR_NULL;
     const int64_t need = (n + 255) / 256;
-    launch(convert_kernel, (unsigned)persistent_grid(convert_kernel, 256, need), 256, 0,
-           reinterpret_cast<cudaStream_t>(stream), fmt, in, n, static_cast<uint8_t*>(out));
-    return launched();
+    return launched(launch(convert_kernel, (unsigned)persistent_grid(convert_kernel, 256, need), 256, 0,
+                           reinterpret_cast<cudaStream_t>(stream), fmt, in, n, static_cast<uint8_t*>(out)));
 }
 
 }  // extern "C"

@@ -291,3 +291,29 @@ def test_host_tensors_are_rejected_before_any_launch():
         kvq.indexer_quant_cache(x, c, c, s, "mxfp8")
     with pytest.raises(ValueError, match="CUDA device"):
         kvq.kv_decompress(c, s, x, 0)
+
+
+def test_calls_run_on_the_tensors_device(monkeypatch):
+    """The library sizes grids and launches on the current device, so the binding
+    makes the tensors' device current for the call when it is not already."""
+    import contextlib
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    assert isinstance(kvq._on(torch.device("cuda", 0)), contextlib.nullcontext)
+    assert isinstance(kvq._on(None), contextlib.nullcontext)
+    ctx = kvq._on(torch.device("cuda", 1))
+    assert isinstance(ctx, torch.cuda.device) and ctx.idx == 1
+
+
+def test_check_flag_reports_fault_bits(monkeypatch, L):
+    """check=True reads the fault word after the call and raises on a set bit."""
+    calls = []
+
+    def fake_get_error(stream, bits):
+        calls.append(stream)
+        ctypes.cast(bits, ctypes.POINTER(ctypes.c_uint32))[0] = kvq.FAULT_SLOT_RANGE
+        return 0
+    monkeypatch.setattr(L, "kvq_get_error", fake_get_error)
+    with pytest.raises(kvq.KvqFault, match="FAULT_SLOT_RANGE"):
+        kvq._faults("op", True, 1234)
+    kvq._faults("op", False, 1234)
+    assert calls == [1234]

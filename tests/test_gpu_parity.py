@@ -90,6 +90,29 @@ def test_compress_pipelined_ragged_counts(T):
     _same(_ce(T, 576, 2, 32, seed=25))
 
 
+# d > 1024: more 64-value segment columns (17, 22, 27) than the pipelined
+# kernel's 16 consumer warps, so each warp walks several columns and packed
+# rows leave by direct stores; 1728 is the widest row whose two-stage ring
+# fits in shared memory.
+@pytest.mark.parametrize("mode,G", [(0, 64), (1, 64), (2, 16), (2, 32), (2, 64)])
+@pytest.mark.parametrize("d", [1088, 1408, 1728])
+def test_compress_pipelined_multi_segment_columns(mode, G, d):
+    _same(_ce(T_PIPE, d, mode, G, kind="wide" if d == 1408 else "normal", seed=31))
+
+
+@pytest.mark.parametrize("mode,G", [(0, 64), (1, 64), (2, 16)])
+@pytest.mark.parametrize("extra,pad", [(1, 0), (7, 5), (16, 1000)])
+def test_compress_pipelined_multi_segment_row_alignments(mode, G, extra, pad):
+    _same(_ce(T_PIPE, 1408, mode, G, extra=extra, pad=pad, seed=33))
+
+
+@pytest.mark.parametrize("mode,G", [(0, 64), (1, 64), (2, 16), (2, 64)])
+def test_compress_widest_rows_at_pipelined_batch_size(mode, G):
+    """d = 8192 with a batch above the pipelined threshold: the ring does not fit
+    in shared memory, so kernel selection must fall back to the direct kernel."""
+    _same(_ce(T_PIPE, 8192, mode, G, seed=35, slot_dtype=np.int64 if mode == 0 else np.int32))
+
+
 def test_compress_max_width_and_int64_slots():
     _same(_ce(40, 8192, 0, seed=9, slot_dtype=np.int64))
     _same(_ce(40, 8192, 2, 16, seed=9, slot_dtype=np.int64))
@@ -357,3 +380,27 @@ def test_drq_named_workload_full_size(name):
 def test_drq_named_workload_narrow_range():
     """Same shapes with |x| <= 2^12, where few int8 codes saturate."""
     _same(W.dequant_rope_quant_page_B16_S1024_H3072(x_range=1 << 12))
+
+
+# ---------------------------------------------------------------------------
+# scatter_rows: the compress access pattern without arithmetic (data movement
+# only, so the expectation is the input bytes themselves)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("out_bytes", [352, 672, 1152])
+def test_scatter_rows_moves_the_row_prefix(out_bytes):
+    from kv_cache_quantize_b200.workloads import dev_cache
+    case = _ce(T_PIPE, 576, 0, seed=41, extra=1152 - oracle.kv_cache_col(576, 0, 64))
+    x, slots, cb = case.arrays["x"], case.arrays["slot_mapping"], case.caches["cache"]
+    st, view = dev_cache(cb, torch.uint8)
+    xt = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    kvq.get_error()
+    kvq.scatter_rows(xt, torch.from_numpy(slots).cuda(), view, out_bytes)
+    torch.cuda.synchronize()
+    assert kvq.get_error() == 0
+    want = cb.storage.copy()
+    xb = x.view(np.uint8).reshape(x.shape[0], -1)
+    for t, s in enumerate(slots.tolist()):
+        if s >= 0:
+            o = cb.offset + (s // cb.block_size) * cb.block_stride + (s % cb.block_size) * cb.row_bytes
+            want[o:o + out_bytes] = xb[t, :out_bytes]
+    assert np.array_equal(st.cpu().numpy(), want)
