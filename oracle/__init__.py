@@ -5,6 +5,9 @@ wrapper, what the four epilogue operations compute.  Only the tests, the
 smoke check (``__graft_entry__.smoke``) and the benchmark's CPU-baseline leg
 may import it.  The CUDA library never uses it and shares no code with it.
 
+The token Compressor (aclnnCompressor, C128A form) is oracle/compressor.py:
+numpy in float64, pinned by tests/test_oracle_compressor.py.
+
 Pinned by tests/test_oracle_codecs.py and tests/test_oracle_ops.py.  Parity
 unpinned (conventions with nothing on the pages to check against): the
 packed-row segment order, the FP4 nibble order, the padding bytes, and the

@@ -91,3 +91,59 @@ def test_every_planted_mistake_is_caught(tmp_path):
     assert rcs[0] == 0, "the pin suites fail on an unmodified copy of the oracle"
     survived = [name for name, rc in zip(MUTANTS, rcs[1:]) if rc == 0]
     assert not survived, f"planted mistakes no pin caught: {survived}"
+
+
+# The Compressor oracle (numpy): mistakes planted in a copy of its source, which
+# is loaded as a module of its own; the pins of tests/test_oracle_compressor.py
+# run against it in this process.
+COMPRESSOR_MUTANTS = {
+    "softmax over channels instead of rows": (
+        "return e / e.sum(axis=1, keepdims=True)", "return e / e.sum(axis=2, keepdims=True)"),
+    "softmax not normalised": ("return e / e.sum(axis=1, keepdims=True)", "return e"),
+    "Ape dropped": ("+ np.asarray(ape, dtype=np.float64)[None, :, :]",
+                    "+ 0.0 * np.asarray(ape, dtype=np.float64)[None, :, :]"),
+    "Ape rows reversed": ("+ np.asarray(ape, dtype=np.float64)[None, :, :]",
+                          "+ np.asarray(ape, dtype=np.float64)[None, ::-1, :]"),
+    "scores weight the scores, not kv_state": ("sh = p * kv.reshape(T // ratio, ratio, D)",
+                                               "sh = p * score.reshape(T // ratio, ratio, D)"),
+    "weights swapped between kv and gate": (
+        "return X @ bf16_to_f64(w_kv).T, X @ bf16_to_f64(w_gate).T",
+        "return X @ bf16_to_f64(w_gate).T, X @ bf16_to_f64(w_kv).T"),
+    "group sum divided by the group size": ("return np.ones(ratio) @ sh", "return np.ones(ratio) @ sh / ratio"),
+    "groups offset by one row": ("s = score.reshape(T // ratio, ratio, D)",
+                                 "s = np.roll(score, 1, axis=0).reshape(T // ratio, ratio, D)"),
+    "bf16 decoded with the wrong shift": ("(b.astype(np.uint32) << 16)", "(b.astype(np.uint32) << 15)"),
+    "stability shift taken per row (over channels)": ("s = s - s.max(axis=1, keepdims=True)",
+                                                      "s = s - s.max(axis=2, keepdims=True)"),
+}
+
+
+def test_every_planted_compressor_mistake_is_caught(tmp_path):
+    import importlib.util
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import test_oracle_compressor as P
+    src = open(os.path.join(ROOT, "oracle", "compressor.py")).read()
+
+    def load(text, name):
+        path = tmp_path / f"{name}.py"
+        path.write_text(text)
+        spec = importlib.util.spec_from_file_location(name, path)
+        mod = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(mod)
+        return mod
+
+    def caught(mod):
+        for pin in P.PINS:
+            try:
+                pin(mod)
+            except Exception:
+                return True
+        return False
+
+    assert not caught(load(src, "control")), "the pins fail on an unmodified copy of the oracle"
+    survived = []
+    for i, (name, (a, b)) in enumerate(COMPRESSOR_MUTANTS.items()):
+        assert a in src, f"mutant site not found: {name}"
+        if not caught(load(src.replace(a, b, 1), f"mutant{i:02d}")):
+            survived.append(name)
+    assert not survived, f"planted mistakes no pin caught: {survived}"

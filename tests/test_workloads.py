@@ -56,3 +56,17 @@ def test_caches_start_with_random_bytes():
     c = W.CONFIGS["compress_mode1_T64_d256"]()
     st = c.caches["cache"].storage
     assert np.unique(st).size > 200
+
+
+def test_compressor_inputs():
+    """The Compressor's inputs: bf16 x ~ N(0, 1), weights ~ N(0, 1/H), float32 Ape; seeded."""
+    c = W.TENSOR_CONFIGS["compressor_c128a_T2048_H1024_D512"]()
+    x, wk, wg, ape = (c.arrays[k] for k in ("x", "w_kv", "w_gate", "ape"))
+    assert x.shape == (2048, 1024) and x.dtype == np.uint16
+    assert wk.shape == wg.shape == (512, 1024) and ape.shape == (128, 512) and ape.dtype == np.float32
+    xv = (x.astype(np.uint32) << 16).view(np.float32)
+    wv = (wk.astype(np.uint32) << 16).view(np.float32)
+    assert abs(float(xv.std()) - 1.0) < 0.01 and abs(float(wv.std()) * 32.0 - 1.0) < 0.02
+    assert not np.array_equal(wk, wg)
+    d = W.TENSOR_CONFIGS["compressor_c128a_T2048_H1024_D512"]()
+    assert all(np.array_equal(c.arrays[k], d.arrays[k]) for k in c.arrays)
