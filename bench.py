@@ -33,7 +33,6 @@ import json
 import os
 import statistics
 import sys
-import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -46,6 +45,7 @@ WORKLOAD = ("kv_compress_epilog large sweep: T=262144 tokens, d=576 bf16 N(0,1) 
             "bf16 scale, rope FP8 E4M3 static x_scale=0.1, 352-B rows); cache blockSize=128, 4096 blocks; "
             "2% slot_mapping -1")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 # ---------------------------------------------------------------------------
@@ -97,6 +97,24 @@ def algorithmic_bytes(case) -> int:
             params += a["indices"].nbytes       # one start position per batch
         return T * per_tok + params
     raise ValueError(case.op)
+
+
+def contraction_flops(case) -> int:
+    """FLOPs of the Compressor's two projections (x @ W^KV^T and x @ W^Gate^T):
+    2 T H D each; the softmax epilogue (a few operations per output of the
+    projections) is not counted."""
+    T, H = case.arrays["x"].shape
+    D = case.arrays["w_kv"].shape[0]
+    return 2 * T * H * 2 * D
+
+
+def bf16_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def token_rows(case) -> int:
@@ -196,70 +214,105 @@ def sum_over_ranks(n: int, dist, device) -> int:
 # ---------------------------------------------------------------------------
 # clocks during the timed region (NVML: the same counters nvidia-smi reads)
 # ---------------------------------------------------------------------------
+_SAMPLER_CHILD = r"""
+import json, select, sys, time
+import pynvml
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByUUID(sys.argv[1].encode())
+period = float(sys.argv[2])
+out = []
+first = True
+while True:
+    t = time.monotonic()
+    try:
+        out.append((t, pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                    int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))))
+    except Exception:
+        pass
+    if first:                      # NVML is warm: the parent may start its timed work
+        sys.stdout.write("ready\n"); sys.stdout.flush()
+        first = False
+    if select.select([sys.stdin], [], [], period)[0]:
+        break
+sys.stdout.write(json.dumps(out) + "\n"); sys.stdout.flush()
+"""
+
+
 class ClockSampler:
-    """SM clock and throttle reasons of THIS process's GPU, sampled in a thread.
+    """SM clock and throttle reasons of THIS process's GPU, sampled by a child
+    process (so the sampling neither competes with the launching thread for the
+    interpreter lock nor is starved by it).
 
     NVML numbers GPUs by physical index and ignores CUDA_VISIBLE_DEVICES, so the
     handle is opened by the CUDA device's UUID (or, failing that, its PCI bus
-    id), never by the CUDA ordinal; the UUID is recorded with the samples."""
+    id), never by the CUDA ordinal; the UUID is recorded with the samples.
+    mark() / mark_end() bracket the timed region on the host's monotonic clock;
+    summary() keeps the samples taken inside it."""
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index: int, period_s: float = 0.001):
+    def __init__(self, device_index: int, period_s: float = 0.0002):
         self.period = period_s
-        self.samples = []
-        self.reasons = set()
         self.max_mhz = None
         self.uuid = None
-        self._stop = threading.Event()
-        self._thr = None
+        self.samples = []
+        self.t0 = self.t1 = None
+        self.proc = None
         try:
             import pynvml
             import torch
             pynvml.nvmlInit()
-            self.nv = pynvml
             props = torch.cuda.get_device_properties(device_index)
             uuid = str(props.uuid)
             uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
             try:
-                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
-                self.uuid = uuid
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
             except Exception:
                 bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
-                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
-                u = pynvml.nvmlDeviceGetUUID(self.h)
-                self.uuid = u.decode() if isinstance(u, bytes) else str(u)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+                h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+                u = pynvml.nvmlDeviceGetUUID(h)
+                uuid = u.decode() if isinstance(u, bytes) else str(u)
+            self.uuid = uuid
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
         except Exception:
-            self.nv = None
-
-    def _run(self):
-        while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for name, b in self.REASONS.items():
-                    if bits & b:
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(self.period)
+            self.uuid = None
 
     def __enter__(self):
-        if self.nv is not None:
-            self._thr = threading.Thread(target=self._run, daemon=True)
-            self._thr.start()
+        import subprocess
+        if self.uuid is not None:
+            try:
+                self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER_CHILD, self.uuid, str(self.period)],
+                                             stdin=subprocess.PIPE, stdout=subprocess.PIPE, text=True)
+                if self.proc.stdout.readline().strip() != "ready":
+                    raise RuntimeError("sampler did not start")
+            except Exception:
+                self.proc = None
         return self
 
+    def mark(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
+
     def __exit__(self, *exc):
-        self._stop.set()
-        if self._thr is not None:
-            self._thr.join()
+        if self.proc is not None:
+            try:
+                out, _ = self.proc.communicate("stop\n", timeout=30)
+                self.samples = json.loads(out.strip().splitlines()[-1])
+            except Exception:
+                self.proc.kill()
+                self.samples = []
 
     def summary(self):
-        med = statistics.median(self.samples) if self.samples else None
-        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                "samples": len(self.samples), "period_ms": 1e3 * self.period, "gpu_uuid": self.uuid}
+        t0 = self.t0 if self.t0 is not None else float("-inf")
+        t1 = self.t1 if self.t1 is not None else float("inf")
+        inside = [(m, b) for t, m, b in self.samples if t0 <= t <= t1]
+        reasons = sorted({n for _, b in inside for n, bit in self.REASONS.items() if b & bit})
+        return {"sm_mhz": statistics.median([m for m, _ in inside]) if inside else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(inside),
+                "period_ms": 1e3 * self.period, "gpu_uuid": self.uuid,
+                "window_ms": None if self.t0 is None or self.t1 is None else 1e3 * (self.t1 - self.t0)}
 
 
 # ---------------------------------------------------------------------------
@@ -409,6 +462,15 @@ def run_profile_workload(args):
         print(f"{args.profile_workload}: {args.profile_reps} launches over 1 input copies, "
               f"{us:.1f} us per launch, {nb / us / 1e3:.0f} GB/s algorithmic")
         return 0
+    if args.profile_workload in W.TENSOR_CONFIGS:
+        case = W.TENSOR_CONFIGS[args.profile_workload]()
+        call, _, _ = W.build_call(case)
+        us = device_us_per_launch([call], stream, args.profile_reps)
+        if kvq.get_error(stream) != 0:
+            raise RuntimeError("device fault bits set")
+        print(f"{args.profile_workload}: {args.profile_reps} launches, {us:.1f} us per launch, "
+              f"{contraction_flops(case) / us / 1e6:.1f} TFLOP/s")
+        return 0
     make = W.CONFIGS[args.profile_workload]
     case = make()
     calls = rotation(case, make, torch.cuda.get_device_properties(0).L2_cache_size)
@@ -432,7 +494,7 @@ def main():
     ap.add_argument("--no-per-config", action="store_true", help="skip the per-workload breakdown")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle timing for cpu_baseline")
     ap.add_argument("--profile-workload", default=None,
-                    help="profiling mode: run only this named workload (a workloads.CONFIGS name, or "
+                    help="profiling mode: run only this named workload (a workloads.CONFIGS or TENSOR_CONFIGS name, or "
                          "decompress_mode0_T262144_d576 / decompress_mode2_G32_T262144_d576 for the decoder) "
                          "--profile-reps times (back to back, cycling input copies larger than L2) and print its "
                          "time per launch; no JSON line")
@@ -471,6 +533,9 @@ def main():
     bytes_a, bytes_b = algorithmic_bytes(case_a), algorithmic_bytes(case_b)
     tokens_per_step = token_rows(case_a) + token_rows(case_b)
 
+    # the clock sampler (a child process) starts before the warm-up, so that it
+    # is sampling steadily when the timed region begins
+    clocks = ClockSampler(local).__enter__()
     for _ in range(args.warmup):
         call_a(stream)
         call_b(stream)
@@ -484,16 +549,18 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(local) as clocks:
-        start.record(stream)
-        for e0, e1, e2 in ev:
-            e0.record(stream)
-            call_a(stream)
-            e1.record(stream)
-            call_b(stream)
-            e2.record(stream)
-        stop.record(stream)
-        torch.cuda.synchronize(dev)
+    clocks.mark()
+    start.record(stream)
+    for e0, e1, e2 in ev:
+        e0.record(stream)
+        call_a(stream)
+        e1.record(stream)
+        call_b(stream)
+        e2.record(stream)
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark_end()
+    clocks.__exit__(None, None, None)
     elapsed = max_over_ranks(start.elapsed_time(stop) / 1e3, dist, dev)
     tokens_all_ranks = sum_over_ranks(tokens_per_step, dist, dev)
     if world > 1:
@@ -572,6 +639,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_per_config:
         per_config = {}
         pc_sampler = ClockSampler(local, 0.005).__enter__()
+        pc_sampler.mark()
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         for name, make in W.CONFIGS.items():
             case = {"compress_mode0_T262144_d576": case_a,
@@ -596,6 +664,20 @@ def main():
                                 "input_copies": 1, "l2": f"{nb >> 20} MB > L2"}
             del dcall
             torch.cuda.empty_cache()
+        # the Compressor (a dense contraction: TFLOP/s against the measured bf16 peak)
+        tpeak, tkind = bf16_peak()
+        for name, make in W.TENSOR_CONFIGS.items():
+            case = make()
+            call, _, _ = W.build_call(case)
+            us = device_us_per_launch([call], stream, 20)
+            fl = contraction_flops(case)
+            per_config[name] = {"tokens": int(case.arrays["x"].shape[0]), "flops": fl, "us_per_launch": us,
+                                "tokens_per_s": case.arrays["x"].shape[0] / us * 1e6, "TFLOPs": fl / us / 1e6,
+                                "frac_of_peak": fl / us / 1e6 / tpeak, "bound": "tensor",
+                                "peak_source": f"{tkind} bf16_tflops (burst)",
+                                "l2": "x larger than L2" if case.arrays["x"].nbytes > l2 else "L2-resident"}
+            del call, case
+            torch.cuda.empty_cache()
         # the same access pattern without arithmetic (kvq_scatter_rows): the DRAM
         # ceiling the two compress passes are compared with
         from kv_cache_quantize_b200.workloads import dev_cache
@@ -618,6 +700,7 @@ def main():
                                 "note": "compress access pattern, no arithmetic"}
             del xt, sl, view, scall
             torch.cuda.empty_cache()
+        pc_sampler.mark_end()
         pc_sampler.__exit__(None, None, None)
         per_config_clocks = pc_sampler.summary()
 

@@ -259,6 +259,33 @@ KVQ_API kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq
                                           kvq_tensor* v_out, kvq_stream stream);
 
 /* ------------------------------------------------------------------------ */
+/* compressor: the token Compressor, C128A form (coff = 1)                   */
+/* Source: aclnnCompressor, 接口功能 / 计算公式 steps 1-5 / 约束说明.          */
+/*                                                                           */
+/* Per group i of cmp_ratio consecutive token rows and per channel c:        */
+/*   kv_state = X @ W^KV^T, score_state = X @ W^Gate^T (step 1),             */
+/*   s_r = score_state[r, c] + ape[r mod cmp_ratio, c] (step 2),             */
+/*   p = softmax over the group's rows of s (step 3, channel by channel),    */
+/*   cmp_kv[i, c] = sum_r p_r kv_state[r, c] (steps 4-5), rounded to bf16.   */
+/* x       bf16 [..., H], contiguous, 16-byte aligned; the leading dims are   */
+/*         the T token rows, T % cmp_ratio == 0 (whole groups: the stateless  */
+/*         case; the page's state cache, start_pos and cu_seqlens are not     */
+/*         modelled).  1024 <= H <= 10240, H % 512 == 0.                     */
+/* w_kv,   bf16 [D, H] (the page's [coff*D, H] with coff = 1), contiguous,    */
+/* w_gate  16-byte aligned; D = 128 or 512.                                   */
+/* ape     f32 [cmp_ratio, D], contiguous.                                    */
+/* cmp_kv  bf16 [T / cmp_ratio, D], contiguous: written.                     */
+/* cmp_ratio  2, 4, 8, 16, 32, 64 or 128 (C128A: 128).                        */
+/* Arithmetic: bf16 products with fp32 accumulation on the tensor cores       */
+/* (tcgen05), the softmax in fp32; the result is within the bound of fp32     */
+/* accumulation of the exact value, not bit-reproducible against another      */
+/* summation order.  One kernel on `stream`; nothing is allocated; no         */
+/* workspace.  KVQ_ERR_CUDA if the TMA descriptors cannot be encoded.         */
+/* ------------------------------------------------------------------------ */
+KVQ_API kvq_status kvq_compressor(const kvq_tensor* x, const kvq_tensor* w_kv, const kvq_tensor* w_gate,
+                                  const kvq_tensor* ape, kvq_tensor* cmp_kv, int32_t cmp_ratio, kvq_stream stream);
+
+/* ------------------------------------------------------------------------ */
 /* Utilities                                                                 */
 /* ------------------------------------------------------------------------ */
 

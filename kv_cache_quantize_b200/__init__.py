@@ -28,7 +28,7 @@ import torch
 __all__ = [
     "KvqError", "KvqFault", "lib", "library_path", "kv_compress_epilog", "kv_decompress", "indexer_quant_cache",
     "kv_rmsnorm_rope_cache",
-    "dequant_rope_quant_kvcache", "get_error", "kv_cache_col", "indexer_scale_col", "convert", "selftest", "scatter_rows",
+    "dequant_rope_quant_kvcache", "compressor", "get_error", "kv_cache_col", "indexer_scale_col", "convert", "selftest", "scatter_rows",
     "FAULT_SLOT_RANGE", "FAULT_TIMEOUT", "STATUS",
 ]
 
@@ -92,6 +92,7 @@ def lib() -> ctypes.CDLL:
                                                      ctypes.POINTER(i64), i32, i32, i32, i32, i32, _P, _P, _P, vp]
         L.kvq_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
         L.kvq_scatter_rows.argtypes = [_P, _P, _P, i64, vp]
+        L.kvq_compressor.argtypes = [_P, _P, _P, _P, _P, i32, vp]
         L.kvq_convert.argtypes = [i32, vp, i64, vp, vp]
         L.kvq_selftest.argtypes = [i32, ctypes.POINTER(ctypes.c_uint64), vp]
         L.kvq_kv_cache_col.argtypes = [i64, i32, i32]
@@ -104,7 +105,7 @@ def lib() -> ctypes.CDLL:
         for name in ("kvq_kv_compress_epilog", "kvq_kv_decompress", "kvq_indexer_quant_cache",
                      "kvq_kv_rmsnorm_rope_cache",
                      "kvq_dequant_rope_quant_kvcache", "kvq_get_error", "kvq_convert", "kvq_selftest",
-                     "kvq_scatter_rows"):
+                     "kvq_scatter_rows", "kvq_compressor"):
             getattr(L, name).restype = i32
         _LIB = L
     return _LIB
@@ -289,6 +290,23 @@ def dequant_rope_quant_kvcache(x: torch.Tensor, cos: torch.Tensor, sin: torch.Te
             _ref(desc(k_out)) if kv_output else None, _ref(desc(v_out)) if kv_output else None, st))
         _faults("dequant_rope_quant_kvcache", check, st)
     return q_out, k_out, v_out
+
+
+def compressor(x: torch.Tensor, w_kv: torch.Tensor, w_gate: torch.Tensor, ape: torch.Tensor,
+               cmp_kv: Optional[torch.Tensor] = None, cmp_ratio: int = 128, stream=None,
+               check: bool = False) -> torch.Tensor:
+    """The token Compressor, C128A form (see kvq_compressor): per group of cmp_ratio token rows
+    and channel, the softmax over the group of (x @ w_gate^T + ape) weights x @ w_kv^T.
+    Returns cmp_kv [T / cmp_ratio, D] (allocated when not given)."""
+    if cmp_kv is None:
+        T = x.numel() // x.shape[-1] if x.dim() else 0
+        cmp_kv = torch.empty((T // max(1, int(cmp_ratio)), w_kv.shape[0]), dtype=torch.bfloat16, device=x.device)
+    with _on(_one_device("compressor", x, w_kv, w_gate, ape, cmp_kv)):
+        st = _stream(stream, x)
+        _check("compressor", lib().kvq_compressor(_ref(desc(x)), _ref(desc(w_kv)), _ref(desc(w_gate)),
+                                                  _ref(desc(ape)), _ref(desc(cmp_kv)), int(cmp_ratio), st))
+        _faults("compressor", check, st)
+    return cmp_kv
 
 
 def scatter_rows(x: torch.Tensor, slot_mapping: torch.Tensor, cache: torch.Tensor, out_bytes: int,

@@ -1,6 +1,8 @@
 // kvq.cu -- host side of the C ABI declared in include/kvq.h: argument
 // validation, kernel selection and launch.  Single translation unit: the
 // kernels live in the .cuh files included below.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -14,6 +16,7 @@
 
 #include "kvq.h"
 #include "compress_epilog.cuh"
+#include "compressor.cuh"
 #include "dequant_rope_quant.cuh"
 #include "indexer_quant.cuh"
 #include "kv_decompress.cuh"
@@ -1095,6 +1098,101 @@ kvq_status kvq_get_error(kvq_stream stream, uint32_t* fault_bits) {
 }
 
 // ---------------------------------------------------------------------------
+namespace {
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (the
+// library links the CUDA runtime statically and never links the driver
+// library itself)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tensor map of a row-major bf16 matrix [rows, cols] (row pitch `pitch`
+// elements) read in boxes of box_rows x 64 columns with the 128-byte swizzle;
+// rows past the end read as zero.
+bool bf16_tile_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t pitch, uint32_t box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(pitch * 2)};
+    const cuuint32_t box[2] = {(cuuint32_t)CP_BK, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+kvq_status kvq_compressor(const kvq_tensor* x, const kvq_tensor* w_kv, const kvq_tensor* w_gate,
+                          const kvq_tensor* ape, kvq_tensor* cmp_kv, int32_t cmp_ratio, kvq_stream stream) {
+    Trace trace("kvq_compressor");
+    if (!x || !w_kv || !w_gate || !ape || !cmp_kv) return KVQ_ERR_NULL;
+    if (!valid_desc(x) || !valid_desc(w_kv) || !valid_desc(w_gate) || !valid_desc(ape) || !valid_desc(cmp_kv))
+        return KVQ_ERR_DTYPE;
+    if (x->dtype != KVQ_BF16 || w_kv->dtype != KVQ_BF16 || w_gate->dtype != KVQ_BF16 || cmp_kv->dtype != KVQ_BF16 ||
+        ape->dtype != KVQ_F32)
+        return KVQ_ERR_DTYPE;
+    if (cmp_ratio < 2 || cmp_ratio > 128 || (cmp_ratio & (cmp_ratio - 1)) != 0) return KVQ_ERR_ATTR;
+    if (x->ndim < 1 || w_kv->ndim != 2 || w_gate->ndim != 2 || ape->ndim != 2 || cmp_kv->ndim != 2)
+        return KVQ_ERR_NDIM;
+    const int64_t H = x->shape[x->ndim - 1];
+    const int64_t T = numel_leading(x);
+    const int64_t D = w_kv->shape[0];
+    if (H < 1024 || H > 10240 || H % 512 != 0) return KVQ_ERR_SHAPE;
+    if (D != 128 && D != 512) return KVQ_ERR_SHAPE;
+    if (w_kv->shape[1] != H || w_gate->shape[0] != D || w_gate->shape[1] != H) return KVQ_ERR_SHAPE;
+    if (ape->shape[0] != cmp_ratio || ape->shape[1] != D) return KVQ_ERR_SHAPE;
+    if (T % cmp_ratio != 0) return KVQ_ERR_SHAPE;
+    if (cmp_kv->shape[0] != T / cmp_ratio || cmp_kv->shape[1] != D) return KVQ_ERR_SHAPE;
+    if (T > (int64_t)0x7fffffff - CP_BN) return KVQ_ERR_SHAPE;          // TMA coordinates are 32-bit
+    if (!contiguous(x) || !contiguous(w_kv) || !contiguous(w_gate) || !contiguous(ape) || !contiguous(cmp_kv))
+        return KVQ_ERR_LAYOUT;
+    if (T == 0) return KVQ_OK;
+    if (!x->data || !w_kv->data || !w_gate->data || !ape->data || !cmp_kv->data) return KVQ_ERR_NULL;
+    auto a16 = [](const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; };
+    if (!a16(x->data) || !a16(w_kv->data) || !a16(w_gate->data)) return KVQ_ERR_LAYOUT;   // TMA base alignment
+
+    CUtensorMap mx, mk, mg;
+    if (!bf16_tile_map(&mx, x->data, T, H, H, CP_BN) || !bf16_tile_map(&mk, w_kv->data, D, H, H, CP_BM) ||
+        !bf16_tile_map(&mg, w_gate->data, D, H, H, CP_BM))
+        return KVQ_ERR_CUDA;
+    CompressorArgs a;
+    a.T = T;
+    a.H = (int32_t)H;
+    a.D = (int32_t)D;
+    a.n_ch_tiles = (int32_t)(D / CP_BM);
+    a.n_tok_tiles = (T + CP_BN - 1) / CP_BN;
+    a.ape = static_cast<const float*>(ape->data);
+    a.out = static_cast<uint16_t*>(cmp_kv->data);
+    const int64_t tiles = a.n_tok_tiles * a.n_ch_tiles;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    auto run = [&](auto kernel) {
+        return launched(launch(kernel, (unsigned)persistent_grid(kernel, CP_THREADS, tiles, CP_SMEM_BYTES),
+                               CP_THREADS, CP_SMEM_BYTES, s, mx, mk, mg, a));
+    };
+    switch (cmp_ratio) {
+        case 2: return run(compressor_kernel<2>);
+        case 4: return run(compressor_kernel<4>);
+        case 8: return run(compressor_kernel<8>);
+        case 16: return run(compressor_kernel<16>);
+        case 32: return run(compressor_kernel<32>);
+        case 64: return run(compressor_kernel<64>);
+        default: return run(compressor_kernel<128>);
+    }
+}
+
+// ---------------------------------------------------------------------------
 kvq_status kvq_scatter_rows(const kvq_tensor* x, const kvq_tensor* slot_mapping, kvq_tensor* cache,
                             int64_t out_bytes, kvq_stream stream) {
     Trace trace("kvq_scatter_rows");
@@ -1105,7 +1203,7 @@ kvq_status kvq_scatter_rows(const kvq_tensor* x, const kvq_tensor* slot_mapping,
     if (!flatten_rows(x, &T, &rs)) return KVQ_ERR_LAYOUT;
     const int64_t eb = elem_bytes(x->dtype);
     const int64_t in_bytes = x->shape[x->ndim - 1] * eb;
-    if (in_bytes % 16 != 0 || in_bytes < 16 || in_bytes > 16 * 32 * SC_MAX_CHUNKS_PER_LANE) return KVQ_ERR_SHAPE;
+    if (in_bytes % 16 != 0 || in_bytes < 16 || in_bytes > SB_MAX_ROW_BYTES) return KVQ_ERR_SHAPE;
     if (out_bytes < 16 || out_bytes % 16 != 0 || out_bytes > in_bytes) return KVQ_ERR_ATTR;
     if (!is_index_dtype(slot_mapping->dtype)) return KVQ_ERR_DTYPE;
     if (numel(slot_mapping) != T) return KVQ_ERR_SHAPE;
@@ -1131,18 +1229,13 @@ kvq_status kvq_scatter_rows(const kvq_tensor* x, const kvq_tensor* slot_mapping,
     a.slots = slot_mapping->data;
     a.slots_i64 = slot_mapping->dtype == KVQ_I64;
     a.cache = rows;
-    a.in_chunks = (int32_t)(in_bytes / 16);
-    a.out_chunks = (int32_t)(out_bytes / 16);
-    const int ncl = (a.in_chunks + 31) / 32;
-    const int64_t need = ((T + 1) / 2 + (SC_THREADS / 32) - 1) / (SC_THREADS / 32);
+    a.in_bytes = (int32_t)in_bytes;
+    a.out_bytes = (int32_t)out_bytes;
+    const size_t smem = sb_smem_bytes((int)in_bytes);
+    const int64_t tiles = (T + SB_ROWS - 1) / SB_ROWS;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    auto run = [&](auto kernel) {
-        return launched(launch(kernel, (unsigned)persistent_grid(kernel, SC_THREADS, need), SC_THREADS, 0, s, a));
-    };
-    if (ncl == 1) return run(scatter_copy_kernel<1>);
-    if (ncl == 2) return run(scatter_copy_kernel<2>);
-    if (ncl == 3) return run(scatter_copy_kernel<3>);
-    return run(scatter_copy_kernel<4>);
+    return launched(launch(scatter_bulk_kernel, (unsigned)persistent_grid(scatter_bulk_kernel, SB_THREADS, tiles, smem),
+                           SB_THREADS, smem, s, a));
 }
 
 kvq_status kvq_convert(int32_t fmt, const float* in, int64_t n, void* out, kvq_stream stream) {

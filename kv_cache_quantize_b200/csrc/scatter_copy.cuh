@@ -2,18 +2,21 @@
 // kernels with none of their arithmetic: each valid token's whole input row is
 // read (contiguous rows) and the first out_bytes of it are written to the
 // token's slot row (scattered rows), skipping -1.  It has no counterpart on the
-// pages; it measures what DRAM delivers for this pattern, the ceiling that the
-// compress kernels are compared with.
+// pages; it measures what DRAM delivers for this pattern through the same
+// engine the pipelined compress kernel uses, the ceiling that kernel is
+// compared with.
 //
-// A warp copies two rows per round: lane l loads the 16-byte chunks l, l + 32,
-// ... of both rows (streaming loads, nothing allocated in L1) before storing
-// any, so a warp keeps up to 2 * NCL * 512 bytes in flight.  Chunks past
-// out_bytes are read but not written; they are folded into a per-thread value
-// whose only use is a store that happens when it equals a fixed 128-bit
-// pattern, which keeps the loads without adding work per chunk.
+// A CTA is a producer warp and a storer warp around a ring of SB_STAGES stages
+// of 32 rows.  The producer loads the tile's slots, keeps the destination row
+// pointers beside the stage and brings each valid row in with one 1-D bulk copy
+// (global -> shared, completion counted in bytes on the stage's `full`
+// mbarrier).  The storer sends each row's first out_bytes out with one bulk
+// copy (shared -> global) and releases the stage once the bulk engine has read
+// it.  No thread reads or writes the row data itself.
 #pragma once
 
 #include "kvq_device.cuh"
+#include "tma_pipe.cuh"
 
 namespace kvq {
 
@@ -24,69 +27,102 @@ struct ScatterCopyArgs {
     const void* slots;
     int32_t slots_i64;
     PagedRows cache;             // rows 16-byte aligned
-    int32_t in_chunks;           // bytes read per row / 16
-    int32_t out_chunks;          // bytes written per row / 16 (<= in_chunks)
+    int32_t in_bytes;            // bytes read per row (a multiple of 16)
+    int32_t out_bytes;           // bytes written per row (a multiple of 16, <= in_bytes)
 };
 
-constexpr int SC_THREADS = 256;
-constexpr int SC_MAX_CHUNKS_PER_LANE = 4;      // rows up to 2048 bytes
+constexpr int SB_ROWS = 32;
+constexpr int SB_STAGES = 3;
+constexpr int SB_THREADS = 64;
+constexpr int SB_MAX_ROW_BYTES = 2048;
 
-__device__ uint4 g_scatter_sink;
-
-__device__ __forceinline__ uint4 ld_nc16(const uint8_t* p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
+__host__ __device__ inline uint32_t sb_header_bytes() {
+    return ((uint32_t)(16 * SB_STAGES + 8 * SB_STAGES * SB_ROWS) + 127u) & ~127u;
 }
 
-template <int NCL>
-__global__ void __launch_bounds__(SC_THREADS) scatter_copy_kernel(const ScatterCopyArgs a) {
+__host__ __device__ inline uint32_t sb_smem_bytes(int in_bytes) {
+    return sb_header_bytes() + (uint32_t)SB_STAGES * SB_ROWS * (uint32_t)in_bytes;
+}
+
+// all but the most recent committed bulk store group of this thread have
+// finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all_but_one() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(SB_THREADS) scatter_bulk_kernel(const ScatterCopyArgs a) {
     pdl_wait();
     pdl_trigger();
-    const int lane = threadIdx.x & 31;
-    const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    uint4 sink = make_uint4(0u, 0u, 0u, 0u);
-    for (int64_t r0 = 2 * gwarp; r0 < a.T; r0 += 2 * nwarps) {
-        int64_t s[2];
-        uint4 v[2][NCL];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int64_t row = r0 + u;
-            s[u] = row < a.T ? load_slot(a.slots, a.slots_i64, row) : -1;
-            if (s[u] != -1 && !slot_ok(s[u], a.cache.num_slots)) {
-                if (lane == 0) raise_fault(FAULT_SLOT_RANGE);
-                s[u] = -1;
-            }
-#pragma unroll
-            for (int k = 0; k < NCL; ++k) {
-                const int c = lane + 32 * k;
-                v[u][k] = (s[u] >= 0 && c < a.in_chunks) ? ld_nc16(a.x + row * a.x_row_bytes + 16 * c)
-                                                         : make_uint4(0u, 0u, 0u, 0u);
-            }
+    extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int S = SB_STAGES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + S;
+    uint8_t** rowptr = reinterpret_cast<uint8_t**>(smem + 16 * S);
+    uint8_t* xs = smem + sb_header_bytes();
+    const uint32_t pitch = (uint32_t)a.in_bytes;
+    const uint32_t stage_bytes = SB_ROWS * pitch;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t ntiles = (a.T + SB_ROWS - 1) / SB_ROWS;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < S; ++st) {
+            mbar_init(&full[st], 1);
+            mbar_init(&empty[st], 1);
         }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            if (s[u] < 0) continue;
-            uint8_t* dst = slot_row(a.cache, s[u]);
-#pragma unroll
-            for (int k = 0; k < NCL; ++k) {
-                const int c = lane + 32 * k;
-                if (c < a.out_chunks) {
-                    *reinterpret_cast<uint4*>(dst + 16 * c) = v[u][k];
-                } else {
-                    sink.x ^= v[u][k].x;
-                    sink.y ^= v[u][k].y;
-                    sink.z ^= v[u][k].z;
-                    sink.w ^= v[u][k].w;
-                }
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        auto lane_slot = [&](int64_t tile) -> int64_t {
+            const int64_t r = tile * SB_ROWS + lane;
+            return (tile < ntiles && r < a.T) ? load_slot(a.slots, a.slots_i64, r) : -1;
+        };
+        int it = 0;
+        int64_t next_slot = lane_slot(blockIdx.x);
+        for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+            const int st = it % S;
+            const uint32_t round = (uint32_t)(it / S);
+            const int64_t slot = next_slot;
+            next_slot = lane_slot(tile + gridDim.x);
+            if (!__all_sync(FULL_MASK, mbar_wait(&empty[st], (round & 1u) ^ 1u))) break;
+            uint8_t* p = nullptr;
+            if (slot != -1) {
+                if (slot_ok(slot, a.cache.num_slots)) p = slot_row(a.cache, slot);
+                else raise_fault(FAULT_SLOT_RANGE);
             }
+            rowptr[st * SB_ROWS + lane] = p;
+            const unsigned valid = __ballot_sync(FULL_MASK, p != nullptr);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_expect_tx(&full[st], (uint32_t)__popc(valid) * pitch);
+            __syncwarp();
+            if (p != nullptr)
+                bulk_copy_g2s(xs + (size_t)st * stage_bytes + (size_t)lane * pitch,
+                              a.x + (tile * SB_ROWS + lane) * a.x_row_bytes, pitch, &full[st]);
+        }
+        // no copy may still be in flight when the CTA exits
+        if (lane == 0)
+            for (int k = it > S ? it - S : 0; k < it; ++k) mbar_wait(&full[k % S], (uint32_t)(k / S) & 1u);
+        return;
+    }
+
+    // ---------------- storer ----------------
+    int it = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+        const int st = it % S;
+        const uint32_t round = (uint32_t)(it / S);
+        if (!__all_sync(FULL_MASK, mbar_wait(&full[st], round & 1u))) break;
+        uint8_t* p = rowptr[st * SB_ROWS + lane];
+        if (p != nullptr) bulk_copy_s2g(p, xs + (size_t)st * stage_bytes + (size_t)lane * pitch, (uint32_t)a.out_bytes);
+        bulk_commit();
+        if (it > 0) {
+            bulk_wait_read_all_but_one();             // tile it-1's rows have left its stage
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[(it - 1) % S]);
         }
     }
-    if (sink.x == 0x9e3779b9u && sink.y == 0x7f4a7c15u && sink.z == 0xf39cc060u && sink.w == 0x5cedc834u)
-        g_scatter_sink = sink;
+    bulk_wait_all();                                  // every store is complete before the CTA exits
 }
 
 }  // namespace kvq

@@ -63,6 +63,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
     return false;
 }
 
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait until the phase of the given parity has completed; false (and the
+// FAULT_TIMEOUT bit) once about `ns` nanoseconds have passed without it.  For
+// waits whose legitimate length varies with the problem (a whole GEMM main
+// loop), where a bound in tries would be either too short or far too long.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uint64_t ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > ns) break;
+    }
+    raise_fault(FAULT_TIMEOUT);
+    return false;
+}
+
 // 1-D bulk copy HBM -> this CTA's shared memory.  dst, src 16-byte aligned,
 // bytes a multiple of 16; completion is counted on bar.
 __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {

@@ -317,3 +317,24 @@ def test_check_flag_reports_fault_bits(monkeypatch, L):
         kvq._faults("op", True, 1234)
     kvq._faults("op", False, 1234)
     assert calls == [1234]
+
+
+def test_compressor_validation(L):
+    x, wk, ape, out = D([2048, 1024], "bf16"), D([512, 1024], "bf16"), D([128, 512], "f32"), D([16, 512], "bf16")
+
+    def f(x=x, wk=wk, wg=wk, ape=ape, out=out, ratio=128):
+        return L.kvq_compressor(R(x), R(wk), R(wg), R(ape), R(out), ratio, None)
+    assert f() == ENULL                                              # valid; stops at the NULL data
+    assert f(ratio=96) == EATTR and f(ratio=1) == EATTR and f(ratio=256) == EATTR
+    assert f(x=D([2048, 1024], "f16")) == EDTYPE and f(ape=D([128, 512], "bf16")) == EDTYPE
+    assert f(x=D([2048, 1000], "bf16"), wk=D([512, 1000], "bf16")) == ESHAPE      # H % 512
+    assert f(x=D([2048, 512], "bf16"), wk=D([512, 512], "bf16")) == ESHAPE        # H < 1024
+    assert f(wk=D([256, 1024], "bf16"), wg=D([256, 1024], "bf16"), ape=D([128, 256], "f32"),
+             out=D([16, 256], "bf16")) == ESHAPE                                   # D is 128 or 512
+    assert f(x=D([2000, 1024], "bf16"), out=D([15, 512], "bf16")) == ESHAPE       # T % cmp_ratio
+    assert f(out=D([15, 512], "bf16")) == ESHAPE and f(ape=D([64, 512], "f32")) == ESHAPE
+    assert f(wk=D([512, 1024], "bf16", [2048, 1])) == ELAYOUT
+    assert f(x=D([2, 1024, 1024], "bf16"), out=D([16, 512], "bf16")) == ENULL     # leading dims are tokens
+    assert f(x=D([0, 1024], "bf16"), out=D([0, 512], "bf16")) == OK               # nothing to do
+    assert f(x=D([2048, 1024], "bf16"), wk=D([128, 1024], "bf16"), wg=D([128, 1024], "bf16"),
+             ape=D([128, 128], "f32"), out=D([16, 128], "bf16")) == ENULL          # D = 128
