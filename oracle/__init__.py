@@ -71,7 +71,7 @@ def lib() -> ctypes.CDLL:
         L.kvqo_decode_array.argtypes = [ctypes.c_int, _vp, _i64, _vp]
         L.kvqo_e8m0_ceil_array.argtypes = [_vp, _i64, _vp]
         L.kvqo_int8_static_array.argtypes = [_vp, _i64, _vp]
-        L.kvqo_kv_compress_epilog.argtypes = [_vp, _i64, _i64, _i64, _vp, ctypes.POINTER(_Paged),
+        L.kvqo_kv_compress_epilog.argtypes = [_vp, ctypes.c_int, _i64, _i64, _i64, _vp, ctypes.POINTER(_Paged),
                                               ctypes.c_int, _i64, ctypes.c_float, _vp]
         L.kvqo_indexer_quant_cache.argtypes = [_vp, ctypes.c_int, _i64, _i64, _i64, _vp,
                                                ctypes.POINTER(_Paged), ctypes.c_int,
@@ -81,7 +81,7 @@ def lib() -> ctypes.CDLL:
                                                  ctypes.POINTER(_CacheOut), ctypes.c_float, _vp]
         L.kvqo_dequant_rope_quant_kvcache.argtypes = [ctypes.POINTER(_DrqArgs), _vp]
         L.kvqo_kv_decompress.argtypes = [ctypes.POINTER(_Paged), _vp, _i64, _i64, ctypes.c_int, _i64,
-                                         ctypes.c_float, _vp, _i64, _vp]
+                                         ctypes.c_float, ctypes.c_int, _vp, _i64, _vp]
         _LIB = L
     return _LIB
 
@@ -184,8 +184,10 @@ def _parallel_rows(T: int, threads: int, fn) -> int:
 
 
 def kv_compress_epilog(x_bits: np.ndarray, slot_mapping, cache: Paged, quant_mode: int,
-                       quant_group_size: int = 64, x_scale: float = 1.0, threads: int = 1) -> int:
-    """x_bits: uint16 bf16 bit patterns [..., d].  Updates cache.storage; returns fault bits."""
+                       quant_group_size: int = 64, x_scale: float = 1.0, threads: int = 1,
+                       x_dtype: str = "bf16") -> int:
+    """x_bits: uint16 bit patterns [..., d] of bf16 (or, in quantMode 0/1, f16) values.
+    Updates cache.storage; returns fault bits."""
     x = np.ascontiguousarray(x_bits, dtype=np.uint16)
     d = x.shape[-1]
     T = x.size // d
@@ -196,7 +198,7 @@ def kv_compress_epilog(x_bits: np.ndarray, slot_mapping, cache: Paged, quant_mod
 
     def run(lo, hi):
         faults = np.zeros(1, dtype=np.uint32)
-        rc = lib().kvqo_kv_compress_epilog(x[lo:].ctypes.data, hi - lo, d, d, s[lo:].ctypes.data,
+        rc = lib().kvqo_kv_compress_epilog(x[lo:].ctypes.data, IN_DTYPES[x_dtype], hi - lo, d, d, s[lo:].ctypes.data,
                                            ctypes.byref(pc), quant_mode, quant_group_size,
                                            ctypes.c_float(x_scale), _ptr(faults))
         _check(rc, "kv_compress_epilog")
@@ -205,10 +207,10 @@ def kv_compress_epilog(x_bits: np.ndarray, slot_mapping, cache: Paged, quant_mod
 
 
 def kv_decompress(cache: Paged, slot_mapping, d: int, quant_mode: int, quant_group_size: int = 64,
-                  x_scale: float = 1.0, y: Optional[np.ndarray] = None, threads: int = 1):
-    """Decode the packed rows named by slot_mapping into bf16 bit patterns y [T, d]
-    (rows of skipped tokens keep y's initial contents, zeros by default).
-    Returns (y, fault bits)."""
+                  x_scale: float = 1.0, y: Optional[np.ndarray] = None, threads: int = 1, y_dtype: str = "bf16"):
+    """Decode the packed rows named by slot_mapping into bit patterns y [T, d] of bf16
+    (or f16 in quantMode 0/1: the dtype of the compressed x) values; rows of skipped
+    tokens keep y's initial contents, zeros by default.  Returns (y, fault bits)."""
     s = _slots(slot_mapping)
     T = s.size
     if y is None:
@@ -219,7 +221,8 @@ def kv_decompress(cache: Paged, slot_mapping, d: int, quant_mode: int, quant_gro
     def run(lo, hi):
         faults = np.zeros(1, dtype=np.uint32)
         rc = lib().kvqo_kv_decompress(ctypes.byref(pc), s[lo:].ctypes.data, hi - lo, d, quant_mode,
-                                      quant_group_size, ctypes.c_float(x_scale), y[lo:].ctypes.data, d,
+                                      quant_group_size, ctypes.c_float(x_scale), IN_DTYPES[y_dtype],
+                                      y[lo:].ctypes.data, d,
                                       _ptr(faults))
         _check(rc, "kv_decompress")
         return int(faults[0])

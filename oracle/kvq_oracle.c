@@ -302,7 +302,8 @@ int64_t kvqo_kv_cache_col(int64_t d, int quant_mode, int64_t group_size)
 }
 
 /*
- * One token row (d elements, bf16) -> packed cache row of kvCacheCol bytes.
+ * One token row (d elements, bf16, or f16 in modes 0/1) -> packed cache row
+ * of kvCacheCol bytes.
  *
  * Formula ([EPI] 计算公式):
  *   mode 0: groups of 64 over the nope columns [0, d-64):
@@ -320,10 +321,13 @@ int64_t kvqo_kv_cache_col(int64_t d, int quant_mode, int64_t group_size)
  * replaced by FP8 E4M3; the 2-byte scales are bfloat16.
  * Row layout (parity unpinned: a convention): [nope codes][rope][scales]
  * then zero bytes up to kvCacheCol.  FP4 codes two per byte, the even
- * element in the low nibble.
+ * element in the low nibble.  In modes 0/1 the rope columns are kept
+ * unchanged: their 16-bit input values (bf16 or f16, `raw`) are copied,
+ * little-endian; the 2-byte scale of mode 0 is bfloat16 whatever x's dtype
+ * (the page names the mode "group (bf16 scale)").
  */
-static void compress_row(const float* x, int64_t d, int quant_mode, int64_t G, float x_scale,
-                         uint8_t* row, int64_t col)
+static void compress_row(const float* x, const uint16_t* raw, int64_t d, int quant_mode, int64_t G,
+                         float x_scale, uint8_t* row, int64_t col)
 {
     const int64_t n = d - 64;
     memset(row, 0, (size_t)col);
@@ -349,9 +353,9 @@ static void compress_row(const float* x, int64_t d, int quant_mode, int64_t G, f
                 for (int64_t i = 0; i < 64; ++i) row[64 * g + i] = enc_e4m3(xg[i] * mul);
             }
         }
-        /* rope columns copied unchanged as bf16, little-endian */
+        /* rope columns copied unchanged (the input's own 16-bit values), little-endian */
         for (int64_t j = 0; j < 64; ++j) {
-            uint16_t h = f32_to_bf16(x[n + j]);   /* exact: x[n+j] is a bf16 value */
+            uint16_t h = raw[n + j];
             row[n + 2 * j + 0] = (uint8_t)(h & 0xFF);
             row[n + 2 * j + 1] = (uint8_t)(h >> 8);
         }
@@ -377,11 +381,13 @@ static void compress_row(const float* x, int64_t d, int quant_mode, int64_t G, f
     }
 }
 
-int kvqo_kv_compress_epilog(const uint16_t* x, int64_t T, int64_t d, int64_t x_row_stride,
+int kvqo_kv_compress_epilog(const uint16_t* x, int x_dtype, int64_t T, int64_t d, int64_t x_row_stride,
                             const int64_t* slot_mapping, const kvqo_paged* cache, int quant_mode,
                             int64_t quant_group_size, float x_scale, uint32_t* faults)
 {
     if (d <= 64 || d % 64 != 0 || d > 8192) return KVQO_EINVAL;
+    if (x_dtype != KVQO_IN_BF16 && x_dtype != KVQO_IN_F16) return KVQO_EINVAL;
+    if (quant_mode == 2 && x_dtype != KVQO_IN_BF16) return KVQO_EINVAL;   /* mode 2 needs bf16 x */
     if (quant_mode == 2) {
         if (quant_group_size != 16 && quant_group_size != 32 && quant_group_size != 64) return KVQO_EINVAL;
         if ((d - 64) % quant_group_size != 0) return KVQO_EINVAL;
@@ -395,8 +401,8 @@ int kvqo_kv_compress_epilog(const uint16_t* x, int64_t T, int64_t d, int64_t x_r
         int64_t s = slot_mapping[t];
         if (s == -1) continue;                               /* skipped token */
         if (s < 0 || s >= num_slots(cache)) { *faults |= KVQO_FAULT_SLOT_RANGE; continue; }
-        for (int64_t i = 0; i < d; ++i) xf[i] = bf16_to_f32(x[t * x_row_stride + i]);
-        compress_row(xf, d, quant_mode, quant_group_size, x_scale, row, col);
+        for (int64_t i = 0; i < d; ++i) xf[i] = load_half(x + t * x_row_stride, i, x_dtype);
+        compress_row(xf, x + t * x_row_stride, d, quant_mode, quant_group_size, x_scale, row, col);
         memcpy(slot_row(cache, s), row, (size_t)col);
     }
     free(xf);
@@ -419,7 +425,10 @@ int kvqo_kv_compress_epilog(const uint16_t* x, int64_t T, int64_t d, int64_t x_r
 /* Readings: the pages define only the encoding; decoding with the stored   */
 /* scale and one rounding to bf16 is the plain inverse.                     */
 /* ------------------------------------------------------------------------ */
-static void decompress_row(const uint8_t* row, int64_t d, int quant_mode, int64_t G, float x_scale, uint16_t* y)
+static uint16_t round_out(int y_dtype, float v) { return y_dtype == KVQO_IN_F16 ? f32_to_f16(v) : f32_to_bf16(v); }
+
+static void decompress_row(const uint8_t* row, int64_t d, int quant_mode, int64_t G, float x_scale, int y_dtype,
+                           uint16_t* y)
 {
     const int64_t n = d - 64;
     if (quant_mode == 0 || quant_mode == 1) {
@@ -434,7 +443,7 @@ static void decompress_row(const uint8_t* row, int64_t d, int quant_mode, int64_
             }
             for (int64_t i = 0; i < 64; ++i) {
                 float v = decode_bits(&FMT_E4M3, row[64 * g + i]);
-                y[64 * g + i] = f32_to_bf16(v * sf);
+                y[64 * g + i] = round_out(y_dtype, v * sf);
             }
         }
         for (int64_t j = 0; j < 64; ++j) y[n + j] = (uint16_t)(row[n + 2 * j] | (row[n + 2 * j + 1] << 8));
@@ -455,13 +464,17 @@ static void decompress_row(const uint8_t* row, int64_t d, int quant_mode, int64_
 }
 
 /* Decode the rows of slot_mapping into y [T, d] (row stride y_row_stride   */
-/* elements).  Tokens whose slot is -1 leave their y row untouched; other   */
-/* slots outside the cache also leave it and raise the fault bit.           */
+/* elements; bf16, or f16 in modes 0/1 -- the dtype of the x that was       */
+/* compressed, whose rope bytes the row holds).  Tokens whose slot is -1    */
+/* leave their y row untouched; other slots outside the cache also leave it */
+/* and raise the fault bit.                                                 */
 int kvqo_kv_decompress(const kvqo_paged* cache, const int64_t* slot_mapping, int64_t T, int64_t d,
-                       int quant_mode, int64_t quant_group_size, float x_scale, uint16_t* y,
+                       int quant_mode, int64_t quant_group_size, float x_scale, int y_dtype, uint16_t* y,
                        int64_t y_row_stride, uint32_t* faults)
 {
     if (d <= 64 || d % 64 != 0 || d > 8192) return KVQO_EINVAL;
+    if (y_dtype != KVQO_IN_BF16 && y_dtype != KVQO_IN_F16) return KVQO_EINVAL;
+    if (quant_mode == 2 && y_dtype != KVQO_IN_BF16) return KVQO_EINVAL;
     if (quant_mode < 0 || quant_mode > 2) return KVQO_EINVAL;
     if (quant_mode == 2) {
         if (quant_group_size != 16 && quant_group_size != 32 && quant_group_size != 64) return KVQO_EINVAL;
@@ -473,7 +486,7 @@ int kvqo_kv_decompress(const kvqo_paged* cache, const int64_t* slot_mapping, int
         int64_t s = slot_mapping[t];
         if (s == -1) continue;
         if (s < 0 || s >= num_slots(cache)) { *faults |= KVQO_FAULT_SLOT_RANGE; continue; }
-        decompress_row(slot_row(cache, s), d, quant_mode, quant_group_size, x_scale, y + t * y_row_stride);
+        decompress_row(slot_row(cache, s), d, quant_mode, quant_group_size, x_scale, y_dtype, y + t * y_row_stride);
     }
     return KVQO_OK;
 }

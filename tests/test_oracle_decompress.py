@@ -162,3 +162,38 @@ def test_decoded_codes_follow_the_format_tables():
         want = np.array([code_value("e4m3", int(c)) * 3.0 for c in chunk])
         got = _bits_to_f64(y[0, :len(chunk)])
         assert np.array_equal(got, _bits_to_f64(W.to_bf16_bits(want.astype(np.float32)))), c0
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_f16_roundtrip_keeps_the_rope_and_bounds_the_codes(mode):
+    """float16 x (quantMode 0/1): decoding into float16 gives back the rope bit for bit
+    (it is stored unchanged) and every nope value within half a code step in its group's
+    scale plus half an f16 ulp; exactly representable rows come back exactly."""
+    T, d = 120, 320
+    rng = np.random.default_rng(40 + mode)
+    xf = (rng.standard_normal((T, d)) * 20).astype(np.float16)
+    x_bits = xf.view(np.uint16)
+    slots = rng.choice(2 * T, T, replace=False).astype(np.int32)
+    slots[::9] = -1
+    cache = _cache_for(T, d, mode, 64, seed=5)
+    st = cache.storage.copy()
+    assert oracle.kv_compress_epilog(x_bits, slots, paged(cache, st), mode, 64, 1.0, x_dtype="f16") == 0
+    y, f = oracle.kv_decompress(paged(cache, st), slots, d, mode, 64, 1.0, y_dtype="f16")
+    assert f == 0
+    live = slots != -1
+    n = d - 64
+    assert np.array_equal(y[live, n:], x_bits[live, n:])
+    x = xf.astype(np.float64)
+    yv = y.view(np.float16).astype(np.float64)
+    amax = np.abs(x[:, :n]).reshape(T, n // 64, 64).max(axis=2)
+    if mode == 1:
+        scale = 2.0 ** np.ceil(np.log2(np.maximum(amax / 448.0, 2.0 ** -127)))
+    else:
+        scale = _bits_to_f64(W.to_bf16_bits((amax / 448.0).astype(np.float32)))
+    s = np.repeat(scale, 64, axis=1)
+    v = np.where(s > 0, x[:, :n] / s, 0.0)
+    bound = s * _half_step("e4m3", v) * (1 + 2.0 ** -20) + np.abs(yv[:, :n]) * 2.0 ** -11
+    assert np.all(np.abs(yv[:, :n] - x[:, :n])[live] <= bound[live])
+    # and the decoder refuses float16 output in quantMode 2 (bfloat16 x only there)
+    with pytest.raises(Exception):
+        oracle.kv_decompress(paged(cache, st), slots, d, 2, 32, 0.1, y_dtype="f16")

@@ -54,7 +54,8 @@ MUTANTS = {
         "const float fmax = quant_mode == KVQO_IDX_MXFP8 ? fp8_max : 6.0f;",
         "const float fmax = quant_mode == KVQO_IDX_MXFP8 ? 6.0f : fp8_max;"),
     "bf16 ties away from zero": ("return nearbyint(k) * quantum;", "return floor(k + 0.5) * quantum;"),
-    "decoder drops the group scale": ("y[64 * g + i] = f32_to_bf16(v * sf);", "y[64 * g + i] = f32_to_bf16(v);"),
+    "decoder drops the group scale": ("y[64 * g + i] = round_out(y_dtype, v * sf);",
+                                      "y[64 * g + i] = round_out(y_dtype, v);"),
     "decoder multiplies the rope by xScale": (
         "y[n + j] = f32_to_bf16(decode_bits(&FMT_E4M3, rope[j]) / x_scale);",
         "y[n + j] = f32_to_bf16(decode_bits(&FMT_E4M3, rope[j]) * x_scale);"),
@@ -62,6 +63,12 @@ MUTANTS = {
         "uint32_t c = (row[e / 2] >> (4 * (e % 2))) & 0xFu;", "uint32_t c = (row[e / 2] >> (4 * (1 - e % 2))) & 0xFu;"),
     "decoder E8M0 exponent bias": ("sf = (float)ldexp(1.0, (int)scales[g] - 127);",
                                    "sf = (float)ldexp(1.0, (int)scales[g] - 126);"),
+    "rope re-encoded as bf16 instead of copied": ("uint16_t h = raw[n + j];", "uint16_t h = f32_to_bf16(x[n + j]);"),
+    "f16 x read as bf16": ("xf[i] = load_half(x + t * x_row_stride, i, x_dtype);",
+                           "xf[i] = load_half(x + t * x_row_stride, i, KVQO_IN_BF16);"),
+    "decoder rounds f16 output as bf16": (
+        "static uint16_t round_out(int y_dtype, float v) { return y_dtype == KVQO_IN_F16 ? f32_to_f16(v) : f32_to_bf16(v); }",
+        "static uint16_t round_out(int y_dtype, float v) { return y_dtype == KVQO_IN_F16 ? f32_to_bf16(v) : f32_to_bf16(v); }"),
 }
 
 

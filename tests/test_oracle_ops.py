@@ -56,11 +56,13 @@ def test_layout_sizes_printed_and_closed_form():
 def test_compress_worked_rows(name):
     c = WORKED[name]
     d, n = int(c["d"]), int(c["row_len"])
-    x = bf16_bits(expand(c["x"], d))[None, :]
+    xdt = c.get("x_dtype", "bf16")
+    vals = expand(c["x"], d)
+    x = (bf16_bits(vals) if xdt == "bf16" else np.asarray(vals, dtype=np.float16).view(np.uint16))[None, :]
     cache = filled_cache(1, 2, n + 16)
     st = cache.storage.copy()
     f = oracle.kv_compress_epilog(x, [1], oracle.Paged(st, cache.offset, 1, 2, n + 16, 2 * (n + 16)),
-                                  int(c["mode"]), int(c["G"]), float(c["x_scale"]))
+                                  int(c["mode"]), int(c["G"]), float(c["x_scale"]), x_dtype=xdt)
     assert f == 0
     assert oracle.kv_cache_col(d, int(c["mode"]), int(c["G"])) == n
     row = row_view(cache, st, 1, n + 16)
@@ -628,3 +630,34 @@ def test_half_rotation_rope_with_unequal_cos_sin_halves():
     want = u * c + np.concatenate([-u[..., h:], u[..., :h]], -1) * s
     np.testing.assert_allclose(bf16_value(outs["q_out"]).reshape(-1, Nq, D), want[:, :Nq], rtol=1e-2, atol=1e-4)
     np.testing.assert_allclose(bf16_value(outs["k_out"]).reshape(-1, Nkv, D), want[:, Nq:], rtol=1e-2, atol=1e-4)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_compress_f16_rope_bytes_are_the_input_bytes(mode):
+    """aclnnKvCompressEpilog keeps the rope segment unchanged: with float16 x (allowed in
+    quantMode 0 and 1) the rope bytes of every written row are x's own 16-bit values."""
+    T, d = 40, 320
+    rng = np.random.default_rng(mode)
+    x = (rng.standard_normal((T, d)) * 3).astype(np.float16).view(np.uint16)
+    col = oracle.kv_cache_col(d, mode, 64)
+    cache = filled_cache(8, 8, col + 3)
+    st = cache.storage.copy()
+    slots = rng.choice(64, T, replace=False).astype(np.int32)
+    slots[::7] = -1
+    assert oracle.kv_compress_epilog(x, slots, oracle.Paged(st, cache.offset, 8, 8, col + 3, 8 * (col + 3)), mode,
+                                     64, 1.0, x_dtype="f16") == 0
+    n = d - 64
+    for t, s in enumerate(slots.tolist()):
+        if s < 0:
+            continue
+        row = row_view(cache, st, s, col)
+        assert bytes(row[n:n + 128]) == x[t, n:].tobytes()
+
+
+def test_compress_f16_is_refused_in_mode_2():
+    """quantMode 2 needs bfloat16 x (aclnnKvCompressEpilog, 约束说明)."""
+    cache = filled_cache(1, 2, 352)
+    x = np.zeros((1, 576), dtype=np.uint16)
+    with pytest.raises(Exception):
+        oracle.kv_compress_epilog(x, [0], oracle.Paged(cache.storage.copy(), cache.offset, 1, 2, 352, 704), 2, 32,
+                                  0.1, x_dtype="f16")
