@@ -100,8 +100,9 @@ typedef enum {
 /* kv_compress_epilog                                                        */
 /* Source: aclnnKvCompressEpilog, 接口功能 / 计算公式 / 约束说明.               */
 /*                                                                           */
-/* x            bf16 [..., d]; the last dimension contiguous, the leading     */
-/*              dimensions flattenable to T rows with one row stride.         */
+/* x            bf16 [..., d] (f16 also in quant_mode 0/1: the page requires  */
+/*              bf16 only in mode 2); the last dimension contiguous, the      */
+/*              leading dimensions flattenable to T rows with one row stride. */
 /*              64 < d <= 8192, d % 64 == 0.  Columns [0, d-64) are the nope  */
 /*              segment, [d-64, d) the rope segment.                          */
 /* slot_mapping int32 or int64, T elements (x's leading dims flattened),     */
@@ -121,7 +122,9 @@ typedef enum {
 /* Codes are round-to-nearest-even with saturation of x divided by the       */
 /* STORED scale; a stored bf16 scale of 0 gives all-zero codes.              */
 /* Packed row (kvCacheCol bytes, written from byte 0 of the slot row):       */
-/*   modes 0/1: [d-64 code bytes][64 bf16 rope values][(d-64)/64 scales]     */
+/*   modes 0/1: [d-64 code bytes][the 64 rope values as given: bf16 or f16   */
+/*              bytes][(d-64)/64 scales: bf16 (mode 0, whatever x's dtype)   */
+/*              or E8M0 (mode 1)]                                            */
 /*   mode 2:    [(d-64)/2 bytes of FP4 pairs, even element in the low nibble] */
 /*              [64 E4M3 rope codes][(d-64)/G bf16 scales]                   */
 /*   then 0x00 up to kvCacheCol (32-byte alignment in modes 0 and 2).        */
@@ -143,9 +146,12 @@ KVQ_API kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor*
 /*              output row; -1 leaves the row untouched.                      */
 /* y            bf16 [..., d] (the last dimension contiguous, the leading     */
 /*              dimensions flattenable to T rows with one row stride),        */
-/*              written row by row:                                           */
-/*   modes 0/1: nope y = bf16_rn(code value * group scale) (the bf16 scale,  */
-/*              or 2^(b-127) for the E8M0 byte b); rope = the stored bf16;   */
+/*              written row by row; in modes 0/1 y may be f16 instead, for    */
+/*              rows compressed from f16 x (y's dtype must be x's: the rope   */
+/*              is stored as x's own 16-bit values):                          */
+/*   modes 0/1: nope y = round_to_y(code value * group scale) (the bf16      */
+/*              scale, or 2^(b-127) for the E8M0 byte b); rope = the stored  */
+/*              16-bit values;                                                */
 /*   mode 2:    nope y = bf16_rn(E2M1 value * group scale); rope =           */
 /*              bf16_rn(E4M3 value / x_scale) (IEEE division).                */
 /* Validation as kv_compress_epilog; a slot outside the cache leaves its row */
@@ -327,7 +333,11 @@ KVQ_API kvq_status kvq_convert(int32_t fmt, const float* in, int64_t n, void* ou
  * format) cases, among 2^28 random bf16 / f16 pairs with |value| <= maximum,
  * each encoded as E4M3 and as E5M2, whose code from the indexer fp8 mode's
  * two-step quotient by maximum / FP8_MAX differs from the code of the IEEE
- * quotient.  Blocks until done; *result receives the count (0 means the
+ * quotient; 9: the number of (x, rms) pairs, among 2^28 random ones inside
+ * the rmsnorm kernel's guard (rms in [2^-60, 2^50], x a bf16 value with |x| >=
+ * max(RN(rms 2^-125), 2^-103), half of them within a few ulps of a rounding
+ * tie), whose unscaled two-step quotient x / rms differs in any bit from IEEE
+ * division.  Blocks until done; *result receives the count (0 means the
  * shortcut is exact on the domain). */
 KVQ_API kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream);
 

@@ -1,7 +1,8 @@
 // compress_epilog.cuh -- kv_compress_epilog kernel (aclnnKvCompressEpilog,
 // 计算公式 scenarios 1-3 and 约束说明 for the packed-row size).
 //
-// Work decomposition.  A row of d bf16 values is d/64 SEGMENTS of 64 values:
+// Work decomposition.  A row of d 16-bit values (bf16; f16 is accepted in
+// modes 0/1, whose rope is copied as it is) is d/64 SEGMENTS of 64 values:
 // the (d-64)/64 nope segments and the rope segment last.  A segment is handled
 // by a TEAM of 8 lanes, each lane one 16-byte chunk of 8 values, so a warp
 // works on 4 segments at a time and a 64-value quantisation group is one team
@@ -21,7 +22,7 @@
 namespace kvq {
 
 struct CompressArgs {
-    const uint16_t* x;      // bf16 bit patterns
+    const uint16_t* x;      // bf16 bit patterns (f16 in modes 0/1 when the kernel's F16 is set)
     int64_t x_row_stride;   // elements
     int64_t T;              // rows
     const void* slots;      // int32 or int64
@@ -82,7 +83,7 @@ __device__ __forceinline__ void div_by_scale8(const float (&f)[8], float sf, flo
 // One segment of 64 values, one 16-byte chunk per lane of an 8-lane team.
 // All lanes call this (the shuffles need the whole warp); row == nullptr for
 // lanes whose segment is inactive or whose token is skipped.
-template <int MODE, int G>
+template <int MODE, int G, bool F16>
 __device__ __forceinline__ void ce_segment(const CompressArgs& a, const uint4& v, uint8_t* row, int j, int sub) {
     constexpr int GL = (MODE == 2 ? G : 64) / 8;   // lanes per quantisation group
     uint32_t m = absmax_bits8(v);
@@ -93,8 +94,8 @@ __device__ __forceinline__ void ce_segment(const CompressArgs& a, const uint4& v
 
     const bool rope = (j == a.nseg - 1);
     float f[8];
-    widen8<false>(v, f);
-    const float amax = __uint_as_float(m << 16);
+    widen8<F16>(v, f);
+    const float amax = half_value<F16>(m);
 
     if (MODE == 0) {
         if (!rope) {
@@ -150,7 +151,7 @@ __device__ __forceinline__ void ce_segment(const CompressArgs& a, const uint4& v
     }
 }
 
-template <int MODE, int G>
+template <int MODE, int G, bool F16>
 __global__ void __launch_bounds__(CE_THREADS) compress_epilog_kernel(const CompressArgs a) {
     pdl_wait();
     pdl_trigger();
@@ -195,7 +196,7 @@ __global__ void __launch_bounds__(CE_THREADS) compress_epilog_kernel(const Compr
             }
 #pragma unroll
             for (int u = 0; u < CE_UNROLL; ++u)
-                ce_segment<MODE, G>(a, v[u], live[u] ? slot_row(a.cache, sl[u]) : nullptr, jj[u], sub);
+                ce_segment<MODE, G, F16>(a, v[u], live[u] ? slot_row(a.cache, sl[u]) : nullptr, jj[u], sub);
         }
     }
 }
@@ -222,12 +223,14 @@ __host__ __device__ inline uint32_t ct_pitch(int nseg) { return (uint32_t)nseg *
 
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
 
-// |x| maximum of the bf16 values of nchunks 16-byte chunks (as bits)
+// |x| maximum of the bf16 (or f16) values of nchunks 16-byte chunks (as bits)
+template <bool F16>
 __device__ __forceinline__ uint32_t seg_absmax_bits(const uint8_t* seg, int nchunks) {
     uint32_t m2 = 0u;
     for (int k = 0; k < nchunks; ++k) {
         const uint4 v = lds128(seg + 16 * k);
-        m2 = absmax_bf16x2(m2, absmax_bf16x2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w)));
+        if (F16) m2 = absmax_f16x2(m2, absmax_f16x2(absmax_f16x2(v.x, v.y), absmax_f16x2(v.z, v.w)));
+        else m2 = absmax_bf16x2(m2, absmax_bf16x2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w)));
     }
     m2 &= 0x7fff7fffu;
     return max(m2 & 0xffffu, m2 >> 16);
@@ -266,10 +269,10 @@ __device__ __forceinline__ int seg_words(bool rope) {
     return MODE == 2 ? 8 : 16;
 }
 
-template <int MODE, int G>
+template <int MODE, int G, bool F16>
 __device__ __forceinline__ void ct_compute_nope(const uint8_t* seg, SegOut& o) {
     if (MODE == 0 || MODE == 1) {
-        const float amax = __uint_as_float(seg_absmax_bits(seg, 8) << 16);
+        const float amax = half_value<F16>(seg_absmax_bits<F16>(seg, 8));
         float sf, r = 0.0f;
         bool fast = true;
         if (MODE == 0) {
@@ -284,7 +287,7 @@ __device__ __forceinline__ void ct_compute_nope(const uint8_t* seg, SegOut& o) {
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
             float f[8], q[8];
-            widen8<false>(lds128(seg + 16 * k), f);
+            widen8<F16>(lds128(seg + 16 * k), f);
             if (MODE == 1) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(f[i], sf);
@@ -311,7 +314,7 @@ __device__ __forceinline__ void ct_compute_nope(const uint8_t* seg, SegOut& o) {
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
             const uint8_t* gseg = seg + g * G * 2;
-            const float amax = __uint_as_float(seg_absmax_bits(gseg, GC) << 16);
+            const float amax = __uint_as_float(seg_absmax_bits<false>(gseg, GC) << 16);
             sb[g] = to_bf16_bits(div_by_fmax(amax, 6.0f));
             const float sf = __uint_as_float(sb[g] << 16);
             const bool fast = scale_in_fast_range(sf);
@@ -427,7 +430,7 @@ __host__ __device__ inline uint32_t ct_out_pitch(int col) { return (uint32_t)(((
 // S: the number of input stages (a.stages holds the same value), a template
 // parameter so that the ring's stage and phase arithmetic folds to constants
 // (measured 3 % faster on the mode-2 row kernel than reading it at run time).
-template <int MODE, int G, int S>
+template <int MODE, int G, int S, bool F16 = false>
 __global__ void __launch_bounds__(CT_MAX_THREADS, 1) compress_tma_kernel(const CompressArgs a) {
     static_assert(S == 2 || S == 3, "stages");
     pdl_wait();
@@ -519,7 +522,7 @@ __global__ void __launch_bounds__(CT_MAX_THREADS, 1) compress_tma_kernel(const C
             uint8_t* orow = obuf + (size_t)lane * opitch;
             SegOut o;
             if (row != nullptr) {
-                if (!rope) ct_compute_nope<MODE, G>(xrow + j * 128, o);
+                if (!rope) ct_compute_nope<MODE, G, F16>(xrow + j * 128, o);
                 else if (MODE == 2) ct_compute_rope2(a, xrow + j * 128, o);
             }
             if (rope) {
@@ -559,7 +562,7 @@ __global__ void __launch_bounds__(CT_MAX_THREADS, 1) compress_tma_kernel(const C
             for (int j = warp; j < a.nseg; j += NCW) {
                 const bool rope = (j == a.nseg - 1);
                 SegOut o;
-                if (!rope) ct_compute_nope<MODE, G>(xrow + j * 128, o);
+                if (!rope) ct_compute_nope<MODE, G, F16>(xrow + j * 128, o);
                 else if (MODE == 2) ct_compute_rope2(a, xrow + j * 128, o);
                 ct_write<MODE, G, false>(a, row, j, rope, o, xrow + j * 128, aligned);
             }

@@ -1,17 +1,24 @@
 // kv_decompress.cuh -- packed-row decoder: the inverse of kv_compress_epilog
 // (aclnnKvCompressEpilog, 计算公式 scenarios 1-3 and the row layout of its
 // 约束说明, read backwards: code value x stored group scale, one rounding to
-// bf16; the bf16 rope of modes 0/1 is copied, the FP8 rope of mode 2 is
-// divided by xScale).
+// bf16 -- or to f16 in modes 0/1 for rows written from f16 x; the 16-bit rope
+// of modes 0/1 is copied, the FP8 rope of mode 2 is divided by xScale).
 //
 // Work decomposition.  A row of d values is d/32 SLICES of 32 values: the
-// (d-64)/32 nope slices, then the two rope slices.  One lane owns one slice:
-// it reads the slice's codes (32 bytes FP8 or 16 bytes FP4) and its group's
-// scale from the packed row, and writes the slice's 64 bytes of bf16 output.
-// A warp takes 32 consecutive slices of the flattened [T, d/32] slice array,
-// so a warp's stores cover one contiguous stretch of y.  Grid-stride over
-// those 32-slice chunks, software-pipelined: the slots of chunk i+2 and the
-// packed bytes of chunk i+1 are in flight while chunk i is decoded.
+// nn = (d-64)/32 nope slices (nn is even), then the two rope slices.  One
+// lane owns one slice: it reads the slice's codes (32 bytes FP8 or 16 bytes
+// FP4) and its group's scale from the packed row, and writes the slice's 64
+// bytes of 16-bit output.  A warp takes a CHUNK of 32 slices:
+//   modes 0/1: 32 consecutive slices of the flattened [T, d/32] slice array,
+//     so a warp's stores cover one contiguous stretch of y (the rope is a
+//     plain copy, as cheap as a nope slice);
+//   mode 2: rows in blocks of 16, whose 16 nn nope slices form nn/2 chunks
+//     (row-major) and whose 32 rope slices one more chunk, so every chunk is
+//     all nope or all rope and the decode path is uniform across the warp
+//     (the rope's table lookups and the FP4 path would otherwise run one
+//     after the other in every warp that holds both).
+// Grid-stride over the chunks, software-pipelined: the slots of chunk i+2 and
+// the packed bytes of chunk i+1 are in flight while chunk i is decoded.
 #pragma once
 
 #include "kvq_device.cuh"
@@ -25,7 +32,7 @@ struct DecompressArgs {
     const void* slots;      // int32 or int64
     int32_t slots_i64;
     int64_t T;
-    uint16_t* y;            // bf16 [T, d], row stride y_row_stride elements
+    uint16_t* y;            // bf16 (or f16, modes 0/1) [T, d], row stride y_row_stride elements
     int64_t y_row_stride;
     int32_t nslice;         // d / 32
     int32_t n;              // d - 64
@@ -79,6 +86,18 @@ __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
     return r;
 }
 
+__device__ __forceinline__ uint32_t f16x2_rn(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// the output pair in y's dtype (YF16: f16, modes 0/1 only; else bf16)
+template <bool YF16>
+__device__ __forceinline__ uint32_t out_x2(float lo, float hi) {
+    return YF16 ? f16x2_rn(lo, hi) : bf16x2_rn(lo, hi);
+}
+
 // 2^(b-127) for an E8M0 byte b (b = 0: the subnormal 2^-127; b = 255: inf)
 __device__ __forceinline__ float e8m0_value(uint32_t b) {
     return b == 0 ? __uint_as_float(0x00400000u) : __uint_as_float(b << 23);
@@ -86,7 +105,7 @@ __device__ __forceinline__ float e8m0_value(uint32_t b) {
 
 // one slice of a live row: decode w (codes, or the stored rope) with scale bits sc
 // rope_tab (mode 2): bf16_rn(E4M3 value / xScale) for each of the 256 codes
-template <int MODE, int G>
+template <int MODE, int G, bool YF16>
 __device__ __forceinline__ void dc_slice(const DecompressArgs& a, int nn, const uint32_t (&w)[16], uint32_t sc,
                                          int j, uint16_t* yrow, const uint16_t* rope_tab) {
     uint32_t out[16];
@@ -108,7 +127,7 @@ __device__ __forceinline__ void dc_slice(const DecompressArgs& a, int nn, const 
         for (int k = 0; k < 16; ++k) {
             float lo, hi;
             e4m3x2_to_f32(w[k >> 1] >> (16 * (k & 1)), lo, hi);
-            out[k] = bf16x2_rn(__fmul_rn(lo, sf), __fmul_rn(hi, sf));
+            out[k] = out_x2<YF16>(__fmul_rn(lo, sf), __fmul_rn(hi, sf));
         }
     } else {
         // 16 bytes of FP4 codes; G = 16: two scales (sc low half first), else one
@@ -168,8 +187,8 @@ __device__ __forceinline__ const uint8_t* dc_row(const DecompressArgs& a, int64_
 
 // NS: slices per row (d / 32) when known at compile time (18: d = 576), else 0
 // and a.nslice; the constant form measured 11 % faster in mode 0 at d = 576.
-template <int MODE, int G, int NS>
-__global__ void __launch_bounds__(DC_THREADS) kv_decompress_kernel(const DecompressArgs a) {
+template <int MODE, int G, int NS, bool YF16 = false>
+__global__ void __launch_bounds__(DC_THREADS, (MODE == 2 || NS != 0) ? 4 : 3) kv_decompress_kernel(const DecompressArgs a) {
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
@@ -177,7 +196,7 @@ __global__ void __launch_bounds__(DC_THREADS) kv_decompress_kernel(const Decompr
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int ns = NS ? NS : a.nslice;
     const int nn = ns - 2;
-    const int64_t nchunks = (a.T * ns + 31) / 32;
+    const int64_t nchunks = MODE == 2 ? ((a.T + 15) / 16) * (nn / 2 + 1) : (a.T * ns + 31) / 32;
     // mode 2: the decoded rope value of every E4M3 code, one IEEE division each
     __shared__ uint16_t rope_tab[MODE == 2 ? 256 : 1];
     if (MODE == 2) {
@@ -189,10 +208,10 @@ __global__ void __launch_bounds__(DC_THREADS) kv_decompress_kernel(const Decompr
         __syncthreads();
     }
     if (gwarp >= nchunks) return;
-    // the lane's slice (row, j) in chunk c, and its step from chunk c to c + nwarps
-    const int64_t hs = gwarp * 32 + lane;
-    int64_t row0 = hs / ns;
-    int j0 = (int)(hs - row0 * ns);
+    // the lane's slice (row, j) in chunk c: modes 0/1 step through the flat
+    // slice array (chunk c + nwarps is nwarps * 32 slices further, added
+    // without a division); mode 2 locates it in its 16-row block
+    const int hn = nn / 2;                      // mode 2: nope chunks per block of 16 rows
     const int64_t step = nwarps * 32;
     const int64_t qs = step / ns;
     const int rs = (int)(step - qs * ns);
@@ -204,9 +223,31 @@ __global__ void __launch_bounds__(DC_THREADS) kv_decompress_kernel(const Decompr
             ++r;
         }
     };
-    int64_t row1 = row0;
-    int j1 = j0;
-    advance(row1, j1);
+    auto locate = [&](int64_t c, int64_t& r, int& j) {
+        const int64_t blk = c / (hn + 1);
+        const int w = (int)(c - blk * (hn + 1));
+        if (w < hn) {
+            const int sl = 32 * w + lane;
+            r = 16 * blk + sl / nn;
+            j = sl - (sl / nn) * nn;
+        } else {
+            r = 16 * blk + (lane >> 1);
+            j = nn + (lane & 1);
+        }
+    };
+    int64_t row0, row1;
+    int j0, j1;
+    if (MODE == 2) {
+        locate(gwarp, row0, j0);
+        locate(gwarp + nwarps, row1, j1);
+    } else {
+        const int64_t hs = gwarp * 32 + lane;
+        row0 = hs / ns;
+        j0 = (int)(hs - row0 * ns);
+        row1 = row0;
+        j1 = j0;
+        advance(row1, j1);
+    }
     const int64_t s0 = dc_slot(a, row0, row0 < a.T);
     int64_t s1 = dc_slot(a, row1, row1 < a.T && gwarp + nwarps < nchunks);
     const uint8_t* p0 = dc_row(a, s0, j0);
@@ -215,11 +256,12 @@ __global__ void __launch_bounds__(DC_THREADS) kv_decompress_kernel(const Decompr
     for (int64_t c = gwarp; c < nchunks; c += nwarps) {
         int64_t row2 = row1;
         int j2 = j1;
-        advance(row2, j2);
+        if (MODE == 2) locate(c + 2 * nwarps, row2, j2);
+        else advance(row2, j2);
         const int64_t s2 = dc_slot(a, row2, row2 < a.T && c + 2 * nwarps < nchunks);
         const uint8_t* p1 = dc_row(a, s1, j1);
         if (p1) dc_fetch<MODE, G>(a, nn, p1, j1, w1, sc1);
-        if (p0) dc_slice<MODE, G>(a, nn, w0, sc0, j0, a.y + row0 * a.y_row_stride, rope_tab);
+        if (p0) dc_slice<MODE, G, YF16>(a, nn, w0, sc0, j0, a.y + row0 * a.y_row_stride, rope_tab);
 #pragma unroll
         for (int i = 0; i < 16; ++i) w0[i] = w1[i];
         sc0 = sc1;

@@ -411,6 +411,47 @@ __global__ void selftest_fp8_row_kernel() {
     if (bad) atomicAdd(&g_selftest_count, bad);
 }
 
+// The unscaled two-step quotient of the rmsnorm kernel (div2_x2 with r =
+// RN(1/rms)) against IEEE division, 2^28 random pairs per call: rms a random
+// binary32 of binade 2^-60 .. 2^49; x a random bf16 of either sign with |x| of
+// binade max(e(rms) - 124, -103) .. e(rms) + 12; for half of the pairs rms is
+// then replaced by RN(x / t) nudged by up to two ulps, t halfway between
+// x / rms and its next binary32 value, so that x / rms lies within a few ulps
+// of a rounding tie.  Pairs outside the kernel's guard (rms in [2^-60, 2^50],
+// |x| >= max(RN(rms 2^-125), 2^-103)) are skipped; counts the pairs whose
+// quotient (of x and of -x) differs from the IEEE quotient in any bit.
+__global__ void selftest_rms_quot_kernel() {
+    const uint64_t i0 = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) * 16u;
+    unsigned long long bad = 0;
+    for (uint64_t i = i0; i < i0 + 16u; ++i) {
+        const uint64_t h1 = st_mix(3 * i), h2 = st_mix(3 * i + 1), h3 = st_mix(3 * i + 2);
+        float rms = st_float(h1, -60, 49);
+        const int er = (int)((__float_as_uint(rms) >> 23) & 0xffu) - 127;
+        const int lo = er - 124 > -103 ? er - 124 : -103, hi = er + 12;
+        const int ex = lo + (int)((h2 >> 8) % (uint64_t)(hi - lo + 1));
+        const uint32_t xb = ((uint32_t)(ex + 127) << 23) | ((uint32_t)(h2 & 0x7fu) << 16) |
+                            ((uint32_t)((h2 >> 7) & 1u) << 31);
+        const float x = __uint_as_float(xb);
+        if (h3 & 1u) {
+            const float q = __fdiv_rn(x, rms);
+            const double qa = fabs((double)q);
+            const double t = 0.5 * (qa + (double)__uint_as_float(__float_as_uint((float)qa) + 1u));
+            float r2 = (float)(fabs((double)x) / t);
+            r2 = __uint_as_float(__float_as_uint(r2) + (uint32_t)((int)((h3 >> 8) % 5u) - 2));
+            rms = r2;
+        }
+        if (!(rms >= 8.673617379884035e-19f && rms <= 1.125899906842624e15f)) continue;
+        const float thr = fmaxf(__fmul_rn(rms, 2.350988701644575e-38f), 9.860761315262648e-32f);
+        if (fabsf(x) < thr) continue;
+        float q0, q1;
+        div2_x2(x, -x, rms, __frcp_rn(rms), q0, q1);
+        const float ref = __fdiv_rn(x, rms);
+        bad += (__float_as_uint(q0) != __float_as_uint(ref) || __float_as_uint(q1) != __float_as_uint(-ref)) ? 1ull
+                                                                                                              : 0ull;
+    }
+    if (bad) atomicAdd(&g_selftest_count, bad);
+}
+
 // every positive finite bf16 amax (bits < 0x7f80) and every positive finite
 // f16 amax (bits < 0x7c00) over the three format maxima
 __global__ void selftest_fmax_kernel() {
@@ -456,7 +497,7 @@ extern "C" {
 
 kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream) {
     if (!result) return KVQ_ERR_NULL;
-    if (which < 0 || which > 8) return KVQ_ERR_ATTR;
+    if (which < 0 || which > 9) return KVQ_ERR_ATTR;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const unsigned long long zero = 0ull;
     unsigned long long h = 0ull;
@@ -466,6 +507,7 @@ kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream) {
     else if (which == 6) selftest_int8_kernel<<<65536, 256, 0, s>>>();
     else if (which == 7) selftest_timeout_kernel<<<1, 32, 0, s>>>();
     else if (which == 8) selftest_fp8_row_kernel<<<65536, 256, 0, s>>>();
+    else if (which == 9) selftest_rms_quot_kernel<<<65536, 256, 0, s>>>();
     else selftest_div_kernel<<<65536, 256, 0, s>>>(which);
     if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
     if (cudaMemcpyFromSymbolAsync(&h, g_selftest_count, sizeof(h), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -523,13 +565,15 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
     Trace trace("kvq_kv_compress_epilog");
     if (!x || !slot_mapping || !cache) return KVQ_ERR_NULL;
     if (!valid_desc(x) || !valid_desc(slot_mapping) || !valid_desc(cache)) return KVQ_ERR_DTYPE;
-    if (x->dtype != KVQ_BF16) return KVQ_ERR_DTYPE;
+    if (x->dtype != KVQ_BF16 && x->dtype != KVQ_F16) return KVQ_ERR_DTYPE;
     if (x->ndim < 1) return KVQ_ERR_NDIM;
     int64_t T, rs;
     if (!flatten_rows(x, &T, &rs)) return KVQ_ERR_LAYOUT;
     const int64_t d = x->shape[x->ndim - 1];
     if (d <= 64 || d % 64 != 0 || d > 8192) return KVQ_ERR_SHAPE;
     if (quant_mode < 0 || quant_mode > 2) return KVQ_ERR_ATTR;
+    if (quant_mode == 2 && x->dtype != KVQ_BF16) return KVQ_ERR_DTYPE;     // mode 2 needs bf16 x
+    const bool xf16 = x->dtype == KVQ_F16;
     const int32_t G = quant_mode == 2 ? quant_group_size : 64;
     if (quant_mode == 2 && ((G != 16 && G != 32 && G != 64) || (d - 64) % G != 0)) return KVQ_ERR_ATTR;
     if (!is_index_dtype(slot_mapping->dtype)) return KVQ_ERR_DTYPE;
@@ -591,16 +635,20 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
         const int64_t tiles = (T + CT_ROWS - 1) / CT_ROWS;
         const int threads = (a.ncw + 1) * 32;
         cudaError_t err = cudaSuccess;
-#define KVQ_LAUNCH_CT(M, GG)                                                                   \
+#define KVQ_LAUNCH_CT(M, GG, F)                                                                \
     do {                                                                                       \
-        auto k = ct_stages == 2 ? compress_tma_kernel<M, GG, 2> : compress_tma_kernel<M, GG, 3>; \
+        auto k = ct_stages == 2 ? compress_tma_kernel<M, GG, 2, F> : compress_tma_kernel<M, GG, 3, F>; \
         err = launch(k, (unsigned)persistent_grid(k, threads, tiles, smem), threads, smem, s, a); \
     } while (0)
-        if (quant_mode == 0) KVQ_LAUNCH_CT(0, 64);
-        else if (quant_mode == 1) KVQ_LAUNCH_CT(1, 64);
-        else if (G == 16) KVQ_LAUNCH_CT(2, 16);
-        else if (G == 32) KVQ_LAUNCH_CT(2, 32);
-        else KVQ_LAUNCH_CT(2, 64);
+        if (quant_mode == 0) {
+            if (xf16) KVQ_LAUNCH_CT(0, 64, true);
+            else KVQ_LAUNCH_CT(0, 64, false);
+        } else if (quant_mode == 1) {
+            if (xf16) KVQ_LAUNCH_CT(1, 64, true);
+            else KVQ_LAUNCH_CT(1, 64, false);
+        } else if (G == 16) KVQ_LAUNCH_CT(2, 16, false);
+        else if (G == 32) KVQ_LAUNCH_CT(2, 32, false);
+        else KVQ_LAUNCH_CT(2, 64, false);
 #undef KVQ_LAUNCH_CT
         return launched(err);
     }
@@ -611,16 +659,20 @@ kvq_status kvq_kv_compress_epilog(const kvq_tensor* x, const kvq_tensor* slot_ma
     const int64_t tiles = (T + a.ce_rows - 1) / a.ce_rows;
     const int64_t need = (tiles + (CE_THREADS / 32) - 1) / (CE_THREADS / 32);
     cudaError_t err = cudaSuccess;
-#define KVQ_LAUNCH_CE(M, GG)                                                                   \
+#define KVQ_LAUNCH_CE(M, GG, F)                                                                \
     do {                                                                                       \
-        auto k = compress_epilog_kernel<M, GG>;                                                \
+        auto k = compress_epilog_kernel<M, GG, F>;                                             \
         err = launch(k, (unsigned)persistent_grid(k, CE_THREADS, need), CE_THREADS, 0, s, a);    \
     } while (0)
-    if (quant_mode == 0) KVQ_LAUNCH_CE(0, 64);
-    else if (quant_mode == 1) KVQ_LAUNCH_CE(1, 64);
-    else if (G == 16) KVQ_LAUNCH_CE(2, 16);
-    else if (G == 32) KVQ_LAUNCH_CE(2, 32);
-    else KVQ_LAUNCH_CE(2, 64);
+    if (quant_mode == 0) {
+        if (xf16) KVQ_LAUNCH_CE(0, 64, true);
+        else KVQ_LAUNCH_CE(0, 64, false);
+    } else if (quant_mode == 1) {
+        if (xf16) KVQ_LAUNCH_CE(1, 64, true);
+        else KVQ_LAUNCH_CE(1, 64, false);
+    } else if (G == 16) KVQ_LAUNCH_CE(2, 16, false);
+    else if (G == 32) KVQ_LAUNCH_CE(2, 32, false);
+    else KVQ_LAUNCH_CE(2, 64, false);
 #undef KVQ_LAUNCH_CE
     return launched(err);
 }
@@ -631,7 +683,9 @@ kvq_status kvq_kv_decompress(const kvq_tensor* cache, const kvq_tensor* slot_map
     Trace trace("kvq_kv_decompress");
     if (!cache || !slot_mapping || !y) return KVQ_ERR_NULL;
     if (!valid_desc(cache) || !valid_desc(slot_mapping) || !valid_desc(y)) return KVQ_ERR_DTYPE;
-    if (y->dtype != KVQ_BF16) return KVQ_ERR_DTYPE;
+    if (y->dtype != KVQ_BF16 && y->dtype != KVQ_F16) return KVQ_ERR_DTYPE;
+    if (quant_mode == 2 && y->dtype != KVQ_BF16) return KVQ_ERR_DTYPE;     // mode 2 rows come from bf16 x
+    const bool yf16 = y->dtype == KVQ_F16;
     if (y->ndim < 1) return KVQ_ERR_NDIM;
     int64_t T, ys;
     if (!flatten_rows(y, &T, &ys)) return KVQ_ERR_LAYOUT;
@@ -667,20 +721,25 @@ kvq_status kvq_kv_decompress(const kvq_tensor* cache, const kvq_tensor* slot_map
     a.rows_vec16 = (reinterpret_cast<uintptr_t>(cache->data) % 16 == 0) && rows.row_bytes % 16 == 0 &&
                    rows.block_stride % 16 == 0;
     a.y_vec32 = (reinterpret_cast<uintptr_t>(y->data) % 32 == 0) && (ys * 2) % 32 == 0;
-    const int64_t nchunks = (T * a.nslice + 31) / 32;
+    const int64_t nchunks = quant_mode == 2 ? ((T + 15) / 16) * ((a.nslice - 2) / 2 + 1)   // see kv_decompress_kernel
+                                            : (T * a.nslice + 31) / 32;
     const int64_t need = (nchunks + (DC_THREADS / 32) - 1) / (DC_THREADS / 32);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t err = cudaSuccess;
-#define KVQ_LAUNCH_DC(M, GG)                                                                   \
+#define KVQ_LAUNCH_DC(M, GG, F)                                                                \
     do {                                                                                       \
-        auto k = a.nslice == 18 ? kv_decompress_kernel<M, GG, 18> : kv_decompress_kernel<M, GG, 0>; \
+        auto k = a.nslice == 18 ? kv_decompress_kernel<M, GG, 18, F> : kv_decompress_kernel<M, GG, 0, F>; \
         err = launch(k, (unsigned)persistent_grid(k, DC_THREADS, need), DC_THREADS, 0, s, a);    \
     } while (0)
-    if (quant_mode == 0) KVQ_LAUNCH_DC(0, 64);
-    else if (quant_mode == 1) KVQ_LAUNCH_DC(1, 64);
-    else if (G == 16) KVQ_LAUNCH_DC(2, 16);
-    else if (G == 32) KVQ_LAUNCH_DC(2, 32);
-    else KVQ_LAUNCH_DC(2, 64);
+    if (quant_mode == 0) {
+        if (yf16) KVQ_LAUNCH_DC(0, 64, true);
+        else KVQ_LAUNCH_DC(0, 64, false);
+    } else if (quant_mode == 1) {
+        if (yf16) KVQ_LAUNCH_DC(1, 64, true);
+        else KVQ_LAUNCH_DC(1, 64, false);
+    } else if (G == 16) KVQ_LAUNCH_DC(2, 16, false);
+    else if (G == 32) KVQ_LAUNCH_DC(2, 32, false);
+    else KVQ_LAUNCH_DC(2, 64, false);
 #undef KVQ_LAUNCH_DC
     return launched(err);
 }
@@ -743,9 +802,9 @@ kvq_status kvq_indexer_quant_cache(const kvq_tensor* x, kvq_tensor* cache, kvq_t
     a.code_vec32 = (reinterpret_cast<uintptr_t>(cache->data) % 32 == 0) && crow.row_bytes % 32 == 0 &&
                    crow.block_stride % 32 == 0;
     const bool f16 = x->dtype == KVQ_F16, e5m2 = cache->dtype == KVQ_F8E5M2;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int64_t passes = (T + (32 >> a.team_shift) - 1) / (32 >> a.team_shift);
     const int64_t need = (passes + (IX_THREADS / 32) - 1) / (IX_THREADS / 32);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t err = cudaSuccess;
 #define KVQ_LAUNCH_IX(M, F, E)                                                                 \
     do {                                                                                       \
@@ -887,13 +946,19 @@ kvq_status kvq_kv_rmsnorm_rope_cache(const kvq_tensor* kv, const kvq_tensor* gam
     const int64_t nch = Dv / 8;
     // the register-chunk kernels stage an int8 ckv cache's parameters in shared memory
     a.ckv_stage = vec && nch <= 128 && cc.dt == CDT_I8;
+    a.inv_dv = (Dv & (Dv - 1)) == 0 ? 1.0f / (float)Dv : 0.0f;     // exact: a power of two
     const size_t smem = a.ckv_stage ? (size_t)3 * Dv * sizeof(float) : 0;
     auto run = [&](auto kernel, size_t sm) {
         return launched(launch(kernel, (unsigned)persistent_grid(kernel, RR_THREADS, need, sm), RR_THREADS, sm, s, a));
     };
-    if (vec && nch <= 32) return run(rmsnorm_rope_kernel<1>, smem);
-    if (vec && nch <= 64) return run(rmsnorm_rope_kernel<2>, smem);
-    if (vec && nch <= 128) return run(rmsnorm_rope_kernel<4>, smem);
+    const int ck = ckv_class(cc.dt);
+#define KVQ_RR_CK(N)                                                                           \
+    return ck == 0 ? run(rmsnorm_rope_kernel<N, 0>, smem)                                      \
+                   : (ck == 1 ? run(rmsnorm_rope_kernel<N, 1>, smem) : run(rmsnorm_rope_kernel<N, 2>, smem))
+    if (vec && nch <= 32) KVQ_RR_CK(1);
+    if (vec && nch <= 64) KVQ_RR_CK(2);
+    if (vec && nch <= 128) KVQ_RR_CK(4);
+#undef KVQ_RR_CK
     return run(rmsnorm_rope_kernel<0>, (size_t)0);
 }
 

@@ -264,6 +264,19 @@ __device__ __forceinline__ void div2_x2(float a0, float a1, float s, float r, fl
     q1 = with_sign_of(q1, a1);
 }
 
+// (a0 b0, a1 b1), each product rounded once (mul.rn.f32x2: each half is the
+// IEEE round-to-nearest-even product).  Used only where the products feed
+// another multiply or a conversion, never an add (no contraction can arise).
+__device__ __forceinline__ void mul_x2(float a0, float a1, float b0, float b1, float& r0, float& r1) {
+    asm("{\n\t.reg .b64 a, b, r;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 r, a, b;\n\t"
+        "mov.b64 {%0, %1}, r;\n\t}"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // Four binary32 values rounded half to even to integers and saturated to
 // int8, packed little-endian (value 0 in byte 0).  NaN gives 0.
 __device__ __forceinline__ uint32_t int8x4_rne_sat(float v0, float v1, float v2, float v3) {
@@ -324,6 +337,19 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
     uint32_t r;
     asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
     return r;
+}
+
+// The same for two f16 halves.
+__device__ __forceinline__ uint32_t absmax_f16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// The value of a 16-bit float's bit pattern (bf16 or f16)
+template <bool F16>
+__device__ __forceinline__ float half_value(uint32_t bits) {
+    return F16 ? __half2float(__ushort_as_half((unsigned short)bits)) : __uint_as_float(bits << 16);
 }
 
 // eight quotients f[i] / s through div_scale1_x2

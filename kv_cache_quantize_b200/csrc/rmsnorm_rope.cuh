@@ -43,6 +43,7 @@ struct RmsRopeArgs {
     CacheOut ckv;           // Dv values per row
     float eps;
     int32_t ckv_stage;      // int8 ckv: scales, offsets and reciprocals staged in shared memory ([3][Dv])
+    float inv_dv;           // 1 / Dv when Dv is a power of two (exact), else 0
 };
 
 constexpr int RR_THREADS = 128;
@@ -112,19 +113,31 @@ __device__ __forceinline__ int64_t rr_resolve(const RmsRopeArgs& a, int64_t b, i
 // multiple of 2^-149, so the fused operations form it exactly, and the
 // quotient stays normal); a smaller |y| has |y / s| < 2^-63, whose code is
 // the zero of y's sign either way.
+// A per-tensor ckv scale that is a normal power of two, s = 2^e: r = 1/s is
+// exact, and RN(y r) and RN(y / s) are the same single rounding of the same
+// real number (subnormal results included), so the codes come from one
+// multiply (pow2).
 struct CkvDiv {
     float s, r;
     bool fast;
+    bool pow2;
 };
 
+// The ckv cache's dtype class, a template parameter of the register kernels
+// so that each instantiation carries only its own store path: 0 bf16 / f16,
+// 1 FP8 (E4M3 / E5M2), 2 int8.
+__host__ __device__ inline int ckv_class(int32_t dt) {
+    return dt == CDT_I8 ? 2 : ((dt == CDT_E4M3 || dt == CDT_E5M2) ? 1 : 0);
+}
+
 // y[0..7] = chunk c of the RMSNorm segment normalised and scaled, stored as
-// the ckv cache's dtype (8 values at row element 8c)
+// the ckv cache's dtype (8 values at row element 8c); CK: ckv_class(c.dt)
+template <int CK>
 __device__ __forceinline__ void rr_store_chunk(const CacheOut& c, uint8_t* row, int ch, const float (&y)[8],
                                                const CkvDiv& dv, const float* stg, int Dv) {
     const int j0 = 8 * ch;
-    switch (c.dt) {
-        case CDT_BF16:
-        case CDT_F16: {
+    switch (CK == 0 ? CDT_BF16 : (CK == 1 ? CDT_E4M3 : CDT_I8)) {
+        case CDT_BF16: {
             uint32_t w[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -135,9 +148,14 @@ __device__ __forceinline__ void rr_store_chunk(const CacheOut& c, uint8_t* row, 
             st_b128(row + 2 * j0, make_uint4(w[0], w[1], w[2], w[3]));
             break;
         }
-        case CDT_E4M3:
-        case CDT_E5M2: {
+        case CDT_E4M3: {
             float q[8];
+            if (dv.pow2) {
+#pragma unroll
+                for (int k = 0; k < 8; k += 2) mul_x2(y[k], y[k + 1], dv.r, dv.r, q[k], q[k + 1]);
+                st_b64(row + j0, c.dt == CDT_E4M3 ? fp8x8<false>(q) : fp8x8<true>(q));
+                break;
+            }
             float ym = 0.0f;
 #pragma unroll
             for (int k = 0; k < 8; ++k) ym = fmaxf(ym, fabsf(y[k]));
@@ -189,7 +207,7 @@ __device__ __forceinline__ void rr_store_chunk(const CacheOut& c, uint8_t* row, 
 // Eight CTAs of four warps per SM (at most 64 registers): the kernel is bound
 // by latency and the two IEEE divisions per value, and runs faster with more
 // warps resident (79 us at 8 CTAs per SM vs 93 us at 5 for 65,536 tokens).
-template <int NCH>
+template <int NCH, int CK = 0>
 __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRopeArgs a) {
     pdl_wait();
     pdl_trigger();
@@ -231,7 +249,7 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
     // of int8x4_quant, staged once per CTA
     extern __shared__ __align__(16) float rr_stage[];
     const float* stg = nullptr;
-    if (NCH > 0 && a.ckv_stage) {
+    if (NCH > 0 && CK == 2 && a.ckv_stage) {
         for (int i = threadIdx.x; i < a.Dv; i += blockDim.x) {
             const float sc = a.ckv.scale[a.ckv.scale_n == 1 ? 0 : i];
             const float of = a.ckv.offset ? a.ckv.offset[a.ckv.offset_n == 1 ? 0 : i] : 0.0f;
@@ -242,11 +260,13 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
         __syncthreads();
         stg = rr_stage;
     }
-    CkvDiv dv{0.0f, 0.0f, false};
-    if (NCH > 0 && (a.ckv.dt == CDT_E4M3 || a.ckv.dt == CDT_E5M2) && a.ckv.scale_n == 1) {
+    CkvDiv dv{0.0f, 0.0f, false, false};
+    if (NCH > 0 && CK == 1 && a.ckv.scale_n == 1) {
         dv.s = a.ckv.scale[0];
-        dv.fast = dv.s >= 9.094947017729282e-13f && dv.s <= 1.099511627776e12f;   // [2^-40, 2^40]
-        dv.r = dv.fast ? __frcp_rn(dv.s) : 0.0f;
+        const uint32_t sb = __float_as_uint(dv.s);
+        dv.pow2 = (sb & 0x807fffffu) == 0u && (sb >> 23) >= 1u && (sb >> 23) <= 254u;   // +2^e, normal
+        dv.fast = dv.s >= 9.094947017729282e-13f && dv.s <= 1.099511627776e12f;        // [2^-40, 2^40]
+        dv.r = (dv.fast || dv.pow2) ? __frcp_rn(dv.s) : 0.0f;
     }
     if (NCH > 0) load_chunks(gwarp, xn);
     prefetch(gwarp);
@@ -288,22 +308,21 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
             }
 #pragma unroll
             for (int k = 16; k >= 1; k >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(FULL_MASK, acc, k));
-            const float mean = __fdiv_rn(acc, (float)a.Dv);
+            const float mean = a.inv_dv != 0.0f ? __fmul_rn(acc, a.inv_dv) : __fdiv_rn(acc, (float)a.Dv);
             const float rms = __fsqrt_rn(__fadd_rn(mean, a.eps));
-            // x / rms as (x 2^64) / (rms 2^64), the same real quotient, by the
-            // two-step form.  For rms in [2^-60, 2^50] every |x| is below
-            // rms sqrt(Dv) < 2^56, so the scaled numerators (bf16 / f16: at
-            // least 2^-133 unscaled), divisor, reciprocal and residuals are
-            // normal; the lane also needs every nonzero |x| >= RN(rms 2^-125)
-            // (a normal quotient, with a factor 2 for the rounding of the
-            // bound: a subnormal quotient can be an exact rounding tie, which
-            // the two-step form may break the wrong way).  Then the quotient
-            // is RN(x / rms).
-            const float thr = __fmul_rn(rms, 2.350988701644575e-38f);            // rms 2^-125
-            const bool nfast = rms >= 8.673617379884035e-19f && rms <= 1.125899906842624e15f &&
-                               xmin2 >= 2u * __float_as_uint(thr) - 2u;
-            const float rs64 = __fmul_rn(rms, 1.8446744073709552e19f);
-            const float rr64 = nfast ? __frcp_rn(rs64) : 0.0f;
+            // x / rms by the two-step form (div2_x2): RN(x / rms) when rms is in
+            // [2^-60, 2^50] and, per lane, every nonzero |x| is at least
+            // max(RN(rms 2^-125), 2^-103) -- the quotient is then normal and each
+            // residual x - q rms a multiple of 2^-149, formed exactly by the
+            // fused operations (kvq_selftest 9 checks the domain; a subnormal
+            // quotient can be an exact rounding tie, which the two-step form
+            // may break the wrong way, hence the first bound).  The bound is
+            // tracked during the sum of squares (xmin2); a lane with a smaller
+            // nonzero value divides with IEEE division.
+            const float uthr = fmaxf(__fmul_rn(rms, 2.350988701644575e-38f), 9.860761315262648e-32f);
+            const bool ufast = rms >= 8.673617379884035e-19f && rms <= 1.125899906842624e15f &&
+                               xmin2 >= 2u * __float_as_uint(uthr) - 2u;
+            const float rr1 = ufast ? __frcp_rn(rms) : 0.0f;
 #pragma unroll
             for (int m = 0; m < NCH; ++m) {
                 const int c = lane + 32 * m;
@@ -317,18 +336,16 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
                     widen8<false>(xv[m], f);
                     widen8<false>(gv, g);
                 }
-                if (nfast) {
+                if (ufast) {
 #pragma unroll
-                    for (int i = 0; i < 8; i += 2)
-                        div2_x2(__fmul_rn(f[i], 1.8446744073709552e19f), __fmul_rn(f[i + 1], 1.8446744073709552e19f),
-                                rs64, rr64, y[i], y[i + 1]);
+                    for (int i = 0; i < 8; i += 2) div2_x2(f[i], f[i + 1], rms, rr1, y[i], y[i + 1]);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(y[i], g[i]);
+                    for (int i = 0; i < 8; i += 2) mul_x2(y[i], y[i + 1], g[i], g[i + 1], y[i], y[i + 1]);
                 } else {
 #pragma unroll
                     for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fdiv_rn(f[i], rms), g[i]);
                 }
-                rr_store_chunk(a.ckv, crow, c, y, dv, stg, a.Dv);
+                rr_store_chunk<CK>(a.ckv, crow, c, y, dv, stg, a.Dv);
             }
         } else {
             // RMSNorm: sum of squares in the fixed lane order

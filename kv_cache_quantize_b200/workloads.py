@@ -111,21 +111,26 @@ def gen_compress(name: str, T: int, d: int, quant_mode: int, num_blocks: int, bl
                  head_dim: int, group_size: int = 64, x_scale: float = 1.0, skip_frac: float = 0.0,
                  outlier_frac: float = 0.0, outlier_mult: float = 50.0, seed: int = 0,
                  slot_dtype=np.int32, block_pad_bytes: int = 0, x_kind: str = "normal",
-                 guard: int = GUARD_BYTES) -> Case:
+                 guard: int = GUARD_BYTES, x_dtype: str = "bf16") -> Case:
+    """x_dtype "f16" (quantMode 0/1): the same samples rounded to float16; the
+    "wide" kind then keeps every exponent but the infinity / NaN one."""
     if x_kind == "normal":
         xf = _rng(seed, 1).standard_normal((T, d), dtype=np.float32)
         if outlier_frac > 0:
             rows = _rng(seed, 2).choice(T, size=int(np.floor(outlier_frac * T)), replace=False)
             xf[rows] *= np.float32(outlier_mult)
-        x = to_bf16_bits(xf)
+        x = to_half_bits(xf, x_dtype)
     elif x_kind == "wide":
         x = wide_bf16_bits(_rng(seed, 1), (T, d))
+        if x_dtype == "f16":       # the all-ones f16 exponent (inf / NaN) becomes a subnormal
+            x = np.where((x & 0x7C00) == 0x7C00, x & 0x83FF, x).astype(np.uint16)
     else:
         raise ValueError(x_kind)
     cache = make_cache(_rng(seed, 3), num_blocks, block_size, head_dim, 1, 1, block_pad_bytes, guard)
     slots = slots_with_skips(_rng(seed, 4), num_blocks * block_size, T, skip_frac, slot_dtype)
     return Case(name, "kv_compress_epilog", {"x": x, "slot_mapping": slots}, {"cache": cache},
-                {"quant_mode": quant_mode, "quant_group_size": group_size, "x_scale": x_scale})
+                {"quant_mode": quant_mode, "quant_group_size": group_size, "x_scale": x_scale,
+                 "x_dtype": x_dtype})
 
 
 def gen_indexer(name: str, T: int, d: int, quant_mode: int, num_blocks: int, block_size: int,
@@ -297,6 +302,12 @@ def compress_mode0_T262144_d576(seed: int = 0) -> Case:
                         block_size=128, head_dim=672, skip_frac=0.02, outlier_frac=0.01, seed=seed)
 
 
+def compress_mode0_f16_T262144_d576(seed: int = 0) -> Case:
+    """The quantMode-0 sweep with float16 x (the page requires bfloat16 only in mode 2)."""
+    return gen_compress("compress_mode0_f16_T262144_d576", T=262144, d=576, quant_mode=0, num_blocks=4096,
+                        block_size=128, head_dim=672, skip_frac=0.02, outlier_frac=0.01, seed=seed, x_dtype="f16")
+
+
 def compress_mode2_G32_T262144_d576(seed: int = 0) -> Case:
     return gen_compress("compress_mode2_G32_T262144_d576", T=262144, d=576, quant_mode=2, group_size=32, x_scale=0.1,
                         num_blocks=4096, block_size=128, head_dim=352, skip_frac=0.02, outlier_frac=0.01,
@@ -394,6 +405,7 @@ CONFIGS = {
     "dequant_rope_quant_page_B16_S1024_H3072": dequant_rope_quant_page_B16_S1024_H3072,
     "compress_mode0_T262144_d576": compress_mode0_T262144_d576,
     "compress_mode2_G32_T262144_d576": compress_mode2_G32_T262144_d576,
+    "compress_mode0_f16_T262144_d576": compress_mode0_f16_T262144_d576,
     "indexer_fp8_T65536_d128": indexer_fp8_T65536_d128,
     "indexer_mxfp8_e5m2_T65536_d128": indexer_mxfp8_e5m2_T65536_d128,
     "rmsnorm_rope_int8_prefill_B65536_D576": rmsnorm_rope_int8_prefill_B65536_D576,
@@ -457,7 +469,7 @@ def build_call(case: Case, misalign: bool = False):
     st, views, outs = {}, {}, {}
     if case.op == "kv_compress_epilog":
         st["cache"], views["cache"] = dev_cache(case.caches["cache"], torch.uint8)
-        x, s = half_tensor(a["x"], "bf16"), idx(a["slot_mapping"])
+        x, s = half_tensor(a["x"], at.get("x_dtype", "bf16")), idx(a["slot_mapping"])
 
         def call(stream=None):
             kvq.kv_compress_epilog(x, s, views["cache"], at["quant_mode"], at["quant_group_size"], at["x_scale"],

@@ -20,7 +20,8 @@ def run_oracle(case: Case, threads: int = 1):
     outs = {}
     if case.op == "kv_compress_epilog":
         f = oracle.kv_compress_epilog(a["x"], a["slot_mapping"], paged(case.caches["cache"], st["cache"]),
-                                      at["quant_mode"], at["quant_group_size"], at["x_scale"], threads)
+                                      at["quant_mode"], at["quant_group_size"], at["x_scale"], threads,
+                                      x_dtype=at.get("x_dtype", "bf16"))
     elif case.op == "indexer_quant_cache":
         f = oracle.indexer_quant_cache(a["x"], at["x_dtype"], a["slot_mapping"],
                                        paged(case.caches["cache"], st["cache"]),

@@ -106,7 +106,10 @@ def test_compress_validation(L):
     x, s, c = D([64, 576], "bf16"), D([64], "i32"), D([8, 16, 1, 672], "u8")
     assert ce(L, x, s, c) == ENULL                        # valid up to the (absent) data
     assert L.kvq_kv_compress_epilog(None, R(s), R(c), 0, 64, ctypes.c_float(1), None) == ENULL
-    assert ce(L, D([64, 576], "f16"), s, c) == EDTYPE
+    assert ce(L, D([64, 576], "f16"), s, c) == ENULL      # float16 x in quantMode 0 (and 1)
+    assert ce(L, D([64, 576], "f16"), s, D([8, 16, 1, 648], "u8"), mode=1) == ENULL
+    assert ce(L, D([64, 576], "f16"), s, D([8, 16, 1, 352], "u8"), mode=2, G=32) == EDTYPE   # mode 2: bf16 only
+    assert ce(L, D([64, 576], "f32"), s, c) == EDTYPE
     assert ce(L, D([64, 600], "bf16"), s, c) == ESHAPE    # d % 64
     assert ce(L, D([64, 64], "bf16"), s, c) == ESHAPE     # d > 64
     assert ce(L, D([64, 8256], "bf16"), s, c) == ESHAPE   # d <= 8192
@@ -137,7 +140,9 @@ def test_decompress_validation(L):
     y, s, c = D([64, 576], "bf16"), D([64], "i32"), D([8, 16, 1, 672], "u8")
     assert kd(L, c, s, y) == ENULL                        # valid up to the (absent) data
     assert L.kvq_kv_decompress(R(c), R(s), None, 0, 64, ctypes.c_float(1), None) == ENULL
-    assert kd(L, c, s, D([64, 576], "f16")) == EDTYPE
+    assert kd(L, c, s, D([64, 576], "f16")) == ENULL      # float16 y for rows of float16 x (mode 0/1)
+    assert kd(L, D([8, 16, 1, 352], "u8"), s, D([64, 576], "f16"), mode=2, G=32) == EDTYPE
+    assert kd(L, c, s, D([64, 576], "f32")) == EDTYPE
     assert kd(L, c, s, D([64, 600], "bf16")) == ESHAPE    # d % 64
     assert kd(L, c, s, D([64, 64], "bf16")) == ESHAPE
     assert kd(L, c, D([63], "i32"), y) == ESHAPE
@@ -272,9 +277,9 @@ def test_row_widths_beyond_32_bit_indexing_are_rejected(L):
 
 
 def test_selftest_numbering(L):
-    """Self-tests 0..8 exist; other numbers and a NULL result are rejected before any device work."""
+    """Self-tests 0..9 exist; other numbers and a NULL result are rejected before any device work."""
     out = ctypes.c_uint64(0)
-    assert L.kvq_selftest(9, ctypes.byref(out), None) == EATTR
+    assert L.kvq_selftest(10, ctypes.byref(out), None) == EATTR
     assert L.kvq_selftest(-1, ctypes.byref(out), None) == EATTR
     assert L.kvq_selftest(0, None, None) == ENULL
 

@@ -21,7 +21,7 @@ def _encoded(case):
     st = case.caches["cache"].storage.copy()
     a, at = case.arrays, case.attrs
     oracle.kv_compress_epilog(a["x"], a["slot_mapping"], paged(case.caches["cache"], st), at["quant_mode"],
-                              at["quant_group_size"], at["x_scale"], THREADS)
+                              at["quant_group_size"], at["x_scale"], THREADS, x_dtype=at.get("x_dtype", "bf16"))
     return st
 
 
@@ -32,15 +32,16 @@ def _same(case, slots=None, y_extra=0, y_shift=0):
     slots = case.arrays["slot_mapping"] if slots is None else slots
     T, d = case.arrays["x"].shape
     mode, G, xs = at["quant_mode"], at["quant_group_size"], at["x_scale"]
+    ydt = at.get("x_dtype", "bf16")
     y_o, f_o = oracle.kv_decompress(paged(cb, st.copy()), slots, d, mode, G, xs,
-                                    y=np.full((T, d), MARK, dtype=np.uint16), threads=THREADS)
+                                    y=np.full((T, d), MARK, dtype=np.uint16), threads=THREADS, y_dtype=ydt)
     # device: the same packed bytes; y rows possibly strided / shifted
     dst = torch.from_numpy(st).cuda()
     view = dst[cb.offset:].as_strided((cb.num_blocks, cb.block_size, 1, cb.head_dim),
                                       (cb.block_stride, cb.head_dim, cb.head_dim, 1))
     row = d + y_extra
     buf = torch.full((T * row + y_shift + 16,), MARK, dtype=torch.int16, device="cuda")
-    y = buf[y_shift:y_shift + T * row].view(T, row)[:, :d].view(torch.bfloat16)
+    y = buf[y_shift:y_shift + T * row].view(T, row)[:, :d].view(torch.bfloat16 if ydt == "bf16" else torch.float16)
     kvq.get_error()
     kvq.kv_decompress(view, torch.from_numpy(np.ascontiguousarray(slots)).cuda(), y, mode, G, xs)
     torch.cuda.synchronize()
@@ -59,12 +60,14 @@ def _same(case, slots=None, y_extra=0, y_shift=0):
     return y_g
 
 
-def _case(T, d, mode, G=64, kind="normal", extra=13, pad=0, seed=0, skip=0.1, slot_dtype=np.int32, xs=0.1):
+def _case(T, d, mode, G=64, kind="normal", extra=13, pad=0, seed=0, skip=0.1, slot_dtype=np.int32, xs=0.1,
+          x_dtype="bf16"):
     col = oracle.kv_cache_col(d, mode, G)
     nblk = max(1, (2 * T + 15) // 16)
-    return W.gen_compress(f"kd_m{mode}_g{G}_d{d}_T{T}_{kind}", T=T, d=d, quant_mode=mode, num_blocks=nblk,
-                          block_size=16, head_dim=col + extra, group_size=G, x_scale=xs, skip_frac=skip,
-                          outlier_frac=0.05, seed=seed, x_kind=kind, block_pad_bytes=pad, slot_dtype=slot_dtype)
+    return W.gen_compress(f"kd_m{mode}_g{G}_d{d}_T{T}_{kind}_{x_dtype}", T=T, d=d, quant_mode=mode,
+                          num_blocks=nblk, block_size=16, head_dim=col + extra, group_size=G, x_scale=xs,
+                          skip_frac=skip, outlier_frac=0.05, seed=seed, x_kind=kind, block_pad_bytes=pad,
+                          slot_dtype=slot_dtype, x_dtype=x_dtype)
 
 
 @pytest.mark.parametrize("kind", ["normal", "wide"])
@@ -104,3 +107,15 @@ def test_decompress_bad_slots_fault_and_int64():
                                   "compress_mode1_T64_d256"])
 def test_decompress_named_workloads_full_size(name):
     _same(W.CONFIGS[name]())
+
+
+@pytest.mark.parametrize("kind", ["normal", "wide"])
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("d", [128, 576, 1088])
+def test_decompress_f16_rows(mode, d, kind):
+    """Rows compressed from float16 x decode into float16 y (quantMode 0/1)."""
+    _same(_case(203, d, mode, kind=kind, seed=41, x_dtype="f16"))
+
+
+def test_decompress_f16_full_size():
+    _same(W.CONFIGS["compress_mode0_f16_T262144_d576"]())

@@ -40,12 +40,13 @@ def _same(case, check_outputs=True, misalign=False):
 # kv_compress_epilog
 # ---------------------------------------------------------------------------
 def _ce(T, d, mode, G=64, kind="normal", pad=0, extra=13, skip=0.1, seed=0, slot_dtype=np.int32, xs=0.1,
-        block_size=16):
+        block_size=16, x_dtype="bf16"):
     col = oracle.kv_cache_col(d, mode, G)
     nblk = max(1, (2 * T + block_size - 1) // block_size)
-    return W.gen_compress(f"ce_m{mode}_g{G}_d{d}_T{T}_{kind}", T=T, d=d, quant_mode=mode, num_blocks=nblk,
-                          block_size=block_size, head_dim=col + extra, group_size=G, x_scale=xs, skip_frac=skip,
-                          outlier_frac=0.05, seed=seed, x_kind=kind, block_pad_bytes=pad, slot_dtype=slot_dtype)
+    return W.gen_compress(f"ce_m{mode}_g{G}_d{d}_T{T}_{kind}_{x_dtype}", T=T, d=d, quant_mode=mode,
+                          num_blocks=nblk, block_size=block_size, head_dim=col + extra, group_size=G, x_scale=xs,
+                          skip_frac=skip, outlier_frac=0.05, seed=seed, x_kind=kind, block_pad_bytes=pad,
+                          slot_dtype=slot_dtype, x_dtype=x_dtype)
 
 
 @pytest.mark.parametrize("kind", ["normal", "wide"])
@@ -157,8 +158,23 @@ def test_compress_all_skipped():
     assert np.array_equal(st_g["cache"], case.caches["cache"].storage)
 
 
+# float16 x (quantMode 0/1: the page requires bfloat16 only in mode 2), on the
+# direct kernel (decode-sized batches, misaligned rows) and the pipelined one
+@pytest.mark.parametrize("kind", ["normal", "wide"])
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("T,d", [(203, 576), (T_PIPE, 576), (T_PIPE, 1408), (45, 8192)])
+def test_compress_f16_x(mode, T, d, kind):
+    _same(_ce(T, d, mode, kind=kind, seed=43, x_dtype="f16"))
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("extra,pad", [(1, 0), (3, 40)])
+def test_compress_f16_x_row_alignments(mode, extra, pad):
+    _same(_ce(T_PIPE, 320, mode, extra=extra, pad=pad, seed=45, x_dtype="f16"))
+
+
 @pytest.mark.parametrize("name", ["compress_mode1_T64_d256", "compress_mode0_T262144_d576",
-                                  "compress_mode2_G32_T262144_d576"])
+                                  "compress_mode2_G32_T262144_d576", "compress_mode0_f16_T262144_d576"])
 def test_compress_named_workloads_full_size(name):
     _same(W.CONFIGS[name]())
 

@@ -13,7 +13,9 @@ whole input domain against IEEE division:
     (value, scale, offset) triples;
   * the indexer fp8 mode's division by the row scale (two-step Markstein form
     where the row maximum is a finite value >= 2^-60): the same E4M3 and E5M2
-    codes as IEEE division on 2^28 random bf16 / f16 (value, maximum) pairs.
+    codes as IEEE division on 2^28 random bf16 / f16 (value, maximum) pairs;
+  * the rmsnorm kernel's unscaled x / rms (two-step Markstein form inside its
+    guard): bit-identical to IEEE division on 2^28 random and near-tie pairs.
 Also the failure path of the pipelined kernels' bounded waits: a wait on a
 barrier that nothing completes gives up after its limit and reports
 FAULT_TIMEOUT through the fault word (no GPU fault, hang or trap)."""
@@ -28,7 +30,8 @@ pytestmark = pytest.mark.gpu
                                         (3, "E2M1 codes of the one-step quotient"),
                                         (4, "constant-divisor scale quotients"),
                                         (6, "int8 codes of the reciprocal-based quotient"),
-                                        (8, "fp8 row-scale codes of the two-step quotient")])
+                                        (8, "fp8 row-scale codes of the two-step quotient"),
+                                        (9, "unscaled two-step quotient x / rms")])
 def test_shortcut_is_exact(which, what):
     assert kvq.selftest(which) == 0, what
 
