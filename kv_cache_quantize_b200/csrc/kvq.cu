@@ -411,8 +411,9 @@ __global__ void selftest_fp8_row_kernel() {
     if (bad) atomicAdd(&g_selftest_count, bad);
 }
 
-// The unscaled two-step quotient of the rmsnorm kernel (div2_x2 with r =
-// RN(1/rms)) against IEEE division, 2^28 random pairs per call: rms a random
+// The unscaled two-step quotient of the rmsnorm kernel (div2_x2_nz with r =
+// RN(1/rms), numerators never zero) against IEEE division, 2^28 random pairs
+// per call: rms a random
 // binary32 of binade 2^-60 .. 2^49; x a random bf16 of either sign with |x| of
 // binade max(e(rms) - 124, -103) .. e(rms) + 12; for half of the pairs rms is
 // then replaced by RN(x / t) nudged by up to two ulps, t halfway between
@@ -444,7 +445,7 @@ __global__ void selftest_rms_quot_kernel() {
         const float thr = fmaxf(__fmul_rn(rms, 2.350988701644575e-38f), 9.860761315262648e-32f);
         if (fabsf(x) < thr) continue;
         float q0, q1;
-        div2_x2(x, -x, rms, __frcp_rn(rms), q0, q1);
+        div2_x2_nz(x, -x, rms, __frcp_rn(rms), q0, q1);
         const float ref = __fdiv_rn(x, rms);
         bad += (__float_as_uint(q0) != __float_as_uint(ref) || __float_as_uint(q1) != __float_as_uint(-ref)) ? 1ull
                                                                                                               : 0ull;

@@ -277,6 +277,23 @@ __device__ __forceinline__ void mul_x2(float a0, float a1, float b0, float b1, f
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
+// div2_x2 for nonzero numerators: the quotient of a nonzero a carries a's sign
+// through every correction, so the signed-zero fix of div2_x2 is not needed.
+__device__ __forceinline__ void div2_x2_nz(float a0, float a1, float s, float r, float& q0, float& q1) {
+    asm("{\n\t.reg .b64 a, ns, rr, q, e;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 ns, {%4, %4};\n\t"
+        "mov.b64 rr, {%5, %5};\n\t"
+        "mul.rn.f32x2 q, a, rr;\n\t"
+        "fma.rn.f32x2 e, q, ns, a;\n\t"
+        "fma.rn.f32x2 q, e, rr, q;\n\t"
+        "fma.rn.f32x2 e, q, ns, a;\n\t"
+        "fma.rn.f32x2 q, e, rr, q;\n\t"
+        "mov.b64 {%0, %1}, q;\n\t}"
+        : "=f"(q0), "=f"(q1)
+        : "f"(a0), "f"(a1), "f"(-s), "f"(r));
+}
+
 // Four binary32 values rounded half to even to integers and saturated to
 // int8, packed little-endian (value 0 in byte 0).  NaN gives 0.
 __device__ __forceinline__ uint32_t int8x4_rne_sat(float v0, float v1, float v2, float v3) {

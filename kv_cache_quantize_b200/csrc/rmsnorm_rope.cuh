@@ -290,10 +290,12 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
 
         if (NCH > 0) {
             // RMSNorm: sum of squares in the fixed lane order, chunks from registers;
-            // also the lane's smallest nonzero |x|, as 2 |x|bits - 2 (zeros wrap
-            // to the largest value)
+            // also the smallest exponent field of the lane's values (per 16-bit
+            // half, on the raw bits): every value then has |x| >= 2^(e - bias),
+            // and a zero or subnormal value gives e = 0
             float acc = 0.0f;
-            uint32_t xmin2 = 0xffffffffu;
+            const uint32_t emask = a.kv_f16 ? 0x7c007c00u : 0x7f807f80u;
+            uint32_t emin2 = emask;
 #pragma unroll
             for (int m = 0; m < NCH; ++m) {
                 if (lane + 32 * m >= nch) break;
@@ -301,27 +303,28 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
                 if (a.kv_f16) widen8<true>(xv[m], f);
                 else widen8<false>(xv[m], f);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    acc = __fadd_rn(acc, __fmul_rn(f[i], f[i]));
-                    xmin2 = min(xmin2, 2u * __float_as_uint(f[i]) - 2u);
-                }
+                for (int i = 0; i < 8; ++i) acc = __fadd_rn(acc, __fmul_rn(f[i], f[i]));
+                emin2 = __vminu2(emin2, __vminu2(xv[m].x & emask, xv[m].y & emask));
+                emin2 = __vminu2(emin2, __vminu2(xv[m].z & emask, xv[m].w & emask));
             }
+            const uint32_t emin = min(emin2 & 0xffffu, emin2 >> 16);     // 2^(e - bias) as 16-bit float bits
 #pragma unroll
             for (int k = 16; k >= 1; k >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(FULL_MASK, acc, k));
             const float mean = a.inv_dv != 0.0f ? __fmul_rn(acc, a.inv_dv) : __fdiv_rn(acc, (float)a.Dv);
             const float rms = __fsqrt_rn(__fadd_rn(mean, a.eps));
-            // x / rms by the two-step form (div2_x2): RN(x / rms) when rms is in
-            // [2^-60, 2^50] and, per lane, every nonzero |x| is at least
+            // x / rms by the two-step form (div2_x2_nz): RN(x / rms) when rms is
+            // in [2^-60, 2^50] and, per lane, every |x| is nonzero and at least
             // max(RN(rms 2^-125), 2^-103) -- the quotient is then normal and each
             // residual x - q rms a multiple of 2^-149, formed exactly by the
             // fused operations (kvq_selftest 9 checks the domain; a subnormal
             // quotient can be an exact rounding tie, which the two-step form
-            // may break the wrong way, hence the first bound).  The bound is
-            // tracked during the sum of squares (xmin2); a lane with a smaller
-            // nonzero value divides with IEEE division.
+            // may break the wrong way, hence the first bound), and a nonzero
+            // numerator's quotient keeps its sign without a fix.  The lane's
+            // smallest power of two 2^(e - bias) stands for its values; a lane
+            // with a zero or a smaller value divides with IEEE division.
             const float uthr = fmaxf(__fmul_rn(rms, 2.350988701644575e-38f), 9.860761315262648e-32f);
             const bool ufast = rms >= 8.673617379884035e-19f && rms <= 1.125899906842624e15f &&
-                               xmin2 >= 2u * __float_as_uint(uthr) - 2u;
+                               half_bits(emin, a.kv_f16) >= uthr;
             const float rr1 = ufast ? __frcp_rn(rms) : 0.0f;
 #pragma unroll
             for (int m = 0; m < NCH; ++m) {
@@ -338,7 +341,7 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
                 }
                 if (ufast) {
 #pragma unroll
-                    for (int i = 0; i < 8; i += 2) div2_x2(f[i], f[i + 1], rms, rr1, y[i], y[i + 1]);
+                    for (int i = 0; i < 8; i += 2) div2_x2_nz(f[i], f[i + 1], rms, rr1, y[i], y[i + 1]);
 #pragma unroll
                     for (int i = 0; i < 8; i += 2) mul_x2(y[i], y[i + 1], g[i], g[i + 1], y[i], y[i + 1]);
                 } else {
