@@ -146,11 +146,19 @@ __device__ __forceinline__ void dc_slice(const DecompressArgs& a, int nn, const 
 
 // packed bytes a slice needs: its codes (or the 64 bytes of a bf16 rope) in w,
 // its group scale bits in sc (nn: the number of nope slices)
-template <int MODE, int G>
+template <int MODE, int G, bool DBL>
 __device__ __forceinline__ void dc_fetch(const DecompressArgs& a, int nn, const uint8_t* row, int j,
                                          uint32_t (&w)[16], uint32_t& sc) {
     const bool v16 = a.rows_vec16 != 0;
     sc = 0u;
+    if (DBL && j < nn) {
+        // mode 2, G = 32 or 64: the two nope slices j, j + 1 (j even): 32 code bytes
+        // and their scale(s), the slice-j scale in the low half
+        dc_load<32>(row + 16 * j, v16, w);
+        const uint8_t* sp = row + a.n / 2 + 64;
+        sc = G == 32 ? (dc_ld16(sp + 2 * j) | (dc_ld16(sp + 2 * j + 2) << 16)) : dc_ld16(sp + 2 * (j >> 1));
+        return;
+    }
     if (j >= nn) {
         if (MODE != 2) dc_load<64>(row + a.n + 64 * (j - nn), v16, w);
         else dc_load<32>(row + a.n / 2 + 32 * (j - nn), v16, w);
@@ -187,8 +195,11 @@ __device__ __forceinline__ const uint8_t* dc_row(const DecompressArgs& a, int64_
 
 // NS: slices per row (d / 32) when known at compile time (18: d = 576), else 0
 // and a.nslice; the constant form measured 11 % faster in mode 0 at d = 576.
-template <int MODE, int G, int NS, bool YF16 = false>
-__global__ void __launch_bounds__(DC_THREADS, (MODE == 2 || NS != 0) ? 4 : 3) kv_decompress_kernel(const DecompressArgs a) {
+// DBL (mode 2, G = 32 or 64, (d - 64) / 32 a multiple of 4): a nope lane takes
+// two adjacent slices (32 bytes of FP4 codes, as many as a mode-0 slice), so a
+// 16-row block is (d - 64) / 128 nope chunks and one rope chunk.
+template <int MODE, int G, int NS, bool YF16 = false, bool DBL = false>
+__global__ void __launch_bounds__(DC_THREADS, (NS != 0 || (MODE == 2 && !DBL)) ? 4 : 3) kv_decompress_kernel(const DecompressArgs a) {
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
@@ -196,7 +207,8 @@ __global__ void __launch_bounds__(DC_THREADS, (MODE == 2 || NS != 0) ? 4 : 3) kv
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int ns = NS ? NS : a.nslice;
     const int nn = ns - 2;
-    const int64_t nchunks = MODE == 2 ? ((a.T + 15) / 16) * (nn / 2 + 1) : (a.T * ns + 31) / 32;
+    const int hn = DBL ? nn / 4 : nn / 2;       // mode 2: nope chunks per block of 16 rows
+    const int64_t nchunks = MODE == 2 ? ((a.T + 15) / 16) * (hn + 1) : (a.T * ns + 31) / 32;
     // mode 2: the decoded rope value of every E4M3 code, one IEEE division each
     __shared__ uint16_t rope_tab[MODE == 2 ? 256 : 1];
     if (MODE == 2) {
@@ -211,7 +223,6 @@ __global__ void __launch_bounds__(DC_THREADS, (MODE == 2 || NS != 0) ? 4 : 3) kv
     // the lane's slice (row, j) in chunk c: modes 0/1 step through the flat
     // slice array (chunk c + nwarps is nwarps * 32 slices further, added
     // without a division); mode 2 locates it in its 16-row block
-    const int hn = nn / 2;                      // mode 2: nope chunks per block of 16 rows
     const int64_t step = nwarps * 32;
     const int64_t qs = step / ns;
     const int rs = (int)(step - qs * ns);
@@ -227,9 +238,10 @@ __global__ void __launch_bounds__(DC_THREADS, (MODE == 2 || NS != 0) ? 4 : 3) kv
         const int64_t blk = c / (hn + 1);
         const int w = (int)(c - blk * (hn + 1));
         if (w < hn) {
+            const int per = DBL ? nn / 2 : nn;          // lanes per row
             const int sl = 32 * w + lane;
-            r = 16 * blk + sl / nn;
-            j = sl - (sl / nn) * nn;
+            r = 16 * blk + sl / per;
+            j = (sl - (sl / per) * per) * (DBL ? 2 : 1);
         } else {
             r = 16 * blk + (lane >> 1);
             j = nn + (lane & 1);
@@ -252,7 +264,7 @@ __global__ void __launch_bounds__(DC_THREADS, (MODE == 2 || NS != 0) ? 4 : 3) kv
     int64_t s1 = dc_slot(a, row1, row1 < a.T && gwarp + nwarps < nchunks);
     const uint8_t* p0 = dc_row(a, s0, j0);
     uint32_t w0[16], w1[16], sc0 = 0u, sc1 = 0u;
-    if (p0) dc_fetch<MODE, G>(a, nn, p0, j0, w0, sc0);
+    if (p0) dc_fetch<MODE, G, DBL>(a, nn, p0, j0, w0, sc0);
     for (int64_t c = gwarp; c < nchunks; c += nwarps) {
         int64_t row2 = row1;
         int j2 = j1;
@@ -260,8 +272,18 @@ __global__ void __launch_bounds__(DC_THREADS, (MODE == 2 || NS != 0) ? 4 : 3) kv
         else advance(row2, j2);
         const int64_t s2 = dc_slot(a, row2, row2 < a.T && c + 2 * nwarps < nchunks);
         const uint8_t* p1 = dc_row(a, s1, j1);
-        if (p1) dc_fetch<MODE, G>(a, nn, p1, j1, w1, sc1);
-        if (p0) dc_slice<MODE, G, YF16>(a, nn, w0, sc0, j0, a.y + row0 * a.y_row_stride, rope_tab);
+        if (p1) dc_fetch<MODE, G, DBL>(a, nn, p1, j1, w1, sc1);
+        if (p0) {
+            uint16_t* yrow = a.y + row0 * a.y_row_stride;
+            dc_slice<MODE, G, YF16>(a, nn, w0, sc0, j0, yrow, rope_tab);
+            if (DBL && j0 < nn) {
+                // the second slice: codes w0[4..7], its own scale (G = 32) or the shared one
+                uint32_t w2[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) w2[i] = i < 4 ? w0[4 + i] : 0u;
+                dc_slice<MODE, G, YF16>(a, nn, w2, G == 32 ? sc0 >> 16 : sc0, j0 + 1, yrow, rope_tab);
+            }
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) w0[i] = w1[i];
         sc0 = sc1;

@@ -722,7 +722,9 @@ kvq_status kvq_kv_decompress(const kvq_tensor* cache, const kvq_tensor* slot_map
     a.rows_vec16 = (reinterpret_cast<uintptr_t>(cache->data) % 16 == 0) && rows.row_bytes % 16 == 0 &&
                    rows.block_stride % 16 == 0;
     a.y_vec32 = (reinterpret_cast<uintptr_t>(y->data) % 32 == 0) && (ys * 2) % 32 == 0;
-    const int64_t nchunks = quant_mode == 2 ? ((T + 15) / 16) * ((a.nslice - 2) / 2 + 1)   // see kv_decompress_kernel
+    const int64_t nn = a.nslice - 2;
+    const bool dbl = quant_mode == 2 && G >= 32 && nn % 4 == 0;            // see kv_decompress_kernel
+    const int64_t nchunks = quant_mode == 2 ? ((T + 15) / 16) * ((dbl ? nn / 4 : nn / 2) + 1)
                                             : (T * a.nslice + 31) / 32;
     const int64_t need = (nchunks + (DC_THREADS / 32) - 1) / (DC_THREADS / 32);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -738,9 +740,21 @@ kvq_status kvq_kv_decompress(const kvq_tensor* cache, const kvq_tensor* slot_map
     } else if (quant_mode == 1) {
         if (yf16) KVQ_LAUNCH_DC(1, 64, true);
         else KVQ_LAUNCH_DC(1, 64, false);
-    } else if (G == 16) KVQ_LAUNCH_DC(2, 16, false);
-    else if (G == 32) KVQ_LAUNCH_DC(2, 32, false);
-    else KVQ_LAUNCH_DC(2, 64, false);
+    } else if (G == 16) {
+        KVQ_LAUNCH_DC(2, 16, false);
+    } else {
+        auto run2 = [&](auto kernel) {
+            return launch(kernel, (unsigned)persistent_grid(kernel, DC_THREADS, need), DC_THREADS, 0, s, a);
+        };
+        if (G == 32) err = dbl ? (a.nslice == 18 ? run2(kv_decompress_kernel<2, 32, 18, false, true>)
+                                                 : run2(kv_decompress_kernel<2, 32, 0, false, true>))
+                               : (a.nslice == 18 ? run2(kv_decompress_kernel<2, 32, 18, false, false>)
+                                                 : run2(kv_decompress_kernel<2, 32, 0, false, false>));
+        else err = dbl ? (a.nslice == 18 ? run2(kv_decompress_kernel<2, 64, 18, false, true>)
+                                         : run2(kv_decompress_kernel<2, 64, 0, false, true>))
+                       : (a.nslice == 18 ? run2(kv_decompress_kernel<2, 64, 18, false, false>)
+                                         : run2(kv_decompress_kernel<2, 64, 0, false, false>));
+    }
 #undef KVQ_LAUNCH_DC
     return launched(err);
 }

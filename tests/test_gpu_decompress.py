@@ -72,9 +72,18 @@ def _case(T, d, mode, G=64, kind="normal", extra=13, pad=0, seed=0, skip=0.1, sl
 
 @pytest.mark.parametrize("kind", ["normal", "wide"])
 @pytest.mark.parametrize("mode,G", [(0, 64), (1, 64), (2, 16), (2, 32), (2, 64)])
-@pytest.mark.parametrize("d", [128, 576, 1024])
+@pytest.mark.parametrize("d", [128, 320, 576, 832, 1024])
 def test_decompress_matches_oracle(mode, G, d, kind):
+    """d = 320, 576, 832: mode 2 with G = 32 / 64 takes two slices per nope lane
+    ((d - 64) / 32 a multiple of 4); d = 128, 1024 and G = 16 one slice."""
     _same(_case(203, d, mode, G, kind, seed=31))
+
+
+@pytest.mark.parametrize("G", [32, 64])
+@pytest.mark.parametrize("T", [1, 15, 16, 17, 6037])
+def test_decompress_mode2_block_tails(G, T):
+    """Row counts around the 16-row blocks of the mode-2 chunk layout."""
+    _same(_case(T, 576, 2, G, seed=47))
 
 
 @pytest.mark.parametrize("mode,G", [(0, 64), (1, 64), (2, 32)])
