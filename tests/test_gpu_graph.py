@@ -3,10 +3,12 @@
 Each call of the C ABI only enqueues kernels on the caller's stream (no
 allocation, no synchronisation), so a serving loop can capture a whole
 epilogue step once and replay it.  Checked here: a graph holding one call of
-every operation (the pipelined and the direct compress kernels, the indexer,
-the rmsnorm/rope kernel, the pipelined dequant kernel and the packed-row
-decoder), replayed on caches reset to their initial bytes, leaves every cache
-and output identical, byte for byte, to the CPU oracle's result.
+every operation (the pipelined and the direct compress kernels, bf16 and
+float16 x, the indexer, the rmsnorm/rope kernel, the pipelined dequant
+kernel, the packed-row decoder and the tcgen05 Compressor), replayed on caches
+reset to their initial bytes, leaves every cache and output identical, byte
+for byte, to the CPU oracle's result -- the Compressor's output to the same
+call run eagerly (its parity with the oracle is a bound, tested elsewhere).
 """
 import numpy as np
 import pytest
@@ -26,6 +28,8 @@ def _cases():
         W.gen_compress("g_ce0", T=5003, d=576, quant_mode=0, num_blocks=640, block_size=16,
                        head_dim=oracle.kv_cache_col(576, 0, 64) + 3, skip_frac=0.1, seed=71),
         W.compress_mode1_T64_d256(),
+        W.gen_compress("g_ce_f16", T=77, d=320, quant_mode=1, num_blocks=16, block_size=16,
+                       head_dim=oracle.kv_cache_col(320, 1, 64) + 5, skip_frac=0.1, seed=74, x_dtype="f16"),
         W.gen_indexer("g_ix", T=3001, d=128, quant_mode=3, num_blocks=128, block_size=64, cache_head_dim=64,
                       scale_head_dim=4, cache_dtype="u8", skip_frac=0.05, seed=72),
         W.rmsnorm_rope_decode_B64_D576(),
@@ -48,11 +52,13 @@ def test_graph_replay_matches_oracle():
                                       (cb.block_stride, cb.head_dim, cb.head_dim, 1))
     slots = torch.from_numpy(np.ascontiguousarray(ce.arrays["slot_mapping"])).cuda()
     y = torch.zeros((T, d), dtype=torch.bfloat16, device="cuda")
+    cp_call, _, cp_outs = W.build_call(W.gen_compressor("g_cp", T=768, H=1024, D=512, ratio=128, seed=75))
 
     def step(stream):
         for call, _, _ in built:
             call(stream)
         kvq.kv_decompress(view, slots, y, 0, 64, 1.0, stream=stream)
+        cp_call(stream)
 
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -60,6 +66,7 @@ def test_graph_replay_matches_oracle():
         step(side)                      # eager warm-up: per-kernel attributes and occupancy are set up once
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
+    cp_eager = cp_outs["cmp_kv"].clone()
 
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
@@ -69,6 +76,7 @@ def test_graph_replay_matches_oracle():
         for k in st:
             st[k].copy_(init[k])
     y.zero_()
+    cp_outs["cmp_kv"].zero_()
     kvq.get_error()
     g.replay()
     torch.cuda.synchronize()
@@ -92,4 +100,5 @@ def test_graph_replay_matches_oracle():
     y_o, _ = oracle.kv_decompress(paged(cb, st_ref), ce.arrays["slot_mapping"], d, 0, 64, 1.0,
                                   y=np.zeros((T, d), dtype=np.uint16), threads=THREADS)
     assert np.array_equal(y.view(torch.int16).cpu().numpy().view(np.uint16), y_o)
+    assert torch.equal(cp_outs["cmp_kv"], cp_eager)
     del g
