@@ -336,9 +336,13 @@ KVQ_API kvq_status kvq_convert(int32_t fmt, const float* in, int64_t n, void* ou
  * quotient; 9: the number of (x, rms) pairs, among 2^28 random ones inside
  * the rmsnorm kernel's guard (rms in [2^-60, 2^50], x a bf16 value with |x| >=
  * max(RN(rms 2^-125), 2^-103), half of them within a few ulps of a rounding
- * tie), whose unscaled two-step quotient x / rms differs in any bit from IEEE
- * division.  Blocks until done; *result receives the count (0 means the
- * shortcut is exact on the domain). */
+ * tie), whose one-step quotient x / rms (q0 = RN(x r), r = RN(1/rms), then
+ * RN(q0 + (x - q0 rms) r)) differs in any bit from IEEE division; 10: the
+ * number of (numerator, divisor) pairs, every bf16 and every f16 numerator
+ * mantissa of either sign against every binary32 divisor mantissa (both in
+ * [1, 2)), whose one-step quotient differs in any bit from IEEE division.
+ * Blocks until done; *result receives the count (0 means the shortcut is
+ * exact on the domain). */
 KVQ_API kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream);
 
 /* The memory access pattern of kv_compress_epilog without its arithmetic (no

@@ -411,7 +411,7 @@ __global__ void selftest_fp8_row_kernel() {
     if (bad) atomicAdd(&g_selftest_count, bad);
 }
 
-// The unscaled two-step quotient of the rmsnorm kernel (div2_x2_nz with r =
+// The one-step quotient of the rmsnorm kernels (div1_x2_nz with r =
 // RN(1/rms), numerators never zero) against IEEE division, 2^28 random pairs
 // per call: rms a random
 // binary32 of binade 2^-60 .. 2^49; x a random bf16 of either sign with |x| of
@@ -445,8 +445,32 @@ __global__ void selftest_rms_quot_kernel() {
         const float thr = fmaxf(__fmul_rn(rms, 2.350988701644575e-38f), 9.860761315262648e-32f);
         if (fabsf(x) < thr) continue;
         float q0, q1;
-        div2_x2_nz(x, -x, rms, __frcp_rn(rms), q0, q1);
+        div1_x2_nz(x, -x, rms, __frcp_rn(rms), q0, q1);
         const float ref = __fdiv_rn(x, rms);
+        bad += (__float_as_uint(q0) != __float_as_uint(ref) || __float_as_uint(q1) != __float_as_uint(-ref)) ? 1ull
+                                                                                                              : 0ull;
+    }
+    if (bad) atomicAdd(&g_selftest_count, bad);
+}
+
+// The one-step quotient (div1_x2_nz) of every bf16 and every f16 numerator
+// mantissa, of both signs, by every binary32 divisor mantissa (one thread per
+// divisor, 2^23 threads), numerator and divisor in [1, 2): counts the pairs
+// whose quotient differs in any bit from IEEE division.  Scaling numerator and
+// divisor by powers of two scales every intermediate exactly while they stay
+// normal, so this covers every pair whose reciprocal, quotient and residual
+// are normal.
+__global__ void selftest_quot_mant_kernel() {
+    const uint32_t j = blockIdx.x * blockDim.x + threadIdx.x;       // 0 .. 2^23 - 1
+    const float b = __uint_as_float(0x3f800000u | (j & 0x7fffffu));
+    const float r = __frcp_rn(b);
+    unsigned long long bad = 0;
+    for (uint32_t i = 0; i < 128u + 1024u; ++i) {
+        const uint32_t m = i < 128u ? i << 16 : (i - 128u) << 13;   // bf16: 7 fraction bits, f16: 10
+        const float x = __uint_as_float(0x3f800000u | m);
+        float q0, q1;
+        div1_x2_nz(x, -x, b, r, q0, q1);
+        const float ref = __fdiv_rn(x, b);
         bad += (__float_as_uint(q0) != __float_as_uint(ref) || __float_as_uint(q1) != __float_as_uint(-ref)) ? 1ull
                                                                                                               : 0ull;
     }
@@ -498,7 +522,7 @@ extern "C" {
 
 kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream) {
     if (!result) return KVQ_ERR_NULL;
-    if (which < 0 || which > 9) return KVQ_ERR_ATTR;
+    if (which < 0 || which > 10) return KVQ_ERR_ATTR;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const unsigned long long zero = 0ull;
     unsigned long long h = 0ull;
@@ -509,6 +533,7 @@ kvq_status kvq_selftest(int32_t which, uint64_t* result, kvq_stream stream) {
     else if (which == 7) selftest_timeout_kernel<<<1, 32, 0, s>>>();
     else if (which == 8) selftest_fp8_row_kernel<<<65536, 256, 0, s>>>();
     else if (which == 9) selftest_rms_quot_kernel<<<65536, 256, 0, s>>>();
+    else if (which == 10) selftest_quot_mant_kernel<<<(1u << 23) / 256u, 256, 0, s>>>();
     else selftest_div_kernel<<<65536, 256, 0, s>>>(which);
     if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
     if (cudaMemcpyFromSymbolAsync(&h, g_selftest_count, sizeof(h), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -966,6 +991,39 @@ kvq_status kvq_kv_rmsnorm_rope_cache(const kvq_tensor* kv, const kvq_tensor* gam
     auto run = [&](auto kernel, size_t sm) {
         return launched(launch(kernel, (unsigned)persistent_grid(kernel, RR_THREADS, need, sm), RR_THREADS, sm, s, a));
     };
+    // the lean kernel: Dv of 256, 512 or 1024, Dk = 64, one index entry per
+    // token, fewer than 2^31 tokens and slots, 32-bit block strides, and cache
+    // rows aligned for its whole-chunk stores (16 bytes for a 16-bit ckv
+    // cache, 8 for FP8 codes; 2 for a 16-bit k cache)
+    auto rows_aligned = [](const PagedRows& r, int64_t q) {
+        return reinterpret_cast<uintptr_t>(r.base) % q == 0 && r.row_bytes % q == 0 && r.block_stride % q == 0;
+    };
+    const bool k16 = kc.dt == CDT_BF16 || kc.dt == CDT_F16;
+    const bool lean = vec && (Dv == 256 || Dv == 512 || Dv == 1024) && Dk == 64 &&
+                      (cache_mode == 1 || cache_mode == 2) && B * S < (1LL << 31) &&
+                      kc.rows.num_slots < (1LL << 31) && cc.rows.block_stride < (1LL << 32) &&
+                      kc.rows.block_stride < (1LL << 32) && bs * cc.rows.row_bytes < (1LL << 32) &&
+                      bs * kc.rows.row_bytes < (1LL << 32) &&
+                      rows_aligned(cc.rows, cc.dt == CDT_BF16 || cc.dt == CDT_F16 ? 16 : 8) &&
+                      (!k16 || rows_aligned(kc.rows, 2));
+    if (lean) {
+        const int lck = cc.dt == CDT_E4M3 ? 1 : (cc.dt == CDT_E5M2 ? 3 : (cc.dt == CDT_I8 ? 2 : 0));
+        const size_t lsm = (size_t)Dv * sizeof(float) * (lck == 2 ? 4 : 1);
+#define KVQ_RR_LEAN(N, C) \
+    return a.kv_f16 ? run(rmsnorm_rope_lean_kernel<N, C, true>, lsm) : run(rmsnorm_rope_lean_kernel<N, C, false>, lsm)
+#define KVQ_RR_LEAN_N(N)                     \
+    switch (lck) {                           \
+        case 0: KVQ_RR_LEAN(N, 0);           \
+        case 1: KVQ_RR_LEAN(N, 1);           \
+        case 2: KVQ_RR_LEAN(N, 2);           \
+        default: KVQ_RR_LEAN(N, 3);          \
+    }
+        if (Dv == 256) KVQ_RR_LEAN_N(1);
+        if (Dv == 512) KVQ_RR_LEAN_N(2);
+        KVQ_RR_LEAN_N(4);
+#undef KVQ_RR_LEAN_N
+#undef KVQ_RR_LEAN
+    }
     const int ck = ckv_class(cc.dt);
 #define KVQ_RR_CK(N)                                                                           \
     return ck == 0 ? run(rmsnorm_rope_kernel<N, 0>, smem)                                      \

@@ -47,6 +47,32 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float f16_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
 __device__ __forceinline__ float f16_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
 
+// acc + x*x over the eight 16-bit values of v in index order (value 2i in the
+// low half of word i), each step one multiply-add on the 16-bit operands
+// (fma.rn.f32.{bf16,f16}: the operands widen exactly and the sum is rounded
+// once).  That equals the separately rounded RN(acc + RN(x*x)) whenever x*x
+// is exact in binary32: for every f16 value (11 significant bits, |x*x| in
+// [2^-48, 2^32]), and for a bf16 value that is zero or has |x| >= 2^-67
+// (8 significant bits, lowest bit >= 2^-74, so x*x is a multiple of 2^-148
+// below 2^128; a square at or above 2^128 is infinite either way).
+template <bool F16>
+__device__ __forceinline__ float sq_acc8(const uint4& v, float acc) {
+#define KVQ_SQ_ACC8(T)                                                          \
+    asm("{\n\t.reg .b16 l0, h0, l1, h1, l2, h2, l3, h3;\n\t"                     \
+        "mov.b32 {l0, h0}, %1;\n\tmov.b32 {l1, h1}, %2;\n\t"                     \
+        "mov.b32 {l2, h2}, %3;\n\tmov.b32 {l3, h3}, %4;\n\t"                     \
+        "fma.rn.f32." T " %0, l0, l0, %0;\n\tfma.rn.f32." T " %0, h0, h0, %0;\n\t" \
+        "fma.rn.f32." T " %0, l1, l1, %0;\n\tfma.rn.f32." T " %0, h1, h1, %0;\n\t" \
+        "fma.rn.f32." T " %0, l2, l2, %0;\n\tfma.rn.f32." T " %0, h2, h2, %0;\n\t" \
+        "fma.rn.f32." T " %0, l3, l3, %0;\n\tfma.rn.f32." T " %0, h3, h3, %0;\n\t}" \
+        : "+f"(acc)                                                             \
+        : "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w))
+    if (F16) KVQ_SQ_ACC8("f16");
+    else KVQ_SQ_ACC8("bf16");
+#undef KVQ_SQ_ACC8
+    return acc;
+}
+
 template <bool F16>
 __device__ __forceinline__ void widen8(const uint4& v, float (&f)[8]) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -277,9 +303,15 @@ __device__ __forceinline__ void mul_x2(float a0, float a1, float b0, float b1, f
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// div2_x2 for nonzero numerators: the quotient of a nonzero a carries a's sign
-// through every correction, so the signed-zero fix of div2_x2 is not needed.
-__device__ __forceinline__ void div2_x2_nz(float a0, float a1, float s, float r, float& q0, float& q1) {
+// a / s for nonzero numerators of at most 11 significant bits (bf16 or f16
+// values) by one correction step: q0 = RN(a r), e = a - q0 s (formed exactly
+// by the fused operation), q = RN(q0 + e r), with r = RN(1/s).  It equals
+// IEEE division whenever the reciprocal, the quotient and the residual stay
+// normal binary32 numbers: kvq_selftest 10 runs every bf16 and f16
+// numerator mantissa against every binary32 divisor mantissa, and 9 the
+// rmsnorm kernels' guard domain (their bounds on rms and |x| keep the three
+// normal).
+__device__ __forceinline__ void div1_x2_nz(float a0, float a1, float s, float r, float& q0, float& q1) {
     asm("{\n\t.reg .b64 a, ns, rr, q, e;\n\t"
         "mov.b64 a, {%2, %3};\n\t"
         "mov.b64 ns, {%4, %4};\n\t"
@@ -287,11 +319,53 @@ __device__ __forceinline__ void div2_x2_nz(float a0, float a1, float s, float r,
         "mul.rn.f32x2 q, a, rr;\n\t"
         "fma.rn.f32x2 e, q, ns, a;\n\t"
         "fma.rn.f32x2 q, e, rr, q;\n\t"
-        "fma.rn.f32x2 e, q, ns, a;\n\t"
-        "fma.rn.f32x2 q, e, rr, q;\n\t"
         "mov.b64 {%0, %1}, q;\n\t}"
         : "=f"(q0), "=f"(q1)
         : "f"(a0), "f"(a1), "f"(-s), "f"(r));
+}
+
+__device__ __forceinline__ void add_x2(float a0, float a1, float b0, float b1, float& r0, float& r1) {
+    asm("{\n\t.reg .b64 a, b, r;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 b, {%4, %5};\n\t"
+        "add.rn.f32x2 r, a, b;\n\t"
+        "mov.b64 {%0, %1}, r;\n\t}"
+        : "=f"(r0), "=f"(r1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// Two binary32 values rounded to bf16 (F16: f16), lo in bits [15:0].
+template <bool F16>
+__device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
+    uint32_t r;
+    if (F16) asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    else asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Eight FP8 codes (E4M3, or E5M2), element 0 in bits [7:0].
+template <bool E5M2>
+__device__ __forceinline__ uint2 fp8x8_packed(const float (&v)[8]) {
+    uint2 r;
+    if (E5M2)
+        asm("{\n\t.reg .b16 c0, c1, c2, c3;\n\t"
+            "cvt.rn.satfinite.e5m2x2.f32 c0, %3, %2;\n\t"
+            "cvt.rn.satfinite.e5m2x2.f32 c1, %5, %4;\n\t"
+            "cvt.rn.satfinite.e5m2x2.f32 c2, %7, %6;\n\t"
+            "cvt.rn.satfinite.e5m2x2.f32 c3, %9, %8;\n\t"
+            "mov.b32 %0, {c0, c1};\n\tmov.b32 %1, {c2, c3};\n\t}"
+            : "=r"(r.x), "=r"(r.y)
+            : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    else
+        asm("{\n\t.reg .b16 c0, c1, c2, c3;\n\t"
+            "cvt.rn.satfinite.e4m3x2.f32 c0, %3, %2;\n\t"
+            "cvt.rn.satfinite.e4m3x2.f32 c1, %5, %4;\n\t"
+            "cvt.rn.satfinite.e4m3x2.f32 c2, %7, %6;\n\t"
+            "cvt.rn.satfinite.e4m3x2.f32 c3, %9, %8;\n\t"
+            "mov.b32 %0, {c0, c1};\n\tmov.b32 %1, {c2, c3};\n\t}"
+            : "=r"(r.x), "=r"(r.y)
+            : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return r;
 }
 
 // Four binary32 values rounded half to even to integers and saturated to
@@ -353,6 +427,17 @@ __device__ __forceinline__ float int8_quant_rcp(float sc, float of) {
 __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
     uint32_t r;
     asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Smallest magnitude of the two 16-bit halves of a and b, per half (the sign
+// bits of the result are not meaningful; a NaN half yields the other
+// operand's half).
+template <bool F16>
+__device__ __forceinline__ uint32_t absmin_x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    if (F16) asm("min.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    else asm("min.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
     return r;
 }
 

@@ -293,35 +293,46 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
             // also the smallest exponent field of the lane's values (per 16-bit
             // half, on the raw bits): every value then has |x| >= 2^(e - bias),
             // and a zero or subnormal value gives e = 0
+            // (fused square-accumulate, sq_acc8: exact for f16, and for bf16
+            // lanes whose values all have |x| >= 2^-67; a lane with a smaller
+            // or zero value sums again with the square rounded first)
             float acc = 0.0f;
             const uint32_t emask = a.kv_f16 ? 0x7c007c00u : 0x7f807f80u;
             uint32_t emin2 = emask;
 #pragma unroll
             for (int m = 0; m < NCH; ++m) {
                 if (lane + 32 * m >= nch) break;
-                float f[8];
-                if (a.kv_f16) widen8<true>(xv[m], f);
-                else widen8<false>(xv[m], f);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc = __fadd_rn(acc, __fmul_rn(f[i], f[i]));
+                acc = a.kv_f16 ? sq_acc8<true>(xv[m], acc) : sq_acc8<false>(xv[m], acc);
                 emin2 = __vminu2(emin2, __vminu2(xv[m].x & emask, xv[m].y & emask));
                 emin2 = __vminu2(emin2, __vminu2(xv[m].z & emask, xv[m].w & emask));
             }
             const uint32_t emin = min(emin2 & 0xffffu, emin2 >> 16);     // 2^(e - bias) as 16-bit float bits
+            if (!a.kv_f16 && emin < 0x1e00u) {                           // 2^-67 as bf16
+                acc = 0.0f;
+#pragma unroll
+                for (int m = 0; m < NCH; ++m) {
+                    if (lane + 32 * m >= nch) break;
+                    float f[8];
+                    widen8<false>(xv[m], f);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc = __fadd_rn(acc, __fmul_rn(f[i], f[i]));
+                }
+            }
 #pragma unroll
             for (int k = 16; k >= 1; k >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(FULL_MASK, acc, k));
             const float mean = a.inv_dv != 0.0f ? __fmul_rn(acc, a.inv_dv) : __fdiv_rn(acc, (float)a.Dv);
             const float rms = __fsqrt_rn(__fadd_rn(mean, a.eps));
-            // x / rms by the two-step form (div2_x2_nz): RN(x / rms) when rms is
-            // in [2^-60, 2^50] and, per lane, every |x| is nonzero and at least
-            // max(RN(rms 2^-125), 2^-103) -- the quotient is then normal and each
-            // residual x - q rms a multiple of 2^-149, formed exactly by the
-            // fused operations (kvq_selftest 9 checks the domain; a subnormal
-            // quotient can be an exact rounding tie, which the two-step form
-            // may break the wrong way, hence the first bound), and a nonzero
-            // numerator's quotient keeps its sign without a fix.  The lane's
-            // smallest power of two 2^(e - bias) stands for its values; a lane
-            // with a zero or a smaller value divides with IEEE division.
+            // x / rms by one correction step (div1_x2_nz): RN(x / rms) when rms
+            // is in [2^-60, 2^50] and, per lane, every |x| is nonzero and at
+            // least max(RN(rms 2^-125), 2^-103) -- the reciprocal and the
+            // quotient are then normal and the residual x - q rms a multiple of
+            // 2^-149, formed exactly by the fused operation (kvq_selftest 9 and
+            // 10 check the domain; a subnormal quotient can be an exact
+            // rounding tie, which the short form may break the wrong way, hence
+            // the first bound), and a nonzero numerator's quotient keeps its
+            // sign without a fix.  The lane's smallest power of two
+            // 2^(e - bias) stands for its values; a lane with a zero or a
+            // smaller value divides with IEEE division.
             const float uthr = fmaxf(__fmul_rn(rms, 2.350988701644575e-38f), 9.860761315262648e-32f);
             const bool ufast = rms >= 8.673617379884035e-19f && rms <= 1.125899906842624e15f &&
                                half_bits(emin, a.kv_f16) >= uthr;
@@ -341,7 +352,7 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
                 }
                 if (ufast) {
 #pragma unroll
-                    for (int i = 0; i < 8; i += 2) div2_x2_nz(f[i], f[i + 1], rms, rr1, y[i], y[i + 1]);
+                    for (int i = 0; i < 8; i += 2) div1_x2_nz(f[i], f[i + 1], rms, rr1, y[i], y[i + 1]);
 #pragma unroll
                     for (int i = 0; i < 8; i += 2) mul_x2(y[i], y[i + 1], g[i], g[i + 1], y[i], y[i + 1]);
                 } else {
@@ -396,6 +407,201 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
             const float y1 = __fadd_rn(__fmul_rn(z1, c1), __fmul_rn(z0, s1));
             store_elem(a.k, krow, j, y0);
             store_elem(a.k, krow, h + j, y1);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// The lean kernel: rows of the common shape -- Dv = 256 NCH RMSNorm values
+// (lane l owns the 16-byte chunks l + 32 m), Dk = 64 RoPE values (one
+// interleaved pair per lane), one index entry per token (PA, PA_BNSD), fewer
+// than 2^31 tokens and slots, cache rows aligned for whole-chunk stores.  It
+// computes exactly what rmsnorm_rope_kernel computes, with less work per
+// token: 32-bit token and slot arithmetic, the dtypes as template parameters
+// (CK: 0 bf16 / f16 ckv, 1 E4M3, 2 int8, 3 E5M2; KF16: f16 kv, gamma, cos,
+// sin), the sum of squares by fused 16-bit multiply-adds (sq_acc8), x / rms
+// by one correction step (div1_x2_nz), and gamma staged per CTA as binary32.
+//
+// For an E4M3 / E5M2 ckv cache with a per-tensor scale s = 2^-k, 0 <= k <= 109,
+// the staged gamma is g r with r = 2^k (exact when every finite g keeps a
+// finite g r), and y r = RN(q g) r becomes RN(q (g r)): in the normal range a
+// power-of-two factor commutes with rounding, an overflow overflows in both
+// forms, and where RN(q g) is subnormal both results are at most 2^-17 in
+// magnitude, which both formats encode as the zero of the same sign.
+// ---------------------------------------------------------------------------
+template <int NCH, int CK, bool KF16>
+__global__ void __launch_bounds__(RR_THREADS, NCH >= 4 ? 6 : 8) rmsnorm_rope_lean_kernel(const RmsRopeArgs a) {
+    constexpr int DV = 256 * NCH;
+    constexpr bool FP8 = CK == 1 || CK == 3;
+    pdl_wait();
+    pdl_trigger();
+    extern __shared__ __align__(16) float rr_stage[];
+    float* gs = rr_stage;                 // [DV] gamma, or gamma * r
+    float* stg = rr_stage + DV;           // int8 ckv: [3][DV] scale, offset, RN(1/scale)
+    const int lane = threadIdx.x & 31;
+
+    // a per-tensor FP8 scale: the folded form, or the CkvDiv forms of rr_store_chunk
+    CkvDiv dv{0.0f, 0.0f, false, false};
+    bool pow2 = false;
+    if (FP8 && a.ckv.scale_n == 1) {
+        dv.s = a.ckv.scale[0];
+        const uint32_t sb = __float_as_uint(dv.s);
+        dv.pow2 = (sb & 0x807fffffu) == 0u && (sb >> 23) >= 1u && (sb >> 23) <= 254u;
+        dv.fast = dv.s >= 9.094947017729282e-13f && dv.s <= 1.099511627776e12f;
+        dv.r = (dv.fast || dv.pow2) ? __frcp_rn(dv.s) : 0.0f;
+        pow2 = dv.pow2 && (sb >> 23) >= 18u && (sb >> 23) <= 127u;   // s = 2^-k, 0 <= k <= 109
+    }
+    int ok = 1;
+    for (int i = threadIdx.x; i < DV; i += RR_THREADS) {
+        const float g = half_bits(a.gamma[i], KF16);
+        gs[i] = g;
+        if (pow2 && fabsf(g) <= 3.4028234663852886e38f && !(fabsf(__fmul_rn(g, dv.r)) <= 3.4028234663852886e38f))
+            ok = 0;
+        if (CK == 2) {
+            const float sc = a.ckv.scale[a.ckv.scale_n == 1 ? 0 : i];
+            const float of = a.ckv.offset ? a.ckv.offset[a.ckv.offset_n == 1 ? 0 : i] : 0.0f;
+            stg[i] = sc;
+            stg[DV + i] = of;
+            stg[2 * DV + i] = int8_quant_rcp(sc, of);
+        }
+    }
+    const bool fold = __syncthreads_and(ok) && pow2;
+    if (fold) {
+        for (int i = threadIdx.x; i < DV; i += RR_THREADS) gs[i] = __fmul_rn(gs[i], dv.r);
+        __syncthreads();
+    }
+
+    const uint32_t ntok = (uint32_t)(a.B * a.S);
+    const uint32_t gwarp = (blockIdx.x * RR_THREADS + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * RR_THREADS) >> 5;
+    const uint32_t rowb = (uint32_t)a.D * 2u;                     // kv row bytes
+    const char* xb = reinterpret_cast<const char*>(a.kv) + 16 * lane;
+    const char* zb = reinterpret_cast<const char*>(a.kv) + 2 * DV + 4 * lane;
+    const uint16_t* cb = a.cos + lane;
+    const uint16_t* sb = a.sin + lane;
+    const uint32_t nslots = (uint32_t)a.k.rows.num_slots;
+    const uint32_t bsz = (uint32_t)a.k.rows.block_size;
+    const int sh = a.k.rows.bs_shift;
+
+    uint4 xn[NCH];
+    int64_t vn = -1;
+    uint32_t zn = 0u, cn = 0u, sn = 0u;
+    auto fetch = [&](uint32_t t) {
+        if (t >= ntok) return;
+        const char* p = xb + (uint64_t)t * rowb;
+#pragma unroll
+        for (int m = 0; m < NCH; ++m) xn[m] = __ldg(reinterpret_cast<const uint4*>(p + 512 * m));
+        vn = a.index_i64 ? __ldg(reinterpret_cast<const long long*>(a.index) + t)
+                         : (int64_t)__ldg(reinterpret_cast<const int32_t*>(a.index) + t);
+        zn = __ldg(reinterpret_cast<const uint32_t*>(zb + (uint64_t)t * rowb));
+        const uint16_t* cp = cb + (uint64_t)t * 64u;
+        const uint16_t* sp = sb + (uint64_t)t * 64u;
+        cn = (uint32_t)__ldg(cp) | ((uint32_t)__ldg(cp + 32) << 16);
+        sn = (uint32_t)__ldg(sp) | ((uint32_t)__ldg(sp + 32) << 16);
+    };
+    fetch(gwarp);
+    for (uint32_t t = gwarp; t < ntok; t += nwarps) {
+        uint4 xv[NCH];
+#pragma unroll
+        for (int m = 0; m < NCH; ++m) xv[m] = xn[m];
+        const int64_t v = vn;
+        const uint32_t zr = zn, cr = cn, sr = sn;
+        fetch(t + nwarps);
+        if (v == -1) continue;
+        if (v < 0 || v >= (int64_t)nslots) {
+            if (lane == 0) raise_fault(FAULT_SLOT_RANGE);
+            continue;
+        }
+        const uint32_t slot = (uint32_t)v;
+        const uint32_t blk = sh >= 0 ? slot >> sh : slot / bsz;
+        const uint32_t row = slot - blk * bsz;
+        uint8_t* crow = a.ckv.rows.base + (uint64_t)blk * (uint32_t)a.ckv.rows.block_stride +
+                        row * (uint32_t)a.ckv.rows.row_bytes;
+        uint8_t* krow = a.k.rows.base + (uint64_t)blk * (uint32_t)a.k.rows.block_stride +
+                        row * (uint32_t)a.k.rows.row_bytes;
+
+        // RMSNorm: the sum of squares in the fixed lane order and the lane's
+        // smallest |x| (as 16-bit float bits)
+        float acc = 0.0f;
+        uint32_t mn = 0x7fff7fffu;
+#pragma unroll
+        for (int m = 0; m < NCH; ++m) {
+            acc = sq_acc8<KF16>(xv[m], acc);
+            mn = absmin_x2<KF16>(mn, absmin_x2<KF16>(absmin_x2<KF16>(xv[m].x, xv[m].y),
+                                                     absmin_x2<KF16>(xv[m].z, xv[m].w)));
+        }
+        mn &= 0x7fff7fffu;
+        const uint32_t emin = min(mn & 0xffffu, mn >> 16);
+        if (!KF16 && emin < 0x1e00u) {                    // a bf16 value below 2^-67, or zero
+            acc = 0.0f;
+#pragma unroll
+            for (int m = 0; m < NCH; ++m) {
+                float f[8];
+                widen8<false>(xv[m], f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc = __fadd_rn(acc, __fmul_rn(f[i], f[i]));
+            }
+        }
+#pragma unroll
+        for (int k = 16; k >= 1; k >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(FULL_MASK, acc, k));
+        const float mean = __fmul_rn(acc, 1.0f / (float)DV);              // exact: DV is a power of two
+        const float rms = __fsqrt_rn(__fadd_rn(mean, a.eps));
+        // the guard of the one-step quotient (as in rmsnorm_rope_kernel)
+        const float uthr = fmaxf(__fmul_rn(rms, 2.350988701644575e-38f), 9.860761315262648e-32f);
+        const bool ufast = rms >= 8.673617379884035e-19f && rms <= 1.125899906842624e15f &&
+                           half_bits(emin, KF16) >= uthr;
+        const float rr1 = ufast ? __frcp_rn(rms) : 0.0f;
+#pragma unroll
+        for (int m = 0; m < NCH; ++m) {
+            const int c = lane + 32 * m;
+            float f[8], y[8];
+            widen8<KF16>(xv[m], f);
+            if (ufast) {
+#pragma unroll
+                for (int i = 0; i < 8; i += 2) div1_x2_nz(f[i], f[i + 1], rms, rr1, y[i], y[i + 1]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] = __fdiv_rn(f[i], rms);
+            }
+            const float4 g0 = *reinterpret_cast<const float4*>(gs + 8 * c);
+            const float4 g1 = *reinterpret_cast<const float4*>(gs + 8 * c + 4);
+            mul_x2(y[0], y[1], g0.x, g0.y, y[0], y[1]);
+            mul_x2(y[2], y[3], g0.z, g0.w, y[2], y[3]);
+            mul_x2(y[4], y[5], g1.x, g1.y, y[4], y[5]);
+            mul_x2(y[6], y[7], g1.z, g1.w, y[6], y[7]);
+            if (CK == 0) {
+                uint4 w;
+                if (a.ckv.dt == CDT_BF16)
+                    w = make_uint4(half2_bits<false>(y[0], y[1]), half2_bits<false>(y[2], y[3]),
+                                   half2_bits<false>(y[4], y[5]), half2_bits<false>(y[6], y[7]));
+                else
+                    w = make_uint4(half2_bits<true>(y[0], y[1]), half2_bits<true>(y[2], y[3]),
+                                   half2_bits<true>(y[4], y[5]), half2_bits<true>(y[6], y[7]));
+                *reinterpret_cast<uint4*>(crow + 16 * c) = w;
+            } else if (FP8) {
+                if (fold) *reinterpret_cast<uint2*>(crow + 8 * c) = fp8x8_packed<CK == 3>(y);
+                else rr_store_chunk<1>(a.ckv, crow, c, y, dv, nullptr, DV);
+            } else {
+                rr_store_chunk<2>(a.ckv, crow, c, y, dv, stg, DV);
+            }
+        }
+
+        // interleaved RoPE on this lane's pair j = lane:
+        // y_j = z_2j c_j - z_2j+1 s_j, y_32+j = z_2j+1 c_32+j + z_2j s_32+j
+        const float z0 = half_bits(zr & 0xffffu, KF16), z1 = half_bits(zr >> 16, KF16);
+        const float c0 = half_bits(cr & 0xffffu, KF16), c1 = half_bits(cr >> 16, KF16);
+        const float s0 = half_bits(sr & 0xffffu, KF16), s1 = half_bits(sr >> 16, KF16);
+        float p0, p1, q0, q1, y0, y1;
+        mul_x2(z0, z1, c0, c1, p0, p1);
+        mul_x2(-z1, z0, s0, s1, q0, q1);
+        add_x2(p0, p1, q0, q1, y0, y1);
+        if (a.k.dt == CDT_BF16 || a.k.dt == CDT_F16) {
+            const uint32_t w = a.k.dt == CDT_BF16 ? half2_bits<false>(y0, y1) : half2_bits<true>(y0, y1);
+            *reinterpret_cast<uint16_t*>(krow + 2 * lane) = (uint16_t)w;
+            *reinterpret_cast<uint16_t*>(krow + 64 + 2 * lane) = (uint16_t)(w >> 16);
+        } else {
+            store_elem(a.k, krow, lane, y0);
+            store_elem(a.k, krow, 32 + lane, y1);
         }
     }
 }

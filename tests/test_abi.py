@@ -277,9 +277,9 @@ def test_row_widths_beyond_32_bit_indexing_are_rejected(L):
 
 
 def test_selftest_numbering(L):
-    """Self-tests 0..9 exist; other numbers and a NULL result are rejected before any device work."""
+    """Self-tests 0..10 exist; other numbers and a NULL result are rejected before any device work."""
     out = ctypes.c_uint64(0)
-    assert L.kvq_selftest(10, ctypes.byref(out), None) == EATTR
+    assert L.kvq_selftest(11, ctypes.byref(out), None) == EATTR
     assert L.kvq_selftest(-1, ctypes.byref(out), None) == EATTR
     assert L.kvq_selftest(0, None, None) == ENULL
 

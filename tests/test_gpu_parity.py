@@ -227,7 +227,7 @@ def test_indexer_bad_slot_fault():
 # ---------------------------------------------------------------------------
 def _rr(cache_mode="PA_BNSD", B=40, S=1, k_dtype="bf16", ckv_dtype="e4m3", kv_dtype="bf16", D=576, Dv=512,
         seed=0, **kw):
-    opt = {}
+    opt = {"block_pad_bytes": 64}
     if ckv_dtype in ("e4m3", "e5m2", "i8"):
         opt["ckv_scale"] = [1 / 64]
     if k_dtype in ("e4m3", "e5m2", "i8"):
@@ -238,7 +238,7 @@ def _rr(cache_mode="PA_BNSD", B=40, S=1, k_dtype="bf16", ckv_dtype="e4m3", kv_dt
     return W.gen_rmsnorm_rope(f"rr_{cache_mode}_{k_dtype}_{ckv_dtype}_{kv_dtype}_D{D}", B=B, S=S, D=D, Dv=Dv,
                               num_blocks=max(B + 1, (2 * B * S) // 32 + 2), block_size=32, k_dtype=k_dtype,
                               ckv_dtype=ckv_dtype, cache_mode=cache_mode, skip_frac=0.1, seed=seed,
-                              kv_dtype=kv_dtype, block_pad_bytes=64, **opt)
+                              kv_dtype=kv_dtype, **opt)
 
 
 @pytest.mark.parametrize("cache_mode,S", [("PA_BNSD", 1), ("PA", 3), ("Norm", 5), ("PA_BLK_BNSD", 70)])
@@ -294,6 +294,65 @@ def test_rmsnorm_rope_subnormal_and_tie_quotients(ckv_dtype):
         kv[r, cols[:6]] = rng.integers(1, 128, size=6).astype(np.uint16) | sign
         kv[r, cols[6:9]] = 0
         kv[r, cols[9:]] = bits(2.0 ** 40)
+    _same(case)
+
+
+# The lean kernel takes Dv of 256, 512 or 1024 with Dk = 64, PA / PA_BNSD,
+# cache rows aligned for whole-chunk stores; the cases below reach each of its
+# template instances and the per-tensor FP8 scale forms.
+@pytest.mark.parametrize("kv_dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("D,Dv", [(320, 256), (576, 512), (1088, 1024)])
+def test_rmsnorm_rope_lean_shapes(D, Dv, kv_dtype):
+    for i, (k_dtype, ckv_dtype) in enumerate([(kv_dtype, kv_dtype), (kv_dtype, "e4m3"), (kv_dtype, "e5m2"),
+                                              ("i8", "i8"), ("e5m2", "e5m2")]):
+        _same(_rr("PA" if i % 2 else "PA_BNSD", B=70, S=1, D=D, Dv=Dv, kv_dtype=kv_dtype, k_dtype=k_dtype,
+                  ckv_dtype=ckv_dtype, seed=100 + i, slot_dtype=np.int64 if i == 3 else np.int32))
+
+
+@pytest.mark.parametrize("ckv_dtype", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("scale", [1 / 64, 2.0 ** -109, 2.0 ** -110, 1.0, 8.0, 0.013, "per_channel", "big_gamma"])
+def test_rmsnorm_rope_fp8_scale_forms(ckv_dtype, scale):
+    """The per-tensor power-of-two scales 2^-k with 0 <= k <= 109 fold into the
+    staged gamma; 2^-110, 8 (k < 0), a scale that is not a power of two, a
+    per-channel scale, and a gamma whose product with 64 overflows take the
+    separate forms."""
+    kw = {}
+    if scale == "per_channel":
+        kw["ckv_scale"] = (2.0 ** np.random.default_rng(3).integers(-8, 0, 512)).tolist()
+    elif scale == "big_gamma":
+        kw["ckv_scale"] = [1 / 64]
+    else:
+        kw["ckv_scale"] = [scale]
+    case = _rr(B=64, ckv_dtype=ckv_dtype, seed=61, **kw)
+    if scale == "big_gamma":
+        case.arrays["gamma"][[5, 300]] = W.to_bf16_bits(np.array([2.0 ** 126, -3.0 * 2.0 ** 125], np.float32))
+    _same(case)
+
+
+@pytest.mark.parametrize("ckv_dtype,pad", [("e4m3", 8), ("bf16", 8), ("e4m3", 4), ("bf16", 2)])
+def test_rmsnorm_rope_cache_row_alignment(ckv_dtype, pad):
+    """Cache blocks padded so that rows are 8-, 4- or 2-byte aligned only:
+    the lean kernel takes the 8-aligned FP8 cache, the general kernel the
+    rest."""
+    _same(_rr(B=60, ckv_dtype=ckv_dtype, seed=67, block_pad_bytes=pad))
+
+
+@pytest.mark.parametrize("ckv_dtype", ["bf16", "e4m3", "i8"])
+def test_rmsnorm_rope_tiny_rows(ckv_dtype):
+    """Rows of tiny values (epsilon 0), so that the squares are subnormal
+    binary32 numbers: bf16 exponent fields drawn from [50, 59] (|x| < 2^-67,
+    x * x not exact in binary32), from [60, 70] (x * x exact), or both mixed
+    in one row; the sum of squares must match the separately rounded
+    RN(acc + RN(x * x)) of the page's formula either way."""
+    case = _rr(B=48, ckv_dtype=ckv_dtype, k_dtype="bf16", seed=47, epsilon=0.0)
+    kv = case.arrays["kv"].reshape(48, 576)
+    rng = np.random.default_rng(53)
+    for r in range(48):
+        lo, hi = ((50, 59), (60, 70), (50, 70))[r % 3]
+        e = rng.integers(lo, hi + 1, size=512).astype(np.uint16)
+        m = rng.integers(0, 128, size=512).astype(np.uint16)
+        sign = (rng.integers(0, 2, size=512) << 15).astype(np.uint16)
+        kv[r, :512] = sign | (e << 7) | m
     _same(case)
 
 

@@ -14,8 +14,10 @@ whole input domain against IEEE division:
   * the indexer fp8 mode's division by the row scale (two-step Markstein form
     where the row maximum is a finite value >= 2^-60): the same E4M3 and E5M2
     codes as IEEE division on 2^28 random bf16 / f16 (value, maximum) pairs;
-  * the rmsnorm kernel's unscaled x / rms (two-step Markstein form inside its
-    guard): bit-identical to IEEE division on 2^28 random and near-tie pairs.
+  * the rmsnorm kernels' unscaled x / rms (one-step Markstein form inside
+    their guard): bit-identical to IEEE division on 2^28 random and near-tie
+    pairs, and for every bf16 and f16 numerator mantissa against every
+    binary32 divisor mantissa.
 Also the failure path of the pipelined kernels' bounded waits: a wait on a
 barrier that nothing completes gives up after its limit and reports
 FAULT_TIMEOUT through the fault word (no GPU fault, hang or trap)."""
@@ -31,7 +33,8 @@ pytestmark = pytest.mark.gpu
                                         (4, "constant-divisor scale quotients"),
                                         (6, "int8 codes of the reciprocal-based quotient"),
                                         (8, "fp8 row-scale codes of the two-step quotient"),
-                                        (9, "unscaled two-step quotient x / rms")])
+                                        (9, "unscaled one-step quotient x / rms"),
+                                        (10, "one-step quotient, every 16-bit numerator mantissa")])
 def test_shortcut_is_exact(which, what):
     assert kvq.selftest(which) == 0, what
 
