@@ -324,16 +324,6 @@ __device__ __forceinline__ void div1_x2_nz(float a0, float a1, float s, float r,
         : "f"(a0), "f"(a1), "f"(-s), "f"(r));
 }
 
-__device__ __forceinline__ void add_x2(float a0, float a1, float b0, float b1, float& r0, float& r1) {
-    asm("{\n\t.reg .b64 a, b, r;\n\t"
-        "mov.b64 a, {%2, %3};\n\t"
-        "mov.b64 b, {%4, %5};\n\t"
-        "add.rn.f32x2 r, a, b;\n\t"
-        "mov.b64 {%0, %1}, r;\n\t}"
-        : "=f"(r0), "=f"(r1)
-        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
-
 // Two binary32 values rounded to bf16 (F16: f16), lo in bits [15:0].
 template <bool F16>
 __device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {

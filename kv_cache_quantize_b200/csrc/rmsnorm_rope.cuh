@@ -591,10 +591,10 @@ __global__ void __launch_bounds__(RR_THREADS, NCH >= 4 ? 6 : 8) rmsnorm_rope_lea
         const float z0 = half_bits(zr & 0xffffu, KF16), z1 = half_bits(zr >> 16, KF16);
         const float c0 = half_bits(cr & 0xffffu, KF16), c1 = half_bits(cr >> 16, KF16);
         const float s0 = half_bits(sr & 0xffffu, KF16), s1 = half_bits(sr >> 16, KF16);
-        float p0, p1, q0, q1, y0, y1;
-        mul_x2(z0, z1, c0, c1, p0, p1);
-        mul_x2(-z1, z0, s0, s1, q0, q1);
-        add_x2(p0, p1, q0, q1, y0, y1);
+        // (scalar products and sums: -fmad=false keeps them separately rounded,
+        // where a packed product followed by a packed add may be fused)
+        const float y0 = __fadd_rn(__fmul_rn(z0, c0), __fmul_rn(-z1, s0));
+        const float y1 = __fadd_rn(__fmul_rn(z1, c1), __fmul_rn(z0, s1));
         if (a.k.dt == CDT_BF16 || a.k.dt == CDT_F16) {
             const uint32_t w = a.k.dt == CDT_BF16 ? half2_bits<false>(y0, y1) : half2_bits<true>(y0, y1);
             *reinterpret_cast<uint16_t*>(krow + 2 * lane) = (uint16_t)w;
