@@ -381,23 +381,17 @@ __device__ __forceinline__ uint32_t int8x4_rne_sat(float v0, float v1, float v2,
 // and result, so it equals the IEEE quotient; below 2^-30 the rounded sum
 // with any binary32 offset, hence the integer, does not depend on the
 // quotient's last bits; above 2^20 the integer saturates either way.  Other
-// lanes divide with IEEE division.  kvq_selftest checks the two paths against
-// each other on random and near-tie triples.
-__device__ __forceinline__ float div2_add(float a, float s, float r, float f) {
-    const float q0 = __fmul_rn(a, r);
-    const float q1 = __fmaf_rn(__fmaf_rn(-q0, s, a), r, q0);
-    const float q2 = __fmaf_rn(__fmaf_rn(-q1, s, a), r, q1);
-    return __fadd_rn(q2, f);
-}
-
+// lanes divide with IEEE division.  kvq_selftest 6 checks the two paths
+// against each other on random and near-tie triples.  The quotients run on
+// packed pairs (div2_add_x2).
 __device__ __forceinline__ uint32_t int8x4_quant(const float (&o)[4], const float (&s)[4], const float (&f)[4],
                                                  const float (&r)[4]) {
     float q[4];
     const float m = fmaxf(fmaxf(fabsf(o[0]), fabsf(o[1])), fmaxf(fabsf(o[2]), fabsf(o[3])));
     const float rmin = fminf(fminf(r[0], r[1]), fminf(r[2], r[3]));
     if (m <= 1.152921504606846976e18f && rmin > 0.0f) {      // |o| <= 2^60, every channel eligible
-#pragma unroll
-        for (int k = 0; k < 4; ++k) q[k] = div2_add(o[k], s[k], r[k], f[k]);
+        div2_add_x2(o[0], o[1], s[0], s[1], r[0], r[1], f[0], f[1], q[0], q[1]);
+        div2_add_x2(o[2], o[3], s[2], s[3], r[2], r[3], f[2], f[3], q[2], q[3]);
     } else {
 #pragma unroll
         for (int k = 0; k < 4; ++k) q[k] = __fadd_rn(__fdiv_rn(o[k], s[k]), f[k]);
