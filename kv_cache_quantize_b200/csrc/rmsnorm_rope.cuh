@@ -429,19 +429,15 @@ __global__ void __launch_bounds__(RR_THREADS, 8) rmsnorm_rope_kernel(const RmsRo
 // forms, and where RN(q g) is subnormal both results are at most 2^-17 in
 // magnitude, which both formats encode as the zero of the same sign.
 // ---------------------------------------------------------------------------
+// The staged gamma (g, or g r when the FP8 scale folds in) and, for an int8
+// ckv cache, its per-channel scale, offset and RN(1/scale) ([3][DV] at stg),
+// written by the CTA's threads; returns whether the scale folded in.  dv
+// receives the per-tensor FP8 scale forms.  Every thread of the CTA calls it.
 template <int NCH, int CK, bool KF16>
-__global__ void __launch_bounds__(RR_THREADS, NCH >= 4 ? 6 : 8) rmsnorm_rope_lean_kernel(const RmsRopeArgs a) {
+__device__ __forceinline__ bool rr_lean_stage(const RmsRopeArgs& a, float* gs, float* stg, CkvDiv& dv) {
     constexpr int DV = 256 * NCH;
     constexpr bool FP8 = CK == 1 || CK == 3;
-    pdl_wait();
-    pdl_trigger();
-    extern __shared__ __align__(16) float rr_stage[];
-    float* gs = rr_stage;                 // [DV] gamma, or gamma * r
-    float* stg = rr_stage + DV;           // int8 ckv: [3][DV] scale, offset, RN(1/scale)
-    const int lane = threadIdx.x & 31;
-
-    // a per-tensor FP8 scale: the folded form, or the CkvDiv forms of rr_store_chunk
-    CkvDiv dv{0.0f, 0.0f, false, false};
+    dv = CkvDiv{0.0f, 0.0f, false, false};
     bool pow2 = false;
     if (FP8 && a.ckv.scale_n == 1) {
         dv.s = a.ckv.scale[0];
@@ -452,7 +448,7 @@ __global__ void __launch_bounds__(RR_THREADS, NCH >= 4 ? 6 : 8) rmsnorm_rope_lea
         pow2 = dv.pow2 && (sb >> 23) >= 18u && (sb >> 23) <= 127u;   // s = 2^-k, 0 <= k <= 109
     }
     int ok = 1;
-    for (int i = threadIdx.x; i < DV; i += RR_THREADS) {
+    for (int i = threadIdx.x; i < DV; i += blockDim.x) {
         const float g = half_bits(a.gamma[i], KF16);
         gs[i] = g;
         if (pow2 && fabsf(g) <= 3.4028234663852886e38f && !(fabsf(__fmul_rn(g, dv.r)) <= 3.4028234663852886e38f))
@@ -467,9 +463,129 @@ __global__ void __launch_bounds__(RR_THREADS, NCH >= 4 ? 6 : 8) rmsnorm_rope_lea
     }
     const bool fold = __syncthreads_and(ok) && pow2;
     if (fold) {
-        for (int i = threadIdx.x; i < DV; i += RR_THREADS) gs[i] = __fmul_rn(gs[i], dv.r);
+        for (int i = threadIdx.x; i < DV; i += blockDim.x) gs[i] = __fmul_rn(gs[i], dv.r);
         __syncthreads();
     }
+    return fold;
+}
+
+// One token of the lean kernels, computed by one warp: RMSNorm of this lane's
+// chunks xv[m] (values 8 (lane + 32 m) .. + 7) into the ckv cache row and
+// RoPE of its pair j = lane (zr: values Dv + 2j, Dv + 2j + 1; cr, sr: cos and
+// sin at j and 32 + j) into the k cache row, both rows of cache slot `slot`.
+template <int NCH, int CK, bool KF16>
+__device__ __forceinline__ void rr_lean_token(const RmsRopeArgs& a, const uint4 (&xv)[NCH], uint32_t zr, uint32_t cr,
+                                              uint32_t sr, uint32_t slot, const float* gs, const float* stg,
+                                              const CkvDiv& dv, bool fold, int lane) {
+    constexpr int DV = 256 * NCH;
+    constexpr bool FP8 = CK == 1 || CK == 3;
+    const uint32_t bsz = (uint32_t)a.k.rows.block_size;
+    const int sh = a.k.rows.bs_shift;
+    const uint32_t blk = sh >= 0 ? slot >> sh : slot / bsz;
+    const uint32_t row = slot - blk * bsz;
+    uint8_t* crow = a.ckv.rows.base + (uint64_t)blk * (uint32_t)a.ckv.rows.block_stride +
+                    row * (uint32_t)a.ckv.rows.row_bytes;
+    uint8_t* krow = a.k.rows.base + (uint64_t)blk * (uint32_t)a.k.rows.block_stride +
+                    row * (uint32_t)a.k.rows.row_bytes;
+
+    // RMSNorm: the sum of squares in the fixed lane order and the lane's
+    // smallest |x| (as 16-bit float bits)
+    float acc = 0.0f;
+    uint32_t mn = 0x7fff7fffu;
+#pragma unroll
+    for (int m = 0; m < NCH; ++m) {
+        acc = sq_acc8<KF16>(xv[m], acc);
+        mn = absmin_x2<KF16>(mn, absmin_x2<KF16>(absmin_x2<KF16>(xv[m].x, xv[m].y),
+                                                 absmin_x2<KF16>(xv[m].z, xv[m].w)));
+    }
+    mn &= 0x7fff7fffu;
+    const uint32_t emin = min(mn & 0xffffu, mn >> 16);
+    if (!KF16 && emin < 0x1e00u) {                    // a bf16 value below 2^-67, or zero
+        acc = 0.0f;
+#pragma unroll
+        for (int m = 0; m < NCH; ++m) {
+            float f[8];
+            widen8<false>(xv[m], f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc = __fadd_rn(acc, __fmul_rn(f[i], f[i]));
+        }
+    }
+#pragma unroll
+    for (int k = 16; k >= 1; k >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(FULL_MASK, acc, k));
+    const float mean = __fmul_rn(acc, 1.0f / (float)DV);              // exact: DV is a power of two
+    const float rms = __fsqrt_rn(__fadd_rn(mean, a.eps));
+    // the guard of the one-step quotient (as in rmsnorm_rope_kernel)
+    const float uthr = fmaxf(__fmul_rn(rms, 2.350988701644575e-38f), 9.860761315262648e-32f);
+    const bool ufast = rms >= 8.673617379884035e-19f && rms <= 1.125899906842624e15f &&
+                       half_bits(emin, KF16) >= uthr;
+    const float rr1 = ufast ? __frcp_rn(rms) : 0.0f;
+#pragma unroll
+    for (int m = 0; m < NCH; ++m) {
+        const int c = lane + 32 * m;
+        float f[8], y[8];
+        widen8<KF16>(xv[m], f);
+        if (ufast) {
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) div1_x2_nz(f[i], f[i + 1], rms, rr1, y[i], y[i + 1]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = __fdiv_rn(f[i], rms);
+        }
+        const float4 g0 = *reinterpret_cast<const float4*>(gs + 8 * c);
+        const float4 g1 = *reinterpret_cast<const float4*>(gs + 8 * c + 4);
+        mul_x2(y[0], y[1], g0.x, g0.y, y[0], y[1]);
+        mul_x2(y[2], y[3], g0.z, g0.w, y[2], y[3]);
+        mul_x2(y[4], y[5], g1.x, g1.y, y[4], y[5]);
+        mul_x2(y[6], y[7], g1.z, g1.w, y[6], y[7]);
+        if (CK == 0) {
+            uint4 w;
+            if (a.ckv.dt == CDT_BF16)
+                w = make_uint4(half2_bits<false>(y[0], y[1]), half2_bits<false>(y[2], y[3]),
+                               half2_bits<false>(y[4], y[5]), half2_bits<false>(y[6], y[7]));
+            else
+                w = make_uint4(half2_bits<true>(y[0], y[1]), half2_bits<true>(y[2], y[3]),
+                               half2_bits<true>(y[4], y[5]), half2_bits<true>(y[6], y[7]));
+            *reinterpret_cast<uint4*>(crow + 16 * c) = w;
+        } else if (FP8) {
+            if (fold) *reinterpret_cast<uint2*>(crow + 8 * c) = fp8x8_packed<CK == 3>(y);
+            else rr_store_chunk<1>(a.ckv, crow, c, y, dv, nullptr, DV);
+        } else {
+            rr_store_chunk<2>(a.ckv, crow, c, y, dv, stg, DV);
+        }
+    }
+
+    // interleaved RoPE on this lane's pair j = lane:
+    // y_j = z_2j c_j - z_2j+1 s_j, y_32+j = z_2j+1 c_32+j + z_2j s_32+j
+    // (scalar products and sums: -fmad=false keeps them separately rounded,
+    // where a packed product followed by a packed add may be fused)
+    const float z0 = half_bits(zr & 0xffffu, KF16), z1 = half_bits(zr >> 16, KF16);
+    const float c0 = half_bits(cr & 0xffffu, KF16), c1 = half_bits(cr >> 16, KF16);
+    const float s0 = half_bits(sr & 0xffffu, KF16), s1 = half_bits(sr >> 16, KF16);
+    const float y0 = __fadd_rn(__fmul_rn(z0, c0), __fmul_rn(-z1, s0));
+    const float y1 = __fadd_rn(__fmul_rn(z1, c1), __fmul_rn(z0, s1));
+    if (a.k.dt == CDT_BF16 || a.k.dt == CDT_F16) {
+        const uint32_t w = a.k.dt == CDT_BF16 ? half2_bits<false>(y0, y1) : half2_bits<true>(y0, y1);
+        *reinterpret_cast<uint16_t*>(krow + 2 * lane) = (uint16_t)w;
+        *reinterpret_cast<uint16_t*>(krow + 64 + 2 * lane) = (uint16_t)(w >> 16);
+    } else {
+        store_elem(a.k, krow, lane, y0);
+        store_elem(a.k, krow, 32 + lane, y1);
+    }
+}
+
+// Each warp loads its next token's chunks, index entry and RoPE inputs one
+// token ahead.
+template <int NCH, int CK, bool KF16>
+__global__ void __launch_bounds__(RR_THREADS, NCH >= 4 ? 6 : 8) rmsnorm_rope_lean_kernel(const RmsRopeArgs a) {
+    constexpr int DV = 256 * NCH;
+    pdl_wait();
+    pdl_trigger();
+    extern __shared__ __align__(16) float rr_stage[];
+    float* gs = rr_stage;                 // [DV] gamma, or gamma * r
+    float* stg = rr_stage + DV;           // int8 ckv: [3][DV] scale, offset, RN(1/scale)
+    const int lane = threadIdx.x & 31;
+    CkvDiv dv;
+    const bool fold = rr_lean_stage<NCH, CK, KF16>(a, gs, stg, dv);
 
     const uint32_t ntok = (uint32_t)(a.B * a.S);
     const uint32_t gwarp = (blockIdx.x * RR_THREADS + threadIdx.x) >> 5;
@@ -480,8 +596,6 @@ __global__ void __launch_bounds__(RR_THREADS, NCH >= 4 ? 6 : 8) rmsnorm_rope_lea
     const uint16_t* cb = a.cos + lane;
     const uint16_t* sb = a.sin + lane;
     const uint32_t nslots = (uint32_t)a.k.rows.num_slots;
-    const uint32_t bsz = (uint32_t)a.k.rows.block_size;
-    const int sh = a.k.rows.bs_shift;
 
     uint4 xn[NCH];
     int64_t vn = -1;
@@ -512,97 +626,7 @@ __global__ void __launch_bounds__(RR_THREADS, NCH >= 4 ? 6 : 8) rmsnorm_rope_lea
             if (lane == 0) raise_fault(FAULT_SLOT_RANGE);
             continue;
         }
-        const uint32_t slot = (uint32_t)v;
-        const uint32_t blk = sh >= 0 ? slot >> sh : slot / bsz;
-        const uint32_t row = slot - blk * bsz;
-        uint8_t* crow = a.ckv.rows.base + (uint64_t)blk * (uint32_t)a.ckv.rows.block_stride +
-                        row * (uint32_t)a.ckv.rows.row_bytes;
-        uint8_t* krow = a.k.rows.base + (uint64_t)blk * (uint32_t)a.k.rows.block_stride +
-                        row * (uint32_t)a.k.rows.row_bytes;
-
-        // RMSNorm: the sum of squares in the fixed lane order and the lane's
-        // smallest |x| (as 16-bit float bits)
-        float acc = 0.0f;
-        uint32_t mn = 0x7fff7fffu;
-#pragma unroll
-        for (int m = 0; m < NCH; ++m) {
-            acc = sq_acc8<KF16>(xv[m], acc);
-            mn = absmin_x2<KF16>(mn, absmin_x2<KF16>(absmin_x2<KF16>(xv[m].x, xv[m].y),
-                                                     absmin_x2<KF16>(xv[m].z, xv[m].w)));
-        }
-        mn &= 0x7fff7fffu;
-        const uint32_t emin = min(mn & 0xffffu, mn >> 16);
-        if (!KF16 && emin < 0x1e00u) {                    // a bf16 value below 2^-67, or zero
-            acc = 0.0f;
-#pragma unroll
-            for (int m = 0; m < NCH; ++m) {
-                float f[8];
-                widen8<false>(xv[m], f);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc = __fadd_rn(acc, __fmul_rn(f[i], f[i]));
-            }
-        }
-#pragma unroll
-        for (int k = 16; k >= 1; k >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(FULL_MASK, acc, k));
-        const float mean = __fmul_rn(acc, 1.0f / (float)DV);              // exact: DV is a power of two
-        const float rms = __fsqrt_rn(__fadd_rn(mean, a.eps));
-        // the guard of the one-step quotient (as in rmsnorm_rope_kernel)
-        const float uthr = fmaxf(__fmul_rn(rms, 2.350988701644575e-38f), 9.860761315262648e-32f);
-        const bool ufast = rms >= 8.673617379884035e-19f && rms <= 1.125899906842624e15f &&
-                           half_bits(emin, KF16) >= uthr;
-        const float rr1 = ufast ? __frcp_rn(rms) : 0.0f;
-#pragma unroll
-        for (int m = 0; m < NCH; ++m) {
-            const int c = lane + 32 * m;
-            float f[8], y[8];
-            widen8<KF16>(xv[m], f);
-            if (ufast) {
-#pragma unroll
-                for (int i = 0; i < 8; i += 2) div1_x2_nz(f[i], f[i + 1], rms, rr1, y[i], y[i + 1]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) y[i] = __fdiv_rn(f[i], rms);
-            }
-            const float4 g0 = *reinterpret_cast<const float4*>(gs + 8 * c);
-            const float4 g1 = *reinterpret_cast<const float4*>(gs + 8 * c + 4);
-            mul_x2(y[0], y[1], g0.x, g0.y, y[0], y[1]);
-            mul_x2(y[2], y[3], g0.z, g0.w, y[2], y[3]);
-            mul_x2(y[4], y[5], g1.x, g1.y, y[4], y[5]);
-            mul_x2(y[6], y[7], g1.z, g1.w, y[6], y[7]);
-            if (CK == 0) {
-                uint4 w;
-                if (a.ckv.dt == CDT_BF16)
-                    w = make_uint4(half2_bits<false>(y[0], y[1]), half2_bits<false>(y[2], y[3]),
-                                   half2_bits<false>(y[4], y[5]), half2_bits<false>(y[6], y[7]));
-                else
-                    w = make_uint4(half2_bits<true>(y[0], y[1]), half2_bits<true>(y[2], y[3]),
-                                   half2_bits<true>(y[4], y[5]), half2_bits<true>(y[6], y[7]));
-                *reinterpret_cast<uint4*>(crow + 16 * c) = w;
-            } else if (FP8) {
-                if (fold) *reinterpret_cast<uint2*>(crow + 8 * c) = fp8x8_packed<CK == 3>(y);
-                else rr_store_chunk<1>(a.ckv, crow, c, y, dv, nullptr, DV);
-            } else {
-                rr_store_chunk<2>(a.ckv, crow, c, y, dv, stg, DV);
-            }
-        }
-
-        // interleaved RoPE on this lane's pair j = lane:
-        // y_j = z_2j c_j - z_2j+1 s_j, y_32+j = z_2j+1 c_32+j + z_2j s_32+j
-        const float z0 = half_bits(zr & 0xffffu, KF16), z1 = half_bits(zr >> 16, KF16);
-        const float c0 = half_bits(cr & 0xffffu, KF16), c1 = half_bits(cr >> 16, KF16);
-        const float s0 = half_bits(sr & 0xffffu, KF16), s1 = half_bits(sr >> 16, KF16);
-        // (scalar products and sums: -fmad=false keeps them separately rounded,
-        // where a packed product followed by a packed add may be fused)
-        const float y0 = __fadd_rn(__fmul_rn(z0, c0), __fmul_rn(-z1, s0));
-        const float y1 = __fadd_rn(__fmul_rn(z1, c1), __fmul_rn(z0, s1));
-        if (a.k.dt == CDT_BF16 || a.k.dt == CDT_F16) {
-            const uint32_t w = a.k.dt == CDT_BF16 ? half2_bits<false>(y0, y1) : half2_bits<true>(y0, y1);
-            *reinterpret_cast<uint16_t*>(krow + 2 * lane) = (uint16_t)w;
-            *reinterpret_cast<uint16_t*>(krow + 64 + 2 * lane) = (uint16_t)(w >> 16);
-        } else {
-            store_elem(a.k, krow, lane, y0);
-            store_elem(a.k, krow, 32 + lane, y1);
-        }
+        rr_lean_token<NCH, CK, KF16>(a, xv, zr, cr, sr, (uint32_t)v, gs, stg, dv, fold, lane);
     }
 }
 

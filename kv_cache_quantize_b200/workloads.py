@@ -461,8 +461,9 @@ def build_call(case: Case, misalign: bool = False):
     Returns (call, storages, outputs): call(stream=None) enqueues the operation;
     storages maps each cache name to the device copy of its whole byte buffer;
     outputs collects the dense outputs (q_out, k_out, v_out) after a call.
-    misalign: dequant_rope_quant_kvcache's x, cos and sin start one element
-    past a 16-byte boundary.
+    misalign: dequant_rope_quant_kvcache's x, cos and sin, and
+    kv_rmsnorm_rope_cache's cos and sin, start one element past a 16-byte
+    boundary.
     """
     import kv_cache_quantize_b200 as kvq
     a, at = case.arrays, case.attrs
@@ -489,6 +490,8 @@ def build_call(case: Case, misalign: bool = False):
         st["ckv_cache"], views["ckv_cache"] = dev_cache(case.caches["ckv_cache"], TORCH_DT[at["ckv_dtype"]])
         kv = half_tensor(a["kv"], kdt)
         gamma, cos, sin = half_tensor(a["gamma"], kdt), half_tensor(a["cos"], kdt), half_tensor(a["sin"], kdt)
+        if misalign:
+            cos, sin = shifted(cos), shifted(sin)
         index = idx(a["index"])
         opt = {k: (f32(a[k]) if k in a else None) for k in ("k_scale", "ckv_scale", "k_offset", "ckv_offset")}
 

@@ -299,14 +299,28 @@ def test_rmsnorm_rope_subnormal_and_tie_quotients(ckv_dtype):
 
 # The lean kernel takes Dv of 256, 512 or 1024 with Dk = 64, PA / PA_BNSD,
 # cache rows aligned for whole-chunk stores; the cases below reach each of its
-# template instances and the per-tensor FP8 scale forms.
+# template instances at a decode-sized and a prefill-sized batch (4803 tokens,
+# several per warp), and the per-tensor FP8 scale forms.
+@pytest.mark.parametrize("B", [70, 4803])
 @pytest.mark.parametrize("kv_dtype", ["bf16", "f16"])
 @pytest.mark.parametrize("D,Dv", [(320, 256), (576, 512), (1088, 1024)])
-def test_rmsnorm_rope_lean_shapes(D, Dv, kv_dtype):
+def test_rmsnorm_rope_lean_shapes(D, Dv, kv_dtype, B):
     for i, (k_dtype, ckv_dtype) in enumerate([(kv_dtype, kv_dtype), (kv_dtype, "e4m3"), (kv_dtype, "e5m2"),
                                               ("i8", "i8"), ("e5m2", "e5m2")]):
-        _same(_rr("PA" if i % 2 else "PA_BNSD", B=70, S=1, D=D, Dv=Dv, kv_dtype=kv_dtype, k_dtype=k_dtype,
+        _same(_rr("PA" if i % 2 else "PA_BNSD", B=B, S=1, D=D, Dv=Dv, kv_dtype=kv_dtype, k_dtype=k_dtype,
                   ckv_dtype=ckv_dtype, seed=100 + i, slot_dtype=np.int64 if i == 3 else np.int32))
+
+
+@pytest.mark.parametrize("scale", [1 / 64, 0.013, "per_channel"])
+def test_rmsnorm_rope_ring_fp8_scales_and_unaligned_rope(scale):
+    """Prefill-sized batches with the folded and the separate FP8 scale
+    forms, with cos / sin 16-byte aligned and one element past a 16-byte
+    boundary."""
+    kw = {"ckv_scale": (2.0 ** np.random.default_rng(3).integers(-8, 0, 512)).tolist()
+          if scale == "per_channel" else [scale]}
+    case = _rr(B=4803, ckv_dtype="e4m3", seed=71, **kw)
+    _same(case)
+    _same(case, misalign=True)
 
 
 @pytest.mark.parametrize("ckv_dtype", ["e4m3", "e5m2"])
