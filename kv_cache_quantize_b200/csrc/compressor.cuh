@@ -4,21 +4,24 @@
 // softmax, the Hadamard product and the group sum in the epilogue.
 //
 // The product is computed transposed, D^T = W X^T: the UMMA M dimension is
-// 128 channels (rows of W^KV and W^Gate), N is 256 tokens, K the hidden size.
+// 128 channels (rows of W^KV and W^Gate), N is BN = 256 tokens (128 when the
+// batch is small, for twice the tiles), K the hidden size.
 // In tensor memory an accumulator row is then one channel and a column one
 // token, so the softmax over the rows of a token group (step 3) runs along a
 // single thread's TMEM row: no cross-thread reduction, and the scores never
 // leave the SM.  Two accumulators share every X tile: kv_state in TMEM
-// columns [0, 256), score_state in [256, 512) (all 512 columns of the SM).
+// columns [0, BN), score_state in [BN, 2 BN) (all 512 columns of the SM at
+// BN = 256).
 //
 // Roles (192 threads, one CTA per SM, persistent over tiles of 128 channels
-// x 256 tokens; the four channel tiles of a token tile are adjacent tile
+// x BN tokens; the four channel tiles of a token tile are adjacent tile
 // numbers, so they run together and read the X tile from L2 once):
-//   warp 0, one lane: TMA producer -- a 3-stage ring of K slices of 64
-//     (W^KV 128x64, W^Gate 128x64 and X 256x64 bf16 boxes, 128-byte swizzle),
+//   warp 0, one lane: TMA producer -- a ring (3 stages at BN = 256, 4 at 128)
+//     of K slices of 64 (W^KV 128x64, W^Gate 128x64 and X BNx64 bf16 boxes,
+//     128-byte swizzle),
 //     completion counted in bytes on the stage's `full` mbarrier;
 //   warp 1: allocates TMEM; one lane issues tcgen05.mma (kind::f16, bf16 in,
-//     fp32 accumulate, M 128, N 256, K 16) and commits each stage to its
+//     fp32 accumulate, M 128, N BN, K 16) and commits each stage to its
 //     `empty` barrier and each finished tile to `tmem_full`;
 //   warps 2-5: the epilogue -- warp w reads TMEM lanes 32 (w % 4) .. +31 (the
 //     lane quarter its hardware subpartition may access), i.e. 32 channels,
@@ -39,17 +42,18 @@
 namespace kvq {
 
 constexpr int CP_BM = 128;                      // channels per tile (UMMA M)
-constexpr int CP_BN = 256;                      // tokens per tile (UMMA N)
+constexpr int CP_BN = 256;                      // tokens per tile (UMMA N), the large-batch width
 constexpr int CP_BK = 64;                       // K per stage: one 128-byte swizzle row of bf16
 constexpr int CP_UK = 16;                       // K of one tcgen05.mma kind::f16
-constexpr int CP_STAGES = 3;
 constexpr int CP_THREADS = 192;
 constexpr uint32_t CP_A_BYTES = CP_BM * CP_BK * 2;                  // 16 KB
-constexpr uint32_t CP_B_BYTES = CP_BN * CP_BK * 2;                  // 32 KB
-constexpr uint32_t CP_STAGE_BYTES = 2 * CP_A_BYTES + CP_B_BYTES;    // 64 KB
-constexpr uint32_t CP_TMEM_COLS = 512;
-constexpr uint32_t CP_GATE_COL = 256;
-constexpr uint32_t CP_SMEM_BYTES = CP_STAGES * CP_STAGE_BYTES + 256 + 1024;   // + barriers + alignment slack
+
+// the ring and tensor-memory shape for a token-tile width BN (256 or 128)
+__host__ __device__ constexpr int cp_stages(int bn) { return bn == 256 ? 3 : 4; }
+__host__ __device__ constexpr uint32_t cp_stage_bytes(int bn) { return 2 * CP_A_BYTES + (uint32_t)bn * CP_BK * 2; }
+__host__ __device__ constexpr uint32_t cp_smem_bytes(int bn) {
+    return (uint32_t)cp_stages(bn) * cp_stage_bytes(bn) + 256 + 1024;   // + barriers + alignment slack
+}
 constexpr uint64_t CP_WAIT_NS = 2000000000ull;     // every wait gives up after 2 s (a tile takes < 1 ms)
 
 struct CompressorArgs {
@@ -57,7 +61,7 @@ struct CompressorArgs {
     int32_t H;             // hidden size (a multiple of 64)
     int32_t D;             // channels (a multiple of 128)
     int32_t n_ch_tiles;    // D / 128
-    int64_t n_tok_tiles;   // ceil(T / 256)
+    int64_t n_tok_tiles;   // ceil(T / BN)
     const float* ape;      // [ratio, D]
     uint16_t* out;         // bf16 [T / ratio, D]
 };
@@ -162,10 +166,15 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 
 // ---------------------------------------------------------------------------
-template <int RATIO>
+template <int RATIO, int BN>
 __global__ void __launch_bounds__(CP_THREADS, 1)
     compressor_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wkv,
                       const __grid_constant__ CUtensorMap tm_wg, const CompressorArgs a) {
+    static_assert(BN == 256 || BN == 128, "token tile");
+    constexpr int CP_STAGES = cp_stages(BN);
+    constexpr uint32_t CP_STAGE_BYTES = cp_stage_bytes(BN);
+    constexpr uint32_t CP_TMEM_COLS = 2 * BN;          // a power of two >= 32
+    constexpr uint32_t CP_GATE_COL = BN;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t* tiles = smem_raw + ((1024u - (raw & 1023u)) & 1023u);      // 1024-byte aligned swizzle atoms
@@ -206,7 +215,7 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
             uint32_t it = 0;
             bool dead = false;
             for (int64_t tile = blockIdx.x; tile < ntiles && !dead; tile += gridDim.x) {
-                const int32_t tok0 = (int32_t)((tile / a.n_ch_tiles) * CP_BN);
+                const int32_t tok0 = (int32_t)((tile / a.n_ch_tiles) * BN);
                 const int32_t ch0 = (int32_t)((tile % a.n_ch_tiles) * CP_BM);
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const uint32_t st = it % CP_STAGES, round = it / CP_STAGES;
@@ -228,7 +237,7 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            constexpr uint32_t IDESC = umma_idesc_bf16(CP_BM, CP_BN);
+            constexpr uint32_t IDESC = umma_idesc_bf16(CP_BM, BN);
             uint32_t it = 0, tl = 0;
             bool dead = false;
             for (int64_t tile = blockIdx.x; tile < ntiles && !dead; tile += gridDim.x, ++tl) {
@@ -266,12 +275,12 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
         const uint32_t tbase = tmem + ((uint32_t)(sub * 32) << 16);
         uint32_t tl = 0;
         for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
-            const int64_t tok0 = (tile / a.n_ch_tiles) * CP_BN;
+            const int64_t tok0 = (tile / a.n_ch_tiles) * BN;
             const int ch = (int)((tile % a.n_ch_tiles) * CP_BM) + row;
             if (!__all_sync(FULL_MASK, mbar_wait_ns(tmem_full, tl & 1u, CP_WAIT_NS))) break;
             tc_fence_after();
             float m = -INFINITY, l = 0.0f, acc = 0.0f;
-            for (int c0 = 0; c0 < CP_BN; c0 += 32) {
+            for (int c0 = 0; c0 < BN; c0 += 32) {
                 if (tok0 + c0 >= a.T) break;                 // ragged last tile (warp-uniform)
                 uint32_t kv[32], gs[32];
                 tmem_ld32x2(tbase + (uint32_t)c0, tbase + CP_GATE_COL + (uint32_t)c0, kv, gs);

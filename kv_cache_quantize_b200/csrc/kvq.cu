@@ -1301,33 +1301,42 @@ kvq_status kvq_compressor(const kvq_tensor* x, const kvq_tensor* w_kv, const kvq
     auto a16 = [](const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; };
     if (!a16(x->data) || !a16(w_kv->data) || !a16(w_gate->data)) return KVQ_ERR_LAYOUT;   // TMA base alignment
 
+    // token tiles of 256, or of 128 when 256-token tiles would fill at most
+    // half of the SMs (twice the tiles for a small batch)
+    const int64_t n_ch = D / CP_BM;
+    const int bn = 2 * ((T + 255) / 256) * n_ch <= (int64_t)sm_count() ? 128 : 256;
     CUtensorMap mx, mk, mg;
-    if (!bf16_tile_map(&mx, x->data, T, H, H, CP_BN) || !bf16_tile_map(&mk, w_kv->data, D, H, H, CP_BM) ||
+    if (!bf16_tile_map(&mx, x->data, T, H, H, (uint32_t)bn) || !bf16_tile_map(&mk, w_kv->data, D, H, H, CP_BM) ||
         !bf16_tile_map(&mg, w_gate->data, D, H, H, CP_BM))
         return KVQ_ERR_CUDA;
     CompressorArgs a;
     a.T = T;
     a.H = (int32_t)H;
     a.D = (int32_t)D;
-    a.n_ch_tiles = (int32_t)(D / CP_BM);
-    a.n_tok_tiles = (T + CP_BN - 1) / CP_BN;
+    a.n_ch_tiles = (int32_t)n_ch;
+    a.n_tok_tiles = (T + bn - 1) / bn;
     a.ape = static_cast<const float*>(ape->data);
     a.out = static_cast<uint16_t*>(cmp_kv->data);
     const int64_t tiles = a.n_tok_tiles * a.n_ch_tiles;
+    const size_t smem = cp_smem_bytes(bn);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     auto run = [&](auto kernel) {
-        return launched(launch(kernel, (unsigned)persistent_grid(kernel, CP_THREADS, tiles, CP_SMEM_BYTES),
-                               CP_THREADS, CP_SMEM_BYTES, s, mx, mk, mg, a));
+        return launched(launch(kernel, (unsigned)persistent_grid(kernel, CP_THREADS, tiles, smem), CP_THREADS, smem,
+                               s, mx, mk, mg, a));
     };
-    switch (cmp_ratio) {
-        case 2: return run(compressor_kernel<2>);
-        case 4: return run(compressor_kernel<4>);
-        case 8: return run(compressor_kernel<8>);
-        case 16: return run(compressor_kernel<16>);
-        case 32: return run(compressor_kernel<32>);
-        case 64: return run(compressor_kernel<64>);
-        default: return run(compressor_kernel<128>);
+#define KVQ_CP_RATIOS(BN)                                 \
+    switch (cmp_ratio) {                                  \
+        case 2: return run(compressor_kernel<2, BN>);     \
+        case 4: return run(compressor_kernel<4, BN>);     \
+        case 8: return run(compressor_kernel<8, BN>);     \
+        case 16: return run(compressor_kernel<16, BN>);   \
+        case 32: return run(compressor_kernel<32, BN>);   \
+        case 64: return run(compressor_kernel<64, BN>);   \
+        default: return run(compressor_kernel<128, BN>);  \
     }
+    if (bn == 128) KVQ_CP_RATIOS(128);
+    KVQ_CP_RATIOS(256);
+#undef KVQ_CP_RATIOS
 }
 
 // ---------------------------------------------------------------------------

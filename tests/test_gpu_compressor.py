@@ -74,13 +74,24 @@ def _check(case, groups=None):
 @pytest.mark.parametrize("D", [128, 512])
 @pytest.mark.parametrize("ratio", [2, 4, 8, 16, 32, 64, 128])
 def test_compressor_ratios(ratio, D):
-    """Three token tiles (768 rows), every ratio, both channel counts."""
+    """768 rows (six 128-token tiles), every ratio, both channel counts."""
     _check(W.gen_compressor(f"cp_r{ratio}_D{D}", T=768, H=1024, D=D, ratio=ratio, seed=ratio + D))
+
+
+@pytest.mark.parametrize("ratio", [2, 32, 128])
+def test_compressor_wide_token_tiles(ratio):
+    """A batch large enough for 256-token tiles (T 5120, D 512: 80 tiles);
+    the cases above, at most 74 tiles of 256, run 128-token tiles."""
+    _check(W.gen_compressor(f"cp_wide_r{ratio}", T=5120, H=1024, D=512, ratio=ratio, seed=7 + ratio))
+
+
+def test_compressor_wide_token_tiles_d128():
+    _check(W.gen_compressor("cp_wide_d128", T=19200, H=1024, D=128, ratio=64, seed=11))
 
 
 @pytest.mark.parametrize("T", [128, 384, 2176])
 def test_compressor_ragged_token_tiles(T):
-    """T not a multiple of the 256-token tile: the last tile holds one group."""
+    """T not a multiple of the token tile: the last tile holds one group."""
     _check(W.gen_compressor(f"cp_T{T}", T=T, H=2048, D=512, ratio=128, seed=T))
 
 
