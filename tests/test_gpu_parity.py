@@ -226,7 +226,7 @@ def test_indexer_bad_slot_fault():
 # kv_rmsnorm_rope_cache
 # ---------------------------------------------------------------------------
 def _rr(cache_mode="PA_BNSD", B=40, S=1, k_dtype="bf16", ckv_dtype="e4m3", kv_dtype="bf16", D=576, Dv=512,
-        seed=0, **kw):
+        seed=0, block_size=32, **kw):
     opt = {"block_pad_bytes": 64}
     if ckv_dtype in ("e4m3", "e5m2", "i8"):
         opt["ckv_scale"] = [1 / 64]
@@ -236,7 +236,8 @@ def _rr(cache_mode="PA_BNSD", B=40, S=1, k_dtype="bf16", ckv_dtype="e4m3", kv_dt
         opt["ckv_offset"] = [2.0]
     opt.update(kw)
     return W.gen_rmsnorm_rope(f"rr_{cache_mode}_{k_dtype}_{ckv_dtype}_{kv_dtype}_D{D}", B=B, S=S, D=D, Dv=Dv,
-                              num_blocks=max(B + 1, (2 * B * S) // 32 + 2), block_size=32, k_dtype=k_dtype,
+                              num_blocks=max(B + 1, (2 * B * S) // block_size + 2), block_size=block_size,
+                              k_dtype=k_dtype,
                               ckv_dtype=ckv_dtype, cache_mode=cache_mode, skip_frac=0.1, seed=seed,
                               kv_dtype=kv_dtype, **opt)
 
@@ -349,6 +350,31 @@ def test_rmsnorm_rope_cache_row_alignment(ckv_dtype, pad):
     the lean kernel takes the 8-aligned FP8 cache, the general kernel the
     rest."""
     _same(_rr(B=60, ckv_dtype=ckv_dtype, seed=67, block_pad_bytes=pad))
+
+
+@pytest.mark.parametrize("ckv_dtype,block_size", [("bf16", 48), ("e4m3", 96)])
+@pytest.mark.parametrize("B", [70, 4803])
+def test_rmsnorm_rope_block_size_not_power_of_two(ckv_dtype, block_size, B):
+    """Slots map to (block, row) by division when blockSize is not a power of
+    two (48 for 16-bit caches, 96 for a 1-byte ckv cache: the page's multiples
+    of 16 and 32)."""
+    _same(_rr(B=B, ckv_dtype=ckv_dtype, seed=73, block_size=block_size))
+
+
+@pytest.mark.parametrize("D,Dv,cache_mode", [(576, 512, "PA_BNSD"), (576, 512, "PA"), (192, 128, "PA_BNSD")])
+@pytest.mark.parametrize("slot_dtype", [np.int32, np.int64])
+def test_rmsnorm_rope_bad_index_fault(D, Dv, cache_mode, slot_dtype):
+    """Index entries past the cache, negative ones other than -1, and (int64)
+    one at 2^31: each such token is skipped and the fault bit is raised, as
+    the oracle does."""
+    case = _rr(cache_mode, B=60, D=D, Dv=Dv, seed=79, slot_dtype=slot_dtype)
+    idx = case.arrays["index"].reshape(-1)
+    n = case.caches["k_cache"].num_slots
+    idx[5] = n
+    idx[17] = -7
+    if slot_dtype == np.int64:
+        idx[31] = 2 ** 31
+    _same(case)
 
 
 @pytest.mark.parametrize("ckv_dtype", ["bf16", "e4m3", "i8"])
