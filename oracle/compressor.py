@@ -5,7 +5,9 @@ import this module.  It shares no code with the CUDA library and the library
 never calls it.
 
 Source: aclnnCompressor (CANN ops-transformer), 接口功能 and 计算公式 steps 1-5,
-the C128A form (coff = 1, no overlap between neighbouring groups):
+the C128A form (coff = 1, no overlap between neighbouring groups) in
+compressor(), and the C4A form (coff = 2, cmp_ratio = 4, each group's eight
+rows reaching into the next group) in compressor_c4a():
 
   1. [kv_state, score_state] = X @ [W^KV, W^Gate]   (W given as [coff*D, H] rows,
      so the product with a weight is X @ W^T)
@@ -34,7 +36,10 @@ rounding only), so the oracle's result is the exact value of the formula to
 about 1e-15 relative, and the bf16 output of the device is compared with it
 within a tolerance derived from binary32 accumulation and one bf16 rounding.
 
-Pinned by tests/test_oracle_compressor.py: hand-worked examples
+Pinned by tests/test_oracle_compressor.py (C4A: the eight-row mean when
+W^Gate = 0 and Ape = 0, selection of an a row or a b row by a dominant Ape
+entry, the last group's four rows, locality, convexity, per-channel shift
+invariance): hand-worked examples
 (tests/golden/compressor_examples.txt), the group mean when W^Gate = 0 and
 Ape = 0, row selection by a dominant Ape entry, invariance under a
 per-channel shift of the scores, sensitivity to a per-row shift,
@@ -96,6 +101,52 @@ def compressor(x: np.ndarray, w_kv: np.ndarray, w_gate: np.ndarray, ape: np.ndar
         x = x[rows]
     kv, score = states(x, w_kv, w_gate)
     return compress_states(kv, score, ape, ratio)
+
+
+def compressor_c4a(x: np.ndarray, w_kv: np.ndarray, w_gate: np.ndarray, ape: np.ndarray,
+                   groups: Optional[Sequence[int]] = None) -> np.ndarray:
+    """The C4A-form Compressor (coff = 2, cmp_ratio = 4) in float64, by the
+    page's steps (计算公式, C4A lines), group by group:
+
+      1. [kv^a, score^a] = X @ [W^aKV, W^aGate], [kv^b, score^b] = X @ [W^bKV, W^bGate]
+      2. score'_i = [score^a[rows 4(i-1)+1 .. 4i] ; score^b[rows 4i+1 .. 4(i+1)]] + Ape
+      3. S'_i = softmax(score'_i)
+      4. (S_H)_i = S'_i (Hadamard) [kv^a[rows 4(i-1)+1 .. 4i] ; kv^b[rows 4i+1 .. 4(i+1)]]
+      5. C_i = [1]_{1 x 8} @ (S_H)_i
+
+    Readings: W^KV and W^Gate are [2D, H] (the page's [coff*D, H]) with the a
+    weights in rows [0, D) and the b weights in rows [D, 2D); Ape is
+    [4, 2D] (the page's [cmp_ratio, coff*D]): columns [0, D) are added to the
+    a rows (row r to the r-th token of the group's own four) and columns
+    [D, 2D) to the b rows (row r to the r-th token of the next four); ";"
+    stacks rows, so a group spans eight rows, its own four tokens through the
+    a projections and the next group's four through the b projections.  The
+    last group of the chunk has no next four tokens: those rows do not exist,
+    and its softmax and sum run over its own four a rows.
+
+    x: bf16 bits [T, H] (T a multiple of 4); w_kv, w_gate: bf16 bits [2D, H];
+    ape: float32 [4, 2D].  Returns C [T / 4, D] (float64), or the listed
+    groups' rows in the listed order."""
+    x = np.asarray(x)
+    T, H = x.shape
+    if T % 4:
+        raise ValueError("T must be a multiple of 4")
+    D = np.asarray(w_kv).shape[0] // 2
+    a_kv, b_kv = np.asarray(w_kv)[:D], np.asarray(w_kv)[D:]
+    a_gate, b_gate = np.asarray(w_gate)[:D], np.asarray(w_gate)[D:]
+    ape = np.asarray(ape, dtype=np.float64)
+    G = T // 4
+    out = []
+    for i in (range(G) if groups is None else groups):
+        own, nxt = x[4 * i:4 * i + 4], x[4 * i + 4:4 * i + 8]          # nxt is empty for the last group
+        kv_a, score_a = states(own, a_kv, a_gate)                        # step 1, the rows group i uses
+        kv_b, score_b = states(nxt, b_kv, b_gate)
+        score = np.vstack([score_a + ape[:, :D], score_b + ape[:len(nxt), D:]])     # step 2
+        kv = np.vstack([kv_a, kv_b])
+        e = np.exp(score - score.max(axis=0, keepdims=True))             # step 3 (an exact shift)
+        p = e / e.sum(axis=0, keepdims=True)
+        out.append(np.ones(len(score)) @ (p * kv))                       # steps 4, 5
+    return np.array(out).reshape(-1, D)
 
 
 def abs_states(x: np.ndarray, w_kv: np.ndarray, w_gate: np.ndarray, groups: Sequence[int], ratio: int):

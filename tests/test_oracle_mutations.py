@@ -122,6 +122,19 @@ COMPRESSOR_MUTANTS = {
     "bf16 decoded with the wrong shift": ("(b.astype(np.uint32) << 16)", "(b.astype(np.uint32) << 15)"),
     "stability shift taken per row (over channels)": ("s = s - s.max(axis=1, keepdims=True)",
                                                       "s = s - s.max(axis=2, keepdims=True)"),
+    "C4A: b rows from the previous group": ("nxt = x[4 * i:4 * i + 4], x[4 * i + 4:4 * i + 8]",
+                                            "nxt = x[4 * i:4 * i + 4], x[max(4 * i - 4, 0):4 * i]"),
+    "C4A: a and b weights swapped": ("a_kv, b_kv = np.asarray(w_kv)[:D], np.asarray(w_kv)[D:]",
+                                     "b_kv, a_kv = np.asarray(w_kv)[:D], np.asarray(w_kv)[D:]"),
+    "C4A: Ape's a and b columns swapped": ("np.vstack([score_a + ape[:, :D], score_b + ape[:len(nxt), D:]])",
+                                           "np.vstack([score_a + ape[:, D:], score_b + ape[:len(nxt), :D]])"),
+    "C4A: last group padded with zero rows": (
+        "own, nxt = x[4 * i:4 * i + 4], x[4 * i + 4:4 * i + 8]",
+        "own, nxt = x[4 * i:4 * i + 4], np.vstack([x[4 * i + 4:4 * i + 8], "
+        "np.zeros((4 - len(x[4 * i + 4:4 * i + 8]), x.shape[1]), x.dtype)])"),
+    "C4A: softmax over channels": ("p = e / e.sum(axis=0, keepdims=True)", "p = e / e.sum(axis=1, keepdims=True)"),
+    "C4A: gate weights of a used for b": ("a_gate, b_gate = np.asarray(w_gate)[:D], np.asarray(w_gate)[D:]",
+                                          "a_gate, b_gate = np.asarray(w_gate)[:D], np.asarray(w_gate)[:D]"),
 }
 
 
