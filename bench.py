@@ -104,8 +104,8 @@ def algorithmic_bytes(case) -> int:
 
 def contraction_flops(case) -> int:
     """FLOPs of the Compressor's two projections (x @ W^KV^T and x @ W^Gate^T):
-    2 T H D each; the softmax epilogue (a few operations per output of the
-    projections) is not counted."""
+    2 T H R each for weights of R = coff D rows; the softmax epilogue (a few
+    operations per output of the projections) is not counted."""
     T, H = case.arrays["x"].shape
     D = case.arrays["w_kv"].shape[0]
     return 2 * T * H * 2 * D

@@ -265,23 +265,32 @@ KVQ_API kvq_status kvq_dequant_rope_quant_kvcache(const kvq_tensor* x, const kvq
                                           kvq_tensor* v_out, kvq_stream stream);
 
 /* ------------------------------------------------------------------------ */
-/* compressor: the token Compressor, C128A form (coff = 1)                   */
+/* compressor: the token Compressor, C128A form (coff = 1) and C4A / C4Li   */
+/* form (coff = 2, cmp_ratio = 4)                                            */
 /* Source: aclnnCompressor, 接口功能 / 计算公式 steps 1-5 / 约束说明.          */
 /*                                                                           */
-/* Per group i of cmp_ratio consecutive token rows and per channel c:        */
+/* C128A (w_kv [D, H]): per group i of cmp_ratio consecutive token rows and  */
+/* per channel c:                                                            */
 /*   kv_state = X @ W^KV^T, score_state = X @ W^Gate^T (step 1),             */
 /*   s_r = score_state[r, c] + ape[r mod cmp_ratio, c] (step 2),             */
 /*   p = softmax over the group's rows of s (step 3, channel by channel),    */
 /*   cmp_kv[i, c] = sum_r p_r kv_state[r, c] (steps 4-5), rounded to bf16.   */
+/* C4A (w_kv [2D, H], cmp_ratio 4): rows [0, D) of w_kv / w_gate are the a   */
+/*   weights, rows [D, 2D) the b weights; group i takes its own four tokens  */
+/*   4i .. 4i+3 through the a weights (scores + ape[p, c]) and the next four */
+/*   4i+4 .. 4i+7 through the b weights (scores + ape[p, D + c]); the        */
+/*   softmax and the sum run over those eight rows, and over the own four    */
+/*   alone for the last group of the chunk (no next tokens).                 */
 /* x       bf16 [..., H], contiguous, 16-byte aligned; the leading dims are   */
 /*         the T token rows, T % cmp_ratio == 0 (whole groups: the stateless  */
 /*         case; the page's state cache, start_pos and cu_seqlens are not     */
 /*         modelled).  1024 <= H <= 10240, H % 512 == 0.                     */
-/* w_kv,   bf16 [D, H] (the page's [coff*D, H] with coff = 1), contiguous,    */
-/* w_gate  16-byte aligned; D = 128 or 512.                                   */
-/* ape     f32 [cmp_ratio, D], contiguous.                                    */
+/* w_kv,   bf16 [coff*D, H], contiguous, 16-byte aligned; D = 128 or 512;     */
+/* w_gate  coff (1 or 2) follows from w_kv's rows and cmp_kv's D.             */
+/* ape     f32 [cmp_ratio, coff*D], contiguous.                               */
 /* cmp_kv  bf16 [T / cmp_ratio, D], contiguous: written.                     */
-/* cmp_ratio  2, 4, 8, 16, 32, 64 or 128 (C128A: 128).                        */
+/* cmp_ratio  2, 4, 8, 16, 32, 64 or 128 (C128A: 128); 4 when coff = 2,       */
+/*         else KVQ_ERR_ATTR.                                                 */
 /* Arithmetic: bf16 products with fp32 accumulation on the tensor cores       */
 /* (tcgen05), the softmax in fp32; the result is within the bound of fp32     */
 /* accumulation of the exact value, not bit-reproducible against another      */

@@ -295,12 +295,17 @@ def dequant_rope_quant_kvcache(x: torch.Tensor, cos: torch.Tensor, sin: torch.Te
 def compressor(x: torch.Tensor, w_kv: torch.Tensor, w_gate: torch.Tensor, ape: torch.Tensor,
                cmp_kv: Optional[torch.Tensor] = None, cmp_ratio: int = 128, stream=None,
                check: bool = False) -> torch.Tensor:
-    """The token Compressor, C128A form (see kvq_compressor): per group of cmp_ratio token rows
-    and channel, the softmax over the group of (x @ w_gate^T + ape) weights x @ w_kv^T.
-    Returns cmp_kv [T / cmp_ratio, D] (allocated when not given)."""
+    """The token Compressor (see kvq_compressor): C128A form with w_kv [D, H] -- per group of
+    cmp_ratio token rows and channel, the softmax over the group of (x @ w_gate^T + ape)
+    weights x @ w_kv^T -- or C4A / C4Li form with w_kv [2D, H] and cmp_ratio 4 (a group's own
+    four tokens through the first D weight rows, the next four through the last D).
+    Returns cmp_kv [T / cmp_ratio, D] (allocated when not given: D is w_kv's rows when they
+    are 128 or 512, else half of them)."""
     if cmp_kv is None:
         T = x.numel() // x.shape[-1] if x.dim() else 0
-        cmp_kv = torch.empty((T // max(1, int(cmp_ratio)), w_kv.shape[0]), dtype=torch.bfloat16, device=x.device)
+        rows = w_kv.shape[0]
+        D = rows if rows in (128, 512) else rows // 2
+        cmp_kv = torch.empty((T // max(1, int(cmp_ratio)), D), dtype=torch.bfloat16, device=x.device)
     with _on(_one_device("compressor", x, w_kv, w_gate, ape, cmp_kv)):
         st = _stream(stream, x)
         _check("compressor", lib().kvq_compressor(_ref(desc(x)), _ref(desc(w_kv)), _ref(desc(w_gate)),

@@ -78,6 +78,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+// 4-D tiled TMA load of box {x, y, z, w} (x innermost) into this CTA's shared memory
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int32_t x, int32_t y, int32_t z,
+                                            int32_t w, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::
+            "r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
                  : "memory");
@@ -166,11 +176,20 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 
 // ---------------------------------------------------------------------------
-template <int RATIO, int BN>
+template <int RATIO, int BN, int COFF = 1>
 __global__ void __launch_bounds__(CP_THREADS, 1)
     compressor_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wkv,
                       const __grid_constant__ CUtensorMap tm_wg, const CompressorArgs a) {
     static_assert(BN == 256 || BN == 128, "token tile");
+    static_assert(COFF == 1 || (COFF == 2 && RATIO == 4), "the C4A form has cmp_ratio 4");
+    // COFF 2: 64 channels per tile, their a and b weight rows interleaved in
+    // blocks of 8 (rows 16k .. 16k+7: a channels ch0 + 8k .. +7, rows
+    // 16k+8 .. +15: the b channels of the same; one 4-D TMA box per weight
+    // and stage), and token tiles overlapping
+    // by one 4-token window (each tile starts BN - 4 tokens after the
+    // previous one), so that every group's next four tokens sit in its tile
+    constexpr int CH_TILE = COFF == 1 ? CP_BM : CP_BM / 2;
+    constexpr int TOK_STEP = COFF == 1 ? BN : BN - 4;
     constexpr int CP_STAGES = cp_stages(BN);
     constexpr uint32_t CP_STAGE_BYTES = cp_stage_bytes(BN);
     constexpr uint32_t CP_TMEM_COLS = 2 * BN;          // a power of two >= 32
@@ -215,8 +234,8 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
             uint32_t it = 0;
             bool dead = false;
             for (int64_t tile = blockIdx.x; tile < ntiles && !dead; tile += gridDim.x) {
-                const int32_t tok0 = (int32_t)((tile / a.n_ch_tiles) * BN);
-                const int32_t ch0 = (int32_t)((tile % a.n_ch_tiles) * CP_BM);
+                const int32_t tok0 = (int32_t)((tile / a.n_ch_tiles) * TOK_STEP);
+                const int32_t ch0 = (int32_t)((tile % a.n_ch_tiles) * CH_TILE);
                 for (int kb = 0; kb < kblocks; ++kb, ++it) {
                     const uint32_t st = it % CP_STAGES, round = it / CP_STAGES;
                     if (!mbar_wait_ns(&empty[st], (round & 1u) ^ 1u, CP_WAIT_NS)) {
@@ -225,8 +244,16 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
                     }
                     uint8_t* s = tiles + st * CP_STAGE_BYTES;
                     mbar_arrive_expect_tx(&full[st], CP_STAGE_BYTES);
-                    tma_load_2d(s, &tm_wkv, kb * CP_BK, ch0, &full[st]);
-                    tma_load_2d(s + CP_A_BYTES, &tm_wg, kb * CP_BK, ch0, &full[st]);
+                    if (COFF == 1) {
+                        tma_load_2d(s, &tm_wkv, kb * CP_BK, ch0, &full[st]);
+                        tma_load_2d(s + CP_A_BYTES, &tm_wg, kb * CP_BK, ch0, &full[st]);
+                    } else {
+                        // the weights seen as [D / 8][2][8][H] (block of 8 channels, a / b
+                        // half, row, k): one box of 8 blocks x 2 halves x 8 rows x 64 k
+                        // lands rows in the interleaved order 16 block + 8 half + row
+                        tma_load_4d(s, &tm_wkv, kb * CP_BK, 0, 0, ch0 / 8, &full[st]);
+                        tma_load_4d(s + CP_A_BYTES, &tm_wg, kb * CP_BK, 0, 0, ch0 / 8, &full[st]);
+                    }
                     tma_load_2d(s + 2 * CP_A_BYTES, &tm_x, kb * CP_BK, tok0, &full[st]);
                 }
             }
@@ -275,10 +302,77 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
         const uint32_t tbase = tmem + ((uint32_t)(sub * 32) << 16);
         uint32_t tl = 0;
         for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
-            const int64_t tok0 = (tile / a.n_ch_tiles) * BN;
-            const int ch = (int)((tile % a.n_ch_tiles) * CP_BM) + row;
+            const int64_t tok0 = (tile / a.n_ch_tiles) * TOK_STEP;
             if (!__all_sync(FULL_MASK, mbar_wait_ns(tmem_full, tl & 1u, CP_WAIT_NS))) break;
             tc_fence_after();
+            if (COFF == 2) {
+                // lane l and l ^ 8 hold the a and b rows of one channel; the a
+                // lane keeps the group of each 4-token window u (its own a rows)
+                // and closes it at window u + 1 with the b lane's rows there
+                const bool is_a = (row & 8) == 0;
+                const int ch = (int)((tile % a.n_ch_tiles) * CH_TILE) + 8 * (row >> 4) + (row & 7);
+                const float* ape_a = a.ape + ch;                   // Ape[p][ch], rows of 2 D
+                const float* ape_b = a.ape + a.D + ch;             // Ape[p][D + ch]
+                float m = -INFINITY, l = 0.0f, acc = 0.0f;
+                auto update = [&](const float (&sc)[4], const float (&v)[4]) {
+                    const float mn = fmaxf(m, fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])));
+                    const float corr = ex2_approx(__fmul_rn(__fsub_rn(m, mn), LOG2E));
+                    l = __fmul_rn(l, corr);
+                    acc = __fmul_rn(acc, corr);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float p = ex2_approx(__fmul_rn(__fsub_rn(sc[i], mn), LOG2E));
+                        l = __fadd_rn(l, p);
+                        acc = __fmaf_rn(p, v[i], acc);
+                    }
+                    m = mn;
+                };
+                for (int c0 = 0; c0 < BN; c0 += 32) {
+                    if (tok0 + c0 >= a.T) break;                   // past the chunk (warp-uniform)
+                    uint32_t kv[32], gs[32];
+                    tmem_ld32x2(tbase + (uint32_t)c0, tbase + CP_GATE_COL + (uint32_t)c0, kv, gs);
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+                        const int u = c0 / 4 + w;                  // window within the tile
+                        const int64_t t4 = tok0 + 4 * u;           // its first token
+                        if (t4 >= a.T) break;                      // warp-uniform
+                        float bk[4], bg[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            bk[i] = __uint_as_float(__shfl_xor_sync(FULL_MASK, kv[4 * w + i], 8));
+                            bg[i] = __uint_as_float(__shfl_xor_sync(FULL_MASK, gs[4 * w + i], 8));
+                        }
+                        if (!is_a) continue;
+                        if (u > 0) {
+                            // window u is the b part of the group of window u - 1
+                            float sc[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) sc[i] = __fadd_rn(bg[i], __ldg(ape_b + (int64_t)i * 2 * a.D));
+                            update(sc, bk);
+                            a.out[(t4 / 4 - 1) * a.D + ch] = (uint16_t)to_bf16_bits(__fdiv_rn(acc, l));
+                        }
+                        if (u < BN / 4 - 1) {
+                            // the group of window u: its own four a rows
+                            m = -INFINITY;
+                            l = 0.0f;
+                            acc = 0.0f;
+                            float sc[4], v[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                sc[i] = __fadd_rn(__uint_as_float(gs[4 * w + i]), __ldg(ape_a + (int64_t)i * 2 * a.D));
+                                v[i] = __uint_as_float(kv[4 * w + i]);
+                            }
+                            update(sc, v);
+                            if (t4 + 4 >= a.T)                     // the last group: no next four tokens
+                                a.out[(t4 / 4) * a.D + ch] = (uint16_t)to_bf16_bits(__fdiv_rn(acc, l));
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(tmem_empty);
+                continue;
+            }
+            const int ch = (int)((tile % a.n_ch_tiles) * CP_BM) + row;
             float m = -INFINITY, l = 0.0f, acc = 0.0f;
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 if (tok0 + c0 >= a.T) break;                 // ragged last tile (warp-uniform)

@@ -1270,6 +1270,22 @@ bool bf16_tile_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The C4A weights [2 D, H] bf16 (rows [0, D) the a half, [D, 2 D) the b half)
+// as a 4-D tensor {k: H, row: 8, half: 2, block: D / 8} with 128-byte swizzled
+// boxes {64, 8, 2, 8}: one box holds 64 channels' a and b rows, interleaved in
+// blocks of 8 rows (a then b) along k slices of 64.
+bool bf16_pair_map(CUtensorMap* m, const void* base, int64_t D, int64_t H) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)H, 8, 2, (cuuint64_t)(D / 8)};
+    const cuuint64_t strides[3] = {(cuuint64_t)(H * 2), (cuuint64_t)(D * H * 2), (cuuint64_t)(8 * H * 2)};
+    const cuuint32_t box[4] = {(cuuint32_t)CP_BK, 8, 2, 8};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 kvq_status kvq_compressor(const kvq_tensor* x, const kvq_tensor* w_kv, const kvq_tensor* w_gate,
@@ -1286,13 +1302,18 @@ kvq_status kvq_compressor(const kvq_tensor* x, const kvq_tensor* w_kv, const kvq
         return KVQ_ERR_NDIM;
     const int64_t H = x->shape[x->ndim - 1];
     const int64_t T = numel_leading(x);
-    const int64_t D = w_kv->shape[0];
+    const int64_t D = cmp_kv->shape[1];
     if (H < 1024 || H > 10240 || H % 512 != 0) return KVQ_ERR_SHAPE;
     if (D != 128 && D != 512) return KVQ_ERR_SHAPE;
-    if (w_kv->shape[1] != H || w_gate->shape[0] != D || w_gate->shape[1] != H) return KVQ_ERR_SHAPE;
-    if (ape->shape[0] != cmp_ratio || ape->shape[1] != D) return KVQ_ERR_SHAPE;
+    // coff from the weights: [D, H] (the C128A form) or [2 D, H] (C4A / C4Li,
+    // cmp_ratio 4)
+    const int64_t coff = w_kv->shape[0] == D ? 1 : (w_kv->shape[0] == 2 * D ? 2 : 0);
+    if (coff == 0) return KVQ_ERR_SHAPE;
+    if (coff == 2 && cmp_ratio != 4) return KVQ_ERR_ATTR;
+    if (w_kv->shape[1] != H || w_gate->shape[0] != coff * D || w_gate->shape[1] != H) return KVQ_ERR_SHAPE;
+    if (ape->shape[0] != cmp_ratio || ape->shape[1] != coff * D) return KVQ_ERR_SHAPE;
     if (T % cmp_ratio != 0) return KVQ_ERR_SHAPE;
-    if (cmp_kv->shape[0] != T / cmp_ratio || cmp_kv->shape[1] != D) return KVQ_ERR_SHAPE;
+    if (cmp_kv->shape[0] != T / cmp_ratio) return KVQ_ERR_SHAPE;
     if (T > (int64_t)0x7fffffff - CP_BN) return KVQ_ERR_SHAPE;          // TMA coordinates are 32-bit
     if (!contiguous(x) || !contiguous(w_kv) || !contiguous(w_gate) || !contiguous(ape) || !contiguous(cmp_kv))
         return KVQ_ERR_LAYOUT;
@@ -1302,19 +1323,25 @@ kvq_status kvq_compressor(const kvq_tensor* x, const kvq_tensor* w_kv, const kvq
     if (!a16(x->data) || !a16(w_kv->data) || !a16(w_gate->data)) return KVQ_ERR_LAYOUT;   // TMA base alignment
 
     // token tiles of 256, or of 128 when 256-token tiles would fill at most
-    // half of the SMs (twice the tiles for a small batch)
-    const int64_t n_ch = D / CP_BM;
-    const int bn = 2 * ((T + 255) / 256) * n_ch <= (int64_t)sm_count() ? 128 : 256;
+    // half of the SMs (twice the tiles for a small batch).  C128A: 128 channels
+    // and BN tokens per tile; C4A: 64 channel pairs (a and b) and BN tokens,
+    // consecutive tiles BN - 4 tokens apart (BN / 4 - 1 groups each)
+    const int64_t n_ch = coff == 1 ? D / CP_BM : D / (CP_BM / 2);
+    auto tok_tiles = [&](int bn) {
+        return coff == 1 ? (T + bn - 1) / bn : (T / 4 + bn / 4 - 2) / (bn / 4 - 1);
+    };
+    const int bn = 2 * tok_tiles(256) * n_ch <= (int64_t)sm_count() ? 128 : 256;
     CUtensorMap mx, mk, mg;
-    if (!bf16_tile_map(&mx, x->data, T, H, H, (uint32_t)bn) || !bf16_tile_map(&mk, w_kv->data, D, H, H, CP_BM) ||
-        !bf16_tile_map(&mg, w_gate->data, D, H, H, CP_BM))
+    if (!bf16_tile_map(&mx, x->data, T, H, H, (uint32_t)bn)) return KVQ_ERR_CUDA;
+    if (coff == 1 ? !bf16_tile_map(&mk, w_kv->data, D, H, H, CP_BM) || !bf16_tile_map(&mg, w_gate->data, D, H, H, CP_BM)
+                  : !bf16_pair_map(&mk, w_kv->data, D, H) || !bf16_pair_map(&mg, w_gate->data, D, H))
         return KVQ_ERR_CUDA;
     CompressorArgs a;
     a.T = T;
     a.H = (int32_t)H;
     a.D = (int32_t)D;
     a.n_ch_tiles = (int32_t)n_ch;
-    a.n_tok_tiles = (T + bn - 1) / bn;
+    a.n_tok_tiles = tok_tiles(bn);
     a.ape = static_cast<const float*>(ape->data);
     a.out = static_cast<uint16_t*>(cmp_kv->data);
     const int64_t tiles = a.n_tok_tiles * a.n_ch_tiles;
@@ -1334,6 +1361,7 @@ kvq_status kvq_compressor(const kvq_tensor* x, const kvq_tensor* w_kv, const kvq
         case 64: return run(compressor_kernel<64, BN>);   \
         default: return run(compressor_kernel<128, BN>);  \
     }
+    if (coff == 2) return bn == 128 ? run(compressor_kernel<4, 128, 2>) : run(compressor_kernel<4, 256, 2>);
     if (bn == 128) KVQ_CP_RATIOS(128);
     KVQ_CP_RATIOS(256);
 #undef KVQ_CP_RATIOS

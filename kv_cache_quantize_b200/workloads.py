@@ -369,16 +369,20 @@ def dequant_rope_quant_bf16_page_B16_S1024_H3072(seed: int = 0) -> Case:
 # the token Compressor (aclnnCompressor, C128A form: D = 512, coff = 1,
 # cmp_ratio = 128; H in the page's 1K..10K range, 7168 as in DeepSeek-V3)
 # ---------------------------------------------------------------------------
-def gen_compressor(name: str, T: int, H: int, D: int, ratio: int, seed: int = 0, ape_scale: float = 1.0) -> Case:
-    """x ~ N(0, 1) bf16 [T, H]; W^KV, W^Gate ~ N(0, 1/H) bf16 [D, H] (1/sqrt(H)
+def gen_compressor(name: str, T: int, H: int, D: int, ratio: int, seed: int = 0, ape_scale: float = 1.0,
+                   coff: int = 1) -> Case:
+    """x ~ N(0, 1) bf16 [T, H]; W^KV, W^Gate ~ N(0, 1/H) bf16 [coff*D, H] (1/sqrt(H)
     initialisation, so kv_state and score_state are about N(0, 1)); Ape ~
-    N(0, ape_scale^2) float32 [ratio, D]."""
+    N(0, ape_scale^2) float32 [ratio, coff*D].  coff 2 (with ratio 4) is the
+    C4A / C4Li form."""
     x = to_bf16_bits(_rng(seed, 1).standard_normal((T, H), dtype=np.float32))
     s = np.float32(1.0 / np.sqrt(H))
-    wk = to_bf16_bits(_rng(seed, 2).standard_normal((D, H), dtype=np.float32) * s)
-    wg = to_bf16_bits(_rng(seed, 3).standard_normal((D, H), dtype=np.float32) * s)
-    ape = (_rng(seed, 4).standard_normal((ratio, D), dtype=np.float32) * np.float32(ape_scale)).astype(np.float32)
-    return Case(name, "compressor", {"x": x, "w_kv": wk, "w_gate": wg, "ape": ape}, {}, {"ratio": ratio})
+    wk = to_bf16_bits(_rng(seed, 2).standard_normal((coff * D, H), dtype=np.float32) * s)
+    wg = to_bf16_bits(_rng(seed, 3).standard_normal((coff * D, H), dtype=np.float32) * s)
+    ape = (_rng(seed, 4).standard_normal((ratio, coff * D), dtype=np.float32) * np.float32(ape_scale)).astype(
+        np.float32)
+    return Case(name, "compressor", {"x": x, "w_kv": wk, "w_gate": wg, "ape": ape}, {},
+                {"ratio": ratio, "coff": coff})
 
 
 def compressor_c128a_T65536_H7168_D512(seed: int = 0) -> Case:
@@ -389,10 +393,20 @@ def compressor_c128a_T2048_H1024_D512(seed: int = 0) -> Case:
     return gen_compressor("compressor_c128a_T2048_H1024_D512", T=2048, H=1024, D=512, ratio=128, seed=seed)
 
 
+def compressor_c4a_T65536_H7168_D512(seed: int = 0) -> Case:
+    return gen_compressor("compressor_c4a_T65536_H7168_D512", T=65536, H=7168, D=512, ratio=4, seed=seed, coff=2)
+
+
+def compressor_c4a_T2048_H1024_D512(seed: int = 0) -> Case:
+    return gen_compressor("compressor_c4a_T2048_H1024_D512", T=2048, H=1024, D=512, ratio=4, seed=seed, coff=2)
+
+
 # tensor-core workloads (a dense contraction: timed in TFLOP/s, not HBM bytes)
 TENSOR_CONFIGS = {
     "compressor_c128a_T65536_H7168_D512": compressor_c128a_T65536_H7168_D512,
     "compressor_c128a_T2048_H1024_D512": compressor_c128a_T2048_H1024_D512,
+    "compressor_c4a_T65536_H7168_D512": compressor_c4a_T65536_H7168_D512,
+    "compressor_c4a_T2048_H1024_D512": compressor_c4a_T2048_H1024_D512,
 }
 
 
@@ -527,8 +541,8 @@ def build_call(case: Case, misalign: bool = False):
     elif case.op == "compressor":
         x, wk, wg = half_tensor(a["x"], "bf16"), half_tensor(a["w_kv"], "bf16"), half_tensor(a["w_gate"], "bf16")
         ape = f32(a["ape"])
-        outs["cmp_kv"] = torch.empty((a["x"].shape[0] // at["ratio"], a["w_kv"].shape[0]), dtype=torch.bfloat16,
-                                     device=DEV)
+        outs["cmp_kv"] = torch.empty((a["x"].shape[0] // at["ratio"], a["w_kv"].shape[0] // at.get("coff", 1)),
+                                     dtype=torch.bfloat16, device=DEV)
 
         def call(stream=None):
             kvq.compressor(x, wk, wg, ape, outs["cmp_kv"], at["ratio"], stream=stream)

@@ -343,3 +343,13 @@ def test_compressor_validation(L):
     assert f(x=D([0, 1024], "bf16"), out=D([0, 512], "bf16")) == OK               # nothing to do
     assert f(x=D([2048, 1024], "bf16"), wk=D([128, 1024], "bf16"), wg=D([128, 1024], "bf16"),
              ape=D([128, 128], "f32"), out=D([16, 128], "bf16")) == ENULL          # D = 128
+    # C4A / C4Li: weights of 2 D rows, Ape [4, 2 D], cmp_ratio 4
+    w2, a2, o4 = D([1024, 1024], "bf16"), D([4, 1024], "f32"), D([512, 512], "bf16")
+    assert f(wk=w2, wg=w2, ape=a2, out=o4, ratio=4) == ENULL                       # C4A, valid
+    assert f(wk=D([256, 1024], "bf16"), wg=D([256, 1024], "bf16"), ape=D([4, 256], "f32"),
+             out=D([512, 128], "bf16"), ratio=4) == ENULL                           # C4Li, valid
+    assert f(wk=w2, wg=w2, ape=D([128, 1024], "f32"), out=out, ratio=128) == EATTR  # coff 2 needs ratio 4
+    assert f(wk=w2, wg=wk, ape=a2, out=o4, ratio=4) == ESHAPE                      # gate rows differ
+    assert f(wk=w2, wg=w2, ape=D([4, 512], "f32"), out=o4, ratio=4) == ESHAPE      # Ape [4, 2 D]
+    assert f(wk=D([768, 1024], "bf16"), wg=D([768, 1024], "bf16"), ape=D([4, 768], "f32"), out=o4,
+             ratio=4) == ESHAPE                                                    # rows neither D nor 2 D

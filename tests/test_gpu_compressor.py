@@ -1,5 +1,5 @@
 """The tcgen05 Compressor kernel against the float64 oracle (aclnnCompressor,
-计算公式 steps 1-5, C128A form), through the C ABI.
+计算公式 steps 1-5, C128A and C4A forms), through the C ABI.
 
 The kernel multiplies bf16 inputs on the tensor cores with fp32 accumulation
 and runs the softmax in fp32, so the comparison is within a bound derived
@@ -14,6 +14,10 @@ from that arithmetic, per output (group g, channel c):
                                                 R = max_r |kv_r - ref|
                + 2^-18 M                        the approximate exponential (relative error below 2^-21
                                                 per weight) and fp32 sums of <= 128 weights, M = max |kv_r|
+
+For the C4A form the same bound is taken over a group's eight rows (its own
+four tokens through the a weights, the next four through the b weights; four
+for the last group).
 
 Full-size workloads are checked on sampled groups (the first, the last and a
 spread between), which the oracle computes one by one.
@@ -69,6 +73,105 @@ def _check(case, groups=None):
     assert bad.size == 0, (f"{case.name}: {len(bad)} outputs beyond the bound, first (group, channel) "
                            f"{tuple(bad[0])}: gpu {got[tuple(bad[0])]} ref {ref[tuple(bad[0])]}")
     return got
+
+
+# ---------------------------------------------------------------------------
+# C4A / C4Li (coff = 2, cmp_ratio = 4)
+# ---------------------------------------------------------------------------
+def _bound_c4a(case, groups, ref):
+    a = case.arrays
+    x, wk, wg = a["x"], a["w_kv"], a["w_gate"]
+    T, H = x.shape
+    D = wk.shape[0] // 2
+    ape = a["ape"].astype(np.float64)
+    out = []
+    for n, i in enumerate(groups):
+        parts = [(np.arange(4 * i, 4 * i + 4), slice(0, D)), (np.arange(4 * i + 4, min(4 * i + 8, T)), slice(D, 2 * D))]
+        kv, sc, akv, ag = [], [], [], []
+        for rows, half in parts:
+            if len(rows) == 0:
+                continue
+            k_, s_ = OC.states(x[rows], wk[half], wg[half])
+            X = np.abs(OC.bf16_to_f64(x[rows]))
+            kv.append(k_)
+            sc.append(s_ + ape[:len(rows), half])
+            akv.append(X @ np.abs(OC.bf16_to_f64(wk[half])).T)
+            ag.append(X @ np.abs(OC.bf16_to_f64(wg[half])).T)
+        kv, sc, akv, ag = (np.vstack(v) for v in (kv, sc, akv, ag))
+        e_kv = (H / 16) * 2.0 ** -23 * akv.max(axis=0)
+        e_s = (H / 16) * 2.0 ** -23 * ag.max(axis=0) + 2.0 ** -24 * np.abs(sc).max(axis=0)
+        R = np.abs(kv - ref[n][None, :]).max(axis=0)
+        M = np.abs(kv).max(axis=0)
+        out.append(2.0 ** -8 * np.abs(ref[n]) + e_kv + 2 * e_s * R + 2.0 ** -18 * M)
+    return np.array(out)
+
+
+def _check_c4a(case, groups=None):
+    call, _, outs = W.build_call(case)
+    kvq.get_error()
+    call()
+    torch.cuda.synchronize()
+    assert kvq.get_error() == 0
+    got = outs["cmp_kv"].float().cpu().numpy().astype(np.float64)
+    G = case.arrays["x"].shape[0] // 4
+    groups = list(range(G)) if groups is None else list(groups)
+    a = case.arrays
+    ref = OC.compressor_c4a(a["x"], a["w_kv"], a["w_gate"], a["ape"], groups=groups)
+    got = got[groups]
+    err = np.abs(got - ref)
+    bound = _bound_c4a(case, groups, ref)
+    bad = np.argwhere(err > bound)
+    print(f"{case.name}: max |err| {err.max():.3e}, max err/bound {float((err / bound).max()):.3f}")
+    assert bad.size == 0, (f"{case.name}: {len(bad)} outputs beyond the bound, first (group, channel) "
+                           f"{tuple(bad[0])}: gpu {got[tuple(bad[0])]} ref {ref[tuple(bad[0])]}")
+    return got
+
+
+@pytest.mark.parametrize("T", [4, 8, 400, 2048, 5120])
+def test_compressor_c4a(T):
+    """D 512: one group (no next tokens at all), two groups, a ragged last tile,
+    128-token tiles (T 2048: 17 tiles of 31 groups per channel tile) and
+    256-token tiles (T 5120: 21 tiles of 63 groups)."""
+    _check_c4a(W.gen_compressor(f"c4a_T{T}", T=T, H=1024, D=512, ratio=4, seed=T, coff=2))
+
+
+@pytest.mark.parametrize("T", [2048, 20480])
+def test_compressor_c4li(T):
+    """D 128 (C4Li): 128- and 256-token tiles."""
+    _check_c4a(W.gen_compressor(f"c4li_T{T}", T=T, H=1536, D=128, ratio=4, seed=T + 1, coff=2))
+
+
+@pytest.mark.parametrize("H", [1536, 10240])
+def test_compressor_c4a_hidden_sizes(H):
+    _check_c4a(W.gen_compressor(f"c4a_H{H}", T=512, H=H, D=512, ratio=4, seed=H, coff=2, ape_scale=3.0))
+
+
+def test_compressor_c4a_selects_rows():
+    """Dominant Ape entries in the a columns for half of the channels and in the
+    b columns for the other half: every output equals one kv value of the own
+    four tokens (a) or of the next four (b), which pins the pairing of the a
+    and b rows and the window of the b part on the device, up to the output
+    rounding."""
+    case = W.gen_compressor("c4a_select", T=1024, H=1024, D=128, ratio=4, seed=5, coff=2)
+    D = 128
+    rng = np.random.default_rng(11)
+    pick = rng.integers(0, 4, D)
+    ape = np.zeros((4, 2 * D), np.float32)
+    ape[pick[:64], np.arange(64)] = 80.0
+    ape[pick[64:], D + np.arange(64, 128)] = 80.0
+    case.arrays["ape"] = ape
+    _check_c4a(case)
+
+
+def test_compressor_c4a_full_size_sampled_groups():
+    case = W.compressor_c4a_T65536_H7168_D512()
+    G = case.arrays["x"].shape[0] // 4
+    # the first and last groups, tile edges of the 256-token tiles (63 groups each) and a spread
+    _check_c4a(case, groups=[0, 1, 62, 63, 64, 125, 126, 127, 4000, 9999, G - 64, G - 63, G - 2, G - 1])
+
+
+def test_compressor_c4a_small_named_workload():
+    _check_c4a(W.compressor_c4a_T2048_H1024_D512())
 
 
 @pytest.mark.parametrize("D", [128, 512])
