@@ -306,27 +306,19 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
             if (!__all_sync(FULL_MASK, mbar_wait_ns(tmem_full, tl & 1u, CP_WAIT_NS))) break;
             tc_fence_after();
             if (COFF == 2) {
-                // lane l and l ^ 8 hold the a and b rows of one channel; the a
-                // lane keeps the group of each 4-token window u (its own a rows)
-                // and closes it at window u + 1 with the b lane's rows there
+                // lane l and l ^ 8 hold the a and b rows of one channel.  In every
+                // 4-token window both lanes reduce their own four rows (softmax
+                // maximum, weight sum, weighted kv sum): the a lane those of the
+                // group that the window opens, the b lane the next-window half of
+                // the group that the window closes; the b lane's three values then
+                // cross to the a lane, which merges them with the a part it kept
+                // from the previous window and writes the closed group.
                 const bool is_a = (row & 8) == 0;
                 const int ch = (int)((tile % a.n_ch_tiles) * CH_TILE) + 8 * (row >> 4) + (row & 7);
-                const float* ape_a = a.ape + ch;                   // Ape[p][ch], rows of 2 D
-                const float* ape_b = a.ape + a.D + ch;             // Ape[p][D + ch]
-                float m = -INFINITY, l = 0.0f, acc = 0.0f;
-                auto update = [&](const float (&sc)[4], const float (&v)[4]) {
-                    const float mn = fmaxf(m, fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])));
-                    const float corr = ex2_approx(__fmul_rn(__fsub_rn(m, mn), LOG2E));
-                    l = __fmul_rn(l, corr);
-                    acc = __fmul_rn(acc, corr);
+                float ap[4];                                       // this lane's Ape column, rows of 2 D
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float p = ex2_approx(__fmul_rn(__fsub_rn(sc[i], mn), LOG2E));
-                        l = __fadd_rn(l, p);
-                        acc = __fmaf_rn(p, v[i], acc);
-                    }
-                    m = mn;
-                };
+                for (int i = 0; i < 4; ++i) ap[i] = __ldg(a.ape + (int64_t)i * 2 * a.D + (is_a ? 0 : a.D) + ch);
+                float pm = 0.0f, pl = 0.0f, pacc = 0.0f;            // the open group's a part (a lanes)
                 for (int c0 = 0; c0 < BN; c0 += 32) {
                     if (tok0 + c0 >= a.T) break;                   // past the chunk (warp-uniform)
                     uint32_t kv[32], gs[32];
@@ -336,35 +328,36 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
                         const int u = c0 / 4 + w;                  // window within the tile
                         const int64_t t4 = tok0 + 4 * u;           // its first token
                         if (t4 >= a.T) break;                      // warp-uniform
-                        float bk[4], bg[4];
+                        float sc[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) sc[i] = __fadd_rn(__uint_as_float(gs[4 * w + i]), ap[i]);
+                        const float cm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+                        float l = 0.0f, acc = 0.0f;
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            bk[i] = __uint_as_float(__shfl_xor_sync(FULL_MASK, kv[4 * w + i], 8));
-                            bg[i] = __uint_as_float(__shfl_xor_sync(FULL_MASK, gs[4 * w + i], 8));
+                            const float p = ex2_approx(__fmul_rn(__fsub_rn(sc[i], cm), LOG2E));
+                            l = __fadd_rn(l, p);
+                            acc = __fmaf_rn(p, __uint_as_float(kv[4 * w + i]), acc);
                         }
+                        const float om = __shfl_xor_sync(FULL_MASK, cm, 8);
+                        const float ol = __shfl_xor_sync(FULL_MASK, l, 8);
+                        const float oacc = __shfl_xor_sync(FULL_MASK, acc, 8);
                         if (!is_a) continue;
                         if (u > 0) {
-                            // window u is the b part of the group of window u - 1
-                            float sc[4];
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) sc[i] = __fadd_rn(bg[i], __ldg(ape_b + (int64_t)i * 2 * a.D));
-                            update(sc, bk);
-                            a.out[(t4 / 4 - 1) * a.D + ch] = (uint16_t)to_bf16_bits(__fdiv_rn(acc, l));
+                            // close the group of window u - 1: its a part and this window's b part
+                            const float mn = fmaxf(pm, om);
+                            const float ca = ex2_approx(__fmul_rn(__fsub_rn(pm, mn), LOG2E));
+                            const float cb = ex2_approx(__fmul_rn(__fsub_rn(om, mn), LOG2E));
+                            const float L = __fmaf_rn(ol, cb, __fmul_rn(pl, ca));
+                            const float A = __fmaf_rn(oacc, cb, __fmul_rn(pacc, ca));
+                            a.out[(t4 / 4 - 1) * a.D + ch] = (uint16_t)to_bf16_bits(__fdiv_rn(A, L));
                         }
                         if (u < BN / 4 - 1) {
-                            // the group of window u: its own four a rows
-                            m = -INFINITY;
-                            l = 0.0f;
-                            acc = 0.0f;
-                            float sc[4], v[4];
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                sc[i] = __fadd_rn(__uint_as_float(gs[4 * w + i]), __ldg(ape_a + (int64_t)i * 2 * a.D));
-                                v[i] = __uint_as_float(kv[4 * w + i]);
-                            }
-                            update(sc, v);
                             if (t4 + 4 >= a.T)                     // the last group: no next four tokens
                                 a.out[(t4 / 4) * a.D + ch] = (uint16_t)to_bf16_bits(__fdiv_rn(acc, l));
+                            pm = cm;
+                            pl = l;
+                            pacc = acc;
                         }
                     }
                 }
