@@ -5,10 +5,11 @@ allocation, no synchronisation), so a serving loop can capture a whole
 epilogue step once and replay it.  Checked here: a graph holding one call of
 every operation (the pipelined and the direct compress kernels, bf16 and
 float16 x, the indexer, the rmsnorm/rope kernel, the pipelined dequant
-kernel, the packed-row decoder and the tcgen05 Compressor), replayed on caches
-reset to their initial bytes, leaves every cache and output identical, byte
-for byte, to the CPU oracle's result -- the Compressor's output to the same
-call run eagerly (its parity with the oracle is a bound, tested elsewhere).
+kernel, the packed-row decoder and the tcgen05 Compressor in its C128A and
+C4A forms), replayed on caches reset to their initial bytes, leaves every
+cache and output identical, byte for byte, to the CPU oracle's result -- the
+Compressor's outputs to the same calls run eagerly (their parity with the
+oracle is a bound, tested elsewhere).
 """
 import numpy as np
 import pytest
@@ -53,12 +54,14 @@ def test_graph_replay_matches_oracle():
     slots = torch.from_numpy(np.ascontiguousarray(ce.arrays["slot_mapping"])).cuda()
     y = torch.zeros((T, d), dtype=torch.bfloat16, device="cuda")
     cp_call, _, cp_outs = W.build_call(W.gen_compressor("g_cp", T=768, H=1024, D=512, ratio=128, seed=75))
+    c4_call, _, c4_outs = W.build_call(W.gen_compressor("g_c4a", T=512, H=1024, D=128, ratio=4, seed=76, coff=2))
 
     def step(stream):
         for call, _, _ in built:
             call(stream)
         kvq.kv_decompress(view, slots, y, 0, 64, 1.0, stream=stream)
         cp_call(stream)
+        c4_call(stream)
 
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -67,6 +70,7 @@ def test_graph_replay_matches_oracle():
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
     cp_eager = cp_outs["cmp_kv"].clone()
+    c4_eager = c4_outs["cmp_kv"].clone()
 
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
@@ -77,6 +81,7 @@ def test_graph_replay_matches_oracle():
             st[k].copy_(init[k])
     y.zero_()
     cp_outs["cmp_kv"].zero_()
+    c4_outs["cmp_kv"].zero_()
     kvq.get_error()
     g.replay()
     torch.cuda.synchronize()
@@ -101,4 +106,5 @@ def test_graph_replay_matches_oracle():
                                   y=np.zeros((T, d), dtype=np.uint16), threads=THREADS)
     assert np.array_equal(y.view(torch.int16).cpu().numpy().view(np.uint16), y_o)
     assert torch.equal(cp_outs["cmp_kv"], cp_eager)
+    assert torch.equal(c4_outs["cmp_kv"], c4_eager)
     del g
